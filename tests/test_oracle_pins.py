@@ -1,0 +1,395 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- hand-worked values, closed forms, brute force with exact rational
+arithmetic, an independent library conversion, or an invariant the pages state.
+
+Sources: "BitNet b1.58: The 1-Bit Ternary LLM Architecture Guide" (P2),
+"BitNet a4.8 Guide: 4-Bit Activation 1-Bit LLMs" (P1),
+"BitNet 2B4T Guide: Scaling Native 1.58-Bit LLMs" (P3).
+"""
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bitlinear_oracle as o
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f32_bits(values):
+    return np.asarray(values, dtype=np.float32).view(np.uint32)
+
+
+def to_bf16_bits_exact(values):
+    """bf16 bit patterns of values that are exactly representable in bf16."""
+    b = f32_bits(values)
+    assert np.all((b & 0xFFFF) == 0), "test value not exactly representable in bf16"
+    return (b >> 16).astype(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# number formats
+# ---------------------------------------------------------------------------
+
+def test_round_rational_matches_ieee_on_exact_doubles():
+    # p/q with q a power of two and p < 2^53 is an exact double, so numpy's
+    # double -> float conversion (IEEE round-to-nearest-even) is a single,
+    # correct rounding to compare against.
+    rng = np.random.default_rng(1)
+    for _ in range(3000):
+        p = int(rng.integers(1, 1 << 53))
+        sh = int(rng.integers(-60, 200))
+        if sh >= 0:
+            num, den = p, 1 << sh
+        else:
+            num, den = p << (-sh), 1
+        want = np.float32(float(Fraction(num, den)))
+        got = o.round_rational_to_f32(num, den)
+        assert got == want and np.signbit(got) == np.signbit(want), (num, den)
+
+
+def test_round_rational_hand_cases():
+    # ties to even on integers: spacing of fp32 in [2^24, 2^25) is 2
+    assert o.round_rational_to_f32((1 << 24) + 1, 1) == np.float32(1 << 24)
+    assert o.round_rational_to_f32((1 << 24) + 3, 1) == np.float32((1 << 24) + 4)
+    # well-known fp32 bit patterns of 1/3, 2/3 and 1/10
+    assert f32_bits(o.round_rational_to_f32(1, 3)) == 0x3EAAAAAB
+    assert f32_bits(o.round_rational_to_f32(2, 3)) == 0x3F2AAAAB
+    assert f32_bits(o.round_rational_to_f32(1, 10)) == 0x3DCCCCCD
+    # subnormal grid 2^-149: half of the smallest subnormal ties to 0,
+    # 1.5 units ties to 2 units
+    assert o.round_rational_to_f32(1, 1 << 150) == np.float32(0.0)
+    assert f32_bits(o.round_rational_to_f32(3, 1 << 150)) == 2
+    assert f32_bits(o.round_rational_to_f32(1, 1 << 149)) == 1
+    # carry into the next binade: 2^24 - 1/2 rounds (tie, even) to 2^24
+    assert o.round_rational_to_f32((1 << 25) - 1, 2) == np.float32(1 << 24)
+
+
+def test_bf16_rounding_hand_cases():
+    cases = {
+        1.0: 0x3F80,
+        1.0 + 2.0 ** -8: 0x3F80,            # tie between 1 and 1+2^-7 -> even
+        1.0 + 3 * 2.0 ** -8: 0x3F82,        # tie -> 1 + 2^-6 (even)
+        1.0 + 3 * 2.0 ** -9: 0x3F81,        # above the tie -> 1 + 2^-7
+        -2.5: 0xC020,
+        0.9148622047: 0x3F6A,               # 234/256
+        0.0: 0x0000,
+    }
+    for v, bits in cases.items():
+        assert int(o.round_to_bf16_bits(np.array([v]))[0]) == bits, v
+
+
+def test_bf16_rounding_matches_torch():
+    # torch's fp32 -> bf16 cast is an independent round-to-nearest-even
+    rng = np.random.default_rng(2)
+    x = np.concatenate([
+        rng.standard_normal(200000).astype(np.float32) * np.float32(10.0) ** rng.integers(-30, 30, 200000).astype(np.float32),
+        # exact ties: bf16 value + half an ulp
+        (f32_bits(rng.standard_normal(10000).astype(np.float32)) & 0xFFFF0000 | 0x8000).view(np.float32),
+    ]).astype(np.float32)
+    x = x[np.isfinite(x)]
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = o.round_to_bf16_bits(x)
+    assert np.array_equal(got, want)
+
+
+def test_bf16_bits_to_f32_exact():
+    b = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = o.bf16_bits_to_f32(b)
+    t = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).float().numpy()
+    fin = np.isfinite(t)
+    assert np.array_equal(f[fin], t[fin])
+
+
+# ---------------------------------------------------------------------------
+# [P2] eq. (1): gamma and the ternary codes
+# ---------------------------------------------------------------------------
+
+def test_exact_abs_sum_brute_force():
+    rng = np.random.default_rng(3)
+    for trial in range(20):
+        n = int(rng.integers(8, 400))
+        mags = rng.integers(-150, 60, n).astype(np.float64)
+        w = (rng.standard_normal(n) * 2.0 ** mags).astype(np.float32)
+        w[rng.random(n) < 0.1] = 0.0
+        if trial % 3 == 0:   # some subnormals
+            w[:5] = np.array([1e-45, -3e-45, 1e-40, 2e-39, -1e-38], np.float32)
+        want = sum(Fraction(float(abs(v))) for v in w) * (1 << 149)
+        assert want.denominator == 1
+        assert o.exact_abs_sum(w) == want.numerator
+        # chunking must not change the result
+        assert o.exact_abs_sum(w, chunk=7) == want.numerator
+
+
+def test_gamma_is_correctly_rounded_mean():
+    # [1, 2^-24, 2^-60, 0]: mean = 1/4 + 2^-26 + 2^-62, just above the
+    # midpoint between 0.25 and 0.25 + 2^-25 -> rounds up.  Summing in
+    # float64 first loses the 2^-60 and lands exactly on the midpoint
+    # (ties-to-even -> 0.25), so this pins the single exact rounding.
+    w = np.array([[1.0, 2.0 ** -24, 2.0 ** -60, 0.0]], np.float32)
+    assert o.absmean_scale(w) == np.float32(0.25 + 2.0 ** -25)
+    naive = np.float32(np.float64(np.abs(w).astype(np.float64).sum()) / 4)
+    assert naive == np.float32(0.25)
+    # [1, 2^-24, 2^-24, 0]: mean = 0.25 + 2^-25, exactly representable;
+    # a sequential fp32 sum gives 0.25
+    w = np.array([[1.0, 2.0 ** -24, 2.0 ** -24, 0.0]], np.float32)
+    assert o.absmean_scale(w) == np.float32(0.25 + 2.0 ** -25)
+
+
+def test_gamma_closed_forms():
+    # all |W| equal -> gamma is that value
+    w = np.full((8, 64), -0.0390625, np.float32)
+    w[::2] *= -1
+    assert o.absmean_scale(w) == np.float32(0.0390625)
+    # dyadic mean: sum |W| = 0.8125 over 4 -> 0.203125
+    assert o.absmean_scale(np.array([[0.375, -0.0625, -0.25, 0.125]], np.float32)) == np.float32(0.203125)
+    # epsilon floor
+    assert o.absmean_scale(np.zeros((3, 16), np.float32)) == o.EPS
+    assert o.absmean_scale(np.full((2, 2), 1e-7, np.float32)) == o.EPS
+    # a mean of exactly 1e-5f stays 1e-5f
+    assert o.absmean_scale(np.full((2, 2), np.float32(1e-5), np.float32)) == o.EPS
+
+
+def test_gamma_gaussian_matches_fsum():
+    # On real data the exact mean and an fp64 sum agree after rounding to
+    # fp32 except with probability ~1e-9; a mismatch here means a bug.
+    rng = np.random.default_rng(4)
+    for std in (0.02, 0.01, 1.0):
+        w = (rng.standard_normal((257, 300)) * std).astype(np.float32)
+        ref = np.float32(math.fsum(np.abs(w).astype(np.float64).ravel()) / w.size)
+        assert o.absmean_scale(w) == ref
+
+
+def test_ternary_codes_ties_and_clip():
+    # W/gamma = [0.5, -0.5, 1.5, -1.5, 0.4, 0.8, -4, 0, 2.5]
+    g = np.float32(0.25)
+    w = np.array([[0.125, -0.125, 0.375, -0.375, 0.1, 0.2, -1.0, 0.0, 0.625]], np.float32)
+    assert o.ternary_codes(w, g).tolist() == [[0, 0, 1, -1, 0, 1, -1, 0, 1]]
+
+
+def test_clip_round_commute():
+    # Round(Clip(v, -1, 1)) (P2 eq. 1) equals Clip(Round(v), -1, 1) (P1, P3)
+    rng = np.random.default_rng(5)
+    v = np.concatenate([rng.standard_normal(100000).astype(np.float32) * 3,
+                        np.array([0.5, -0.5, 1.5, -1.5, 1.0, -1.0, 0.0], np.float32)])
+    a = np.rint(np.clip(v, -1, 1))
+    b = np.clip(np.rint(v), -1, 1)
+    assert np.array_equal(a, b)
+
+
+def test_gaussian_zero_fraction():
+    # For W ~ N(0, s^2), gamma ~ E|W| = s*sqrt(2/pi) and a weight is coded 0
+    # when |W| < gamma/2: P = erf(0.5*sqrt(2/pi)/sqrt(2)) = erf(1/(2*sqrt(pi))).
+    rng = np.random.default_rng(6)
+    w = (rng.standard_normal((1000, 1000)) * 0.02).astype(np.float32)
+    c = o.ternary_codes(w, o.absmean_scale(w))
+    p0 = math.erf(1.0 / (2.0 * math.sqrt(math.pi)))
+    assert abs(p0 - 0.3101) < 1e-3
+    assert abs(float(np.mean(c == 0)) - p0) < 3e-3
+    assert set(np.unique(c).tolist()) <= {-1, 0, 1}
+    # symmetric
+    assert abs(float(np.mean(c == 1)) - float(np.mean(c == -1))) < 3e-3
+
+
+# ---------------------------------------------------------------------------
+# 2-bit storage (P1 Step 4 byte count; the bit layout is this library's)
+# ---------------------------------------------------------------------------
+
+def test_packed_layout_golden():
+    g = json.load(open(os.path.join(GOLDEN, "packed_layout.json")))
+    K = g["K"]
+    codes = np.zeros((1, K), np.int8)
+    for k, v in g["nonzero_codes"].items():
+        codes[0, int(k)] = v
+    packed = o.pack_ternary(codes)
+    assert packed.tolist() == [g["packed_bytes"]]
+    assert np.array_equal(o.unpack_ternary(packed, K), codes)
+
+
+def test_pack_roundtrip_and_size():
+    rng = np.random.default_rng(7)
+    for N, K in [(1, 16), (3, 64), (17, 256), (64, 1024)]:
+        c = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        p = o.pack_ternary(c)
+        assert p.shape == (N, K // 4) and p.nbytes == N * K * 2 // 8
+        assert np.array_equal(o.unpack_ternary(p, K), c)
+        # field value 3 never written
+        w = p.view("<u4")
+        for sh in range(0, 32, 2):
+            assert not np.any(((w >> sh) & 3) == 3)
+
+
+def test_unpack_bytewise_definition():
+    # decode one random row bit by bit from the layout definition
+    rng = np.random.default_rng(8)
+    K = 64
+    c = rng.integers(-1, 2, (1, K)).astype(np.int8)
+    p = o.pack_ternary(c)[0]
+    for k in range(K):
+        g, r = divmod(k, 16)
+        j, b = divmod(r, 4)
+        byte = p[4 * g + b]
+        assert ((int(byte) >> (2 * j)) & 3) - 1 == c[0, k]
+
+
+# ---------------------------------------------------------------------------
+# [P2] eq. (2), [P1] section 1: activation quantisation
+# ---------------------------------------------------------------------------
+
+def test_act_quant_hand_cases():
+    x = to_bf16_bits_exact([[1, -2, 0.5, 4],
+                            [127, 2.5, 3.5, -0.5],
+                            [0, 0, 0, 0],
+                            [3, 1.5, -3, 0.75]])
+    q, s = o.act_quant(x, 8)
+    assert s[0] == np.float32(31.75)
+    assert q[0].tolist() == [32, -64, 16, 127]      # -63.5 ties to -64
+    assert s[1] == np.float32(1.0)
+    assert q[1].tolist() == [127, 2, 4, 0]          # 2.5 -> 2, 3.5 -> 4, -0.5 -> -0
+    assert s[2] == np.float32(127) / np.float32(1e-5)
+    assert q[2].tolist() == [0, 0, 0, 0]
+    # fp32 product decides the code: s = f32(127/3) = 11097429 * 2^-18 and
+    # 1.5*s = 16646143.5 * 2^-18 is a tie in fp32 that rounds (to even) up
+    # to 63.5, then rint(63.5) = 64.  In exact arithmetic it would be 63.
+    assert s[3] == np.float32(11097429 * 2.0 ** -18)
+    assert q[3].tolist() == [127, 64, -127, 32]
+    assert float(Fraction(3, 2) * Fraction(127, 3)) == 63.5
+
+
+def test_act_quant_int4_hand_cases():
+    x = to_bf16_bits_exact([[7, -3.5, 2.5, 0.375, -7, 0]])
+    q, s = o.act_quant(x, 4)
+    assert s[0] == np.float32(1.0)
+    assert q[0].tolist() == [7, -4, 2, 0, -7, 0]
+
+
+def test_act_quant_invariants():
+    rng = np.random.default_rng(9)
+    xf = rng.standard_normal((64, 512)).astype(np.float32)
+    xf[:, :3] *= 20
+    xf[5] = 0
+    x = (xf.view(np.uint32) >> 16).astype(np.uint16)     # truncation is fine: any bf16 data
+    for bits in (8, 4):
+        Q = o.QMAX[bits]
+        q, s = o.act_quant(x, bits)
+        assert np.all(np.abs(q.astype(np.int32)) <= Q)          # never -Q-1
+        nz = np.any(o.bf16_bits_to_f32(x) != 0, axis=1)
+        assert np.all(np.max(np.abs(q[nz].astype(np.int32)), axis=1) == Q)
+        assert np.all(q[~nz] == 0)
+
+
+def test_a4_divide_form_is_close():
+    # P1's literal form x / (a/7) and the multiply form x * (7/a) agree on
+    # nearly every code; where they differ, by exactly one (a tie moved by
+    # one rounding).
+    rng = np.random.default_rng(10)
+    z = rng.standard_normal((256, 1024)).astype(np.float32)
+    x = (np.maximum(z, 0) ** 2).astype(np.float32)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    q1, _ = o.act_quant(xb, 4)
+    q2, _ = o.act_quant(xb, 4, a4_divide_form=True)
+    d = np.abs(q1.astype(np.int32) - q2.astype(np.int32))
+    assert d.max() <= 1
+    assert np.mean(d) < 1e-3
+
+
+# ---------------------------------------------------------------------------
+# [P2] eq. (3), "Why 1.58 Bits?": integer matmul and rescale
+# ---------------------------------------------------------------------------
+
+def naive_acc(q, c):
+    M, K = q.shape
+    N = c.shape[0]
+    out = [[0] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            t = 0
+            for k in range(K):
+                t += int(q[m, k]) * int(c[n, k])
+            out[m][n] = t
+    return np.array(out, dtype=np.int64)
+
+
+def test_matmul_brute_force_and_add_sub_form():
+    rng = np.random.default_rng(11)
+    for (M, K, N) in [(1, 16, 1), (3, 64, 5), (7, 48, 9)]:
+        q = rng.integers(-128, 128, (M, K)).astype(np.int8)
+        c = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        acc = o.matmul_i32(q, c)
+        assert np.array_equal(acc, naive_acc(q, c))
+        # ternary weight adds (+1), subtracts (-1) or skips (0) the activation
+        for m in range(M):
+            for n in range(N):
+                plus = int(q[m][c[n] == 1].astype(np.int64).sum())
+                minus = int(q[m][c[n] == -1].astype(np.int64).sum())
+                assert acc[m, n] == plus - minus
+
+
+def test_matmul_extremes():
+    K = 8192
+    q = np.full((2, K), 127, np.int8)
+    q[1] = -127
+    c = np.ones((2, K), np.int8)
+    c[1] = -1
+    acc = o.matmul_i32(q, c)
+    assert acc.tolist() == [[127 * K, -127 * K], [-127 * K, 127 * K]]
+
+
+def test_rescale_against_exact_rational():
+    rng = np.random.default_rng(12)
+    acc = rng.integers(-300000, 300000, (5, 7)).astype(np.int32)
+    s = (np.float32(127) / (np.abs(rng.standard_normal(5)) + 0.1).astype(np.float32)).astype(np.float32)
+    g = np.float32(0.0123)
+    y64, y32 = o.rescale(acc, g, s)
+    for m in range(5):
+        for n in range(7):
+            exact = Fraction(int(acc[m, n])) * Fraction(float(g)) / Fraction(float(s[m]))
+            assert abs(Fraction(float(y64[m, n])) - exact) <= abs(exact) * Fraction(1, 1 << 51)
+            assert abs(Fraction(float(y32[m, n])) - exact) <= abs(exact) * Fraction(1, 1 << 22)
+
+
+def test_dequantized_float_matmul_brute_force():
+    # The pages' simulated integer GEMM (F.linear on dequantised operands)
+    # equals the integer path: y = (q/s) . (c*gamma)^T, in exact arithmetic.
+    rng = np.random.default_rng(13)
+    M, K, N = 4, 64, 6
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xf = rng.standard_normal((M, K)).astype(np.float32)
+    x = (xf.view(np.uint32) >> 16).astype(np.uint16)
+    r = o.forward(x, W)
+    g = Fraction(float(r["gamma"]))
+    for m in range(M):
+        sm = Fraction(float(r["s"][m]))
+        for n in range(N):
+            exact = sum(Fraction(int(r["q"][m, k])) / sm * (int(r["codes"][n, k]) * g) for k in range(K))
+            assert abs(Fraction(float(r["y64"][m, n])) - exact) <= abs(exact) * Fraction(1, 1 << 50)
+
+
+def test_worked_example_golden():
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    W = np.array([g["W"]], np.float32)
+    x = to_bf16_bits_exact([g["x"]])
+    r = o.forward(x, W)
+    assert r["gamma"] == np.float32(g["gamma"])
+    assert r["codes"][0].tolist() == g["codes"]
+    assert r["s"][0] == np.float32(g["s"])
+    assert r["q"][0].tolist() == g["q"]
+    assert int(r["acc"][0, 0]) == g["acc"]
+    exact = Fraction(g["y_exact_num"]) / Fraction(g["y_exact_den"])
+    assert abs(Fraction(float(r["y64"][0, 0])) - exact) <= exact * Fraction(1, 1 << 50)
+    assert int(r["Y"][0, 0]) == g["Y_bf16_bits"]
+
+
+def test_zero_row_and_zero_weights():
+    W = np.zeros((3, 32), np.float32)
+    x = to_bf16_bits_exact([[0.0] * 32, [1.0] * 32])
+    r = o.forward(x, W)
+    assert r["gamma"] == o.EPS
+    assert np.all(r["codes"] == 0)
+    assert np.all(r["acc"] == 0)
+    assert np.all(r["Y"] == 0)
