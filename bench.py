@@ -1,0 +1,535 @@
+"""BitLinear forward benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Headline workload: the 2B-class decode layer set (batch 1; up and gate
+2560 -> 6912, down 6912 -> 2560).  A step is one pass of the forward hot path
+(per-token quantisation, ternary GEMV, rescale to bf16) over all three layers.
+Weights are quantised once before timing (the offline part of the method, timed
+separately).  Metric: HBM GB/s of algorithmic bytes
+(packed weights + bf16 activations in + bf16 out + scales).  Secondary lines
+report tensor-core TOPS on the prefill workloads.
+
+Timing: CUDA graphs of back-to-back steps, CUDA events on the launching stream,
+barrier + synchronize on both sides of exactly K steps, max over ranks.  Each
+step uses one of several rotated copies of the weights so the weight stream is
+larger than the 126 MB L2.  With --gpus N > 1 (torchrun), every rank runs an
+independent replica (the decode path has no exchange step), and the value is
+the work of all ranks over the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear TOPS (prefill) and HBM GB/s (decode) vs roofline, 1×B200"
+INT8_NOMINAL_RATIO = 2.0   # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+
+
+# ---------------------------------------------------------------------------
+# shared helpers
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(M, K, N):
+    """Packed weights + bf16 X + bf16 Y + fp32 scales and gamma."""
+    return N * K // 4 + 2 * M * K + 2 * M * N + 4 * M + 4
+
+
+def algorithmic_ops(M, K, N):
+    return 2 * M * N * K
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def ncu_traffic(kernel_key):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel source; otherwise None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, "bitlinear_bl_forward_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(src)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(src, fn), "rb").read())
+    sha = h.hexdigest()[:16]
+    for line in open(path):
+        if line.startswith("#") or "=" not in line:
+            continue
+        kv = dict(t.split("=", 1) for t in line.split())
+        if kv.get("key") == kernel_key and kv.get("src_sha") == sha:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *a):
+        time.sleep(0.15)
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            p = [t.strip() for t in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append((float(p[1]), float(p[2]), float(p[3]), p[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        busy = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in busy), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(busy),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle arm (CPU): the CPU baseline and --impl reference
+# ---------------------------------------------------------------------------
+
+def oracle_step_fn(workload_name, row_fraction=1.0):
+    """Return (fn, bytes_per_call, description): fn() runs the oracle's forward
+    scope (activation quantisation, integer matmul, rescale, bf16 rounding)
+    over every layer of the workload, restricted to the first
+    ceil(row_fraction * N) output features of each layer."""
+    from bitlinear_bl_forward_b200.inputs import WORKLOADS, layer_inputs
+    from oracle import bitlinear_oracle as o
+    w = WORKLOADS[workload_name]
+    layers = []
+    nbytes = 0
+    for i, L in enumerate(w.layers):
+        X, W = layer_inputs(w, i)
+        n = max(1, int(math.ceil(row_fraction * L.N)))
+        W = W[:n]
+        g = o.absmean_scale(W)
+        c = o.ternary_codes(W, g)
+        layers.append((X, g, c))
+        nbytes += algorithmic_bytes(w.M, L.K, n)
+
+    def fn():
+        for X, g, c in layers:
+            q, s = o.act_quant(X, w.bits)
+            acc = o.matmul_i32(q, c)
+            _, y32 = o.rescale(acc, g, s)
+            o.round_to_bf16_bits(y32)
+
+    desc = f"{workload_name}, first {row_fraction:.4g} of each layer's output rows"
+    return fn, nbytes, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(workload_name, budget_s=10.0):
+    fn, nbytes, desc = oracle_step_fn(workload_name)
+    fn()   # warm
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": nbytes * n / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} full steps of {desc} in {dt:.1f} s (weight quantisation excluded)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    name = args.workload
+    K, W = args.steps, args.warmup
+    # calibrate one full step, then size each step so the run stays within ~2 minutes
+    fn, nbytes, _ = oracle_step_fn(name)
+    t0 = time.perf_counter()
+    fn()
+    t_full = time.perf_counter() - t0
+    frac = min(1.0, 120.0 / max(1e-9, (K + W) * t_full))
+    if frac < 1.0:
+        fn, nbytes, _ = oracle_step_fn(name, frac)
+    for _ in range(W):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        fn()
+    dt = time.perf_counter() - t0
+    value = nbytes * K / dt / 1e9
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": K,
+        "warmup": W, "ms_per_step": dt / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": name},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {name}, fraction {frac:.4g} of each layer's output rows"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------
+
+class GpuWorkload:
+    """Device buffers for one workload: R rotated copies of the packed weights
+    of every layer, one bf16 input and output per layer, workspace."""
+
+    def __init__(self, name, rotations, seed=0, device="cuda"):
+        import torch
+        from bitlinear_bl_forward_b200 import bl
+        from bitlinear_bl_forward_b200.inputs import WORKLOADS, make_activation
+        self.w = WORKLOADS[name]
+        self.name = name
+        self.layers = []
+        g = torch.Generator(device=device).manual_seed(seed)
+        for i, L in enumerate(self.w.layers):
+            Wf = torch.randn(L.N, L.K, generator=g, device=device, dtype=torch.float32) * self.w.w_std
+            Wp, gamma = bl.bl_quantize_weights(Wf)
+            del Wf
+            copies = [(Wp, gamma)] + [(Wp.clone(), gamma.clone()) for _ in range(rotations - 1)]
+            xb = make_activation(self.w.M, L.K, self.w.x_kind, seed + 1 + 10 * i, self.w.outliers_for(L.K),
+                                 self.w.outlier_mult)
+            X = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(device)
+            Y = torch.empty((self.w.M, L.N), dtype=torch.bfloat16, device=device)
+            ws_n = bl.bl_forward_workspace_bytes(self.w.M, L.K, L.N, self.w.bits)
+            ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=device)
+            self.layers.append(dict(L=L, copies=copies, X=X, Y=Y, ws=ws, xb=xb))
+        self.rotations = rotations
+        self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N) for d in self.layers)
+        self.ops_per_step = sum(algorithmic_ops(self.w.M, d["L"].K, d["L"].N) for d in self.layers)
+        self.launches_per_step = sum(1 if self.w.M <= 2 else 2 for _ in self.layers)
+
+    def step(self, i, events=None):
+        from bitlinear_bl_forward_b200 import bl
+        r = i % self.rotations
+        for j, d in enumerate(self.layers):
+            Wp, gamma = d["copies"][r]
+            if events is not None:
+                events[j][0].record()
+            bl.bl_forward(d["X"], Wp, gamma, d["L"].N, self.w.bits, out=d["Y"], workspace=d["ws"])
+            if events is not None:
+                events[j][1].record()
+
+
+def capture(wl, nsteps, start, with_events):
+    import torch
+    events = None
+    if with_events:
+        events = [[(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for _ in wl.layers] for _ in range(nsteps)]
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(nsteps):
+                wl.step(start + i, events[i] if events else None)
+    torch.cuda.current_stream().wait_stream(s)
+    return g, events
+
+
+def time_workload(wl, steps, warmup, dist_ctx, sample_clocks=True, chunk=None):
+    """Warm up, then time exactly `steps` steps (graph replays) with events."""
+    import torch
+    for i in range(warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+    chunk = chunk or min(steps, 64 * wl.rotations // math.gcd(64, wl.rotations))
+    chunk = max(1, min(chunk, steps))
+    g_main, ev = capture(wl, chunk, 0, with_events=True)
+    rem = steps % chunk
+    g_rem = capture(wl, rem, (steps // chunk) * chunk, with_events=False)[0] if rem else None
+    g_main.replay()        # upload + untimed warm replay
+    if g_rem is not None:
+        g_rem.replay()
+    torch.cuda.synchronize()
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device()) if sample_clocks else None
+    if sampler:
+        sampler.__enter__()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(steps // chunk):
+        g_main.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    if sampler:
+        sampler.__exit__()
+    ms = t0.elapsed_time(t1)
+    ms_max = dist_ctx.max(ms)
+    # per-launch durations of the last replayed chunk of the timed region
+    per_layer = [[] for _ in wl.layers]
+    for step_ev in ev:
+        for j, (a, b) in enumerate(step_ev):
+            per_layer[j].append(a.elapsed_time(b))
+    return ms_max, per_layer, (sampler.summary() if sampler else None)
+
+
+def time_e2e(wl, steps, warmup, dist_ctx):
+    """Same metric through the public API with host buffers: each step copies
+    every layer's input from pinned host memory, runs bl_forward and reads the
+    outputs back to pinned host memory."""
+    import torch
+    from bitlinear_bl_forward_b200 import bl
+    hx = [torch.from_numpy(d["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for d in wl.layers]
+    hy = [torch.empty(tuple(d["Y"].shape), dtype=torch.bfloat16).pin_memory() for d in wl.layers]
+    h2d = sum(t.numel() * 2 for t in hx)
+    d2h = sum(t.numel() * 2 for t in hy)
+
+    def one(i):
+        r = i % wl.rotations
+        for j, d in enumerate(wl.layers):
+            d["X"].copy_(hx[j], non_blocking=True)
+            Wp, gamma = d["copies"][r]
+            bl.bl_forward(d["X"], Wp, gamma, d["L"].N, wl.w.bits, out=d["Y"], workspace=d["ws"])
+            hy[j].copy_(d["Y"], non_blocking=True)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        one(i)
+    t1.record()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    ms = dist_ctx.max(t0.elapsed_time(t1))
+    return ms, h2d, d2h
+
+
+class DistCtx:
+    def __init__(self, ngpus):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = None
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v):
+        if self.dist is None:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+def roofline_entry(kind, achieved, peak, unit, traffic):
+    return {"bound": kind, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": traffic}
+
+
+def run_gpu(args):
+    import torch
+    from bitlinear_bl_forward_b200 import build as blbuild
+    from bitlinear_bl_forward_b200 import bl
+    blbuild.build()
+    bl.lib()
+    ctx = DistCtx(args.gpus)
+    peaks = load_peaks()
+    name = args.workload
+    from bitlinear_bl_forward_b200.inputs import WORKLOADS
+    w = WORKLOADS[name]
+    decode = w.M <= 2
+    # enough rotated weight copies that one rotation is > 2x the 126 MB L2
+    wbytes = sum(L.N * L.K // 4 for L in w.layers)
+    rot = max(2, min(64, int(math.ceil(256e6 / wbytes))))
+    wl = GpuWorkload(name, rot)
+    K = args.steps if args.steps is not None else (60000 if decode else 2000)
+    Wm = max(3, args.warmup)
+    ms, per_layer, clocks = time_workload(wl, K, Wm, ctx)
+    N = ctx.world
+    sec = ms / 1e3
+    if decode:
+        value = N * wl.bytes_per_step * K / sec / 1e9
+        unit = "GB/s"
+    else:
+        value = N * wl.ops_per_step * K / sec / 1e12
+        unit = "TOPS"
+
+    # dominant kernel: the launch set with the largest share of time
+    tot = [sum(v) for v in per_layer]
+    launches = sum(len(v) for v in per_layer)
+    if decode:
+        achieved = sum(algorithmic_bytes(w.M, d["L"].K, d["L"].N) * len(per_layer[j])
+                       for j, d in enumerate(wl.layers)) / (sum(tot) / 1e3) / 1e9
+        roof = roofline_entry("hbm", achieved, peaks["hbm_gbs"], "GB/s", ncu_traffic(f"gemv:{name}"))
+    else:
+        achieved = sum(algorithmic_ops(w.M, d["L"].K, d["L"].N) * len(per_layer[j])
+                       for j, d in enumerate(wl.layers)) / (sum(tot) / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO
+        roof = roofline_entry("tensor", achieved, peak, "TFLOP/s", ncu_traffic(f"tc:{name}"))
+    roof["peak_src"] = peaks["src"] + (" hbm copy" if decode else " bf16 sustained x2 (int8/bf16 nominal)")
+    roof["kernel_ms_avg"] = sum(tot) / max(1, launches)
+
+    # end-to-end through the public API with host buffers
+    e2e_steps = min(K, 2000 if decode else 200)
+    ms_e2e, h2d, d2h = time_e2e(wl, e2e_steps, 3, ctx)
+    e2e_val = (N * (wl.bytes_per_step if decode else wl.ops_per_step) * e2e_steps / (ms_e2e / 1e3)
+               / (1e9 if decode else 1e12))
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": N, "steps": K, "warmup": Wm,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8", "data": "synthetic (seeded; weights N(0, std) generated on the GPU, activations on the host)",
+        "config": {"workload": name, "M": w.M, "layers": [[L.name, L.K, L.N] for L in w.layers], "bits": w.bits,
+                   "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
+                   "l2": f"{rot} rotated weight copies ({rot * wbytes / 1e6:.0f} MB, > 126 MB L2)",
+                   "timing": "CUDA graph replays, events on the launching stream"},
+        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": K * wl.launches_per_step,
+        "roofline": roof,
+        "clocks": clocks,
+    }
+    if not args.no_secondary and ctx.world == 1:
+        line["secondary"] = secondary(args, ctx, peaks)
+    if ctx.rank == 0 and not args.no_cpu_baseline and ctx.world == 1:
+        line["cpu_baseline"] = cpu_baseline(name, budget_s=args.cpu_seconds)
+    ctx.close()
+    if ctx.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def secondary(args, ctx, peaks):
+    """Tensor-core workloads and the 70B decode layer, shorter runs."""
+    import torch
+    out = []
+    for name, steps in (("prefill_2b", 300), ("layer_70b_m1", 3000), ("layer_70b_m16", 3000),
+                        ("layer_70b_m128", 2000), ("layer_70b_m2048", 200), ("a48", 300)):
+        if args.secondary and name not in args.secondary.split(","):
+            continue
+        from bitlinear_bl_forward_b200.inputs import WORKLOADS
+        w = WORKLOADS[name]
+        wbytes = sum(L.N * L.K // 4 for L in w.layers)
+        rot = max(2, min(64, int(math.ceil(256e6 / wbytes))))
+        wl = GpuWorkload(name, rot)
+        ms, per_layer, _ = time_workload(wl, steps, 3, ctx, sample_clocks=False)
+        sec = ms / 1e3
+        tot_ms = sum(sum(v) for v in per_layer)
+        nl = sum(len(v) for v in per_layer)
+        gbs = wl.bytes_per_step * steps / sec / 1e9
+        tops = wl.ops_per_step * steps / sec / 1e12
+        kernel_bytes = sum(algorithmic_bytes(w.M, d["L"].K, d["L"].N) * len(per_layer[j])
+                           for j, d in enumerate(wl.layers))
+        kernel_ops = sum(algorithmic_ops(w.M, d["L"].K, d["L"].N) * len(per_layer[j])
+                         for j, d in enumerate(wl.layers))
+        ent = {"workload": name, "M": w.M, "ms_per_step": ms / steps, "GB/s": gbs, "TOPS": tops,
+               "hbm_frac": (kernel_bytes / (tot_ms / 1e3) / 1e9) / peaks["hbm_gbs"],
+               "tensor_frac": (kernel_ops / (tot_ms / 1e3) / 1e12)
+               / (peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO),
+               "forward_ms_avg": tot_ms / max(1, nl), "steps": steps}
+        out.append(ent)
+        del wl
+        torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_2b")
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--secondary", default="", help="comma list restricting the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 20
+        run_reference(args)
+        return
+    run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

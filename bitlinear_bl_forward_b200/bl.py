@@ -1,0 +1,193 @@
+"""Thin Python binding of libbitlinear (include/bitlinear.h).
+
+Argument marshalling only: every function checks dtypes/devices, allocates
+outputs and workspace with torch (device memory plumbing), passes raw device
+pointers and torch's current CUDA stream to the C ABI, and raises BLError on a
+non-OK status.  All arithmetic runs in the library's CUDA kernels; there is no
+fallback of any kind -- if libbitlinear.so is missing the call fails.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+BL_OK = 0
+STATUS_NAMES = {
+    0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGNMENT",
+    4: "BL_ERR_UNSUPPORTED", 5: "BL_ERR_CUDA", 6: "BL_ERR_TIMEOUT", 7: "BL_ERR_WORKSPACE",
+}
+
+# name -> (restype, argtypes), mirroring include/bitlinear.h
+_i64, _sz, _p, _int = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "bl_status_string": (ctypes.c_char_p, [_int]),
+    "bl_version": (_int, []),
+    "bl_packed_weight_bytes": (_sz, [_i64, _i64]),
+    "bl_quantize_weights_workspace_bytes": (_sz, [_i64, _i64]),
+    "bl_quantize_weights": (_int, [_p, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "bl_unpack_weights": (_int, [_p, _i64, _i64, _p, _p]),
+    "bl_quant_act": (_int, [_p, _i64, _i64, _int, _p, _p, _p]),
+    "bl_forward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
+    "bl_forward": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
+    "bl_forward_f32": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
+    "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
+    "bl_selftest_wait_timeout": (_int, [ctypes.c_ulonglong, _p, _p]),
+}
+
+_lib = None
+
+
+class BLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} "
+                         f"({lib().bl_status_string(self.status).decode()})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitlinear.so (built in-tree by bitlinear_bl_forward_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m bitlinear_bl_forward_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != BL_OK:
+        raise BLError(st, where)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dev(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# C-ABI mirrors
+# ---------------------------------------------------------------------------
+
+def bl_packed_weight_bytes(N: int, K: int) -> int:
+    return int(lib().bl_packed_weight_bytes(N, K))
+
+
+def bl_quantize_weights(W: torch.Tensor):
+    """fp32 [N, K] -> (packed uint8 [N, K/4], gamma fp32 [1])."""
+    N, K = W.shape
+    pW = _dev(W, torch.float32, "W")
+    Wp = torch.empty((N, max(K // 4, 1)), dtype=torch.uint8, device=W.device)
+    gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    ws = _workspace(int(lib().bl_quantize_weights_workspace_bytes(N, K)), W.device)
+    _check(lib().bl_quantize_weights(pW, N, K, Wp.data_ptr(), gamma.data_ptr(),
+                                     ws.data_ptr() if ws is not None else None,
+                                     ws.numel() if ws is not None else 0, _stream()),
+           "bl_quantize_weights")
+    return Wp, gamma
+
+
+def bl_unpack_weights(Wp: torch.Tensor, N: int, K: int) -> torch.Tensor:
+    p = _dev(Wp, torch.uint8, "Wp")
+    codes = torch.empty((N, K), dtype=torch.int8, device=Wp.device)
+    _check(lib().bl_unpack_weights(p, N, K, codes.data_ptr(), _stream()), "bl_unpack_weights")
+    return codes
+
+
+def bl_quant_act(X: torch.Tensor, bits: int = 8):
+    """bf16 [M, K] -> (int8 codes [M, K], scale fp32 [M])."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    _check(lib().bl_quant_act(px, M, K, bits, Xq.data_ptr(), s.data_ptr(), _stream()), "bl_quant_act")
+    return Xq, s
+
+
+def bl_forward_workspace_bytes(M: int, K: int, N: int, bits: int = 8) -> int:
+    return int(lib().bl_forward_workspace_bytes(M, K, N, bits))
+
+
+def bl_forward(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8,
+               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """BitLinear forward: bf16 [M, K] activations, packed weights -> bf16 [M, N]."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    need = bl_forward_workspace_bytes(M, K, N, bits)
+    ws = workspace if workspace is not None else _workspace(need, X.device)
+    _check(lib().bl_forward(px, M, K, N, pw, pg, bits, py,
+                            ws.data_ptr() if ws is not None else None,
+                            ws.numel() if ws is not None else 0, _stream()), "bl_forward")
+    return Y
+
+
+def bl_forward_f32(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8) -> torch.Tensor:
+    """As bl_forward, fp32 output before the bf16 rounding (test export)."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    ws = _workspace(bl_forward_workspace_bytes(M, K, N, bits), X.device)
+    _check(lib().bl_forward_f32(px, M, K, N, pw, pg, bits, Y.data_ptr(),
+                                ws.data_ptr() if ws is not None else None,
+                                ws.numel() if ws is not None else 0, _stream()), "bl_forward_f32")
+    return Y
+
+
+def bl_matmul_i32(Xq: torch.Tensor, Wp: torch.Tensor, N: int) -> torch.Tensor:
+    """Exact int32 accumulators of int8 [M, K] codes x packed weights (test export)."""
+    M, K = Xq.shape
+    px = _dev(Xq, torch.int8, "Xq")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    ws = _workspace(int(lib().bl_matmul_i32_workspace_bytes(M, K, N)), Xq.device)
+    _check(lib().bl_matmul_i32(px, M, K, N, pw, acc.data_ptr(),
+                               ws.data_ptr() if ws is not None else None,
+                               ws.numel() if ws is not None else 0, _stream()), "bl_matmul_i32")
+    return acc
+
+
+def bl_device_status(clear: bool = True):
+    """(status, site) recorded by kernels since the last clear."""
+    site = ctypes.c_int(0)
+    st = lib().bl_device_status(1 if clear else 0, ctypes.byref(site))
+    return int(st), int(site.value)
+
+
+def bl_selftest_wait_timeout(limit_ns: int) -> torch.Tensor:
+    out = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(lib().bl_selftest_wait_timeout(limit_ns, out.data_ptr(), _stream()), "bl_selftest_wait_timeout")
+    return out

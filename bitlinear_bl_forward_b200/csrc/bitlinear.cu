@@ -1,0 +1,360 @@
+// libbitlinear: host side of the C ABI declared in include/bitlinear.h.
+//
+// Validation happens before any CUDA call, so a rejected call launches
+// nothing (and needs no GPU).  Dispatch:
+//   M <= 2      decode GEMV with the activation quantisation fused in;
+//   otherwise   activation quantisation into the caller's workspace, then the
+//               tcgen05 kind::i8 GEMM (weights expanded into tensor memory).
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/bitlinear.h"
+#include "bl_act.cuh"
+#include "bl_common.cuh"
+#include "bl_gemm_tc.cuh"
+#include "bl_gemv.cuh"
+#include "bl_weights.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;                       // 0.1.0
+constexpr int64_t kMaxK = 65536;
+constexpr int64_t kMaxElems = int64_t(1) << 40;     // N*K and M*K bound
+constexpr int kGemvMaxM = 2;
+constexpr int kAbsumMaxBlocks = 592;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr int kMaxDevices = 64;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bl_status check_shape_nk(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
+  if (N >= kMaxElems / K) return BL_ERR_SHAPE;
+  return BL_OK;
+}
+
+bl_status check_m(int64_t M, int64_t K) {
+  if (M < 0 || M > INT32_MAX) return BL_ERR_SHAPE;
+  if (M > 0 && M >= kMaxElems / K) return BL_ERR_SHAPE;
+  return BL_OK;
+}
+
+bl_status last_cuda() { return cudaGetLastError() == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
+
+int num_sms() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+// Raise a kernel's dynamic shared memory limit once per device.
+template <typename F>
+bool ensure_smem(F* func, int bytes, std::atomic<uint64_t>* done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done_mask->load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(func), cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done_mask->fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || p == nullptr)
+    return nullptr;
+  f = reinterpret_cast<EncodeTiledFn>(p);
+  fn.store(f, std::memory_order_release);
+  return f;
+}
+
+// 2-D uint8 tensor [rows, cols] (cols contiguous), box [box_rows, box_cols].
+bool encode_u8_2d(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                  uint32_t box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// launches
+// ---------------------------------------------------------------------------
+
+template <int MT, int RT>
+bl_status launch_gemv_t(const void* X, int x_is_i8, int M, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
+                        void* Y, int out_mode, cudaStream_t stream) {
+  static std::atomic<uint64_t> done{0};
+  const int KL = static_cast<int>(align_up(static_cast<size_t>(K), 128));
+  const int smem = MT * KL;
+  if (!ensure_smem(bl::gemv_kernel<MT, RT>, MT * static_cast<int>(kMaxK), &done)) return BL_ERR_CUDA;
+  const int ntiles = (N + RT - 1) / RT;
+  int blocks = (ntiles + bl::kGemvWarps - 1) / bl::kGemvWarps;
+  const int cap = 2 * num_sms();
+  if (blocks > cap) blocks = cap;
+  bl::gemv_kernel<MT, RT><<<blocks, bl::kGemvThreads, smem, stream>>>(
+      X, x_is_i8, M, K, N, reinterpret_cast<const uint4*>(Wp), gamma, Q, Y, out_mode);
+  return last_cuda();
+}
+
+bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
+                      void* Y, int out_mode, cudaStream_t stream) {
+  if (M == 1) return launch_gemv_t<1, 2>(X, x_is_i8, M, K, N, Wp, gamma, Q, Y, out_mode, stream);
+  return launch_gemv_t<2, 2>(X, x_is_i8, M, K, N, Wp, gamma, Q, Y, out_mode, stream);
+}
+
+template <int BN>
+bl_status launch_tc_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
+                      const float* gamma, void* Y, int out_mode, int debug_flags, unsigned long long limit_ns,
+                      cudaStream_t stream) {
+  using C = bl::TcCfg<BN>;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(bl::tc_gemm_kernel<BN>, C::kSmemBytes, &done)) return BL_ERR_CUDA;
+  CUtensorMap tmX, tmW;
+  if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), BN, bl::kTcBK,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return BL_ERR_CUDA;
+  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kTcBK / 4,
+                    CU_TENSOR_MAP_SWIZZLE_32B))
+    return BL_ERR_CUDA;
+  const dim3 grid((N + bl::kTcRows - 1) / bl::kTcRows, (M + BN - 1) / BN);
+  bl::tc_gemm_kernel<BN><<<grid, bl::kTcThreads, C::kSmemBytes, stream>>>(tmX, tmW, M, N, K, R, s, gamma, Y, out_mode,
+                                                                         limit_ns, debug_flags);
+  return last_cuda();
+}
+
+bl_status launch_tc(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
+                    const float* gamma, void* Y, int out_mode, int debug_flags, cudaStream_t stream) {
+  const unsigned long long lim = kWaitLimitNs;
+  if (M <= 16) return launch_tc_t<16>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
+  if (M <= 32) return launch_tc_t<32>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
+  if (M <= 64) return launch_tc_t<64>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
+  if (M <= 128) return launch_tc_t<128>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
+  return launch_tc_t<256>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
+}
+
+struct FwdWs {
+  int8_t* Xq;
+  float* s;
+  int* R;
+};
+
+size_t fwd_ws_bytes(int64_t M, int64_t K) {
+  if (M <= kGemvMaxM) return 0;
+  return align_up(static_cast<size_t>(M) * K, 256) + 2 * align_up(static_cast<size_t>(M) * 4, 256);
+}
+
+FwdWs fwd_ws_split(void* ws, int64_t M, int64_t K) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  FwdWs w;
+  w.Xq = reinterpret_cast<int8_t*>(p);
+  p += align_up(static_cast<size_t>(M) * K, 256);
+  w.s = reinterpret_cast<float*>(p);
+  p += align_up(static_cast<size_t>(M) * 4, 256);
+  w.R = reinterpret_cast<int*>(p);
+  return w;
+}
+
+bl_status forward_common(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
+                         int bits, void* Y, int out_mode, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (M == 0) return BL_OK;
+  if (!X || !Wp || !gamma || !Y) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wp)) return BL_ERR_ALIGNMENT;
+  const size_t need = fwd_ws_bytes(M, K);
+  if (need > 0) {
+    if (!ws || ws_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BL_ERR_ALIGNMENT;
+  }
+  const int Q = bits == 8 ? 127 : 7;
+  const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+  if (M <= kGemvMaxM) return launch_gemv(X, 0, m, k, n, Wp, gamma, Q, Y, out_mode, stream);
+  const FwdWs w = fwd_ws_split(ws, M, K);
+  const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
+  bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, w.Xq, w.s, w.R);
+  if ((st = last_cuda()) != BL_OK) return st;
+  return launch_tc(w.Xq, m, k, n, Wp, w.R, w.s, gamma, Y, out_mode, 0, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bl_status_string(bl_status s) {
+  switch (s) {
+    case BL_OK: return "ok";
+    case BL_ERR_INVALID_ARG: return "invalid argument (null pointer)";
+    case BL_ERR_SHAPE: return "unsupported shape (need N,K > 0, K % 64 == 0, K <= 65536, M >= 0, N*K < 2^40)";
+    case BL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case BL_ERR_UNSUPPORTED: return "unsupported activation width (bits must be 4 or 8)";
+    case BL_ERR_CUDA: return "CUDA error";
+    case BL_ERR_TIMEOUT: return "a kernel wait timed out";
+    case BL_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int bl_version(void) { return kVersion; }
+
+size_t bl_packed_weight_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / 4;
+}
+
+static int absum_blocks(int64_t N, int64_t K) {
+  const int64_t n4 = N * K / 4;
+  int64_t b = (n4 + 255) / 256;
+  if (b > kAbsumMaxBlocks) b = kAbsumMaxBlocks;
+  if (b < 1) b = 1;
+  return static_cast<int>(b);
+}
+
+size_t bl_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
+  if (check_shape_nk(N, K) != BL_OK) return 0;
+  return static_cast<size_t>(absum_blocks(N, K)) * bl::kBins * sizeof(unsigned long long);
+}
+
+bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gamma, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if (!W || !Wp || !gamma) return BL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wp)) return BL_ERR_ALIGNMENT;
+  const size_t need = bl_quantize_weights_workspace_bytes(N, K);
+  if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+  const int blocks = absum_blocks(N, K);
+  auto* bins = static_cast<unsigned long long*>(workspace);
+  const int64_t n = N * K;
+  bl::weight_absum_bins_kernel<<<blocks, bl::kAbsumThreads, 0, stream>>>(W, n, bins);
+  if ((st = last_cuda()) != BL_OK) return st;
+  bl::weight_gamma_kernel<<<1, 256, 0, stream>>>(bins, blocks, static_cast<uint64_t>(n), gamma);
+  if ((st = last_cuda()) != BL_OK) return st;
+  const int64_t nwords = n / 16;
+  bl::weight_pack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
+      W, nwords, gamma, reinterpret_cast<uint32_t*>(Wp));
+  return last_cuda();
+}
+
+bl_status bl_unpack_weights(const uint8_t* Wp, int64_t N, int64_t K, int8_t* codes, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if (!Wp || !codes) return BL_ERR_INVALID_ARG;
+  if (!aligned16(Wp) || !aligned16(codes)) return BL_ERR_ALIGNMENT;
+  const int64_t nwords = N * K / 16;
+  bl::weight_unpack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint32_t*>(Wp), nwords, codes);
+  return last_cuda();
+}
+
+bl_status bl_quant_act(const uint16_t* X, int64_t M, int64_t K, int bits, int8_t* Xq, float* scale,
+                       cudaStream_t stream) {
+  if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
+  bl_status st = check_m(M, K);
+  if (st != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (M == 0) return BL_OK;
+  if (!X || !Xq || !scale) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Xq)) return BL_ERR_ALIGNMENT;
+  const int m = static_cast<int>(M);
+  const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
+  bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale,
+                                                   nullptr);
+  return last_cuda();
+}
+
+size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+  (void)bits;
+  if (check_shape_nk(N, K) != BL_OK || check_m(M, K) != BL_OK) return 0;
+  return fwd_ws_bytes(M, K);
+}
+
+bl_status bl_forward(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
+                     int bits, uint16_t* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return forward_common(X, M, K, N, Wp, gamma, bits, Y, bl::kOutBF16, workspace, workspace_bytes, stream);
+}
+
+bl_status bl_forward_f32(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
+                         int bits, float* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return forward_common(X, M, K, N, Wp, gamma, bits, Y, bl::kOutF32, workspace, workspace_bytes, stream);
+}
+
+size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (check_shape_nk(N, K) != BL_OK || check_m(M, K) != BL_OK) return 0;
+  if (M <= kGemvMaxM) return 0;
+  return align_up(static_cast<size_t>(M) * 4, 256);
+}
+
+bl_status bl_matmul_i32(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, int32_t* acc,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (M == 0) return BL_OK;
+  if (!Xq || !Wp || !acc) return BL_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(Wp)) return BL_ERR_ALIGNMENT;
+  const size_t need = bl_matmul_i32_workspace_bytes(M, K, N);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+  }
+  const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+  if (M <= kGemvMaxM) return launch_gemv(Xq, 1, m, k, n, Wp, nullptr, 0, acc, bl::kOutI32, stream);
+  int* R = static_cast<int*>(workspace);
+  bl::act_rowsum_kernel<<<(m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock, 256, 0, stream>>>(Xq, m, k, R);
+  if ((st = last_cuda()) != BL_OK) return st;
+  return launch_tc(Xq, m, k, n, Wp, R, nullptr, nullptr, acc, bl::kOutI32, 0, stream);
+}
+
+bl_status bl_device_status(int clear, int* site) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return BL_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bl::g_status, sizeof(v)) != cudaSuccess) return BL_ERR_CUDA;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(bl::g_status, &z, sizeof(z)) != cudaSuccess) return BL_ERR_CUDA;
+  }
+  if (site) *site = static_cast<int>((v >> 8) & 0xffu);
+  return static_cast<bl_status>(v & 0xffu);
+}
+
+bl_status bl_selftest_wait_timeout(unsigned long long limit_ns, int* waited_ok, cudaStream_t stream) {
+  if (!waited_ok) return BL_ERR_INVALID_ARG;
+  if (limit_ns > 10ull * kWaitLimitNs) return BL_ERR_INVALID_ARG;
+  bl::wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, waited_ok);
+  return last_cuda();
+}
+
+}  // extern "C"

@@ -1,0 +1,125 @@
+// Per-token absmax activation quantisation.
+//
+// "BitNet b1.58: The 1-Bit Ternary LLM Architecture Guide", section "The
+// Mathematical Formulation of BitLinear", eq. (2): scale_X = Q_b / (max_j |X_ij|
+// + eps) per token, X~ = Round(Clip(X * scale_X, ...)).  Clip range [-128, 127]
+// from "BitNet 2B4T Guide: Scaling Native 1.58-Bit LLMs", section "1. The
+// BitLinear Operator"; the 4-bit mode (Q = 7, range [-8, 7]) from "BitNet a4.8
+// Guide: 4-Bit Activation 1-Bit LLMs", section "1. Hybrid W1.58 / A4
+// Quantization Function".  eps is read as a floor: s = Q / max(a, 1e-5).
+//
+// Every rounding is explicit so results are bit-identical to an IEEE fp32
+// evaluation: __fdiv_rn for the scale, __fmul_rn for x * s (never fused),
+// __float2int_rn (round half to even) for the code.
+#pragma once
+
+#include "bl_common.cuh"
+
+namespace bl {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float absmax8_bf16(uint4 v) {
+  float a = fabsf(bf16_lo(v.x));
+  a = fmaxf(a, fabsf(bf16_hi(v.x)));
+  a = fmaxf(a, fabsf(bf16_lo(v.y)));
+  a = fmaxf(a, fabsf(bf16_hi(v.y)));
+  a = fmaxf(a, fabsf(bf16_lo(v.z)));
+  a = fmaxf(a, fabsf(bf16_hi(v.z)));
+  a = fmaxf(a, fabsf(bf16_lo(v.w)));
+  a = fmaxf(a, fabsf(bf16_hi(v.w)));
+  return a;
+}
+
+__device__ __forceinline__ uint32_t quant1(float x, float s, int Q) {
+  int q = __float2int_rn(__fmul_rn(x, s));
+  q = q < -Q - 1 ? -Q - 1 : (q > Q ? Q : q);
+  return static_cast<uint32_t>(q) & 0xffu;
+}
+
+// 8 bf16 -> 8 int8 codes (as two 32-bit words) and their sum.
+__device__ __forceinline__ uint2 quant8_bf16(uint4 v, float s, int Q, int& sum) {
+  const uint32_t b0 = quant1(bf16_lo(v.x), s, Q), b1 = quant1(bf16_hi(v.x), s, Q);
+  const uint32_t b2 = quant1(bf16_lo(v.y), s, Q), b3 = quant1(bf16_hi(v.y), s, Q);
+  const uint32_t b4 = quant1(bf16_lo(v.z), s, Q), b5 = quant1(bf16_hi(v.z), s, Q);
+  const uint32_t b6 = quant1(bf16_lo(v.w), s, Q), b7 = quant1(bf16_hi(v.w), s, Q);
+  const uint32_t lo = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+  const uint32_t hi = b4 | (b5 << 8) | (b6 << 16) | (b7 << 24);
+  sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+constexpr int kActRowsPerBlock = 8;   // one warp per token row
+constexpr int kActCache = 16;         // 16-byte chunks kept in registers per lane
+
+// X bf16 [M, K] -> Xq int8 [M, K], s[M] = Q / max(a, 1e-5), optional R[M] =
+// sum_k Xq[m, k] (used to undo the +1 offset of the stored weight codes).
+__global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restrict__ X, int M, int K, int Q,
+                                                        int8_t* __restrict__ Xq, float* __restrict__ s_out,
+                                                        int* __restrict__ R_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * kActRowsPerBlock + warp;
+  if (m >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
+  const int nch = K >> 3;
+  uint4 cache[kActCache];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kActCache; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nch) {
+      cache[i] = __ldg(xr + c);
+      amax = fmaxf(amax, absmax8_bf16(cache[i]));
+    }
+  }
+  for (int c = lane + 32 * kActCache; c < nch; c += 32) amax = fmaxf(amax, absmax8_bf16(__ldg(xr + c)));
+  amax = warp_max(amax);
+  const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(amax, 1e-5f));
+  uint2* qr = reinterpret_cast<uint2*>(Xq + static_cast<size_t>(m) * K);
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kActCache; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+  }
+  for (int c = lane + 32 * kActCache; c < nch; c += 32) qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
+  sum = warp_sum(sum);
+  if (lane == 0) {
+    if (s_out) s_out[m] = s;
+    if (R_out) R_out[m] = sum;
+  }
+}
+
+// R[m] = sum_k Xq[m, k] for already-quantised int8 activations.
+__global__ void __launch_bounds__(256) act_rowsum_kernel(const int8_t* __restrict__ Xq, int M, int K,
+                                                         int* __restrict__ R_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * kActRowsPerBlock + warp;
+  if (m >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(Xq + static_cast<size_t>(m) * K);
+  int sum = 0;
+  for (int c = lane; c < (K >> 4); c += 32) {
+    const uint4 v = __ldg(xr + c);
+    sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
+    sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
+    sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
+    sum = __dp4a(static_cast<int>(v.w), 0x01010101, sum);
+  }
+  sum = warp_sum(sum);
+  if (lane == 0) R_out[m] = sum;
+}
+
+}  // namespace bl

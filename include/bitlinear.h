@@ -1,0 +1,176 @@
+/*
+ * libbitlinear -- BitNet b1.58 BitLinear forward on NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every pointer argument that names a tensor is a DEVICE pointer that
+ * the caller allocated and owns; the library allocates no device memory of its
+ * own except one 4-byte status word (see bl_device_status).  Every compute
+ * call is asynchronous on the given CUDA stream (0 = legacy default stream)
+ * and returns a bl_status:
+ *   - arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and leaves every output untouched;
+ *   - BL_ERR_CUDA reports a launch failure (cudaGetLastError);
+ *   - problems found while a kernel runs (a pipeline wait that gave up) are
+ *     recorded in the device status word, read with bl_device_status.
+ * Calls on distinct streams are thread-safe.  Inputs containing NaN or Inf
+ * give undefined (but memory-safe) results.
+ *
+ * Notation: X bf16 [M, K] activations (tokens x in-features, row-major),
+ * W fp32 [N, K] latent weights (out-features x in-features, the nn.Linear
+ * convention), Y [M, N] outputs (row-major).  bf16 tensors are passed as
+ * pointers to their 16-bit patterns.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [b1.58] "BitNet b1.58: The 1-Bit Ternary LLM Architecture Guide",
+ *           section "The Mathematical Formulation of BitLinear", eqs. (1)-(3).
+ *   [a4.8]  "BitNet a4.8 Guide: 4-Bit Activation 1-Bit LLMs", section
+ *           "1. Hybrid W1.58 / A4 Quantization Function".
+ *   [2B4T]  "BitNet 2B4T Guide: Scaling Native 1.58-Bit LLMs", section
+ *           "1. The BitLinear Operator".
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define BL_API __attribute__((visibility("default")))
+#else
+#define BL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BL_OK = 0,
+  BL_ERR_INVALID_ARG = 1, /* null pointer where a tensor is required */
+  BL_ERR_SHAPE = 2,       /* M < 0, N or K <= 0, K % 64 != 0, K > 65536, N*K >= 2^40 */
+  BL_ERR_ALIGNMENT = 3,   /* a pointer that must be 16-byte aligned is not */
+  BL_ERR_UNSUPPORTED = 4, /* bits not in {4, 8} */
+  BL_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
+  BL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait gave up (device status word) */
+  BL_ERR_WORKSPACE = 7    /* workspace pointer null or smaller than required */
+} bl_status;
+
+/* Static, NUL-terminated description of a status code. */
+BL_API const char* bl_status_string(bl_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+BL_API int bl_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Packed ternary weights.
+ *
+ * Storage: 2 bits per weight, N*K/4 bytes (the a4.8 page's verification
+ * harness counts in*out*2/8 bytes; the bit layout is this library's).  Row n
+ * starts at byte n*K/4 and is a run of little-endian 32-bit words; word g holds
+ * weights k = 16g..16g+15; weight k = 16g + 4j + b (j, b in 0..3) sits in bits
+ * [8b+2j, 8b+2j+2) and stores code+1 (0 = -1, 1 = 0, 2 = +1; 3 is never
+ * written).  gamma is one fp32 in device memory.
+ * ------------------------------------------------------------------------- */
+
+/* N*K/4. */
+BL_API size_t bl_packed_weight_bytes(int64_t N, int64_t K);
+
+/* Device workspace bytes bl_quantize_weights needs (independent of the data). */
+BL_API size_t bl_quantize_weights_workspace_bytes(int64_t N, int64_t K);
+
+/*
+ * [b1.58] eq. (1), absmean weight quantisation:
+ *   gamma = max(mean_{n,k} |W[n,k]|, 1e-5)   -- the mean is formed exactly
+ *           and rounded once to fp32 (nearest, ties to even), so gamma does not
+ *           depend on any summation order;
+ *   code  = clamp(round_half_even(W / gamma), -1, 1)   (IEEE fp32 division);
+ *   Wp    = packed codes (layout above), gamma written to *gamma.
+ * W: fp32 [N, K], 16-byte aligned.  Wp: N*K/4 bytes, 16-byte aligned.
+ * workspace: at least bl_quantize_weights_workspace_bytes(N, K) bytes,
+ * 16-byte aligned, contents ignored and clobbered.
+ */
+BL_API bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gamma, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/* Packed weights -> int8 codes in {-1, 0, 1}, row-major [N, K] (16-byte
+ * aligned).  For tests and inspection. */
+BL_API bl_status bl_unpack_weights(const uint8_t* Wp, int64_t N, int64_t K, int8_t* codes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Activations.
+ * ------------------------------------------------------------------------- */
+
+/*
+ * [b1.58] eq. (2) per token, with the [2B4T] clip range and the [a4.8] 4-bit
+ * mode.  For each row m of X:
+ *   a_m  = max_k |X[m,k]|
+ *   s_m  = Q / max(a_m, 1e-5)                     (fp32 division)
+ *   q    = clamp(round_half_even(X * s_m), -Q-1, Q)  (fp32 product)
+ * with Q = 127 for bits = 8 and Q = 7 for bits = 4.
+ * X: bf16 bits [M, K], 16-byte aligned.  Xq: int8 [M, K] (4-bit codes are
+ * stored one per byte), 16-byte aligned.  scale: fp32 [M], receives s_m.
+ * M == 0 is a no-op.
+ */
+BL_API bl_status bl_quant_act(const uint16_t* X, int64_t M, int64_t K, int bits, int8_t* Xq, float* scale,
+                       cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Forward.
+ * ------------------------------------------------------------------------- */
+
+/* Device workspace bytes bl_forward / bl_forward_f32 need for this shape (0
+ * when the decode path is taken, M <= 2). */
+BL_API size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+
+/*
+ * [b1.58] eqs. (2)-(3): the BitLinear forward on packed weights.
+ *   q, s_m  = per-token activation quantisation of X (see bl_quant_act)
+ *   acc     = sum_k q[m,k] * code[n,k]        (exact int32)
+ *   Y[m,n]  = bf16_round_nearest_even( f32(acc) * f32(gamma / s_m) )
+ * Decode (M <= 2): one fused kernel (quantisation prologue + GEMV).
+ * Otherwise: an activation-quantisation kernel writes int8 codes, scales and
+ * row sums into the workspace, then a tcgen05 tensor-core GEMM runs.
+ * X: bf16 bits [M, K], 16-byte aligned.  Wp, gamma: from bl_quantize_weights.
+ * Y: bf16 bits [M, N].  workspace: >= bl_forward_workspace_bytes(M, K, N, bits)
+ * bytes, 16-byte aligned (may be null when that is 0).
+ */
+BL_API bl_status bl_forward(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
+                     int bits, uint16_t* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* As bl_forward but writes the fp32 value f32(acc) * f32(gamma / s_m) before
+ * the bf16 rounding.  For tests. */
+BL_API bl_status bl_forward_f32(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
+                         int bits, float* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
+BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
+
+/*
+ * [b1.58] eq. (3) without the rescale: acc[m,n] = sum_k Xq[m,k] * code[n,k]
+ * as exact int32, on already-quantised int8 activations Xq [M, K] (16-byte
+ * aligned).  acc: int32 [M, N].  Same kernels as bl_forward.  For tests.
+ */
+BL_API bl_status bl_matmul_i32(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, int32_t* acc,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Device status.
+ * ------------------------------------------------------------------------- */
+
+/* Synchronises the current device, then returns the status recorded by
+ * kernels since the last clear (BL_OK if none) and, if clear != 0, resets it.
+ * If site != NULL it receives the identifier of the wait that gave up. */
+BL_API bl_status bl_device_status(int clear, int* site);
+
+/* Launches a one-thread kernel that waits, with the library's bounded wait,
+ * on a barrier nothing ever completes; after limit_ns nanoseconds the wait
+ * gives up and records BL_ERR_TIMEOUT in the device status word.  *waited_ok
+ * (device int) receives 0.  For tests of the failure path. */
+BL_API bl_status bl_selftest_wait_timeout(unsigned long long limit_ns, int* waited_ok, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+* the library loads and exports every entry point include/bitlinear.h declares;
+* the Python binding mirrors exactly those names;
+* argument validation rejects bad calls before any CUDA call.
+
+Every validation call below carries at least one invalid argument, so nothing
+is ever launched (the pointers are fake and are never dereferenced).
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bitlinear_bl_forward_b200 import bl
+from bitlinear_bl_forward_b200 import build as blbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT, WS = range(8)
+A = 0x10000      # fake, 16-byte aligned
+U = 0x10001      # fake, misaligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    blbuild.build()
+    return bl.lib()
+
+
+def header_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^BL_API\s+[\w\s\*]+?\b(bl_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_header_symbols_exported(L):
+    syms = header_symbols()
+    assert len(syms) >= 14
+    for s in syms:
+        assert hasattr(L, s), s
+    # and nothing else with the bl_ prefix is bound by Python
+    assert sorted(bl.SIGNATURES) == syms
+
+
+def test_binding_names_match_header():
+    for s in header_symbols():
+        if s in ("bl_status_string", "bl_version", "bl_quantize_weights_workspace_bytes",
+                 "bl_matmul_i32_workspace_bytes"):
+            continue
+        assert hasattr(bl, s), s
+
+
+def test_status_strings(L):
+    for code in range(8):
+        assert L.bl_status_string(code)
+    assert L.bl_status_string(99) == b"unknown status"
+    assert L.bl_version() >= 100
+
+
+def test_sizes(L):
+    assert L.bl_packed_weight_bytes(6912, 2560) == 6912 * 2560 // 4
+    assert L.bl_packed_weight_bytes(28672, 8192) == 58720256
+    assert L.bl_forward_workspace_bytes(1, 2560, 6912, 8) == 0
+    assert L.bl_forward_workspace_bytes(2, 2560, 6912, 8) == 0
+    ws = L.bl_forward_workspace_bytes(4096, 2560, 6912, 8)
+    assert ws >= 4096 * 2560 + 2 * 4 * 4096
+    assert L.bl_forward_workspace_bytes(4096, 2500, 6912, 8) == 0     # bad shape
+    assert L.bl_quantize_weights_workspace_bytes(512, 256) > 0
+    assert L.bl_matmul_i32_workspace_bytes(17, 256, 512) >= 17 * 4
+
+
+@pytest.mark.parametrize("args,want", [
+    # (X, M, K, N, Wp, gamma, bits, Y, ws, ws_bytes)
+    ((A, 4, 100, 8, A, A, 8, A, A, 1 << 20), SHAPE),       # K % 64
+    ((A, 4, 0, 8, A, A, 8, A, A, 1 << 20), SHAPE),
+    ((A, 4, 131072, 8, A, A, 8, A, A, 1 << 30), SHAPE),    # K too large
+    ((A, 4, 64, 0, A, A, 8, A, A, 1 << 20), SHAPE),        # N <= 0
+    ((A, -1, 64, 8, A, A, 8, A, A, 1 << 20), SHAPE),       # M < 0
+    ((A, 4, 64, 8, A, A, 2, A, A, 1 << 20), UNSUP),        # bits
+    ((A, 4, 64, 8, A, A, 16, A, A, 1 << 20), UNSUP),
+    ((None, 4, 64, 8, A, A, 8, A, A, 1 << 20), INVALID),
+    ((A, 4, 64, 8, None, A, 8, A, A, 1 << 20), INVALID),
+    ((A, 4, 64, 8, A, None, 8, A, A, 1 << 20), INVALID),
+    ((A, 4, 64, 8, A, A, 8, None, A, 1 << 20), INVALID),
+    ((U, 4, 64, 8, A, A, 8, A, A, 1 << 20), ALIGN),
+    ((A, 4, 64, 8, U, A, 8, A, A, 1 << 20), ALIGN),
+    ((A, 4, 64, 8, A, A, 8, A, None, 0), WS),              # workspace needed (M > 2)
+    ((A, 4, 64, 8, A, A, 8, A, A, 16), WS),                # too small
+    ((A, 4, 64, 8, A, A, 8, A, U, 1 << 20), ALIGN),
+    ((A, 0, 64, 8, None, None, 8, None, None, 0), OK),     # M == 0: nothing to do
+])
+def test_forward_validation(L, args, want):
+    X, M, K, N, Wp, g, bits, Y, ws, wsb = args
+    assert L.bl_forward(X, M, K, N, Wp, g, bits, Y, ws, wsb, None) == want
+    assert L.bl_forward_f32(X, M, K, N, Wp, g, bits, Y, ws, wsb, None) == want
+
+
+def test_quantize_weights_validation(L):
+    need = L.bl_quantize_weights_workspace_bytes(8, 64)
+    assert L.bl_quantize_weights(A, 8, 60, A, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_quantize_weights(A, 0, 64, A, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_quantize_weights(A, 1 << 30, 1 << 14, A, A, A, 1 << 20, None) == SHAPE   # N*K >= 2^40... 2^44
+    assert L.bl_quantize_weights(None, 8, 64, A, A, A, need, None) == INVALID
+    assert L.bl_quantize_weights(A, 8, 64, None, A, A, need, None) == INVALID
+    assert L.bl_quantize_weights(A, 8, 64, A, None, A, need, None) == INVALID
+    assert L.bl_quantize_weights(U, 8, 64, A, A, A, need, None) == ALIGN
+    assert L.bl_quantize_weights(A, 8, 64, A, A, None, need, None) == WS
+    assert L.bl_quantize_weights(A, 8, 64, A, A, A, need - 1, None) == WS
+
+
+def test_other_validation(L):
+    assert L.bl_quant_act(A, 4, 64, 3, A, A, None) == UNSUP
+    assert L.bl_quant_act(A, 4, 65, 8, A, A, None) == SHAPE
+    assert L.bl_quant_act(None, 4, 64, 8, A, A, None) == INVALID
+    assert L.bl_quant_act(A, 4, 64, 8, U, A, None) == ALIGN
+    assert L.bl_quant_act(None, 0, 64, 8, None, None, None) == OK
+    assert L.bl_unpack_weights(A, 8, 48, A, None) == SHAPE
+    assert L.bl_unpack_weights(None, 8, 64, A, None) == INVALID
+    assert L.bl_unpack_weights(A, 8, 64, U, None) == ALIGN
+    assert L.bl_matmul_i32(A, 4, 64, 8, A, A, None, 0, None) == WS
+    assert L.bl_matmul_i32(None, 4, 64, 8, A, A, A, 1 << 20, None) == INVALID
+    assert L.bl_matmul_i32(A, 4, 64, -8, A, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_selftest_wait_timeout(1000, None, None) == INVALID
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    # the binding has no fallback: a missing library is an error
+    monkeypatch.setattr(bl, "_lib", None)
+    monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        bl.lib()

@@ -1,0 +1,247 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle.
+
+Bars: bit-exact gamma, packed bytes, ternary codes, int8/int4 activation codes,
+activation scales and int32 accumulators; fp32 rescaled outputs within 1e-3
+relative of the oracle; bf16 outputs within 1 ulp of the oracle's fp32 value
+rounded to bf16.  Inputs are the seeded synthetic workloads; the oracle never
+sees a value produced by the GPU.
+"""
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from bitlinear_bl_forward_b200 import bl
+from bitlinear_bl_forward_b200.inputs import WORKLOADS, layer_inputs, random_case
+from oracle import bitlinear_oracle as o
+from tests.gpu_helpers import (BF16_ULP_TOL, F32_REL_TOL, bf16_dev_to_bits, bf16_ulp_distance, rel_err,
+                               x_to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    bl.lib()
+    bl.bl_device_status(clear=True)
+    yield
+    st, site = bl.bl_device_status(clear=True)
+    assert st == 0, f"device status {st} at wait site {site}"
+
+
+@functools.lru_cache(maxsize=8)
+def oracle_weights(key):
+    """(W, gamma, codes, packed) for a cached weight (key = workload, layer)."""
+    name, i = key
+    _, W = layer_inputs(WORKLOADS[name], i, M=1)
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    return W, g, c, o.pack_ternary(c)
+
+
+def check_weights(W, g, codes, packed):
+    N, K = W.shape
+    Wd = torch.from_numpy(W).cuda()
+    Wp, gd = bl.bl_quantize_weights(Wd)
+    torch.cuda.synchronize()
+    assert gd.cpu().numpy().view(np.uint32)[0] == np.float32(g).view(np.uint32), (gd.item(), g)
+    assert np.array_equal(Wp.cpu().numpy(), packed)
+    cd = bl.bl_unpack_weights(Wp, N, K).cpu().numpy()
+    assert np.array_equal(cd, codes)
+    return Wp, gd
+
+
+def check_act(x_bits, bits):
+    q, s = o.act_quant(x_bits, bits)
+    qd, sd = bl.bl_quant_act(x_to_dev(x_bits), bits)
+    assert np.array_equal(qd.cpu().numpy(), q)
+    assert np.array_equal(sd.cpu().numpy().view(np.uint32), s.view(np.uint32))
+    return q, s
+
+
+def check_forward(x_bits, Wp, g, codes, bits, rows=None):
+    """Compare bl_forward / bl_forward_f32 / bl_matmul_i32 with the oracle;
+    `rows` restricts the oracle to a sample of tokens (per-token quantisation
+    makes each token independent)."""
+    N = codes.shape[0]
+    Xd = x_to_dev(x_bits)
+    q_full, s_full = o.act_quant(x_bits, bits)
+    sel = np.arange(x_bits.shape[0]) if rows is None else np.asarray(rows)
+    q, s = q_full[sel], s_full[sel]
+    acc = o.matmul_i32(q, codes)
+    y64, y32 = o.rescale(acc, g, s)
+    Y = o.round_to_bf16_bits(y32)
+
+    accd = bl.bl_matmul_i32(torch.from_numpy(q_full).cuda(), Wp, N).cpu().numpy()[sel]
+    assert np.array_equal(accd, acc)
+
+    Yd = bf16_dev_to_bits(bl.bl_forward(Xd, Wp, torch.tensor([g], device="cuda"), N, bits))[sel]
+    d = bf16_ulp_distance(Yd, Y)
+    assert d.max() <= BF16_ULP_TOL, f"bf16 ulp distance {d.max()}"
+
+    Yf = bl.bl_forward_f32(Xd, Wp, torch.tensor([g], device="cuda"), N, bits).cpu().numpy()[sel]
+    e = rel_err(Yf, y64)
+    assert e.max() <= F32_REL_TOL, f"fp32 rel err {e.max()}"
+    # the kernels evaluate exactly the oracle's fp32 expression
+    return float(np.mean(Yf.view(np.uint32) == y32.view(np.uint32))), float(np.mean(d == 0))
+
+
+# ---------------------------------------------------------------------------
+# failure path: bounded waits
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_times_out_cleanly():
+    bl.bl_device_status(clear=True)
+    out = bl.bl_selftest_wait_timeout(10_000_000)   # 10 ms
+    st, site = bl.bl_device_status(clear=True)
+    assert int(out.item()) == 0
+    assert st == 6 and site == 0xEE
+    # the context is still usable and the status word was cleared
+    assert bl.bl_device_status(clear=True) == (0, 0)
+    torch.ones(4, device="cuda").sum().item()
+
+
+# ---------------------------------------------------------------------------
+# small and ragged shapes
+# ---------------------------------------------------------------------------
+
+SMALL = [(1, 64, 1), (1, 256, 512), (2, 192, 100), (3, 64, 129), (16, 256, 512), (17, 320, 130),
+         (33, 128, 257), (64, 256, 64), (100, 384, 300), (130, 256, 512), (257, 192, 129), (300, 1024, 700)]
+
+
+@pytest.mark.parametrize("M,K,N", SMALL)
+@pytest.mark.parametrize("bits", [8, 4])
+def test_small_shapes(M, K, N, bits):
+    X, W = random_case(M, K, N, seed=M * 1000 + K + N)
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    Wp, gd = check_weights(W, g, c, o.pack_ternary(c))
+    check_act(X, bits)
+    check_forward(X, Wp, g, c, bits)
+
+
+def test_zero_inputs_and_degenerate_rows():
+    M, K, N = 5, 128, 96
+    X, W = random_case(M, K, N, seed=7)
+    X[1] = 0                       # all-zero token -> zero codes, zero output
+    X[3, :] = X[3, 0]              # constant row
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    Wp, _ = check_weights(W, g, c, o.pack_ternary(c))
+    check_act(X, 8)
+    check_forward(X, Wp, g, c, 8)
+    # all-zero weights: gamma = 1e-5, codes 0
+    Wz = np.zeros((N, K), np.float32)
+    gz = o.absmean_scale(Wz)
+    cz = o.ternary_codes(Wz, gz)
+    Wpz, _ = check_weights(Wz, gz, cz, o.pack_ternary(cz))
+    check_forward(X, Wpz, gz, cz, 8)
+
+
+def test_exact_ties_in_weights_and_activations():
+    # weights at exactly +-gamma/2 and +-3gamma/2, activations with x*s exact .5
+    K, N = 64, 16
+    W = np.zeros((N, K), np.float32)
+    W[:, ::4] = 0.25
+    W[:, 1::4] = -0.25
+    W[:, 2::4] = 0.0625
+    W[:, 3::4] = -0.1875
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    Wp, _ = check_weights(W, g, c, o.pack_ternary(c))
+    xf = np.zeros((3, K), np.float32)
+    xf[:, 0] = 127.0
+    xf[0, 1:8] = [2.5, 3.5, -0.5, -1.5, 0.5, 126.5, -126.5]
+    xf[1, 0] = 3.0
+    xf[1, 1:4] = [1.5, -1.5, 0.75]   # s = f32(127/3): 1.5*s is an fp32 tie -> 64
+    xf[2, 0] = 7.0
+    xf[2, 1:5] = [3.5, -3.5, 2.5, 0.5]
+    xb = (xf.view(np.uint32) >> 16).astype(np.uint16)
+    for bits in (8, 4):
+        q, _ = check_act(xb, bits)
+        check_forward(xb, Wp, g, c, bits)
+    q8, _ = o.act_quant(xb, 8)
+    assert q8[1, 1] == 64
+
+
+def test_m_zero_is_a_noop():
+    N, K = 32, 64
+    Wp = torch.zeros((N, K // 4), dtype=torch.uint8, device="cuda")
+    X = torch.zeros((0, K), dtype=torch.bfloat16, device="cuda")
+    Y = bl.bl_forward(X, Wp, torch.ones(1, device="cuda"), N)
+    assert Y.shape == (0, N)
+
+
+def test_gemv_and_tensor_core_paths_agree():
+    # M = 2 runs the decode kernel, M = 3 the tensor-core kernel; token rows
+    # are independent, so the shared rows must match bit for bit.
+    X, W = random_case(3, 2560, 700, seed=11)
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    Wp, gd = check_weights(W, g, c, o.pack_ternary(c))
+    y2 = bl.bl_forward_f32(x_to_dev(X[:2]), Wp, gd, 700).cpu().numpy()
+    y3 = bl.bl_forward_f32(x_to_dev(X), Wp, gd, 700).cpu().numpy()
+    assert np.array_equal(y2.view(np.uint32), y3[:2].view(np.uint32))
+
+
+def test_streams_are_respected():
+    # two independent problems on two streams give the same results as serial runs
+    X, W = random_case(40, 512, 384, seed=12)
+    Wd = torch.from_numpy(W).cuda()
+    Wp, gd = bl.bl_quantize_weights(Wd)
+    Xd = x_to_dev(X)
+    ref = bl.bl_forward(Xd, Wp, gd, 384).clone()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s1):
+        a = bl.bl_forward(Xd, Wp, gd, 384)
+    with torch.cuda.stream(s2):
+        b = bl.bl_forward(Xd[:1].contiguous(), Wp, gd, 384)
+    torch.cuda.synchronize()
+    assert torch.equal(a, ref) and torch.equal(b[0], ref[0])
+
+
+# ---------------------------------------------------------------------------
+# the workloads at full size
+# ---------------------------------------------------------------------------
+
+def run_workload(name, rows=None):
+    w = WORKLOADS[name]
+    for i, L in enumerate(w.layers):
+        X, _ = layer_inputs(w, i)
+        W, g, c, p = oracle_weights((name if not name.startswith("layer_70b") else "layer_70b_m1", i))
+        Wp, gd = check_weights(W, g, c, p)
+        check_act(X, w.bits)
+        exact32, exact16 = check_forward(X, Wp, g, c, w.bits, rows=rows)
+        print(f"{name}/{L.name}: fp32 bitwise-equal {exact32:.6f}, bf16 equal {exact16:.6f}")
+
+
+def test_workload_tiny():
+    run_workload("tiny")
+
+
+def test_workload_decode_2b():
+    run_workload("decode_2b")
+
+
+def test_workload_prefill_2b():
+    run_workload("prefill_2b")
+
+
+@pytest.mark.parametrize("name", ["layer_70b_m1", "layer_70b_m16", "layer_70b_m128"])
+def test_workload_70b(name):
+    run_workload(name)
+
+
+def test_workload_70b_m2048_sampled():
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(2048, 64, replace=False))
+    run_workload("layer_70b_m2048", rows=rows)
+
+
+def test_workload_a48():
+    run_workload("a48")
