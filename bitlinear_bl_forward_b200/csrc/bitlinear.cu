@@ -126,8 +126,52 @@ bl_status launch_gemv_t(const void* X, int x_is_i8, int M, int K, int N, const u
   return last_cuda();
 }
 
+template <int MT, int CPL, int RT, int D, int THREADS, int MINB>
+bl_status launch_gemv1_t(const void* X, int x_is_i8, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
+                         void* Y, int out_mode, cudaStream_t stream) {
+  constexpr int kWarps = THREADS / 32;
+  const int ntiles = (N + RT - 1) / RT;
+  // spread the tiles over at most MINB CTAs per SM, every CTA a contiguous range
+  const int cap = MINB * num_sms();
+  int tiles_per_cta = (ntiles + cap - 1) / cap;
+  if (tiles_per_cta < kWarps) tiles_per_cta = (ntiles < kWarps) ? ntiles : kWarps;
+  const int blocks = (ntiles + tiles_per_cta - 1) / tiles_per_cta;
+  // programmatic dependent launch: the kernel only prefetches into L2 before
+  // its griddepcontrol.wait, so it may start while the previous kernel drains
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint4* wp4 = reinterpret_cast<const uint4*>(Wp);
+  if (cudaLaunchKernelEx(&cfg, bl::gemv1_kernel<MT, CPL, RT, D, THREADS, MINB>, X, x_is_i8, K, N, wp4, gamma, Q, Y,
+                         out_mode, tiles_per_cta) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return last_cuda();
+}
+
 bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
                       void* Y, int out_mode, cudaStream_t stream) {
+  const int cpl = (K / 64 + 31) / 32;
+  // one CTA of 16 warps per SM (room for the next kernel's CTA to start its
+  // L2 prefetch alongside); D tiles of weights in flight per warp
+  if (M == 1 && K <= 8192) {
+    switch (cpl) {
+      case 1: return launch_gemv1_t<1, 1, 2, 4, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+      case 2: return launch_gemv1_t<1, 2, 1, 4, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+      case 3: return launch_gemv1_t<1, 3, 1, 3, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+      default: return launch_gemv1_t<1, 4, 1, 2, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+    }
+  }
+  if (M == 2 && K <= 4096) {
+    if (cpl == 1) return launch_gemv1_t<2, 1, 2, 2, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+    return launch_gemv1_t<2, 2, 1, 2, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+  }
   if (M == 1) return launch_gemv_t<1, 2>(X, x_is_i8, M, K, N, Wp, gamma, Q, Y, out_mode, stream);
   return launch_gemv_t<2, 2>(X, x_is_i8, M, K, N, Wp, gamma, Q, Y, out_mode, stream);
 }

@@ -226,4 +226,239 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Decode fast path: MT in {1, 2} tokens, K <= 8192 (CPL = ceil(K/64/32) <= 4).
+//
+//   1. each CTA owns a contiguous range of output rows, i.e. one contiguous
+//      byte range of packed weights; one thread asks the TMA unit to stream
+//      that range into L2 (cp.async.bulk.prefetch.L2).  Then the programmatic
+//      dependent-launch handshake: nothing before griddepcontrol.wait reads
+//      or writes memory, so an early start is safe whatever precedes it;
+//   2. the CTA quantises the token(s) once (two block barriers) into shared
+//      memory, XOR-swizzled so that the lanes' 64-byte-strided reads hit
+//      distinct banks; lane l then keeps the int8 activations of its
+//      64-weight chunks l, l+32, ... in registers for every row it visits;
+//   3. each warp walks RT-row tiles of the CTA's range and double-buffers the
+//      packed weights of two tiles in registers;
+//   4. unpacking without shifts: for the 2-bit slice j of a word,
+//      (w & (0x03030303 << 2j)) holds 4^j * u per byte, so an unsigned x
+//      signed dp4a gives 4^j * sum u*q; each slice has its own accumulator
+//      and the exact total is acc0 + (acc1 >> 2) + (acc2 >> 4) + (acc3 >> 6)
+//      (every acc_j is a multiple of 4^j; |acc_3| <= 64*2*127*K/4 < 2^31);
+//   5. warp-shuffle reduction, offset correction, rescale, store.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kPrefetchChunk = 1u << 16;
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+template <int CPL, int RT>
+__device__ __forceinline__ void gemv1_load(uint4 (&w)[RT][CPL], const uint4* __restrict__ Wp, int tile, int tend,
+                                           int N, int KV, int lane) {
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int n = tile * RT + r, c = lane + 32 * i;
+      w[r][i] = (tile < tend && n < N && c < KV) ? ldg_pinned_v4(Wp + static_cast<size_t>(n) * KV + c)
+                                                 : make_uint4(0, 0, 0, 0);
+    }
+}
+
+template <int MT, int CPL, int RT>
+__device__ __forceinline__ void gemv1_tile(const uint4 (&w)[RT][CPL], const uint32_t (&act)[MT][CPL][16], int tile,
+                                           int N, int KV, int lane, const int (&R)[MT], const float (&f)[MT],
+                                           void* __restrict__ Y, int out_mode) {
+  int acc[RT][MT][4];
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[r][m][j] = 0;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    if (i == CPL - 1 && lane + 32 * i >= KV) break;   // only the last chunk slot can be empty
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const uint32_t wd[4] = {w[r][i].x, w[r][i].y, w[r][i].z, w[r][i].w};
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t e = wd[g] & (0x03030303u << (2 * j));
+#pragma unroll
+          for (int m = 0; m < MT; ++m) acc[r][m][j] = dp4a_us(e, act[m][i][4 * g + j], acc[r][m][j]);
+        }
+    }
+  }
+  int tot[RT][MT];
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      tot[r][m] = warp_sum(acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6));
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const int n = tile * RT + r;
+      if (lane == r * MT + m && n < N) {
+        const int a = tot[r][m] - R[m];
+        const size_t o = static_cast<size_t>(m) * N + n;
+        if (out_mode == kOutI32) {
+          static_cast<int*>(Y)[o] = a;
+        } else {
+          const float y = __fmul_rn(__int2float_rn(a), f[m]);
+          if (out_mode == kOutF32)
+            static_cast<float*>(Y)[o] = y;
+          else
+            static_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(y);
+        }
+      }
+    }
+}
+
+template <int MT, int CPL, int RT, int D, int THREADS, int MINB>
+__global__ void __launch_bounds__(THREADS, MINB)
+    gemv1_kernel(const void* __restrict__ X, int x_is_i8, int K, int N, const uint4* __restrict__ Wp,
+                 const float* __restrict__ gamma_p, int Q, void* __restrict__ Y, int out_mode, int tiles_per_cta) {
+  constexpr int WARPS = THREADS / 32;
+  __shared__ __align__(16) uint8_t s_act[MT][8192];
+  __shared__ uint32_t s_red_f[MT][WARPS];
+  __shared__ int s_red_i[MT][WARPS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KV = K >> 6;
+  const int ntiles = (N + RT - 1) / RT;
+  const int tbeg = blockIdx.x * tiles_per_cta;
+  const int tend = min(ntiles, tbeg + tiles_per_cta);
+
+  // 1. stream this CTA's weight rows into L2; dependent-launch handshake
+  if (threadIdx.x == 0 && tbeg < tend) {
+    const size_t row_bytes = static_cast<size_t>(K) >> 2;
+    const size_t r0 = static_cast<size_t>(tbeg) * RT;
+    const size_t r1 = min(static_cast<size_t>(N), static_cast<size_t>(tend) * RT);
+    const char* base = reinterpret_cast<const char*>(Wp) + r0 * row_bytes;
+    const size_t bytes = (r1 - r0) * row_bytes;
+    for (size_t off = 0; off < bytes; off += kPrefetchChunk)
+      bulk_prefetch_l2(base + off, static_cast<uint32_t>(min(static_cast<size_t>(kPrefetchChunk), bytes - off)));
+  }
+  pdl_launch_dependents();
+  pdl_wait();
+
+  // token loads first, then the first D weight tiles of this warp (a ring of
+  // D register buffers, refilled as tiles are consumed)
+  constexpr int U = (8192 / 8 + THREADS - 1) / THREADS;   // 16-byte token loads per thread
+  const int nch = x_is_i8 ? (K >> 4) : (K >> 3);
+  uint4 xv[MT][U];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = threadIdx.x + THREADS * u;
+      xv[m][u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + static_cast<size_t>(m) * nch + c)
+                           : make_uint4(0, 0, 0, 0);
+    }
+  uint4 wr[D][RT][CPL];
+#pragma unroll
+  for (int d = 0; d < D; ++d) gemv1_load<CPL, RT>(wr[d], Wp, tbeg + warp + d * WARPS, tend, N, KV, lane);
+  const float gamma = (out_mode == kOutI32) ? 1.f : __ldg(gamma_p);
+
+  // 2. the CTA quantises the token(s) into s_act (plain byte order)
+  int rsum[MT];
+  float s[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    rsum[m] = 0;
+    s[m] = 1.f;
+  }
+  if (!x_is_i8) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float amax = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) amax = fmaxf(amax, absmax8_bf16(xv[m][u]));
+      // non-negative floats order like their bit patterns
+      const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+      if (lane == 0) s_red_f[m][warp] = wmax;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      uint32_t bmax = s_red_f[m][0];
+#pragma unroll
+      for (int w = 1; w < WARPS; ++w) bmax = max(bmax, s_red_f[m][w]);
+      s[m] = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = threadIdx.x + THREADS * u;
+        if (c < nch) *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = quant8_bf16(xv[m][u], s[m], Q, rsum[m]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = threadIdx.x + THREADS * u;
+        if (c < nch) {
+          const uint4 v = xv[m][u];
+          rsum[m] = __dp4a(static_cast<int>(v.x), 0x01010101, rsum[m]);
+          rsum[m] = __dp4a(static_cast<int>(v.y), 0x01010101, rsum[m]);
+          rsum[m] = __dp4a(static_cast<int>(v.z), 0x01010101, rsum[m]);
+          rsum[m] = __dp4a(static_cast<int>(v.w), 0x01010101, rsum[m]);
+          *reinterpret_cast<uint4*>(&s_act[m][act_swz(16u * c)]) = v;
+        }
+      }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int ws = __reduce_add_sync(0xffffffffu, rsum[m]);
+    if (lane == 0) s_red_i[m][warp] = ws;
+  }
+  __syncthreads();
+  int R[MT];
+  float f[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    R[m] = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) R[m] += s_red_i[m][w];
+    f[m] = (x_is_i8 || out_mode == kOutI32) ? 0.f : __fdiv_rn(gamma, s[m]);
+  }
+
+  // this lane's activation chunks, kept in registers
+  uint32_t act[MT][CPL][16];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int c = lane + 32 * i;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (c < KV) v = *reinterpret_cast<const uint4*>(&s_act[m][act_swz(64u * c + 16u * g)]);
+        act[m][i][4 * g + 0] = v.x;
+        act[m][i][4 * g + 1] = v.y;
+        act[m][i][4 * g + 2] = v.z;
+        act[m][i][4 * g + 3] = v.w;
+      }
+    }
+
+  // 3.-5. this warp's tiles tbeg + warp + k*WARPS; ring buffer d holds tile k with k % D == d
+  for (int t = tbeg + warp; t < tend; t += D * WARPS) {
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      const int td = t + d * WARPS;
+      if (td >= tend) break;
+      gemv1_tile<MT, CPL, RT>(wr[d], act, td, N, KV, lane, R, f, Y, out_mode);
+      gemv1_load<CPL, RT>(wr[d], Wp, td + D * WARPS, tend, N, KV, lane);
+    }
+  }
+}
+
 }  // namespace bl
