@@ -21,6 +21,7 @@ BL_OK = 0
 STATUS_NAMES = {
     0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGNMENT",
     4: "BL_ERR_UNSUPPORTED", 5: "BL_ERR_CUDA", 6: "BL_ERR_TIMEOUT", 7: "BL_ERR_WORKSPACE",
+    8: "BL_ERR_SCRATCH_LIMIT",
 }
 
 # name -> (restype, argtypes), mirroring include/bitlinear.h
@@ -36,6 +37,7 @@ SIGNATURES = {
     "bl_forward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "bl_forward": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_forward_f32": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
+    "bl_forward_noalloc": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
@@ -164,6 +166,22 @@ def bl_forward_f32(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: in
     _check(lib().bl_forward_f32(px, M, K, N, pw, pg, bits, Y.data_ptr(),
                                 ws.data_ptr() if ws is not None else None,
                                 ws.numel() if ws is not None else 0, _stream()), "bl_forward_f32")
+    return Y
+
+
+def bl_forward_noalloc(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8,
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """bl_forward without a workspace: for callers that cannot allocate device
+    memory per call, the library keeps the scratch in a static device array
+    (limits M*K <= 16 MiB, M <= 8192 when M > 2; calls that overlap on the GPU
+    race on it).  Only the output buffer is passed in."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    _check(lib().bl_forward_noalloc(px, M, K, N, pw, pg, bits, py, _stream()), "bl_forward_noalloc")
     return Y
 
 

@@ -266,6 +266,8 @@ const char* bl_status_string(bl_status s) {
     case BL_ERR_CUDA: return "CUDA error";
     case BL_ERR_TIMEOUT: return "a kernel wait timed out";
     case BL_ERR_WORKSPACE: return "workspace missing or too small";
+    case BL_ERR_SCRATCH_LIMIT:
+      return "shape exceeds the built-in scratch of bl_forward_noalloc (M*K <= 16 MiB, M <= 8192)";
   }
   return "unknown status";
 }
@@ -380,6 +382,67 @@ bl_status bl_matmul_i32(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const
   bl::act_rowsum_kernel<<<(m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock, 256, 0, stream>>>(Xq, m, k, R);
   if ((st = last_cuda()) != BL_OK) return st;
   return launch_tc(Xq, m, k, n, Wp, R, nullptr, nullptr, acc, bl::kOutI32, 0, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the tensor-core path's scratch lives in one static
+// device array (one copy per GPU that loads the library, until exit) instead
+// of a caller workspace.  For callers that cannot allocate device memory or
+// pass a workspace, e.g. engines that budget all memory at start-up and give an
+// operator only its inputs and outputs.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+constexpr size_t kNoAllocCodeBytes = size_t(16) << 20;    // int8 codes: M*K <= 16 MiB
+constexpr int64_t kNoAllocMaxM = 8192;                     // tokens: scales and row sums
+constexpr size_t kNoAllocBytes = kNoAllocCodeBytes + 2 * sizeof(int32_t) * kNoAllocMaxM;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+
+// The array's device address on the current device.  Host code must not use
+// the symbol itself (it names a host-side stand-in); the address is looked up
+// once per device with that device current, then cached.
+bl_status noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
+  void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return BL_ERR_CUDA;
+    g_noalloc_addr[dev].store(p, std::memory_order_release);
+  }
+  *out = static_cast<unsigned char*>(p);
+  return BL_OK;
+}
+}  // namespace
+
+extern "C" {
+
+bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
+                             const float* gamma, int bits, uint16_t* Y, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (M == 0) return BL_OK;
+  if (!X || !Wp || !gamma || !Y) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wp)) return BL_ERR_ALIGNMENT;
+  const int Q = bits == 8 ? 127 : 7;
+  const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+  if (M <= kGemvMaxM) return launch_gemv(X, 0, m, k, n, Wp, gamma, Q, Y, bl::kOutBF16, stream);
+  if (static_cast<size_t>(M) * static_cast<size_t>(K) > kNoAllocCodeBytes || M > kNoAllocMaxM)
+    return BL_ERR_SCRATCH_LIMIT;
+  unsigned char* base = nullptr;
+  if ((st = noalloc_scratch(&base)) != BL_OK) return st;
+  int8_t* Xq = reinterpret_cast<int8_t*>(base);
+  float* s = reinterpret_cast<float*>(base + kNoAllocCodeBytes);
+  int* R = reinterpret_cast<int*>(base + kNoAllocCodeBytes + sizeof(float) * kNoAllocMaxM);
+  const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
+  bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
+  if ((st = last_cuda()) != BL_OK) return st;
+  return launch_tc(Xq, m, k, n, Wp, R, s, gamma, Y, bl::kOutBF16, 0, stream);
 }
 
 bl_status bl_device_status(int clear, int* site) {

@@ -53,7 +53,8 @@ typedef enum {
   BL_ERR_UNSUPPORTED = 4, /* bits not in {4, 8} */
   BL_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
   BL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait gave up (device status word) */
-  BL_ERR_WORKSPACE = 7    /* workspace pointer null or smaller than required */
+  BL_ERR_WORKSPACE = 7,   /* workspace pointer null or smaller than required */
+  BL_ERR_SCRATCH_LIMIT = 8 /* shape exceeds the built-in scratch of bl_forward_noalloc */
 } bl_status;
 
 /* Static, NUL-terminated description of a status code. */
@@ -142,6 +143,33 @@ BL_API bl_status bl_forward(const uint16_t* X, int64_t M, int64_t K, int64_t N, 
  * the bf16 rounding.  For tests. */
 BL_API bl_status bl_forward_f32(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
                          int bits, float* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Allocation-free forward.  The pages have no counterpart of this call; it is
+ * an integration aid.  Some callers cannot allocate device memory or hand the
+ * library a workspace: for example an engine that budgets all device memory
+ * once at start-up and gives its operators only their input and output
+ * buffers, or a plug-in whose host framework owns every allocation.  This call
+ * computes exactly what bl_forward computes, with the same kernels, but keeps
+ * the tensor-core path's scratch (int8 activation codes, per-token scales and
+ * row sums) in one static device array of the library instead of a caller
+ * workspace.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Limits: M*K <= 16 MiB (the int8 codes) and M <= 8192 on the tensor-core path
+ * (M > 2); larger shapes return BL_ERR_SCRATCH_LIMIT before anything runs.
+ * The decode path (M <= 2) needs no scratch and has no such limit.  The array
+ * (16 MiB + 64 KiB) exists on every GPU that loads the library, until the
+ * process exits.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  Every call on a device shares the one array: calls whose
+ * kernels overlap on the GPU (different streams, or several host threads) race
+ * on it and must be serialised by the caller.  Nothing in the array needs to
+ * start at zero: every byte a call reads is first written by the same call.
+ * Arguments, layouts and status codes are otherwise those of bl_forward.
+ */
+BL_API bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
+                                    const float* gamma, int bits, uint16_t* Y, cudaStream_t stream);
 
 /* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
 BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
