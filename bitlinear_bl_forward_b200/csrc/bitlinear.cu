@@ -155,8 +155,52 @@ bl_status launch_gemv1_t(const void* X, int x_is_i8, int K, int N, const uint8_t
   return last_cuda();
 }
 
+template <int MT, int CPL>
+bl_status launch_gemv2_t(const void* X, int x_is_i8, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
+                         void* Y, int out_mode, cudaStream_t stream) {
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(bl::gemv2_kernel<MT, CPL>, bl::kG2SmemBytes, &done)) return BL_ERR_CUDA;
+  const int sms = num_sms();
+  const int rows_per_cta = (N + sms - 1) / sms;
+  const int blocks = (N + rows_per_cta - 1) / rows_per_cta;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(bl::kG2Threads);
+  cfg.dynamicSmemBytes = bl::kG2SmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const unsigned long long lim = kWaitLimitNs;
+  if (cudaLaunchKernelEx(&cfg, bl::gemv2_kernel<MT, CPL>, X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, rows_per_cta,
+                         lim) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return last_cuda();
+}
+
+// Decode kernel selection (build-time, for experiments): 0 = by shape,
+// 1 = register-ring GEMV only, 2 = TMA-staged GEMV whenever M == 1.
+#ifndef BL_DECODE_KERNEL
+#define BL_DECODE_KERNEL 0
+#endif
+constexpr int kDecodeKernel = BL_DECODE_KERNEL;
+
 bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
                       void* Y, int out_mode, cudaStream_t stream) {
+  const int cplx = (K / 64 + 31) / 32;
+  // one token: the TMA-staged kernel (measured at least as fast on every
+  // decode shape); two tokens: the register-ring kernel
+  const bool staged = (kDecodeKernel == 2) || (kDecodeKernel == 0 && M == 1);
+  if (staged && M == 1 && K <= 8192) {
+    switch (cplx) {
+      case 1: return launch_gemv2_t<1, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+      case 2: return launch_gemv2_t<1, 2>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+      case 3: return launch_gemv2_t<1, 3>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+      default: return launch_gemv2_t<1, 4>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+    }
+  }
   const int cpl = (K / 64 + 31) / 32;
   // one CTA of 16 warps per SM (room for the next kernel's CTA to start its
   // L2 prefetch alongside); D tiles of weights in flight per warp

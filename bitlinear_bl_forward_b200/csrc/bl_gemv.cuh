@@ -269,10 +269,11 @@ __device__ __forceinline__ void gemv1_load(uint4 (&w)[RT][CPL], const uint4* __r
     }
 }
 
+// Partial dot products of one RT-row tile for this lane: one accumulator per
+// token and 2-bit slice j (each a multiple of 4^j), folded into one partial.
 template <int MT, int CPL, int RT>
-__device__ __forceinline__ void gemv1_tile(const uint4 (&w)[RT][CPL], const uint32_t (&act)[MT][CPL][16], int tile,
-                                           int N, int KV, int lane, const int (&R)[MT], const float (&f)[MT],
-                                           void* __restrict__ Y, int out_mode) {
+__device__ __forceinline__ void gemv1_accumulate(const uint4 (&w)[RT][CPL], const uint32_t (&act)[MT][CPL][16],
+                                                 int KV, int lane, int (&part)[RT][MT]) {
   int acc[RT][MT][4];
 #pragma unroll
   for (int r = 0; r < RT; ++r)
@@ -296,19 +297,26 @@ __device__ __forceinline__ void gemv1_tile(const uint4 (&w)[RT][CPL], const uint
         }
     }
   }
-  int tot[RT][MT];
 #pragma unroll
   for (int r = 0; r < RT; ++r)
 #pragma unroll
     for (int m = 0; m < MT; ++m)
-      tot[r][m] = warp_sum(acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6));
+      part[r][m] = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6);
+}
+
+// Warp-wide sum of the partials (one redux per row and token), correction and
+// rescale, store.
+template <int MT, int RT>
+__device__ __forceinline__ void gemv1_finish(const int (&part)[RT][MT], int tile, int N, int lane, const int (&R)[MT],
+                                             const float (&f)[MT], void* __restrict__ Y, int out_mode) {
 #pragma unroll
   for (int r = 0; r < RT; ++r)
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
+      const int tot = __reduce_add_sync(0xffffffffu, part[r][m]);
       const int n = tile * RT + r;
       if (lane == r * MT + m && n < N) {
-        const int a = tot[r][m] - R[m];
+        const int a = tot - R[m];
         const size_t o = static_cast<size_t>(m) * N + n;
         if (out_mode == kOutI32) {
           static_cast<int*>(Y)[o] = a;
@@ -329,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, MINB)
                  const float* __restrict__ gamma_p, int Q, void* __restrict__ Y, int out_mode, int tiles_per_cta) {
   constexpr int WARPS = THREADS / 32;
   __shared__ __align__(16) uint8_t s_act[MT][8192];
-  __shared__ uint32_t s_red_f[MT][WARPS];
+  __shared__ __align__(16) uint32_t s_red_f[MT][WARPS];
   __shared__ int s_red_i[MT][WARPS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KV = K >> 6;
@@ -389,9 +397,12 @@ __global__ void __launch_bounds__(THREADS, MINB)
     __syncthreads();
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      uint32_t bmax = s_red_f[m][0];
+      uint32_t bmax = 0;
 #pragma unroll
-      for (int w = 1; w < WARPS; ++w) bmax = max(bmax, s_red_f[m][w]);
+      for (int w = 0; w < WARPS; w += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(&s_red_f[m][w]);
+        bmax = max(bmax, max(max(v.x, v.y), max(v.z, v.w)));
+      }
       s[m] = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -449,16 +460,223 @@ __global__ void __launch_bounds__(THREADS, MINB)
       }
     }
 
-  // 3.-5. this warp's tiles tbeg + warp + k*WARPS; ring buffer d holds tile k with k % D == d
+  // 3.-5. this warp's tiles tbeg + warp + k*WARPS; ring buffer d holds tile k
+  // with k % D == d.  A round accumulates its D tiles together (independent
+  // chains), refills the ring with the next round's loads, then reduces and
+  // stores while those loads are in flight.
   for (int t = tbeg + warp; t < tend; t += D * WARPS) {
+    int part[D][RT][MT];
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const int td = t + d * WARPS;
-      if (td >= tend) break;
-      gemv1_tile<MT, CPL, RT>(wr[d], act, td, N, KV, lane, R, f, Y, out_mode);
-      gemv1_load<CPL, RT>(wr[d], Wp, td + D * WARPS, tend, N, KV, lane);
-    }
+    for (int d = 0; d < D; ++d) gemv1_accumulate<MT, CPL, RT>(wr[d], act, KV, lane, part[d]);
+#pragma unroll
+    for (int d = 0; d < D; ++d) gemv1_load<CPL, RT>(wr[d], Wp, t + (d + D) * WARPS, tend, N, KV, lane);
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+      if (t + d * WARPS < tend) gemv1_finish<MT, RT>(part[d], t + d * WARPS, N, lane, R, f, Y, out_mode);
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Decode, large layers: the same arithmetic as gemv1_kernel, but the packed
+// weights reach the SM through a shared-memory ring filled by the TMA unit.
+//
+// Each CTA (one per SM) owns a contiguous row range, i.e. one contiguous byte
+// range.  Warp 16 is the producer: one thread cuts the range into stages of
+// whole rows (<= 32 KB) and issues one cp.async.bulk per stage onto the
+// stage's mbarrier, so up to kG2Stages x 32 KB are in flight per SM without
+// spending registers.  Warps 0-15 quantise the token (named barriers among
+// themselves, so the producer never waits on them), keep their lanes'
+// activation chunks in registers, and then consume stages: a warp takes rows
+// w, w+16, ... of the stage, its lanes read their 16-byte chunks of the row
+// from shared memory (consecutive lanes, consecutive addresses), accumulate
+// with the masked dp4a scheme, reduce with redux and store.  Each consumer
+// warp releases a stage with one arrive on its "empty" barrier.  All waits are
+// bounded; on a timeout the kernel records BL_ERR_TIMEOUT and unwinds, and
+// the producer waits for the copies it issued before the CTA exits.
+// ---------------------------------------------------------------------------
+constexpr int kG2ConsumerWarps = 16;
+constexpr int kG2Threads = (kG2ConsumerWarps + 1) * 32;
+constexpr int kG2Stages = 6;
+constexpr int kG2StageBytes = 32 * 1024;
+constexpr int kG2SmemBytes = kG2Stages * kG2StageBytes + 2048;
+
+template <int MT, int CPL>
+__global__ void __launch_bounds__(kG2Threads, 1)
+    gemv2_kernel(const void* __restrict__ X, int x_is_i8, int K, int N, const uint8_t* __restrict__ Wp,
+                 const float* __restrict__ gamma_p, int Q, void* __restrict__ Y, int out_mode, int rows_per_cta,
+                 unsigned long long limit_ns) {
+  extern __shared__ __align__(128) uint8_t g2_smem[];
+  __shared__ __align__(16) uint8_t s_act[MT][8192];
+  __shared__ __align__(16) uint32_t s_red_f[MT][kG2ConsumerWarps];
+  __shared__ int s_red_i[MT][kG2ConsumerWarps];
+  __shared__ __align__(8) uint64_t full[kG2Stages], empty[kG2Stages];
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KV = K >> 6;
+  const size_t row_bytes = static_cast<size_t>(K) >> 2;
+  const int r0 = blockIdx.x * rows_per_cta;
+  const int r1 = min(N, r0 + rows_per_cta);
+  const int stage_rows = kG2StageBytes / static_cast<int>(row_bytes);
+  const int nst = (r1 > r0) ? (r1 - r0 + stage_rows - 1) / stage_rows : 0;
+  volatile int* abort_v = &abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kG2Stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kG2ConsumerWarps);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+    if (r1 > r0) {
+      const char* base = reinterpret_cast<const char*>(Wp) + static_cast<size_t>(r0) * row_bytes;
+      const size_t bytes = static_cast<size_t>(r1 - r0) * row_bytes;
+      for (size_t off = 0; off < bytes; off += kPrefetchChunk)
+        bulk_prefetch_l2(base + off, static_cast<uint32_t>(min(static_cast<size_t>(kPrefetchChunk), bytes - off)));
+    }
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (warp == kG2ConsumerWarps) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % kG2Stages;
+        if (st >= kG2Stages && !mbar_wait(&empty[s], ((st / kG2Stages) & 1) ^ 1u, abort_v, limit_ns, 11)) break;
+        const int rows = min(stage_rows, r1 - (r0 + st * stage_rows));
+        const uint32_t bytes = static_cast<uint32_t>(rows * row_bytes);
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_load(g2_smem + s * kG2StageBytes,
+                  Wp + (static_cast<size_t>(r0) + static_cast<size_t>(st) * stage_rows) * row_bytes, bytes, &full[s]);
+        issued = st + 1;
+      }
+      for (int s = 0; s < kG2Stages && s < issued; ++s) {
+        const int last = s + kG2Stages * ((issued - 1 - s) / kG2Stages);
+        mbar_wait(&full[s], (last / kG2Stages) & 1, nullptr, limit_ns, 12);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers: token quantisation ----------------
+  constexpr int CT = kG2ConsumerWarps * 32;
+  constexpr int U = (8192 / 8 + CT - 1) / CT;
+  const int nch = x_is_i8 ? (K >> 4) : (K >> 3);
+  uint4 xv[MT][U];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = threadIdx.x + CT * u;
+      xv[m][u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + static_cast<size_t>(m) * nch + c)
+                           : make_uint4(0, 0, 0, 0);
+    }
+  const float gamma = (out_mode == kOutI32) ? 1.f : __ldg(gamma_p);
+  int rsum[MT];
+  float sc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    rsum[m] = 0;
+    sc[m] = 1.f;
+  }
+  if (!x_is_i8) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float amax = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) amax = fmaxf(amax, absmax8_bf16(xv[m][u]));
+      const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+      if (lane == 0) s_red_f[m][warp] = wmax;
+    }
+    named_bar_sync(1, CT);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      uint32_t bmax = 0;
+#pragma unroll
+      for (int w = 0; w < kG2ConsumerWarps; w += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(&s_red_f[m][w]);
+        bmax = max(bmax, max(max(v.x, v.y), max(v.z, v.w)));
+      }
+      sc[m] = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = threadIdx.x + CT * u;
+        if (c < nch) *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = quant8_bf16(xv[m][u], sc[m], Q, rsum[m]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = threadIdx.x + CT * u;
+        if (c < nch) {
+          const uint4 v = xv[m][u];
+          rsum[m] = __dp4a(static_cast<int>(v.x), 0x01010101, rsum[m]);
+          rsum[m] = __dp4a(static_cast<int>(v.y), 0x01010101, rsum[m]);
+          rsum[m] = __dp4a(static_cast<int>(v.z), 0x01010101, rsum[m]);
+          rsum[m] = __dp4a(static_cast<int>(v.w), 0x01010101, rsum[m]);
+          *reinterpret_cast<uint4*>(&s_act[m][act_swz(16u * c)]) = v;
+        }
+      }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int ws = __reduce_add_sync(0xffffffffu, rsum[m]);
+    if (lane == 0) s_red_i[m][warp] = ws;
+  }
+  named_bar_sync(1, CT);
+  int R[MT];
+  float f[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    R[m] = 0;
+#pragma unroll
+    for (int w = 0; w < kG2ConsumerWarps; ++w) R[m] += s_red_i[m][w];
+    f[m] = (x_is_i8 || out_mode == kOutI32) ? 0.f : __fdiv_rn(gamma, sc[m]);
+  }
+  uint32_t act[MT][CPL][16];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int c = lane + 32 * i;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (c < KV) v = *reinterpret_cast<const uint4*>(&s_act[m][act_swz(64u * c + 16u * g)]);
+        act[m][i][4 * g + 0] = v.x;
+        act[m][i][4 * g + 1] = v.y;
+        act[m][i][4 * g + 2] = v.z;
+        act[m][i][4 * g + 3] = v.w;
+      }
+    }
+
+  // ---------------- consumers: stream the stages ----------------
+  for (int st = 0; st < nst; ++st) {
+    const int s = st % kG2Stages;
+    const bool ok = mbar_wait(&full[s], (st / kG2Stages) & 1, abort_v, limit_ns, 13);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const int row0 = r0 + st * stage_rows;
+    const int rows = min(stage_rows, r1 - row0);
+    const uint8_t* sbase = g2_smem + s * kG2StageBytes;
+    for (int rr = warp; rr < rows; rr += kG2ConsumerWarps) {
+      uint4 w[1][CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const int c = lane + 32 * i;
+        w[0][i] = (c < KV) ? *reinterpret_cast<const uint4*>(sbase + rr * row_bytes + 16 * c) : make_uint4(0, 0, 0, 0);
+      }
+      int part[1][MT];
+      gemv1_accumulate<MT, CPL, 1>(w, act, KV, lane, part);
+      gemv1_finish<MT, 1>(part, row0 + rr, N, lane, R, f, Y, out_mode);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
 }  // namespace bl
