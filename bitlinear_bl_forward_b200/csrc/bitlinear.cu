@@ -16,6 +16,8 @@
 #include "bl_act.cuh"
 #include "bl_common.cuh"
 #include "bl_gemm_tc.cuh"
+#include "bl_gemm_tc2.cuh"
+#include "bl_gemm_2sm.cuh"
 #include "bl_gemv.cuh"
 #include "bl_weights.cuh"
 
@@ -240,8 +242,105 @@ bl_status launch_tc_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, 
   return last_cuda();
 }
 
+template <int BN, int EXPG>
+bl_status launch_tc2_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
+                       const float* gamma, void* Y, int out_mode, cudaStream_t stream) {
+  using C = bl::P2Cfg<BN>;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(bl::tc_gemm_persistent_kernel<BN, EXPG>, C::kSmemBytes, &done)) return BL_ERR_CUDA;
+  CUtensorMap tmX, tmW;
+  if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), BN, bl::kTcBK,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return BL_ERR_CUDA;
+  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kTcBK / 4,
+                    CU_TENSOR_MAP_SWIZZLE_32B))
+    return BL_ERR_CUDA;
+  const int ntiles = ((M + BN - 1) / BN) * ((N + bl::kTcRows - 1) / bl::kTcRows);
+  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  bl::tc_gemm_persistent_kernel<BN, EXPG><<<grid, bl::P2Warps<EXPG>::kThreads, C::kSmemBytes, stream>>>(
+      tmX, tmW, M, N, K, R, s, gamma, Y, out_mode, kWaitLimitNs);
+  return last_cuda();
+}
+
+// Largest number of two-CTA clusters of `kernel` that are resident at once on
+// the current device (cached per device).
+template <typename F>
+int max_active_pairs(F* kernel, int threads, int smem) {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) return 0;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
+                         const float* gamma, void* Y, int out_mode, cudaStream_t stream) {
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(bl::tc_gemm_pair_kernel, bl::kQSmemBytes, &done)) return BL_ERR_CUDA;
+  CUtensorMap tmX, tmW;
+  if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), bl::kQHalf, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return BL_ERR_CUDA;
+  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kQBK / 4,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return BL_ERR_CUDA;
+  const int ntiles = ((M + bl::kQBN - 1) / bl::kQBN) * ((N + bl::kQRows - 1) / bl::kQRows);
+  cudaLaunchConfig_t cfg = {};
+  // a persistent grid must fit in one wave: not every SM can host half of a
+  // two-SM cluster, so ask how many clusters are co-resident (once per device)
+  int npairs = max_active_pairs(bl::tc_gemm_pair_kernel, bl::kQThreads, bl::kQSmemBytes);
+  if (npairs <= 0) return BL_ERR_CUDA;
+  if (npairs > ntiles) npairs = ntiles;
+  cfg.gridDim = dim3(2 * npairs);
+  cfg.blockDim = dim3(bl::kQThreads);
+  cfg.dynamicSmemBytes = bl::kQSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const unsigned long long lim = kWaitLimitNs;
+  if (cudaLaunchKernelEx(&cfg, bl::tc_gemm_pair_kernel, tmX, tmW, M, N, K, R, s, gamma, Y, out_mode, lim) !=
+      cudaSuccess)
+    return BL_ERR_CUDA;
+  return last_cuda();
+}
+
+// Tensor-core kernel selection (build-time, for experiments): 0 = by shape
+// (CTA-pair kernel for M > 64, one-SM persistent kernel otherwise),
+// 1 = one-tile-per-CTA kernel, 2 = one-SM persistent kernel only.
+#ifndef BL_TC_KERNEL
+#define BL_TC_KERNEL 0
+#endif
+
 bl_status launch_tc(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
                     const float* gamma, void* Y, int out_mode, int debug_flags, cudaStream_t stream) {
+  if (BL_TC_KERNEL == 0 && debug_flags == 0 && M > 64)
+    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+  if (BL_TC_KERNEL != 1 && debug_flags == 0) {
+    if (M <= 16) return launch_tc2_t<16, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    if (M <= 32) return launch_tc2_t<32, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    if (M <= 64) return launch_tc2_t<64, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    return launch_tc2_t<128, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+  }
   const unsigned long long lim = kWaitLimitNs;
   if (M <= 16) return launch_tc_t<16>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
   if (M <= 32) return launch_tc_t<32>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);

@@ -1,0 +1,291 @@
+// Persistent tensor-core GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same arithmetic as the other tensor-core kernels ("BitNet b1.58: The 1-Bit
+// Ternary LLM Architecture Guide", section "The Mathematical Formulation of
+// BitLinear", eq. (3)): D[n, m] = sum_k u[n, k] * q[m, k] with u = c + 1 the
+// expanded weight codes (A, tensor memory) and q the int8 activation codes
+// (B, shared memory); the epilogue subtracts R[m] and applies gamma / s_m.
+//
+// A cluster of two CTAs (two SMs) computes one 256 x BN tile per MMA
+// (M = 256 weight rows, N = BN tokens):
+//   * each CTA stages its own 128 weight rows (packed) and HALF of the token
+//     tile (BN/2 rows of int8 codes) in its own shared memory with TMA, and
+//     expands its weight rows into its own tensor memory;
+//   * the leader CTA (rank 0) issues tcgen05.mma.cta_group::2; the pair's
+//     tensor cores share the two halves of B, so each SM loads and serves only
+//     half of the activation tile -- the traffic that bounds the one-SM
+//     kernel;
+//   * the leader's tcgen05.commit arrives on the barriers of both CTAs
+//     (smem stage free, TMEM A slot free, accumulator full); the peer's
+//     expanders and epilogue warps arrive on the leader's barriers remotely.
+// Rings as in the one-SM persistent kernel: S shared-memory stages, 8 TMEM A
+// slots (the slot round trip crosses the pair twice), 2 accumulators (the epilogue of tile i overlaps the MMAs of i+1).
+// Warps: 0 producer, 1 MMA issuer (leader) / TMEM owner, 2-5 expanders,
+// 6-9 epilogue.  All waits are bounded; the pair meets at a cluster barrier
+// before TMEM is freed, after the leader has waited for its last MMA.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "bl_common.cuh"
+#include "bl_gemm_tc.cuh"
+#include "bl_gemv.cuh"
+
+namespace bl {
+
+constexpr int kQThreads = 320;
+constexpr int kQBK = 256;                       // K per pipeline stage: 8 MMAs per hand-off
+constexpr int kQASlots = 4;                     // TMEM: 2 x 128 accumulator + 4 x 64 A columns = 512
+constexpr int kQASlotCols = kQBK / 4;           // int8 codes, 4 per 32-bit column
+constexpr int kQBN = 128;                       // tokens per pair tile (MMA N)
+constexpr int kQHalf = kQBN / 2;                // token rows staged per CTA
+constexpr int kQRows = 256;                     // weight rows per pair tile (MMA M)
+constexpr int kQXBoxBytes = kQHalf * 128;       // one 128-byte-wide activation box (SW128)
+constexpr int kQXStageBytes = kQHalf * kQBK;    // 16 KB: kQBK / 128 boxes
+constexpr int kQWStageBytes = kTcRows * kQBK / 4;   // 8 KB packed, 64-byte rows (SW64)
+constexpr int kQStageBytes = kQXStageBytes + kQWStageBytes;
+constexpr int kQStages = 8;                     // 192 KB
+constexpr int kQAccCols = kQBN;
+constexpr int kQACol = 2 * kQAccCols;
+constexpr int kQTmemCols = 512;
+constexpr int kQBarOffset = kQStages * kQStageBytes;
+constexpr int kQNumBars = 2 * kQStages + 2 * kQASlots + 5;
+constexpr int kQEpiOffset = kQBarOffset + kQNumBars * 8 + 16;
+constexpr int kQSmemBytes = kQEpiOffset + 2 * kQBN * 8 + 1024;
+
+__global__ void __launch_bounds__(kQThreads, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int M, int N,
+                        int K, const int* __restrict__ Rg, const float* __restrict__ sg,
+                        const float* __restrict__ gamma_p, void* __restrict__ Y, int out_mode,
+                        unsigned long long limit_ns) {
+  constexpr int S = kQStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sX = smem;
+  uint8_t* sW = smem + S * kQXStageBytes;
+  static_assert(kQBK % 128 == 0 && kQASlotCols == 64, "stage layout below assumes K = 256 per stage");
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQBarOffset);
+  uint64_t* empty = full + S;
+  uint64_t* afull = empty + S;        // leader's copy counts both CTAs' expander warps
+  uint64_t* aempty = afull + kQASlots;
+  uint64_t* accfull = aempty + kQASlots;
+  uint64_t* accempty = accfull + 2;   // leader's copy counts both CTAs' epilogue threads
+  uint64_t* drain = accempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* sR = reinterpret_cast<int*>(smem + kQEpiOffset);   // [2][BN]
+  float* sF = reinterpret_cast<float*>(sR + 2 * kQBN);    // [2][BN]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nk = (K + kQBK - 1) / kQBK;
+  const int mt = (M + kQBN - 1) / kQBN;
+  const int ntiles = mt * ((N + kQRows - 1) / kQRows);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int t = 0; t < kQASlots; ++t) {
+      mbar_init(&afull[t], 8);   // one arrival per expander warp of each CTA
+      mbar_init(&aempty[t], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 256);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kQTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmW);
+      uint32_t g = 0;
+      bool stop = false;
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+        const int m0 = (tile % mt) * kQBN + static_cast<int>(rank) * kQHalf;
+        const int n0 = (tile / mt) * kQRows + static_cast<int>(rank) * kTcRows;
+        for (int ks = 0; ks < nk; ++ks, ++g) {
+          const int s = g % S;
+          if (g >= static_cast<uint32_t>(S) &&
+              !mbar_wait_cluster(&empty[s], ((g / S) & 1) ^ 1u, abort_flag, limit_ns, kSiteProdEmpty)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kQStageBytes);
+#pragma unroll
+          for (int bx = 0; bx < kQBK / 128; ++bx)
+            tma_load_2d(sX + s * kQXStageBytes + bx * kQXBoxBytes, &tmX, ks * kQBK + bx * 128, m0, &full[s]);
+          tma_load_2d(sW + s * kQWStageBytes, &tmW, ks * (kQBK / 4), n0, &full[s]);
+        }
+      }
+      const uint32_t issued = g;
+      for (uint32_t s = 0; s < static_cast<uint32_t>(S) && s < issued; ++s) {
+        const uint32_t last = s + S * ((issued - 1 - s) / S);
+        mbar_wait(&full[s], (last / S) & 1, nullptr, limit_ns, kSiteDrain);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader only) ----------------
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_i8(kQRows, kQBN);
+      uint32_t g = 0;
+      int i = 0;
+      bool stop = false;
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs, ++i) {
+        const int b = i & 1;
+        if (i >= 2 && !mbar_wait_cluster(&accempty[b], ((i >> 1) & 1) ^ 1u, abort_flag, limit_ns, kSiteAcc)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + b * kQAccCols;
+        for (int ks = 0; ks < nk; ++ks, ++g) {
+          const int s = g % S;
+          const int t = g % kQASlots;
+          if (!mbar_wait_cluster(&afull[t], (g / kQASlots) & 1, abort_flag, limit_ns, kSiteMmaExfull)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xs = smem_u32(sX + s * kQXStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < kQBK / 32; ++kk) {
+            const uint32_t a_tmem = tmem + kQACol + kQASlotCols * t + 8 * kk;
+            const uint32_t b_addr = xs + (kk >> 2) * kQXBoxBytes + 32 * (kk & 3);
+            mma_i8_ts_pair(d_tmem, a_tmem, smem_desc_k_sw128(b_addr), idesc, (ks | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[s], 3);
+          tc_commit_pair(&aempty[t], 3);
+        }
+        if (stop) break;
+        tc_commit_pair(&accfull[b], 3);
+      }
+      // no MMA of the pair may be in flight when either CTA frees its TMEM
+      tc_commit_pair(drain, 1);
+      mbar_wait(drain, 0, nullptr, limit_ns, kSiteDrain);
+    }
+  } else if (warp < 6) {
+    // ---------------- expanders (both CTAs) ----------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t wsw = static_cast<uint32_t>((r >> 1) & 3);   // 64-byte swizzle of the packed box
+    uint32_t g = 0;
+    bool stop = false;
+    for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+      for (int ks = 0; ks < nk; ++ks, ++g) {
+        const int s = g % S;
+        const int t = g % kQASlots;
+        bool ok = mbar_wait(&full[s], (g / S) & 1, abort_flag, limit_ns, kSiteExpFull);
+        if (ok && g >= static_cast<uint32_t>(kQASlots))
+          ok = mbar_wait_cluster(&aempty[t], ((g / kQASlots) & 1) ^ 1u, abort_flag, limit_ns, kSiteExpEmpty);
+        if (!__all_sync(0xffffffffu, ok)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        // row r of the stage: 64 packed bytes = four 16-byte chunks, chunk c
+        // stored at chunk position c ^ ((r >> 1) & 3) (64-byte swizzle)
+        const uint32_t wrow = smem_u32(sW + s * kQWStageBytes) + r * 64;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 lo = ld_shared_v4(wrow + (((2u * h) ^ wsw) << 4));
+          const uint4 hi = ld_shared_v4(wrow + (((2u * h + 1u) ^ wsw) << 4));
+          const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          uint32_t v[32];
+#pragma unroll
+          for (int gw = 0; gw < 8; ++gw)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[4 * gw + j] = (wd[gw] >> (2 * j)) & 0x03030303u;
+          tmem_st_32x32b_x32(tmem + lane_base + kQACol + kQASlotCols * t + 32 * h, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(&afull[t], 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue (both CTAs) ----------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int et = threadIdx.x - 192;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const float gamma = (out_mode == kOutI32) ? 1.f : *gamma_p;
+    int i = 0;
+    for (int tile = pair; tile < ntiles; tile += npairs, ++i) {
+      const int b = i & 1;
+      const int m0 = (tile % mt) * kQBN;
+      const int n0 = (tile / mt) * kQRows + static_cast<int>(rank) * kTcRows;
+      for (int j = et; j < kQBN; j += 128) {
+        const int m = m0 + j;
+        int rv = 0;
+        float fv = 0.f;
+        if (m < M) {
+          rv = Rg[m];
+          if (out_mode != kOutI32) fv = __fdiv_rn(gamma, sg[m]);
+        }
+        sR[b * kQBN + j] = rv;
+        sF[b * kQBN + j] = fv;
+      }
+      __syncwarp();
+      named_bar_sync(2, 128);
+      const bool ok = mbar_wait_cluster(&accfull[b], (i >> 1) & 1, abort_flag, limit_ns, kSiteAcc) && !*abort_flag;
+      __syncwarp();
+      if (!named_bar_and(3, 128, ok)) break;
+      tc_fence_after();
+      const int n = n0 + r;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kQBN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + b * kQAccCols + c0, v);
+        tmem_wait_ld();
+        if (n < N) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const int m = m0 + c0 + t;
+            if (m < M) {
+              const int a = static_cast<int>(v[t]) - sR[b * kQBN + c0 + t];
+              const size_t o = static_cast<size_t>(m) * N + n;
+              if (out_mode == kOutI32) {
+                static_cast<int*>(Y)[o] = a;
+              } else {
+                const float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
+                if (out_mode == kOutF32)
+                  static_cast<float*>(Y)[o] = y;
+                else
+                  static_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(y);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(&accempty[b], 0);
+      __syncwarp();
+      named_bar_sync(2, 128);
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();   // the leader has drained its MMAs; both CTAs may free TMEM
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kQTmemCols);
+  }
+}
+
+}  // namespace bl
