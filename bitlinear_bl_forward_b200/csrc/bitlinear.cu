@@ -299,6 +299,23 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
   if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kQBK / 4,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return BL_ERR_CUDA;
+  // bf16 outputs leave through TMA stores when the rows are 16-byte aligned
+  CUtensorMap tmY;
+  std::memset(&tmY, 0, sizeof(tmY));
+  int tma_store = 0;
+  if (out_mode == bl::kOutBF16 && (N % 8) == 0 && (reinterpret_cast<uintptr_t>(Y) & 15u) == 0) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return BL_ERR_CUDA;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(bl::kQBN)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return BL_ERR_CUDA;
+    tma_store = 1;
+  }
   const int ntiles = ((M + bl::kQBN - 1) / bl::kQBN) * ((N + bl::kQRows - 1) / bl::kQRows);
   cudaLaunchConfig_t cfg = {};
   // a persistent grid must fit in one wave: not every SM can host half of a
@@ -318,8 +335,8 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const unsigned long long lim = kWaitLimitNs;
-  if (cudaLaunchKernelEx(&cfg, bl::tc_gemm_pair_kernel, tmX, tmW, M, N, K, R, s, gamma, Y, out_mode, lim) !=
-      cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, bl::tc_gemm_pair_kernel, tmX, tmW, tmY, M, N, K, R, s, gamma, Y, out_mode, tma_store,
+                         lim) != cudaSuccess)
     return BL_ERR_CUDA;
   return last_cuda();
 }

@@ -44,31 +44,36 @@ constexpr int kQXBoxBytes = kQHalf * 128;       // one 128-byte-wide activation 
 constexpr int kQXStageBytes = kQHalf * kQBK;    // 16 KB: kQBK / 128 boxes
 constexpr int kQWStageBytes = kTcRows * kQBK / 4;   // 8 KB packed, 64-byte rows (SW64)
 constexpr int kQStageBytes = kQXStageBytes + kQWStageBytes;
-constexpr int kQStages = 8;                     // 192 KB
+constexpr int kQStages = 7;                     // 168 KB
+constexpr int kQStageOutBytes = kQBN * 32 * 2;  // bf16 [BN tokens][32 rows] per epilogue warp
 constexpr int kQAccCols = kQBN;
 constexpr int kQACol = 2 * kQAccCols;
 constexpr int kQTmemCols = 512;
-constexpr int kQBarOffset = kQStages * kQStageBytes;
-constexpr int kQNumBars = 2 * kQStages + 2 * kQASlots + 5;
+constexpr int kQOutOffset = kQStages * kQStageBytes;
+constexpr int kQBarOffset = kQOutOffset + 4 * kQStageOutBytes;
+// barriers: full[S], done[S] (stage consumed by the MMAs: frees its shared
+// memory and, kQASlots stages later, its TMEM A slot), afull[4], accfull[2],
+// accempty[2], drain
+constexpr int kQNumBars = 2 * kQStages + kQASlots + 5;
 constexpr int kQEpiOffset = kQBarOffset + kQNumBars * 8 + 16;
 constexpr int kQSmemBytes = kQEpiOffset + 2 * kQBN * 8 + 1024;
 
 __global__ void __launch_bounds__(kQThreads, 1)
-    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int M, int N,
-                        int K, const int* __restrict__ Rg, const float* __restrict__ sg,
-                        const float* __restrict__ gamma_p, void* __restrict__ Y, int out_mode,
-                        unsigned long long limit_ns) {
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const int* __restrict__ Rg,
+                        const float* __restrict__ sg, const float* __restrict__ gamma_p, void* __restrict__ Y,
+                        int out_mode, int tma_store, unsigned long long limit_ns) {
   constexpr int S = kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem;
   uint8_t* sW = smem + S * kQXStageBytes;
   static_assert(kQBK % 128 == 0 && kQASlotCols == 64, "stage layout below assumes K = 256 per stage");
+  uint8_t* sOut = smem + kQOutOffset;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQBarOffset);
-  uint64_t* empty = full + S;
-  uint64_t* afull = empty + S;        // leader's copy counts both CTAs' expander warps
-  uint64_t* aempty = afull + kQASlots;
-  uint64_t* accfull = aempty + kQASlots;
+  uint64_t* done = full + S;
+  uint64_t* afull = done + S;         // leader's copy counts both CTAs' expander warps
+  uint64_t* accfull = afull + kQASlots;
   uint64_t* accempty = accfull + 2;   // leader's copy counts both CTAs' epilogue threads
   uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -86,12 +91,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&done[s], 1);
     }
-    for (int t = 0; t < kQASlots; ++t) {
-      mbar_init(&afull[t], 8);   // one arrival per expander warp of each CTA
-      mbar_init(&aempty[t], 1);
-    }
+    for (int t = 0; t < kQASlots; ++t) mbar_init(&afull[t], 8);   // one arrival per expander warp of each CTA
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 256);
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         for (int ks = 0; ks < nk; ++ks, ++g) {
           const int s = g % S;
           if (g >= static_cast<uint32_t>(S) &&
-              !mbar_wait_cluster(&empty[s], ((g / S) & 1) ^ 1u, abort_flag, limit_ns, kSiteProdEmpty)) {
+              !mbar_wait_cluster(&done[s], ((g / S) & 1) ^ 1u, abort_flag, limit_ns, kSiteProdEmpty)) {
             stop = true;
             break;
           }
@@ -166,8 +168,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
             const uint32_t b_addr = xs + (kk >> 2) * kQXBoxBytes + 32 * (kk & 3);
             mma_i8_ts_pair(d_tmem, a_tmem, smem_desc_k_sw128(b_addr), idesc, (ks | kk) != 0 ? 1u : 0u);
           }
-          tc_commit_pair(&empty[s], 3);
-          tc_commit_pair(&aempty[t], 3);
+          tc_commit_pair(&done[s], 3);
         }
         if (stop) break;
         tc_commit_pair(&accfull[b], 3);
@@ -189,8 +190,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int s = g % S;
         const int t = g % kQASlots;
         bool ok = mbar_wait(&full[s], (g / S) & 1, abort_flag, limit_ns, kSiteExpFull);
-        if (ok && g >= static_cast<uint32_t>(kQASlots))
-          ok = mbar_wait_cluster(&aempty[t], ((g / kQASlots) & 1) ^ 1u, abort_flag, limit_ns, kSiteExpEmpty);
+        if (ok && g >= static_cast<uint32_t>(kQASlots)) {
+          // slot t was last used by stage g - kQASlots: free once that stage is done
+          const uint32_t gp = g - kQASlots;
+          ok = mbar_wait_cluster(&done[gp % S], (gp / S) & 1, abort_flag, limit_ns, kSiteExpEmpty);
+        }
         if (!__all_sync(0xffffffffu, ok)) {
           stop = true;
           break;
@@ -247,6 +251,35 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!named_bar_and(3, 128, ok)) break;
       tc_fence_after();
       const int n = n0 + r;
+      if (tma_store) {
+        // bf16 tile of this warp, [BN tokens][32 rows], then one TMA store
+        uint16_t* so = reinterpret_cast<uint16_t*>(sOut + q * kQStageOutBytes);
+        if (lane == 0) bulk_wait_group_read0();   // the previous store has read the buffer
+        __syncwarp();
+#pragma unroll 1
+        for (int c0 = 0; c0 < kQBN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + b * kQAccCols + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const int a = static_cast<int>(v[t]) - sR[b * kQBN + c0 + t];
+            const float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
+            so[(c0 + t) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(&accempty[b], 0);   // accumulator drained: the MMAs may reuse it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, n0 + q * 32, m0, so);
+          bulk_commit_group();
+        }
+        __syncwarp();
+        named_bar_sync(2, 128);
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < kQBN; c0 += 32) {
         uint32_t v[32];
@@ -278,6 +311,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       named_bar_sync(2, 128);
     }
   }
+  if (warp >= 6 && lane == 0) bulk_wait_group0();   // outputs written before exit
   tc_fence_before();
   __syncwarp();
   cluster_sync_all();   // the leader has drained its MMAs; both CTAs may free TMEM
