@@ -250,24 +250,52 @@ class GpuWorkload:
             Wp, gamma = bl.bl_quantize_weights(Wf)
             del Wf
             copies = [(Wp, gamma)] + [(Wp.clone(), gamma.clone()) for _ in range(rotations - 1)]
-            xb = make_activation(self.w.M, L.K, self.w.x_kind, seed + 1 + 10 * i, self.w.outliers_for(L.K),
-                                 self.w.outlier_mult)
-            X = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(device)
+            if L.x_layer >= 0:          # reads the same hidden state as an earlier layer
+                src = self.layers[L.x_layer]
+                xb, X, own_x = src["xb"], src["X"], False
+            else:
+                xb = make_activation(self.w.M, L.K, self.w.x_kind, seed + 1 + 10 * i, self.w.outliers_for(L.K),
+                                     self.w.outlier_mult)
+                X, own_x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(device), True
             Y = torch.empty((self.w.M, L.N), dtype=torch.bfloat16, device=device)
             ws_n = bl.bl_forward_workspace_bytes(self.w.M, L.K, L.N, self.w.bits)
             ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=device)
-            self.layers.append(dict(L=L, copies=copies, X=X, Y=Y, ws=ws, xb=xb))
+            self.layers.append(dict(L=L, copies=copies, X=X, Y=Y, ws=ws, xb=xb, own_x=own_x))
         self.rotations = rotations
-        self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N) for d in self.layers)
+        # layers run together in one grouped call (e.g. up and gate of a feed-forward block)
+        self.groups = [list(gr) for gr in self.w.groups] or [[i] for i in range(len(self.layers))]
+        self.group_ws = []
+        for gr in self.groups:
+            if len(gr) > 1:
+                probs = [(self.layers[j]["X"], *self.layers[j]["copies"][0], self.layers[j]["L"].N) for j in gr]
+                n = bl.bl_forward_grouped_workspace_bytes(probs, self.w.bits)
+                self.group_ws.append(torch.empty(max(n, 16), dtype=torch.uint8, device=device))
+            else:
+                self.group_ws.append(None)
+        # activations shared by several layers are read (and counted) once
+        self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N)
+                                  - (0 if d["own_x"] else 2 * self.w.M * d["L"].K) for d in self.layers)
         self.ops_per_step = sum(algorithmic_ops(self.w.M, d["L"].K, d["L"].N) for d in self.layers)
-        self.launches_per_step = sum(1 if self.w.M <= 2 else 2 for _ in self.layers)
+        # decode: one launch per call (a grouped call of decode problems is one launch);
+        # otherwise activation quantisation + GEMM per layer
+        self.launches_per_step = len(self.groups) if self.w.M <= 2 else 2 * len(self.layers)
 
-    def step(self, i):
+    def run_group(self, gi, r):
         from bitlinear_bl_forward_b200 import bl
-        r = i % self.rotations
-        for d in self.layers:
+        gr = self.groups[gi]
+        if len(gr) == 1:
+            d = self.layers[gr[0]]
             Wp, gamma = d["copies"][r]
             bl.bl_forward(d["X"], Wp, gamma, d["L"].N, self.w.bits, out=d["Y"], workspace=d["ws"])
+        else:
+            ds = [self.layers[j] for j in gr]
+            bl.bl_forward_grouped([(d["X"], *d["copies"][r], d["L"].N) for d in ds], self.w.bits,
+                                  outs=[d["Y"] for d in ds], workspace=self.group_ws[gi])
+
+    def step(self, i):
+        r = i % self.rotations
+        for gi in range(len(self.groups)):
+            self.run_group(gi, r)
 
 def capture(wl, nsteps, start):
     import torch
@@ -327,18 +355,21 @@ def time_e2e(wl, steps, warmup, dist_ctx):
     outputs back to pinned host memory."""
     import torch
     from bitlinear_bl_forward_b200 import bl
-    hx = [torch.from_numpy(d["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for d in wl.layers]
+    hx = {j: torch.from_numpy(d["xb"].view(np.int16)).view(torch.bfloat16).pin_memory()
+          for j, d in enumerate(wl.layers) if d["own_x"]}
     hy = [torch.empty(tuple(d["Y"].shape), dtype=torch.bfloat16).pin_memory() for d in wl.layers]
-    h2d = sum(t.numel() * 2 for t in hx)
+    h2d = sum(t.numel() * 2 for t in hx.values())
     d2h = sum(t.numel() * 2 for t in hy)
 
     def one(i):
         r = i % wl.rotations
-        for j, d in enumerate(wl.layers):
-            d["X"].copy_(hx[j], non_blocking=True)
-            Wp, gamma = d["copies"][r]
-            bl.bl_forward(d["X"], Wp, gamma, d["L"].N, wl.w.bits, out=d["Y"], workspace=d["ws"])
-            hy[j].copy_(d["Y"], non_blocking=True)
+        for gi, gr in enumerate(wl.groups):
+            for j in gr:
+                if j in hx:
+                    wl.layers[j]["X"].copy_(hx[j], non_blocking=True)
+            wl.run_group(gi, r)
+            for j in gr:
+                hy[j].copy_(wl.layers[j]["Y"], non_blocking=True)
 
     for i in range(warmup):
         one(i)
@@ -436,7 +467,7 @@ def run_gpu(args):
         roof = roofline_entry("tensor", achieved, peak, "TFLOP/s", ncu_traffic(f"tc:{name}"))
     roof["peak_src"] = peaks["src"] + (" hbm copy" if decode else " bf16 sustained x2 (int8/bf16 nominal)")
     roof["kernel"] = "gemv2_kernel" if decode else "tc_gemm_kernel (+ act_quant_kernel in the step)"
-    roof["kernel_us_avg"] = per_rank_ms * 1e3 / (K * len(wl.layers))
+    roof["kernel_us_avg"] = per_rank_ms * 1e3 / launches
 
     # end-to-end through the public API with host buffers
     e2e_steps = min(K, 2000 if decode else 200)
@@ -449,6 +480,7 @@ def run_gpu(args):
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "i8", "data": "synthetic (seeded; weights N(0, std) generated on the GPU, activations on the host)",
         "config": {"workload": name, "M": w.M, "layers": [[L.name, L.K, L.N] for L in w.layers], "bits": w.bits,
+                   "calls_per_step": [[w.layers[j].name for j in gr] for gr in wl.groups],
                    "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
                    "l2": f"{rot} rotated weight copies ({rot * wbytes / 1e6:.0f} MB, > 126 MB L2)",
                    "timing": "CUDA graph replays, events on the launching stream"},

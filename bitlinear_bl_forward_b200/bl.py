@@ -38,6 +38,8 @@ SIGNATURES = {
     "bl_forward": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_forward_f32": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_forward_noalloc": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p]),
+    "bl_forward_grouped_workspace_bytes": (_sz, [_int, _p, _int]),
+    "bl_forward_grouped": (_int, [_int, _p, _int, _p, _sz, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
@@ -45,6 +47,12 @@ SIGNATURES = {
 }
 
 _lib = None
+
+
+class BLLinear(ctypes.Structure):
+    """Mirror of the C struct bl_linear (one problem of bl_forward_grouped)."""
+    _fields_ = [("X", ctypes.c_void_p), ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("Wp", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("Y", ctypes.c_void_p)]
 
 
 class BLError(RuntimeError):
@@ -183,6 +191,37 @@ def bl_forward_noalloc(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N
     py = _dev(Y, torch.bfloat16, "out")
     _check(lib().bl_forward_noalloc(px, M, K, N, pw, pg, bits, py, _stream()), "bl_forward_noalloc")
     return Y
+
+
+def _grouped_structs(problems, outs):
+    arr = (BLLinear * max(1, len(problems)))()
+    for i, ((X, Wp, gamma, N), Y) in enumerate(zip(problems, outs)):
+        M, K = X.shape
+        arr[i] = BLLinear(_dev(X, torch.bfloat16, "X"), M, K, N, _dev(Wp, torch.uint8, "Wp"),
+                          _dev(gamma, torch.float32, "gamma"), _dev(Y, torch.bfloat16, "out"))
+    return arr
+
+
+def bl_forward_grouped_workspace_bytes(problems, bits: int = 8) -> int:
+    """problems: list of (X, Wp, gamma, N)."""
+    outs = [torch.empty((X.shape[0], N), dtype=torch.bfloat16, device=X.device) for (X, _, _, N) in problems]
+    arr = _grouped_structs(problems, outs)
+    return int(lib().bl_forward_grouped_workspace_bytes(len(problems), arr, bits))
+
+
+def bl_forward_grouped(problems, bits: int = 8, outs=None, workspace: torch.Tensor | None = None):
+    """Several independent BitLinear forwards in one call (problems: list of
+    (X bf16 [M, K], Wp, gamma, N)); returns the list of bf16 outputs."""
+    if outs is None:
+        outs = [torch.empty((X.shape[0], N), dtype=torch.bfloat16, device=X.device) for (X, _, _, N) in problems]
+    arr = _grouped_structs(problems, outs)
+    ws = workspace
+    if ws is None:
+        need = int(lib().bl_forward_grouped_workspace_bytes(len(problems), arr, bits))
+        ws = _workspace(need, problems[0][0].device if problems else "cuda")
+    _check(lib().bl_forward_grouped(len(problems), arr, bits, ws.data_ptr() if ws is not None else None,
+                                    ws.numel() if ws is not None else 0, _stream()), "bl_forward_grouped")
+    return outs
 
 
 def bl_matmul_i32(Xq: torch.Tensor, Wp: torch.Tensor, N: int) -> torch.Tensor:

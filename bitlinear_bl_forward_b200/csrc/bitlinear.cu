@@ -158,15 +158,11 @@ bl_status launch_gemv1_t(const void* X, int x_is_i8, int K, int N, const uint8_t
 }
 
 template <int MT, int CPL>
-bl_status launch_gemv2_t(const void* X, int x_is_i8, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
-                         void* Y, int out_mode, cudaStream_t stream) {
+bl_status launch_gemv2_table(const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode, cudaStream_t stream) {
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(bl::gemv2_kernel<MT, CPL>, bl::kG2SmemBytes, &done)) return BL_ERR_CUDA;
-  const int sms = num_sms();
-  const int rows_per_cta = (N + sms - 1) / sms;
-  const int blocks = (N + rows_per_cta - 1) / rows_per_cta;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(blocks);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(bl::kG2Threads);
   cfg.dynamicSmemBytes = bl::kG2SmemBytes;
   cfg.stream = stream;
@@ -176,10 +172,32 @@ bl_status launch_gemv2_t(const void* X, int x_is_i8, int K, int N, const uint8_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const unsigned long long lim = kWaitLimitNs;
-  if (cudaLaunchKernelEx(&cfg, bl::gemv2_kernel<MT, CPL>, X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, rows_per_cta,
-                         lim) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, bl::gemv2_kernel<MT, CPL>, tab, x_is_i8, Q, out_mode, lim) != cudaSuccess)
     return BL_ERR_CUDA;
   return last_cuda();
+}
+
+bl_status launch_gemv2_cpl(int cpl, const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode,
+                           cudaStream_t stream) {
+  switch (cpl) {
+    case 1: return launch_gemv2_table<1, 1>(tab, grid, x_is_i8, Q, out_mode, stream);
+    case 2: return launch_gemv2_table<1, 2>(tab, grid, x_is_i8, Q, out_mode, stream);
+    case 3: return launch_gemv2_table<1, 3>(tab, grid, x_is_i8, Q, out_mode, stream);
+    default: return launch_gemv2_table<1, 4>(tab, grid, x_is_i8, Q, out_mode, stream);
+  }
+}
+
+// Single one-token problem: rows split evenly over one CTA per SM.
+bl_status launch_gemv2_one(const void* X, int x_is_i8, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
+                           void* Y, int out_mode, cudaStream_t stream) {
+  bl::G2Table tab;
+  std::memset(&tab, 0, sizeof(tab));
+  const int sms = num_sms();
+  const int rows_per_cta = (N + sms - 1) / sms;
+  tab.count = 1;
+  tab.p[0] = bl::G2Problem{X, Wp, gamma, Y, K, N, rows_per_cta, 0};
+  const int grid = (N + rows_per_cta - 1) / rows_per_cta;
+  return launch_gemv2_cpl((K / 64 + 31) / 32, tab, grid, x_is_i8, Q, out_mode, stream);
 }
 
 // Decode kernel selection (build-time, for experiments): 0 = by shape,
@@ -195,14 +213,8 @@ bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uin
   // one token: the TMA-staged kernel (measured at least as fast on every
   // decode shape); two tokens: the register-ring kernel
   const bool staged = (kDecodeKernel == 2) || (kDecodeKernel == 0 && M == 1);
-  if (staged && M == 1 && K <= 8192) {
-    switch (cplx) {
-      case 1: return launch_gemv2_t<1, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-      case 2: return launch_gemv2_t<1, 2>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-      case 3: return launch_gemv2_t<1, 3>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-      default: return launch_gemv2_t<1, 4>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-    }
-  }
+  (void)cplx;
+  if (staged && M == 1 && K <= 8192) return launch_gemv2_one(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
   const int cpl = (K / 64 + 31) / 32;
   // one CTA of 16 warps per SM (room for the next kernel's CTA to start its
   // L2 prefetch alongside); D tiles of weights in flight per warp
@@ -603,6 +615,80 @@ bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N,
   bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
   if ((st = last_cuda()) != BL_OK) return st;
   return launch_tc(Xq, m, k, n, Wp, R, s, gamma, Y, bl::kOutBF16, 0, stream);
+}
+
+size_t bl_forward_grouped_workspace_bytes(int count, const bl_linear* problems, int bits) {
+  (void)bits;
+  if (count <= 0 || count > bl::kG2MaxProblems || problems == nullptr) return 0;
+  size_t need = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    if (check_shape_nk(p.N, p.K) != BL_OK || check_m(p.M, p.K) != BL_OK) return 0;
+    const size_t w = fwd_ws_bytes(p.M, p.K);
+    if (w > need) need = w;
+  }
+  return need;
+}
+
+bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+  if (problems == nullptr) return BL_ERR_INVALID_ARG;
+  if (count < 0 || count > bl::kG2MaxProblems) return BL_ERR_UNSUPPORTED;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  // validate everything before launching anything
+  bool all_decode = true;
+  int cpl = 1;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    bl_status st = check_shape_nk(p.N, p.K);
+    if (st != BL_OK) return st;
+    if ((st = check_m(p.M, p.K)) != BL_OK) return st;
+    if (p.M == 0) continue;
+    if (!p.X || !p.Wp || !p.gamma || !p.Y) return BL_ERR_INVALID_ARG;
+    if (!aligned16(p.X) || !aligned16(p.Wp)) return BL_ERR_ALIGNMENT;
+    const size_t need = fwd_ws_bytes(p.M, p.K);
+    if (need > 0) {
+      if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+      if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+    }
+    if (p.M != 1 || p.K > 8192) all_decode = false;
+    const int c = static_cast<int>((p.K / 64 + 31) / 32);
+    if (c > cpl) cpl = c;
+  }
+  const int Q = bits == 8 ? 127 : 7;
+  if (all_decode && kDecodeKernel != 1) {
+    // one launch: CTAs shared out in proportion to each problem's weight bytes
+    bl::G2Table tab;
+    std::memset(&tab, 0, sizeof(tab));
+    const int sms = num_sms();
+    double total = 0.0;
+    for (int i = 0; i < count; ++i)
+      if (problems[i].M > 0) total += static_cast<double>(problems[i].N) * static_cast<double>(problems[i].K);
+    int grid = 0;
+    for (int i = 0; i < count; ++i) {
+      const bl_linear& p = problems[i];
+      if (p.M == 0) continue;
+      int c = static_cast<int>(sms * (static_cast<double>(p.N) * static_cast<double>(p.K)) / total);
+      if (c < 1) c = 1;
+      const int rows_per_cta = static_cast<int>((p.N + c - 1) / c);
+      c = static_cast<int>((p.N + rows_per_cta - 1) / rows_per_cta);
+      tab.p[tab.count] = bl::G2Problem{p.X, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
+                                       rows_per_cta, grid};
+      tab.count += 1;
+      grid += c;
+    }
+    if (tab.count == 0) return BL_OK;
+    return launch_gemv2_cpl(cpl, tab, grid, 0, Q, bl::kOutBF16, stream);
+  }
+  // otherwise the problems run one after another on the stream (the
+  // workspace is reused: stream order serialises them)
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    const bl_status st =
+        forward_common(p.X, p.M, p.K, p.N, p.Wp, p.gamma, bits, p.Y, bl::kOutBF16, workspace, workspace_bytes, stream);
+    if (st != BL_OK) return st;
+  }
+  return BL_OK;
 }
 
 bl_status bl_device_status(int clear, int* site) {

@@ -33,7 +33,11 @@
 
 namespace bl {
 
-constexpr int kQThreads = 320;
+// warps: 0 producer, 1 MMA issuer, 2..(2+4*kQExpGroups-1) expanders (group e
+// expands the stages g with g % kQExpGroups == e), then 4 epilogue warps
+constexpr int kQExpGroups = 1;   // measured: a second group does not help
+constexpr int kQFirstEpi = 2 + 4 * kQExpGroups;
+constexpr int kQThreads = 32 * (kQFirstEpi + 4);
 constexpr int kQBK = 256;                       // K per pipeline stage: 8 MMAs per hand-off
 constexpr int kQASlots = 4;                     // TMEM: 2 x 128 accumulator + 4 x 64 A columns = 512
 constexpr int kQASlotCols = kQBK / 4;           // int8 codes, 4 per 32-bit column
@@ -177,8 +181,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       tc_commit_pair(drain, 1);
       mbar_wait(drain, 0, nullptr, limit_ns, kSiteDrain);
     }
-  } else if (warp < 6) {
+  } else if (warp < kQFirstEpi) {
     // ---------------- expanders (both CTAs) ----------------
+    const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
@@ -187,6 +192,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     bool stop = false;
     for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
       for (int ks = 0; ks < nk; ++ks, ++g) {
+        if (static_cast<int>(g % kQExpGroups) != grp) continue;
         const int s = g % S;
         const int t = g % kQASlots;
         bool ok = mbar_wait(&full[s], (g / S) & 1, abort_flag, limit_ns, kSiteExpFull);
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     // ---------------- epilogue (both CTAs) ----------------
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    const int et = threadIdx.x - 192;
+    const int et = threadIdx.x - 32 * kQFirstEpi;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float gamma = (out_mode == kOutI32) ? 1.f : *gamma_p;
     int i = 0;
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       named_bar_sync(2, 128);
     }
   }
-  if (warp >= 6 && lane == 0) bulk_wait_group0();   // outputs written before exit
+  if (warp >= kQFirstEpi && lane == 0) bulk_wait_group0();   // outputs written before exit
   tc_fence_before();
   __syncwarp();
   cluster_sync_all();   // the leader has drained its MMAs; both CTAs may free TMEM

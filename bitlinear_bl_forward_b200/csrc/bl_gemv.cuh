@@ -495,6 +495,24 @@ __global__ void __launch_bounds__(THREADS, MINB)
 // bounded; on a timeout the kernel records BL_ERR_TIMEOUT and unwinds, and
 // the producer waits for the copies it issued before the CTA exits.
 // ---------------------------------------------------------------------------
+// One launch can serve several independent one-token problems (grouped
+// decode): CTAs [cta_begin, next cta_begin) of the grid work on problem i.
+struct G2Problem {
+  const void* X;
+  const uint8_t* Wp;
+  const float* gamma;
+  void* Y;
+  int K;
+  int N;
+  int rows_per_cta;
+  int cta_begin;
+};
+constexpr int kG2MaxProblems = 8;
+struct G2Table {
+  G2Problem p[kG2MaxProblems];
+  int count;
+};
+
 constexpr int kG2ConsumerWarps = 16;
 constexpr int kG2Threads = (kG2ConsumerWarps + 1) * 32;
 constexpr int kG2Stages = 6;
@@ -503,9 +521,15 @@ constexpr int kG2SmemBytes = kG2Stages * kG2StageBytes + 2048;
 
 template <int MT, int CPL>
 __global__ void __launch_bounds__(kG2Threads, 1)
-    gemv2_kernel(const void* __restrict__ X, int x_is_i8, int K, int N, const uint8_t* __restrict__ Wp,
-                 const float* __restrict__ gamma_p, int Q, void* __restrict__ Y, int out_mode, int rows_per_cta,
-                 unsigned long long limit_ns) {
+    gemv2_kernel(const __grid_constant__ G2Table tab, int x_is_i8, int Q, int out_mode, unsigned long long limit_ns) {
+  int pi = 0;
+  while (pi + 1 < tab.count && static_cast<int>(blockIdx.x) >= tab.p[pi + 1].cta_begin) ++pi;
+  const void* __restrict__ X = tab.p[pi].X;
+  const uint8_t* __restrict__ Wp = tab.p[pi].Wp;
+  const float* __restrict__ gamma_p = tab.p[pi].gamma;
+  void* __restrict__ Y = tab.p[pi].Y;
+  const int K = tab.p[pi].K, N = tab.p[pi].N, rows_per_cta = tab.p[pi].rows_per_cta;
+  const int cta = static_cast<int>(blockIdx.x) - tab.p[pi].cta_begin;
   extern __shared__ __align__(128) uint8_t g2_smem[];
   __shared__ __align__(16) uint8_t s_act[MT][8192];
   __shared__ __align__(16) uint32_t s_red_f[MT][kG2ConsumerWarps];
@@ -516,7 +540,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KV = K >> 6;
   const size_t row_bytes = static_cast<size_t>(K) >> 2;
-  const int r0 = blockIdx.x * rows_per_cta;
+  const int r0 = cta * rows_per_cta;
   const int r1 = min(N, r0 + rows_per_cta);
   const int stage_rows = kG2StageBytes / static_cast<int>(row_bytes);
   const int nst = (r1 > r0) ? (r1 - r0 + stage_rows - 1) / stage_rows : 0;

@@ -9,7 +9,8 @@ Recipe (per workload; ``seed`` defaults to 0):
   * weights:  W fp32 [N, K] = std * N(0, 1), generator seed = seed + 10*i for
     the i-th layer of the workload;
   * activations: X [M, K] drawn in fp32 from N(0, 1) with generator seed
-    seed + 1 + 10*i, then
+    seed + 1 + 10*i (i = the layer whose input it is: up and gate of a
+    feed-forward block share one), then
       - "outliers": n_out channels (columns) chosen by randperm(K) with seed
         seed + 2 + 10*i are multiplied by ``mult`` for every token,
       - "relu2":    X = max(0, z)^2 elementwise,
@@ -31,6 +32,7 @@ class Layer:
     name: str
     K: int          # in-features
     N: int          # out-features
+    x_layer: int = -1   # >= 0: this layer reads the activations of that layer (same hidden state)
 
 
 @dataclass(frozen=True)
@@ -44,6 +46,7 @@ class Workload:
     outlier_mult: float = 1.0
     bits: int = 8
     note: str = ""
+    groups: tuple = ()          # layers a step runs in one grouped call, e.g. ((0, 1), (2,))
 
     def outliers_for(self, K: int) -> int:
         if isinstance(self.n_outliers, str) and self.n_outliers.endswith("%"):
@@ -56,9 +59,10 @@ class Workload:
 WORKLOADS = {
     "tiny": Workload("tiny", 16, (Layer("proj", 256, 512),), 0.02, "outliers", 2, 20.0, 8,
                      "tiny BitLinear 16x256 -> 512"),
+    # up and gate project the same hidden state; down reads its own input
     "decode_2b": Workload("decode_2b", 1,
-                          (Layer("up", 2560, 6912), Layer("gate", 2560, 6912), Layer("down", 6912, 2560)),
-                          0.02, "outliers", "1%", 10.0, 8, "2B-class decode GEMV, batch 1"),
+                          (Layer("up", 2560, 6912), Layer("gate", 2560, 6912, x_layer=0), Layer("down", 6912, 2560)),
+                          0.02, "outliers", "1%", 10.0, 8, "2B-class decode GEMV, batch 1", ((0, 1), (2,))),
     "prefill_2b": Workload("prefill_2b", 4096,
                            (Layer("up", 2560, 6912), Layer("down", 6912, 2560)),
                            0.02, "outliers", "1%", 10.0, 8, "2B-class prefill GEMM, 4096 tokens"),
@@ -100,7 +104,8 @@ def layer_inputs(w: Workload, i: int, seed: int = 0, M: int | None = None):
     L = w.layers[i]
     M = w.M if M is None else M
     W = make_weight(L.N, L.K, w.w_std, seed + 10 * i)
-    X = make_activation(M, L.K, w.x_kind, seed + 1 + 10 * i, w.outliers_for(L.K), w.outlier_mult)
+    xi = i if L.x_layer < 0 else L.x_layer
+    X = make_activation(M, L.K, w.x_kind, seed + 1 + 10 * xi, w.outliers_for(L.K), w.outlier_mult)
     return X, W
 
 

@@ -171,6 +171,32 @@ BL_API bl_status bl_forward_f32(const uint16_t* X, int64_t M, int64_t K, int64_t
 BL_API bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
                                     const float* gamma, int bits, uint16_t* Y, cudaStream_t stream);
 
+/*
+ * Grouped forward: up to 8 independent BitLinear problems in one call, e.g.
+ * the up and gate projections of a feed-forward block (same X, two weight
+ * tensors) or several requests' layers.  Each problem is exactly one
+ * bl_forward (same formulas, same rounding, bit-identical results).  When
+ * every problem has M == 1 and K <= 8192 they share one decode kernel launch
+ * (its CTAs are shared out in proportion to each problem's weight bytes), so
+ * the fixed cost of a launch and of the token-quantisation prologue is paid
+ * once; otherwise the problems run one after another on the stream.
+ * workspace: >= bl_forward_grouped_workspace_bytes(count, problems, bits)
+ * (the largest per-problem bl_forward workspace; 0 for an all-decode group).
+ * count > 8 returns BL_ERR_UNSUPPORTED; problems with M == 0 are skipped.
+ * All problems are validated before anything is launched.
+ */
+typedef struct {
+  const uint16_t* X; /* bf16 bits [M, K], 16-byte aligned */
+  int64_t M, K, N;
+  const uint8_t* Wp;  /* packed weights [N, K/4], 16-byte aligned */
+  const float* gamma; /* device fp32 */
+  uint16_t* Y;        /* bf16 bits [M, N] */
+} bl_linear;
+
+BL_API size_t bl_forward_grouped_workspace_bytes(int count, const bl_linear* problems, int bits);
+BL_API bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream);
+
 /* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
 BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
 

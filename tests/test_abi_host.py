@@ -132,3 +132,22 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         bl.lib()
+
+
+def test_grouped_validation(L):
+    arr = (bl.BLLinear * 9)()
+    for i in range(9):
+        arr[i] = bl.BLLinear(A, 1, 64, 8, A, A, A)
+    assert L.bl_forward_grouped(9, arr, 8, None, 0, None) == UNSUP          # more than 8 problems
+    assert L.bl_forward_grouped(2, None, 8, None, 0, None) == INVALID
+    assert L.bl_forward_grouped(2, arr, 3, None, 0, None) == UNSUP
+    arr[1] = bl.BLLinear(A, 1, 60, 8, A, A, A)                              # K % 64
+    assert L.bl_forward_grouped(2, arr, 8, None, 0, None) == SHAPE
+    arr[1] = bl.BLLinear(A, 1, 64, 8, None, A, A)
+    assert L.bl_forward_grouped(2, arr, 8, None, 0, None) == INVALID
+    arr[1] = bl.BLLinear(U, 1, 64, 8, A, A, A)
+    assert L.bl_forward_grouped(2, arr, 8, None, 0, None) == ALIGN
+    arr[1] = bl.BLLinear(A, 4, 64, 8, A, A, A)                              # M > 2 needs a workspace
+    assert L.bl_forward_grouped(2, arr, 8, None, 0, None) == WS
+    assert L.bl_forward_grouped_workspace_bytes(2, arr, 8) >= 4 * 64
+    assert L.bl_forward_grouped(0, arr, 8, None, 0, None) == OK

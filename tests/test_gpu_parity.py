@@ -245,3 +245,48 @@ def test_workload_70b_m2048_sampled():
 
 def test_workload_a48():
     run_workload("a48")
+
+
+# ---------------------------------------------------------------------------
+# grouped forward
+# ---------------------------------------------------------------------------
+
+def test_grouped_decode_matches_single_calls_and_oracle():
+    # up and gate of the 2B decode layer share X: one grouped launch
+    w = WORKLOADS["decode_2b"]
+    X, _ = layer_inputs(w, 0)
+    Xd = x_to_dev(X)
+    probs, refs = [], []
+    for i in (0, 1):
+        W, g, c, p = oracle_weights(("decode_2b", i))
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        N = W.shape[0]
+        probs.append((Xd, Wp, gd, N))
+        refs.append(bl.bl_forward(Xd, Wp, gd, N))
+        q, s = o.act_quant(X, 8)
+        Y = o.round_to_bf16_bits(o.rescale(o.matmul_i32(q, c), g, s)[1])
+        refs[-1] = (refs[-1], Y)
+    outs = bl.bl_forward_grouped(probs)
+    torch.cuda.synchronize()
+    for Yg, (Ys, Yo) in zip(outs, refs):
+        assert torch.equal(Yg, Ys)
+        assert bf16_ulp_distance(bf16_dev_to_bits(Yg), Yo).max() <= BF16_ULP_TOL
+
+
+def test_grouped_mixed_shapes_fall_back_to_sequential():
+    cases = [(1, 256, 300), (3, 512, 129), (1, 4096, 64), (2, 192, 100), (0, 64, 8)]
+    probs, singles = [], []
+    for j, (M, K, N) in enumerate(cases):
+        X, W = random_case(M, K, N, seed=100 + j)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        Xd = x_to_dev(X) if M > 0 else torch.zeros((0, K), dtype=torch.bfloat16, device="cuda")
+        probs.append((Xd, Wp, gd, N))
+        singles.append(bl.bl_forward(Xd, Wp, gd, N))
+    outs = bl.bl_forward_grouped(probs)
+    torch.cuda.synchronize()
+    for a, b in zip(outs, singles):
+        assert torch.equal(a, b)
+    # all-decode group of different K (one fused launch)
+    probs2 = [probs[0], probs[2]]
+    outs2 = bl.bl_forward_grouped(probs2)
+    assert torch.equal(outs2[0], singles[0]) and torch.equal(outs2[1], singles[2])
