@@ -19,6 +19,7 @@
 #include "bl_gemm_tc2.cuh"
 #include "bl_gemm_2sm.cuh"
 #include "bl_gemv.cuh"
+#include "bl_gemv3.cuh"
 #include "bl_weights.cuh"
 
 namespace {
@@ -187,25 +188,174 @@ bl_status launch_gemv2_cpl(int cpl, const bl::G2Table& tab, int grid, int x_is_i
   }
 }
 
-// Single one-token problem: rows split evenly over one CTA per SM.
-bl_status launch_gemv2_one(const void* X, int x_is_i8, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
-                           void* Y, int out_mode, cudaStream_t stream) {
-  bl::G2Table tab;
-  std::memset(&tab, 0, sizeof(tab));
-  const int sms = num_sms();
-  const int rows_per_cta = (N + sms - 1) / sms;
-  tab.count = 1;
-  tab.p[0] = bl::G2Problem{X, Wp, gamma, Y, K, N, rows_per_cta, 0};
-  const int grid = (N + rows_per_cta - 1) / rows_per_cta;
-  return launch_gemv2_cpl((K / 64 + 31) / 32, tab, grid, x_is_i8, Q, out_mode, stream);
+#ifndef BL_G3_WARPS
+#define BL_G3_WARPS 16
+#endif
+// consumer warps of the decode kernel (16: enough warps to hide shared-memory
+// and dp4a latency, and registers for two CTAs per SM)
+template <int WPL>
+constexpr int g3_warps() { return BL_G3_WARPS; }
+
+template <int WPL>
+bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode, cudaStream_t stream) {
+  auto kern = bl::gemv3_kernel<WPL, g3_warps<WPL>()>;
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
+  if (!(done.load(std::memory_order_acquire) & (uint64_t(1) << dev))) {
+    // two CTAs per SM (this launch's and the next one's) need the largest
+    // shared-memory carve-out
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bl::kG3SmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return BL_ERR_CUDA;
+    done.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(bl::G3Cfg<WPL, g3_warps<WPL>()>::kThreads);
+  // the same footprint for every launch: a third CTA never fits on an SM,
+  // so two CTAs of one launch never share an SM
+  cfg.dynamicSmemBytes = bl::kG3SmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const unsigned long long lim = kWaitLimitNs;
+  if (cudaLaunchKernelEx(&cfg, kern, tab, x_is_i8, Q, out_mode, lim) != cudaSuccess) return BL_ERR_CUDA;
+  return last_cuda();
 }
 
-// Decode kernel selection (build-time, for experiments): 0 = by shape,
-// 1 = register-ring GEMV only, 2 = TMA-staged GEMV whenever M == 1.
+// words of 16 weights per lane: K / 512 rounded up (K <= 8192)
+bl_status launch_gemv3_wpl(int wpl, const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode,
+                           cudaStream_t stream) {
+  switch (wpl) {
+#define BL_G3_CASE(n) \
+  case n: return launch_gemv3_table<n>(tab, grid, x_is_i8, Q, out_mode, stream);
+    BL_G3_CASE(1) BL_G3_CASE(2) BL_G3_CASE(3) BL_G3_CASE(4) BL_G3_CASE(5) BL_G3_CASE(6) BL_G3_CASE(7) BL_G3_CASE(8)
+    BL_G3_CASE(9) BL_G3_CASE(10) BL_G3_CASE(11) BL_G3_CASE(12) BL_G3_CASE(13) BL_G3_CASE(14) BL_G3_CASE(15)
+    BL_G3_CASE(16)
+#undef BL_G3_CASE
+    default: return BL_ERR_UNSUPPORTED;
+  }
+}
+
+// Decode kernel selection (build-time, for experiments): 0 = by shape (one
+// token: the resident decode kernel when the layer's weights fit its ring on
+// every SM, the TMA-staged streaming GEMV otherwise), 1 = register-ring GEMV
+// only, 2 = the TMA-staged GEMV for every one-token layer.
 #ifndef BL_DECODE_KERNEL
 #define BL_DECODE_KERNEL 0
 #endif
 constexpr int kDecodeKernel = BL_DECODE_KERNEL;
+
+// Fill a launch table with one-token problems of one kernel variant: every
+// problem gets CTAs in proportion to its weight bytes (at least one, at most
+// one per row), and the launch has exactly one CTA per SM when the rows allow.
+// Returns the grid size.
+int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms) {
+  std::memset(tab, 0, sizeof(*tab));
+  double total = 0.0;
+  int64_t rows = 0;
+  for (int i = 0; i < n; ++i) {
+    total += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K);
+    rows += probs[i]->N;
+  }
+  const int target = static_cast<int>(rows < sms ? rows : sms);
+  int c[bl::kG2MaxProblems];
+  int sum = 0;
+  for (int i = 0; i < n; ++i) {
+    const double share = static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / total;
+    int v = static_cast<int>(share * target);
+    if (v < 1) v = 1;
+    if (v > probs[i]->N) v = static_cast<int>(probs[i]->N);
+    c[i] = v;
+    sum += v;
+  }
+  // hand out the remaining CTAs to the problems with the most bytes a CTA
+  while (sum < target) {
+    int best = -1;
+    double most = 0.0;
+    for (int i = 0; i < n; ++i) {
+      if (c[i] >= probs[i]->N) continue;
+      const double per = static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / c[i];
+      if (per > most) {
+        most = per;
+        best = i;
+      }
+    }
+    if (best < 0) break;
+    c[best] += 1;
+    sum += 1;
+  }
+  int grid = 0;
+  for (int i = 0; i < n; ++i) {
+    const bl_linear& p = *probs[i];
+    const int rows_per_cta = static_cast<int>((p.N + c[i] - 1) / c[i]);
+    tab->p[i] = bl::G2Problem{p.X, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
+                              rows_per_cta, grid, c[i]};
+    grid += c[i];
+  }
+  tab->count = n;
+  return grid;
+}
+
+// Launch one-token problems that share a kernel variant (at most
+// kG2MaxProblems).
+bl_status launch_decode(const bl_linear* const* probs, int n, int x_is_i8, int Q, int out_mode,
+                        cudaStream_t stream) {
+  if (n <= 0) return BL_OK;
+  const int sms = num_sms();
+  bl::G2Table tab;
+  int maxK = 64;
+  double wbytes = 0.0;
+  for (int i = 0; i < n; ++i) {
+    if (probs[i]->K > maxK) maxK = static_cast<int>(probs[i]->K);
+    wbytes += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / 4.0;
+  }
+  // layers whose weights do not fit the resident kernel's ring on every SM
+  // stream through the deeper TMA-staged GEMV instead
+  const bool streaming = wbytes > static_cast<double>(sms) * bl::kG3Stages * bl::kG3StageBytes;
+  if (kDecodeKernel == 2 || streaming) {
+    // the first TMA-staged GEMV: ceil(N / SMs) rows a CTA
+    std::memset(&tab, 0, sizeof(tab));
+    double total = 0.0;
+    for (int i = 0; i < n; ++i) total += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K);
+    int grid = 0;
+    for (int i = 0; i < n; ++i) {
+      const bl_linear& p = *probs[i];
+      int c = static_cast<int>(sms * (static_cast<double>(p.N) * static_cast<double>(p.K)) / total);
+      if (c < 1) c = 1;
+      const int rows_per_cta = static_cast<int>((p.N + c - 1) / c);
+      c = static_cast<int>((p.N + rows_per_cta - 1) / rows_per_cta);
+      tab.p[i] = bl::G2Problem{p.X, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N), rows_per_cta,
+                               grid, c};
+      grid += c;
+    }
+    tab.count = n;
+    return launch_gemv2_cpl((maxK / 64 + 31) / 32, tab, grid, x_is_i8, Q, out_mode, stream);
+  }
+  const int grid = fill_decode_table(&tab, probs, n, sms);
+  return launch_gemv3_wpl((maxK + 511) / 512, tab, grid, x_is_i8, Q, out_mode, stream);
+}
+
+// Single one-token problem.
+bl_status launch_decode_one(const void* X, int x_is_i8, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
+                            void* Y, int out_mode, cudaStream_t stream) {
+  bl_linear p;
+  p.X = static_cast<const uint16_t*>(X);
+  p.M = 1;
+  p.K = K;
+  p.N = N;
+  p.Wp = Wp;
+  p.gamma = gamma;
+  p.Y = static_cast<uint16_t*>(Y);
+  const bl_linear* pp = &p;
+  return launch_decode(&pp, 1, x_is_i8, Q, out_mode, stream);
+}
 
 bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
                       void* Y, int out_mode, cudaStream_t stream) {
@@ -214,7 +364,7 @@ bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uin
   // decode shape); two tokens: the register-ring kernel
   const bool staged = (kDecodeKernel == 2) || (kDecodeKernel == 0 && M == 1);
   (void)cplx;
-  if (staged && M == 1 && K <= 8192) return launch_gemv2_one(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+  if (staged && M == 1 && K <= 8192) return launch_decode_one(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
   const int cpl = (K / 64 + 31) / 32;
   // one CTA of 16 warps per SM (room for the next kernel's CTA to start its
   // L2 prefetch alongside); D tiles of weights in flight per warp
@@ -637,7 +787,6 @@ bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, voi
   if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
   // validate everything before launching anything
   bool all_decode = true;
-  int cpl = 1;
   for (int i = 0; i < count; ++i) {
     const bl_linear& p = problems[i];
     bl_status st = check_shape_nk(p.N, p.K);
@@ -652,33 +801,26 @@ bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, voi
       if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
     }
     if (p.M != 1 || p.K > 8192) all_decode = false;
-    const int c = static_cast<int>((p.K / 64 + 31) / 32);
-    if (c > cpl) cpl = c;
   }
   const int Q = bits == 8 ? 127 : 7;
   if (all_decode && kDecodeKernel != 1) {
-    // one launch: CTAs shared out in proportion to each problem's weight bytes
-    bl::G2Table tab;
-    std::memset(&tab, 0, sizeof(tab));
-    const int sms = num_sms();
-    double total = 0.0;
-    for (int i = 0; i < count; ++i)
-      if (problems[i].M > 0) total += static_cast<double>(problems[i].N) * static_cast<double>(problems[i].K);
-    int grid = 0;
+    // one launch per kernel variant (words of 16 weights a lane, ceil(K / 512))
+    bool used[bl::kG2MaxProblems] = {};
     for (int i = 0; i < count; ++i) {
-      const bl_linear& p = problems[i];
-      if (p.M == 0) continue;
-      int c = static_cast<int>(sms * (static_cast<double>(p.N) * static_cast<double>(p.K)) / total);
-      if (c < 1) c = 1;
-      const int rows_per_cta = static_cast<int>((p.N + c - 1) / c);
-      c = static_cast<int>((p.N + rows_per_cta - 1) / rows_per_cta);
-      tab.p[tab.count] = bl::G2Problem{p.X, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
-                                       rows_per_cta, grid};
-      tab.count += 1;
-      grid += c;
+      if (used[i] || problems[i].M == 0) continue;
+      const int64_t key = kDecodeKernel == 2 ? 0 : (problems[i].K + 511) / 512;
+      const bl_linear* sel[bl::kG2MaxProblems];
+      int n = 0;
+      for (int j = i; j < count; ++j) {
+        const bl_linear& p = problems[j];
+        if (used[j] || p.M == 0 || (kDecodeKernel != 2 && (p.K + 511) / 512 != key)) continue;
+        used[j] = true;
+        sel[n++] = &p;
+      }
+      const bl_status st = launch_decode(sel, n, 0, Q, bl::kOutBF16, stream);
+      if (st != BL_OK) return st;
     }
-    if (tab.count == 0) return BL_OK;
-    return launch_gemv2_cpl(cpl, tab, grid, 0, Q, bl::kOutBF16, stream);
+    return BL_OK;
   }
   // otherwise the problems run one after another on the stream (the
   // workspace is reused: stream order serialises them)

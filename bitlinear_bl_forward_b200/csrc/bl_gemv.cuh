@@ -504,8 +504,9 @@ struct G2Problem {
   void* Y;
   int K;
   int N;
-  int rows_per_cta;
-  int cta_begin;
+  int rows_per_cta;   // TMA-staged GEMV: CTA c takes rows [c*rows_per_cta, ...)
+  int cta_begin;      // first CTA of this problem in the launch
+  int ctas;           // decode kernel: CTA c takes rows [c*N/ctas, (c+1)*N/ctas)
 };
 constexpr int kG2MaxProblems = 8;
 struct G2Table {

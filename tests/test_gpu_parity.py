@@ -286,7 +286,17 @@ def test_grouped_mixed_shapes_fall_back_to_sequential():
     torch.cuda.synchronize()
     for a, b in zip(outs, singles):
         assert torch.equal(a, b)
-    # all-decode group of different K (one fused launch)
+    # all-decode group of different K (one launch per kernel variant)
     probs2 = [probs[0], probs[2]]
     outs2 = bl.bl_forward_grouped(probs2)
     assert torch.equal(outs2[0], singles[0]) and torch.equal(outs2[1], singles[2])
+    # several one-token problems of one kernel variant with ragged row counts
+    probs3, singles3 = [], []
+    for j, (K, N) in enumerate([(2560, 6912), (2560, 33), (2048, 1000), (2560, 1)]):
+        X, W = random_case(1, K, N, seed=300 + j)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        probs3.append((x_to_dev(X), Wp, gd, N))
+        singles3.append(bl.bl_forward(probs3[-1][0], Wp, gd, N))
+    outs3 = bl.bl_forward_grouped(probs3)
+    for a, b in zip(outs3, singles3):
+        assert torch.equal(a, b)
