@@ -135,6 +135,14 @@ BL_API size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bi
  * X: bf16 bits [M, K], 16-byte aligned.  Wp, gamma: from bl_quantize_weights.
  * Y: bf16 bits [M, N].  workspace: >= bl_forward_workspace_bytes(M, K, N, bits)
  * bytes, 16-byte aligned (may be null when that is 0).
+ * Ordering: the kernels are launched with programmatic dependent launch.  They
+ * read X (and the workspace) only after the preceding kernel on the stream has
+ * completed, but a one-token launch may fetch Wp before that, while the
+ * preceding kernel still runs: Wp must not be written by the kernel launched
+ * immediately before on the same stream if that kernel triggers its dependents
+ * early (this library's forward kernels do; bl_quantize_weights and ordinary
+ * kernels do not, and a dependent launch after them starts only once they
+ * have finished).
  */
 BL_API bl_status bl_forward(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
                      int bits, uint16_t* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -176,10 +184,11 @@ BL_API bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int
  * the up and gate projections of a feed-forward block (same X, two weight
  * tensors) or several requests' layers.  Each problem is exactly one
  * bl_forward (same formulas, same rounding, bit-identical results).  When
- * every problem has M == 1 and K <= 8192 they share one decode kernel launch
- * (its CTAs are shared out in proportion to each problem's weight bytes), so
- * the fixed cost of a launch and of the token-quantisation prologue is paid
- * once; otherwise the problems run one after another on the stream.
+ * every problem has M == 1 and K <= 8192, the problems with the same
+ * ceil(K / 512) share one decode kernel launch (its CTAs are shared out in
+ * proportion to each problem's weight bytes), so the fixed cost of a launch is
+ * paid once per such set; otherwise the problems run one after another on the
+ * stream.  The ordering rule of bl_forward applies to every Wp.
  * workspace: >= bl_forward_grouped_workspace_bytes(count, problems, bits)
  * (the largest per-problem bl_forward workspace; 0 for an all-decode group).
  * count > 8 returns BL_ERR_UNSUPPORTED; problems with M == 0 are skipped.
