@@ -63,22 +63,23 @@ def load_peaks():
 
 def ncu_traffic(kernel_key):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
-    the current kernel source; otherwise None."""
+    the kernel's current source (hash of the source files the line lists);
+    otherwise None."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
     src = os.path.join(ROOT, "bitlinear_bl_forward_b200", "csrc")
-    h = hashlib.sha256()
-    for fn in sorted(os.listdir(src)):
-        if fn.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(src, fn), "rb").read())
-    sha = h.hexdigest()[:16]
     for line in open(path):
         if line.startswith("#") or "=" not in line:
             continue
         kv = dict(t.split("=", 1) for t in line.split())
-        if kv.get("key") == kernel_key and kv.get("src_sha") == sha:
+        if kv.get("key") != kernel_key or "files" not in kv:
+            continue
+        h = hashlib.sha256()
+        for fn in kv["files"].split(","):
+            h.update(open(os.path.join(src, fn), "rb").read())
+        if kv.get("src_sha") == h.hexdigest()[:16]:
             return float(kv["dram_bytes_per_launch"])
     return None
 

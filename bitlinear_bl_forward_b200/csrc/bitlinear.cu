@@ -384,6 +384,22 @@ bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uin
   return launch_gemv_t<2, 2>(X, x_is_i8, M, K, N, Wp, gamma, Q, Y, out_mode, stream);
 }
 
+// Per-token activation quantisation: a warp per row when there are rows enough
+// to fill the GPU, a CTA per row otherwise.
+bl_status launch_act_quant(const uint16_t* X, int m, int k, int Q, int8_t* Xq, float* s, int* R, cudaStream_t stream) {
+  if (m < bl::kActRowsPerBlock * num_sms()) {
+    bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R);
+  } else {
+    const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
+    bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
+  }
+  return last_cuda();
+}
+
+#ifndef BL_P2_EXPG
+#define BL_P2_EXPG 1
+#endif
+
 template <int BN>
 bl_status launch_tc_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
                       const float* gamma, void* Y, int out_mode, int debug_flags, unsigned long long limit_ns,
@@ -414,8 +430,8 @@ bl_status launch_tc2_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp,
   if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), BN, bl::kTcBK,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BL_ERR_CUDA;
-  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kTcBK / 4,
-                    CU_TENSOR_MAP_SWIZZLE_32B))
+  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kP2BK / 4,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
     return BL_ERR_CUDA;
   const int ntiles = ((M + BN - 1) / BN) * ((N + bl::kTcRows - 1) / bl::kTcRows);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
@@ -505,7 +521,7 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
 
 // Tensor-core kernel selection (build-time, for experiments): 0 = by shape
 // (CTA-pair kernel for M > 64, one-SM persistent kernel otherwise),
-// 1 = one-tile-per-CTA kernel, 2 = one-SM persistent kernel only.
+// 1 = one-tile-per-CTA kernel.
 #ifndef BL_TC_KERNEL
 #define BL_TC_KERNEL 0
 #endif
@@ -515,10 +531,10 @@ bl_status launch_tc(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, co
   if (BL_TC_KERNEL == 0 && debug_flags == 0 && M > 64)
     return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
   if (BL_TC_KERNEL != 1 && debug_flags == 0) {
-    if (M <= 16) return launch_tc2_t<16, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
-    if (M <= 32) return launch_tc2_t<32, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
-    if (M <= 64) return launch_tc2_t<64, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
-    return launch_tc2_t<128, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    if (M <= 16) return launch_tc2_t<16, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    if (M <= 32) return launch_tc2_t<32, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    if (M <= 64) return launch_tc2_t<64, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
   }
   const unsigned long long lim = kWaitLimitNs;
   if (M <= 16) return launch_tc_t<16>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
@@ -568,9 +584,7 @@ bl_status forward_common(const uint16_t* X, int64_t M, int64_t K, int64_t N, con
   const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
   if (M <= kGemvMaxM) return launch_gemv(X, 0, m, k, n, Wp, gamma, Q, Y, out_mode, stream);
   const FwdWs w = fwd_ws_split(ws, M, K);
-  const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
-  bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, w.Xq, w.s, w.R);
-  if ((st = last_cuda()) != BL_OK) return st;
+  if ((st = launch_act_quant(X, m, k, Q, w.Xq, w.s, w.R, stream)) != BL_OK) return st;
   return launch_tc(w.Xq, m, k, n, Wp, w.R, w.s, gamma, Y, out_mode, 0, stream);
 }
 
@@ -656,11 +670,8 @@ bl_status bl_quant_act(const uint16_t* X, int64_t M, int64_t K, int bits, int8_t
   if (M == 0) return BL_OK;
   if (!X || !Xq || !scale) return BL_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Xq)) return BL_ERR_ALIGNMENT;
-  const int m = static_cast<int>(M);
-  const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
-  bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale,
-                                                   nullptr);
-  return last_cuda();
+  return launch_act_quant(X, static_cast<int>(M), static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr,
+                          stream);
 }
 
 size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {

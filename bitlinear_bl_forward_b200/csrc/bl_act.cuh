@@ -103,6 +103,64 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restri
   }
 }
 
+// The same quantisation with one CTA per token row, for few rows: the
+// absmax is a block reduction, so a row of K = 8192 costs four 16-byte loads
+// a thread instead of 32 a lane.  Bit-identical to act_quant_kernel (the max
+// and the integer sum do not depend on the order).
+constexpr int kActRowThreads = 256;
+constexpr int kActRowCache = 8;   // 16-byte chunks kept in registers per thread (K <= 16384)
+
+__global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uint16_t* __restrict__ X, int K, int Q,
+                                                                       int8_t* __restrict__ Xq,
+                                                                       float* __restrict__ s_out,
+                                                                       int* __restrict__ R_out) {
+  constexpr int W = kActRowThreads / 32;
+  __shared__ uint32_t s_max[W];
+  __shared__ int s_sum[W];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const size_t m = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(X + m * K);
+  const int nch = K >> 3;
+  uint4 cache[kActRowCache];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kActRowCache; ++i) {
+    const int c = t + kActRowThreads * i;
+    if (c < nch) {
+      cache[i] = __ldg(xr + c);
+      amax = fmaxf(amax, absmax8_bf16(cache[i]));
+    }
+  }
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+    amax = fmaxf(amax, absmax8_bf16(__ldg(xr + c)));
+  const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+  if (lane == 0) s_max[warp] = wmax;
+  __syncthreads();
+  uint32_t bmax = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) bmax = max(bmax, s_max[w]);
+  const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
+  uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kActRowCache; ++i) {
+    const int c = t + kActRowThreads * i;
+    if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+  }
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+    qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
+  const int wsum = __reduce_add_sync(0xffffffffu, sum);
+  if (lane == 0) s_sum[warp] = wsum;
+  __syncthreads();
+  if (t == 0) {
+    int tot = 0;
+#pragma unroll
+    for (int w = 0; w < W; ++w) tot += s_sum[w];
+    if (s_out) s_out[m] = s;
+    if (R_out) R_out[m] = tot;
+  }
+}
+
 // R[m] = sum_k Xq[m, k] for already-quantised int8 activations.
 __global__ void __launch_bounds__(256) act_rowsum_kernel(const int8_t* __restrict__ Xq, int M, int K,
                                                          int* __restrict__ R_out) {

@@ -9,9 +9,13 @@
 //
 // One CTA per SM walks a static list of tiles (128 weight rows x BN tokens),
 // token tiles fastest so the CTAs of a wave share weight tiles through L2.
+// A pipeline stage covers K = 512: the packed weight tile is 128 rows of 128
+// contiguous bytes (one 128-byte-swizzled TMA box, so every DRAM burst is a
+// whole 128-byte row segment), the tokens four 128-byte boxes; expanders and
+// MMAs work on it in four sub-stages of K = 128.
 // Four rings decouple the roles:
 //   smem ring (S stages):  TMA producer -> expanders (packed W) and MMA (X);
-//                          freed by the MMA's commit;
+//                          freed by the MMA's commit after the last sub-stage;
 //   TMEM A ring (4 slots): expanders (tcgen05.st of int8 codes) -> MMA;
 //                          freed by the MMA's commit;
 //   accumulators (2):      MMA -> epilogue; freed by the epilogue warps,
@@ -33,7 +37,16 @@
 
 namespace bl {
 
-constexpr int kP2ASlots = 4;
+#ifndef BL_P2_KACC
+#define BL_P2_KACC 4
+#endif
+#ifndef BL_P2_SLOTS
+#define BL_P2_SLOTS 8
+#endif
+constexpr int kP2ASlots = BL_P2_SLOTS;
+constexpr int kP2Sub = 4;                        // sub-stages of K = 128 per stage
+constexpr int kP2BK = kTcBK * kP2Sub;            // K per stage (512)
+constexpr int kP2WStageBytes = kTcRows * kP2BK / 4;   // 16 KB packed
 // warps: producer, MMA issuer, EXPG groups of 4 expander warps, 4 epilogue warps
 template <int EXPG>
 struct P2Warps {
@@ -46,13 +59,18 @@ constexpr int kP2SmemBudget = 200 * 1024;
 template <int BN>
 struct P2Cfg {
   static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128, "unsupported token tile");
-  static constexpr int kXStageBytes = BN * kTcBK;
-  static constexpr int kStageBytes = kXStageBytes + kTcWStageBytes;
+  static constexpr int kXSubBytes = BN * kTcBK;               // one 128-byte-wide token box
+  static constexpr int kXStageBytes = kP2Sub * kXSubBytes;
+  static constexpr int kStageBytes = kXStageBytes + kP2WStageBytes;
   static constexpr int kStagesRaw = kP2SmemBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 24 ? 24 : kStagesRaw;
-  static constexpr int kAccCols = BN < 32 ? 32 : BN;             // per accumulator buffer
-  static constexpr int kACol = 2 * kAccCols;                      // first TMEM column of the A ring
+  static constexpr int kAccCols = BN < 32 ? 32 : BN;             // per accumulator
+  // independent accumulators a tile's sub-stages rotate through (summed in
+  // the epilogue): consecutive MMAs never wait on each other's result
+  static constexpr int kKAcc = BN <= 32 ? BL_P2_KACC : (BL_P2_KACC > 2 ? 2 : BL_P2_KACC);
+  static constexpr int kACol = 2 * kKAcc * kAccCols;              // first TMEM column of the A ring
   static constexpr int kTmemCols = (kACol + 32 * kP2ASlots <= 256) ? 256 : 512;
+  static_assert(kACol + 32 * kP2ASlots <= 512, "accumulators and A slots exceed tensor memory");
   static constexpr int kBarOffset = kStages * kStageBytes;
   // barriers: full[S], empty[S], afull[4], aempty[4], accfull[2], accempty[2], drain
   static constexpr int kNumBars = 2 * kStages + 2 * kP2ASlots + 5;
@@ -86,7 +104,7 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
   float* sF = reinterpret_cast<float*>(sR + 2 * BN);        // [2][BN]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = (K + kTcBK - 1) / kTcBK;
+  const int nk = (K + kP2BK - 1) / kP2BK;   // stages per tile (K beyond the end reads zeros)
   const int mt = (M + BN - 1) / BN;
   const int ntiles = mt * ((N + kTcRows - 1) / kTcRows);
 
@@ -133,8 +151,10 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-          tma_load_2d(sX + s * C::kXStageBytes, &tmX, ks * kTcBK, m0, &full[s]);
-          tma_load_2d(sW + s * kTcWStageBytes, &tmW, ks * (kTcBK / 4), n0, &full[s]);
+          tma_load_2d(sW + s * kP2WStageBytes, &tmW, ks * (kP2BK / 4), n0, &full[s]);
+#pragma unroll
+          for (int j = 0; j < kP2Sub; ++j)
+            tma_load_2d(sX + s * C::kXStageBytes + j * C::kXSubBytes, &tmX, ks * kP2BK + j * kTcBK, m0, &full[s]);
         }
       }
       // every copy issued into this CTA's shared memory must land before exit
@@ -155,23 +175,25 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
         const int b = i & 1;
         if (i >= 2 && !mbar_wait(&accempty[b], ((i >> 1) & 1) ^ 1u, abort_flag, limit_ns, kSiteAcc)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + b * C::kAccCols;
-        for (int ks = 0; ks < nk; ++ks, ++g) {
-          const int s = g % S;
+        const uint32_t d_base = tmem + b * C::kKAcc * C::kAccCols;
+        for (int kq = 0; kq < nk * kP2Sub; ++kq, ++g) {   // g counts sub-stages
+          const int s = (g / kP2Sub) % S;
           const int t = g % kP2ASlots;
           if (!mbar_wait(&afull[t], (g / kP2ASlots) & 1, abort_flag, limit_ns, kSiteMmaExfull)) {
             stop = true;
             break;
           }
           tc_fence_after();
-          const uint32_t xs = smem_u32(sX + s * C::kXStageBytes);
+          const uint32_t xs = smem_u32(sX + s * C::kXStageBytes + (g % kP2Sub) * C::kXSubBytes);
+          const uint32_t d_tmem = d_base + (kq % C::kKAcc) * C::kAccCols;
 #pragma unroll
           for (int kk = 0; kk < kTcBK / 32; ++kk) {
             const uint32_t a_tmem = tmem + C::kACol + 32 * t + 8 * kk;
-            mma_i8_ts(d_tmem, a_tmem, smem_desc_k_sw128(xs + 32 * kk), idesc, (ks | kk) != 0 ? 1u : 0u);
+            mma_i8_ts(d_tmem, a_tmem, smem_desc_k_sw128(xs + 32 * kk), idesc,
+                      (kq >= C::kKAcc || kk != 0) ? 1u : 0u);
           }
-          tc_commit(&empty[s]);
           tc_commit(&aempty[t]);
+          if (g % kP2Sub == kP2Sub - 1) tc_commit(&empty[g / kP2Sub % S]);
         }
         if (stop) break;
         tc_commit(&accfull[b]);
@@ -186,15 +208,16 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t wsw = static_cast<uint32_t>((r >> 2) & 1) << 4;
-    uint32_t g = 0;
+    const uint32_t rsw = static_cast<uint32_t>(r & 7);   // 128-byte swizzle: 16-byte chunk c sits at c ^ (r % 8)
+    uint32_t g = 0;   // sub-stage counter
     bool stop = false;
     for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
-      for (int ks = 0; ks < nk; ++ks, ++g) {
+      for (int kq = 0; kq < nk * kP2Sub; ++kq, ++g) {
         if (static_cast<int>(g % EXPG) != grp) continue;
-        const int s = g % S;
+        const uint32_t st = g / kP2Sub;
+        const int s = st % S;
         const int t = g % kP2ASlots;
-        bool ok = mbar_wait(&full[s], (g / S) & 1, abort_flag, limit_ns, kSiteExpFull);
+        bool ok = mbar_wait(&full[s], (st / S) & 1, abort_flag, limit_ns, kSiteExpFull);
         if (ok && g >= static_cast<uint32_t>(kP2ASlots))
           ok = mbar_wait(&aempty[t], ((g / kP2ASlots) & 1) ^ 1u, abort_flag, limit_ns, kSiteExpEmpty);
         if (!__all_sync(0xffffffffu, ok)) {
@@ -202,9 +225,10 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t wrow = smem_u32(sW + s * kTcWStageBytes) + r * 32;
-        const uint4 lo = ld_shared_v4(wrow + (0u ^ wsw));
-        const uint4 hi = ld_shared_v4(wrow + (16u ^ wsw));
+        const uint32_t wrow = smem_u32(sW + s * kP2WStageBytes) + r * 128;
+        const uint32_t c0 = 2u * (g % kP2Sub);
+        const uint4 lo = ld_shared_v4(wrow + (((c0 + 0u) ^ rsw) << 4));
+        const uint4 hi = ld_shared_v4(wrow + (((c0 + 1u) ^ rsw) << 4));
         const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         uint32_t v[32];
 #pragma unroll
@@ -252,11 +276,24 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += kChunk) {
         uint32_t v[32];
+        const uint32_t acc0 = tmem + lane_base + b * C::kKAcc * C::kAccCols + c0;
         if constexpr (kChunk == 32)
-          tmem_ld_32x32b_x32(tmem + lane_base + b * C::kAccCols + c0, v);
+          tmem_ld_32x32b_x32(acc0, v);
         else
-          tmem_ld_32x32b_x16(tmem + lane_base + b * C::kAccCols + c0, v);
+          tmem_ld_32x32b_x16(acc0, v);
         tmem_wait_ld();
+        // the tile's other accumulators (a tile has at least kKAcc sub-stages)
+#pragma unroll 1
+        for (int a = 1; a < C::kKAcc; ++a) {
+          uint32_t u[32];
+          if constexpr (kChunk == 32)
+            tmem_ld_32x32b_x32(acc0 + a * C::kAccCols, u);
+          else
+            tmem_ld_32x32b_x16(acc0 + a * C::kAccCols, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) v[j] += u[j];
+        }
         if (n < N) {
 #pragma unroll
           for (int t = 0; t < kChunk; ++t) {
