@@ -1,4 +1,4 @@
-// Persistent tensor-core GEMM for the prefill / batched path.
+// Persistent tensor-core GEMM for few tokens (M <= 64).
 //
 // Same arithmetic as tc_gemm_kernel ("BitNet b1.58: The 1-Bit Ternary LLM
 // Architecture Guide", section "The Mathematical Formulation of BitLinear",
@@ -10,19 +10,22 @@
 // One CTA per SM walks a static list of tiles (128 weight rows x BN tokens),
 // token tiles fastest so the CTAs of a wave share weight tiles through L2.
 // A pipeline stage covers K = 512: the packed weight tile is 128 rows of 128
-// contiguous bytes (one 128-byte-swizzled TMA box, so every DRAM burst is a
-// whole 128-byte row segment), the tokens four 128-byte boxes; expanders and
-// MMAs work on it in four sub-stages of K = 128.
-// Four rings decouple the roles:
+// contiguous bytes (one 128-byte-swizzled TMA box: whole 128-byte row
+// segments from DRAM), the tokens four 128-byte boxes.  With few tokens an
+// MMA (M = 128, N <= 64, K = 32) is short (about 46 cycles, measured), so the
+// fixed costs around it decide the speed: each hand-off between roles moves a
+// whole stage (16 MMAs), and one commit per stage frees both the shared
+// memory stage and, three stages later, the tensor-memory slot.
+// Rings:
 //   smem ring (S stages):  TMA producer -> expanders (packed W) and MMA (X);
-//                          freed by the MMA's commit after the last sub-stage;
-//   TMEM A ring (4 slots): expanders (tcgen05.st of int8 codes) -> MMA;
-//                          freed by the MMA's commit;
+//                          freed by the MMA's commit to empty[s];
+//   TMEM A ring (3 slots of 128 columns, one stage each): expanders
+//                          (tcgen05.st of int8 codes) -> MMA; slot reuse waits
+//                          on the empty[] phase of the stage that last used it;
 //   accumulators (2):      MMA -> epilogue; freed by the epilogue warps,
 //                          so tile i's epilogue overlaps tile i+1's MMAs.
 // Warps: 0 producer, 1 MMA issuer (owns TMEM), then EXPG groups of four
-// expander warps (group e takes the k-stages g with g % EXPG == e, so the
-// latency of tcgen05.st + wait::st is paid EXPG stages at a time), then four
+// expander warps (group e takes the stages g with g % EXPG == e), then four
 // epilogue warps.
 // Every wait is bounded; a stalled pipeline records BL_ERR_TIMEOUT, each
 // role unwinds, the producer drains its copies, the MMA thread waits for its
@@ -37,16 +40,11 @@
 
 namespace bl {
 
-#ifndef BL_P2_KACC
-#define BL_P2_KACC 4
-#endif
-#ifndef BL_P2_SLOTS
-#define BL_P2_SLOTS 8
-#endif
-constexpr int kP2ASlots = BL_P2_SLOTS;
+constexpr int kP2ASlots = 3;                     // tensor-memory A slots, one K = 512 stage each
 constexpr int kP2Sub = 4;                        // sub-stages of K = 128 per stage
 constexpr int kP2BK = kTcBK * kP2Sub;            // K per stage (512)
 constexpr int kP2WStageBytes = kTcRows * kP2BK / 4;   // 16 KB packed
+constexpr int kP2ASlotCols = kP2BK / 4;               // 128 columns of int8x4 per slot
 // warps: producer, MMA issuer, EXPG groups of 4 expander warps, 4 epilogue warps
 template <int EXPG>
 struct P2Warps {
@@ -64,16 +62,13 @@ struct P2Cfg {
   static constexpr int kStageBytes = kXStageBytes + kP2WStageBytes;
   static constexpr int kStagesRaw = kP2SmemBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 24 ? 24 : kStagesRaw;
-  static constexpr int kAccCols = BN < 32 ? 32 : BN;             // per accumulator
-  // independent accumulators a tile's sub-stages rotate through (summed in
-  // the epilogue): consecutive MMAs never wait on each other's result
-  static constexpr int kKAcc = BN <= 32 ? BL_P2_KACC : (BL_P2_KACC > 2 ? 2 : BL_P2_KACC);
-  static constexpr int kACol = 2 * kKAcc * kAccCols;              // first TMEM column of the A ring
-  static constexpr int kTmemCols = (kACol + 32 * kP2ASlots <= 256) ? 256 : 512;
-  static_assert(kACol + 32 * kP2ASlots <= 512, "accumulators and A slots exceed tensor memory");
+  static constexpr int kAccCols = BN < 32 ? 32 : BN;             // per accumulator buffer
+  static constexpr int kACol = 2 * kAccCols;                      // first TMEM column of the A ring
+  static constexpr int kTmemCols = 512;
+  static_assert(kACol + kP2ASlotCols * kP2ASlots <= 512, "accumulators and A slots exceed tensor memory");
   static constexpr int kBarOffset = kStages * kStageBytes;
-  // barriers: full[S], empty[S], afull[4], aempty[4], accfull[2], accempty[2], drain
-  static constexpr int kNumBars = 2 * kStages + 2 * kP2ASlots + 5;
+  // barriers: full[S], empty[S], afull[slots], accfull[2], accempty[2], drain
+  static constexpr int kNumBars = 2 * kStages + kP2ASlots + 5;
   static constexpr int kEpiOffset = kBarOffset + kNumBars * 8 + 16;
   static constexpr int kUsedBytes = kEpiOffset + 2 * BN * 8;
   static constexpr int kSmemBytes = kUsedBytes + 1024;
@@ -94,8 +89,7 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* empty = full + S;
   uint64_t* afull = empty + S;
-  uint64_t* aempty = afull + kP2ASlots;
-  uint64_t* accfull = aempty + kP2ASlots;
+  uint64_t* accfull = afull + kP2ASlots;
   uint64_t* accempty = accfull + 2;
   uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -115,7 +109,6 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
     }
     for (int t = 0; t < kP2ASlots; ++t) {
       mbar_init(&afull[t], 128);
-      mbar_init(&aempty[t], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
@@ -175,25 +168,26 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
         const int b = i & 1;
         if (i >= 2 && !mbar_wait(&accempty[b], ((i >> 1) & 1) ^ 1u, abort_flag, limit_ns, kSiteAcc)) break;
         tc_fence_after();
-        const uint32_t d_base = tmem + b * C::kKAcc * C::kAccCols;
-        for (int kq = 0; kq < nk * kP2Sub; ++kq, ++g) {   // g counts sub-stages
-          const int s = (g / kP2Sub) % S;
+        const uint32_t d_tmem = tmem + b * C::kAccCols;
+        for (int ks = 0; ks < nk; ++ks, ++g) {   // g counts stages
+          const int s = g % S;
           const int t = g % kP2ASlots;
           if (!mbar_wait(&afull[t], (g / kP2ASlots) & 1, abort_flag, limit_ns, kSiteMmaExfull)) {
             stop = true;
             break;
           }
           tc_fence_after();
-          const uint32_t xs = smem_u32(sX + s * C::kXStageBytes + (g % kP2Sub) * C::kXSubBytes);
-          const uint32_t d_tmem = d_base + (kq % C::kKAcc) * C::kAccCols;
+          const uint32_t xs = smem_u32(sX + s * C::kXStageBytes);
+          const uint32_t as = tmem + C::kACol + kP2ASlotCols * t;
 #pragma unroll
-          for (int kk = 0; kk < kTcBK / 32; ++kk) {
-            const uint32_t a_tmem = tmem + C::kACol + 32 * t + 8 * kk;
-            mma_i8_ts(d_tmem, a_tmem, smem_desc_k_sw128(xs + 32 * kk), idesc,
-                      (kq >= C::kKAcc || kk != 0) ? 1u : 0u);
-          }
-          tc_commit(&aempty[t]);
-          if (g % kP2Sub == kP2Sub - 1) tc_commit(&empty[g / kP2Sub % S]);
+          for (int j = 0; j < kP2Sub; ++j)
+#pragma unroll
+            for (int kk = 0; kk < kTcBK / 32; ++kk)
+              mma_i8_ts(d_tmem, as + 32 * j + 8 * kk, smem_desc_k_sw128(xs + j * C::kXSubBytes + 32 * kk), idesc,
+                        (ks | j | kk) != 0 ? 1u : 0u);
+          // one commit frees both the smem stage (producer) and, three stages
+          // later, the tensor-memory slot (expanders wait on the same phase)
+          tc_commit(&empty[s]);
         }
         if (stop) break;
         tc_commit(&accfull[b]);
@@ -209,33 +203,40 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t rsw = static_cast<uint32_t>(r & 7);   // 128-byte swizzle: 16-byte chunk c sits at c ^ (r % 8)
-    uint32_t g = 0;   // sub-stage counter
+    uint32_t g = 0;   // stage counter
     bool stop = false;
     for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
-      for (int kq = 0; kq < nk * kP2Sub; ++kq, ++g) {
+      for (int ks = 0; ks < nk; ++ks, ++g) {
         if (static_cast<int>(g % EXPG) != grp) continue;
-        const uint32_t st = g / kP2Sub;
-        const int s = st % S;
+        const int s = g % S;
         const int t = g % kP2ASlots;
-        bool ok = mbar_wait(&full[s], (st / S) & 1, abort_flag, limit_ns, kSiteExpFull);
-        if (ok && g >= static_cast<uint32_t>(kP2ASlots))
-          ok = mbar_wait(&aempty[t], ((g / kP2ASlots) & 1) ^ 1u, abort_flag, limit_ns, kSiteExpEmpty);
+        bool ok = mbar_wait(&full[s], (g / S) & 1, abort_flag, limit_ns, kSiteExpFull);
+        // slot t was last read by the MMAs of stage g - kP2ASlots, whose commit
+        // completes that stage's phase of empty[]; no later phase of that
+        // barrier can complete before this stage is expanded
+        if (ok && g >= static_cast<uint32_t>(kP2ASlots)) {
+          const uint32_t prev = g - kP2ASlots;
+          ok = mbar_wait(&empty[prev % S], (prev / S) & 1, abort_flag, limit_ns, kSiteExpEmpty);
+        }
         if (!__all_sync(0xffffffffu, ok)) {
           stop = true;
           break;
         }
         tc_fence_after();
         const uint32_t wrow = smem_u32(sW + s * kP2WStageBytes) + r * 128;
-        const uint32_t c0 = 2u * (g % kP2Sub);
-        const uint4 lo = ld_shared_v4(wrow + (((c0 + 0u) ^ rsw) << 4));
-        const uint4 hi = ld_shared_v4(wrow + (((c0 + 1u) ^ rsw) << 4));
-        const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        uint32_t v[32];
+        // four sub-steps of K = 128 (32 bytes of the row each); one wait for all stores
+#pragma unroll 1
+        for (uint32_t j = 0; j < kP2Sub; ++j) {
+          const uint4 lo = ld_shared_v4(wrow + (((2u * j + 0u) ^ rsw) << 4));
+          const uint4 hi = ld_shared_v4(wrow + (((2u * j + 1u) ^ rsw) << 4));
+          const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          uint32_t v[32];
 #pragma unroll
-        for (int gw = 0; gw < 8; ++gw)
+          for (int gw = 0; gw < 8; ++gw)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) v[4 * gw + j] = (wd[gw] >> (2 * j)) & 0x03030303u;
-        tmem_st_32x32b_x32(tmem + lane_base + C::kACol + 32 * t, v);
+            for (int jj = 0; jj < 4; ++jj) v[4 * gw + jj] = (wd[gw] >> (2 * jj)) & 0x03030303u;
+          tmem_st_32x32b_x32(tmem + lane_base + C::kACol + kP2ASlotCols * t + 32 * j, v);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&afull[t]);
@@ -276,24 +277,11 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += kChunk) {
         uint32_t v[32];
-        const uint32_t acc0 = tmem + lane_base + b * C::kKAcc * C::kAccCols + c0;
         if constexpr (kChunk == 32)
-          tmem_ld_32x32b_x32(acc0, v);
+          tmem_ld_32x32b_x32(tmem + lane_base + b * C::kAccCols + c0, v);
         else
-          tmem_ld_32x32b_x16(acc0, v);
+          tmem_ld_32x32b_x16(tmem + lane_base + b * C::kAccCols + c0, v);
         tmem_wait_ld();
-        // the tile's other accumulators (a tile has at least kKAcc sub-stages)
-#pragma unroll 1
-        for (int a = 1; a < C::kKAcc; ++a) {
-          uint32_t u[32];
-          if constexpr (kChunk == 32)
-            tmem_ld_32x32b_x32(acc0 + a * C::kAccCols, u);
-          else
-            tmem_ld_32x32b_x16(acc0 + a * C::kAccCols, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < kChunk; ++j) v[j] += u[j];
-        }
         if (n < N) {
 #pragma unroll
           for (int t = 0; t < kChunk; ++t) {
