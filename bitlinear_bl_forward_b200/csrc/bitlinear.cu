@@ -486,7 +486,7 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
     if (!enc) return BL_ERR_CUDA;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(bl::kQBN)};
+    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(bl::kQEpiCols)};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=

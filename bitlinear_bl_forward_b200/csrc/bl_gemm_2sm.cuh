@@ -21,7 +21,9 @@
 // Rings as in the one-SM persistent kernel: S shared-memory stages, 8 TMEM A
 // slots (the slot round trip crosses the pair twice), 2 accumulators (the epilogue of tile i overlaps the MMAs of i+1).
 // Warps: 0 producer, 1 MMA issuer (leader) / TMEM owner, 2-5 expanders,
-// 6-9 epilogue.  All waits are bounded; the pair meets at a cluster barrier
+// 6-13 epilogue (two per TMEM lane quadrant, 64 tokens each: the epilogue of
+// a tile must finish within the next tile's main loop, which for K = 2560 is
+// only ten stages).  All waits are bounded; the pair meets at a cluster barrier
 // before TMEM is freed, after the leader has waited for its last MMA.
 #pragma once
 
@@ -37,7 +39,8 @@ namespace bl {
 // expands the stages g with g % kQExpGroups == e), then 4 epilogue warps
 constexpr int kQExpGroups = 1;   // measured: a second group does not help
 constexpr int kQFirstEpi = 2 + 4 * kQExpGroups;
-constexpr int kQThreads = 32 * (kQFirstEpi + 4);
+constexpr int kQEpiWarps = 8;   // two per TMEM lane quadrant, each takes half of the tile's tokens
+constexpr int kQThreads = 32 * (kQFirstEpi + kQEpiWarps);
 constexpr int kQBK = 256;                       // K per pipeline stage: 8 MMAs per hand-off
 constexpr int kQASlots = 4;                     // TMEM: 2 x 128 accumulator + 4 x 64 A columns = 512
 constexpr int kQASlotCols = kQBK / 4;           // int8 codes, 4 per 32-bit column
@@ -49,12 +52,13 @@ constexpr int kQXStageBytes = kQHalf * kQBK;    // 16 KB: kQBK / 128 boxes
 constexpr int kQWStageBytes = kTcRows * kQBK / 4;   // 8 KB packed, 64-byte rows (SW64)
 constexpr int kQStageBytes = kQXStageBytes + kQWStageBytes;
 constexpr int kQStages = 7;                     // 168 KB
-constexpr int kQStageOutBytes = kQBN * 32 * 2;  // bf16 [BN tokens][32 rows] per epilogue warp
+constexpr int kQEpiCols = kQBN / 2;             // tokens per epilogue warp
+constexpr int kQStageOutBytes = kQEpiCols * 32 * 2;  // bf16 [64 tokens][32 rows] per epilogue warp
 constexpr int kQAccCols = kQBN;
 constexpr int kQACol = 2 * kQAccCols;
 constexpr int kQTmemCols = 512;
 constexpr int kQOutOffset = kQStages * kQStageBytes;
-constexpr int kQBarOffset = kQOutOffset + 4 * kQStageOutBytes;
+constexpr int kQBarOffset = kQOutOffset + kQEpiWarps * kQStageOutBytes;
 // barriers: full[S], done[S] (stage consumed by the MMAs: frees its shared
 // memory and, kQASlots stages later, its TMEM A slot), afull[4], accfull[2],
 // accempty[2], drain
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     for (int t = 0; t < kQASlots; ++t) mbar_init(&afull[t], 8);   // one arrival per expander warp of each CTA
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], 256);
+      mbar_init(&accempty[b], 2 * 32 * kQEpiWarps);   // every epilogue thread of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -232,6 +236,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const int et = threadIdx.x - 32 * kQFirstEpi;
+    const int col0 = ((warp - kQFirstEpi) >> 2) * kQEpiCols;   // this warp's half of the tokens
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float gamma = (out_mode == kOutI32) ? 1.f : *gamma_p;
     int i = 0;
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const int b = i & 1;
       const int m0 = (tile % mt) * kQBN;
       const int n0 = (tile / mt) * kQRows + static_cast<int>(rank) * kTcRows;
-      for (int j = et; j < kQBN; j += 128) {
+      for (int j = et; j < kQBN; j += 32 * kQEpiWarps) {
         const int m = m0 + j;
         int rv = 0;
         float fv = 0.f;
@@ -251,19 +256,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
         sF[b * kQBN + j] = fv;
       }
       __syncwarp();
-      named_bar_sync(2, 128);
+      named_bar_sync(2, 32 * kQEpiWarps);
       const bool ok = mbar_wait_cluster(&accfull[b], (i >> 1) & 1, abort_flag, limit_ns, kSiteAcc) && !*abort_flag;
       __syncwarp();
-      if (!named_bar_and(3, 128, ok)) break;
+      if (!named_bar_and(3, 32 * kQEpiWarps, ok)) break;
       tc_fence_after();
       const int n = n0 + r;
       if (tma_store) {
         // bf16 tile of this warp, [BN tokens][32 rows], then one TMA store
-        uint16_t* so = reinterpret_cast<uint16_t*>(sOut + q * kQStageOutBytes);
+        uint16_t* so = reinterpret_cast<uint16_t*>(sOut + (warp - kQFirstEpi) * kQStageOutBytes);
         if (lane == 0) bulk_wait_group_read0();   // the previous store has read the buffer
         __syncwarp();
 #pragma unroll 1
-        for (int c0 = 0; c0 < kQBN; c0 += 32) {
+        for (int c0 = col0; c0 < col0 + kQEpiCols; c0 += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tmem + lane_base + b * kQAccCols + c0, v);
           tmem_wait_ld();
@@ -271,23 +276,23 @@ __global__ void __launch_bounds__(kQThreads, 1)
           for (int t = 0; t < 32; ++t) {
             const int a = static_cast<int>(v[t]) - sR[b * kQBN + c0 + t];
             const float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
-            so[(c0 + t) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+            so[(c0 - col0 + t) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
           }
         }
         tc_fence_before();
         mbar_arrive_cluster(&accempty[b], 0);   // accumulator drained: the MMAs may reuse it
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmY, n0 + q * 32, m0, so);
+        if (lane == 0 && m0 + col0 < M) {   // (a box starting past the last token writes nothing)
+          tma_store_2d(&tmY, n0 + q * 32, m0 + col0, so);
           bulk_commit_group();
         }
         __syncwarp();
-        named_bar_sync(2, 128);
+        named_bar_sync(2, 32 * kQEpiWarps);
         continue;
       }
 #pragma unroll 1
-      for (int c0 = 0; c0 < kQBN; c0 += 32) {
+      for (int c0 = col0; c0 < col0 + kQEpiCols; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lane_base + b * kQAccCols + c0, v);
         tmem_wait_ld();
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       tc_fence_before();
       mbar_arrive_cluster(&accempty[b], 0);
       __syncwarp();
-      named_bar_sync(2, 128);
+      named_bar_sync(2, 32 * kQEpiWarps);
     }
   }
   if (warp >= kQFirstEpi && lane == 0) bulk_wait_group0();   // outputs written before exit
