@@ -475,7 +475,7 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BL_ERR_CUDA;
   if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kQBK / 4,
-                    CU_TENSOR_MAP_SWIZZLE_64B))
+                    bl::kQBK == 512 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return BL_ERR_CUDA;
   // bf16 outputs leave through TMA stores when the rows are 16-byte aligned
   CUtensorMap tmY;

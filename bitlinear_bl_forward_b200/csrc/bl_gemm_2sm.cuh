@@ -18,8 +18,11 @@
 //   * the leader's tcgen05.commit arrives on the barriers of both CTAs
 //     (smem stage free, TMEM A slot free, accumulator full); the peer's
 //     expanders and epilogue warps arrive on the leader's barriers remotely.
-// Rings as in the one-SM persistent kernel: S shared-memory stages, 8 TMEM A
-// slots (the slot round trip crosses the pair twice), 2 accumulators (the epilogue of tile i overlaps the MMAs of i+1).
+// Rings: S shared-memory stages of K = 512 (16 MMAs per hand-off: a commit
+// costs about as much pipe time as two short MMAs, so fewer hand-offs), two
+// TMEM A slots of 128 columns (a slot is free again once the stage that last
+// used it is done), 2 accumulators (the epilogue of tile i overlaps the MMAs
+// of i+1).
 // Warps: 0 producer, 1 MMA issuer (leader) / TMEM owner, 2-5 expanders,
 // 6-13 epilogue (two per TMEM lane quadrant, 64 tokens each: the epilogue of
 // a tile must finish within the next tile's main loop, which for K = 2560 is
@@ -41,17 +44,21 @@ constexpr int kQExpGroups = 1;   // measured: a second group does not help
 constexpr int kQFirstEpi = 2 + 4 * kQExpGroups;
 constexpr int kQEpiWarps = 8;   // two per TMEM lane quadrant, each takes half of the tile's tokens
 constexpr int kQThreads = 32 * (kQFirstEpi + kQEpiWarps);
-constexpr int kQBK = 256;                       // K per pipeline stage: 8 MMAs per hand-off
-constexpr int kQASlots = 4;                     // TMEM: 2 x 128 accumulator + 4 x 64 A columns = 512
+#ifndef BL_Q_BK
+#define BL_Q_BK 512
+#endif
+constexpr int kQBK = BL_Q_BK;                   // K per pipeline stage: kQBK / 32 MMAs per hand-off
+constexpr int kQASlots = kQBK == 512 ? 2 : 4;   // TMEM: 2 x 128 accumulator + A slots = 512 columns
 constexpr int kQASlotCols = kQBK / 4;           // int8 codes, 4 per 32-bit column
 constexpr int kQBN = 128;                       // tokens per pair tile (MMA N)
 constexpr int kQHalf = kQBN / 2;                // token rows staged per CTA
 constexpr int kQRows = 256;                     // weight rows per pair tile (MMA M)
 constexpr int kQXBoxBytes = kQHalf * 128;       // one 128-byte-wide activation box (SW128)
 constexpr int kQXStageBytes = kQHalf * kQBK;    // 16 KB: kQBK / 128 boxes
-constexpr int kQWStageBytes = kTcRows * kQBK / 4;   // 8 KB packed, 64-byte rows (SW64)
+constexpr int kQWRowBytes = kQBK / 4;           // packed bytes of a weight row per stage
+constexpr int kQWStageBytes = kTcRows * kQWRowBytes;   // 64-byte rows (SW64) or 128-byte rows (SW128)
 constexpr int kQStageBytes = kQXStageBytes + kQWStageBytes;
-constexpr int kQStages = 7;                     // 168 KB
+constexpr int kQStages = kQBK == 512 ? 3 : 7;   // 144 KB / 168 KB
 constexpr int kQEpiCols = kQBN / 2;             // tokens per epilogue warp
 constexpr int kQStageOutBytes = kQEpiCols * 32 * 2;  // bf16 [64 tokens][32 rows] per epilogue warp
 constexpr int kQAccCols = kQBN;
@@ -76,7 +83,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem;
   uint8_t* sW = smem + S * kQXStageBytes;
-  static_assert(kQBK % 128 == 0 && kQASlotCols == 64, "stage layout below assumes K = 256 per stage");
+  static_assert(kQBK == 256 || kQBK == 512, "stage layout below assumes K = 256 or 512 per stage");
+  static_assert(2 * kQAccCols + kQASlots * kQASlotCols <= kQTmemCols, "tensor memory budget");
   uint8_t* sOut = smem + kQOutOffset;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQBarOffset);
   uint64_t* done = full + S;
@@ -191,7 +199,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t wsw = static_cast<uint32_t>((r >> 1) & 3);   // 64-byte swizzle of the packed box
+    // swizzle of the packed box: 16-byte chunk c of row r sits at chunk c ^ wsw
+    const uint32_t wsw = kQWRowBytes == 64 ? static_cast<uint32_t>((r >> 1) & 3) : static_cast<uint32_t>(r & 7);
     uint32_t g = 0;
     bool stop = false;
     for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
@@ -210,11 +219,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
           break;
         }
         tc_fence_after();
-        // row r of the stage: 64 packed bytes = four 16-byte chunks, chunk c
-        // stored at chunk position c ^ ((r >> 1) & 3) (64-byte swizzle)
-        const uint32_t wrow = smem_u32(sW + s * kQWStageBytes) + r * 64;
+        // row r of the stage: kQWRowBytes packed bytes in 16-byte chunks, 32
+        // bytes (K = 128) per tcgen05.st of 32 columns
+        const uint32_t wrow = smem_u32(sW + s * kQWStageBytes) + r * kQWRowBytes;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kQWRowBytes / 32; ++h) {
           const uint4 lo = ld_shared_v4(wrow + (((2u * h) ^ wsw) << 4));
           const uint4 hi = ld_shared_v4(wrow + (((2u * h + 1u) ^ wsw) << 4));
           const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
