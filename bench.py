@@ -467,7 +467,9 @@ def run_gpu(args):
         peak = peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO
         roof = roofline_entry("tensor", achieved, peak, "TFLOP/s", ncu_traffic(f"tc:{name}"))
     roof["peak_src"] = peaks["src"] + (" hbm copy" if decode else " bf16 sustained x2 (int8/bf16 nominal)")
-    roof["kernel"] = "gemv3_kernel" if decode else "tc_gemm_pair_kernel (+ act_quant_kernel in the step)"
+    roof["kernel"] = ("gemv3_kernel" if decode else
+                      ("tc_gemm_persistent_kernel" if w.M <= 64 else "tc_gemm_pair_kernel")
+                      + " (+ activation quantisation in the step)")
     roof["kernel_us_avg"] = per_rank_ms * 1e3 / launches
 
     # end-to-end through the public API with host buffers

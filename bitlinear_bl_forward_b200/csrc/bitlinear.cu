@@ -385,9 +385,11 @@ bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uin
 }
 
 // Per-token activation quantisation: a warp per row when there are rows enough
-// to fill the GPU, a CTA per row otherwise.
+// to fill the GPU and a row fits a warp's registers, a CTA per row otherwise.
 bl_status launch_act_quant(const uint16_t* X, int m, int k, int Q, int8_t* Xq, float* s, int* R, cudaStream_t stream) {
-  if (m < bl::kActRowsPerBlock * num_sms()) {
+  // measured: the CTA-per-row kernel also wins for long rows (K > 4096, where
+  // a warp can no longer keep its row in registers and reads part of it twice)
+  if (m < bl::kActRowsPerBlock * num_sms() || k > 32 * 8 * bl::kActCache) {
     bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R);
   } else {
     const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
