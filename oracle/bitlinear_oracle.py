@@ -20,7 +20,11 @@ Sources (web pages, cited by title and section):
          activation codes clipped to [-8, 7], scale max|X| / 7.
   [P3] "BitNet 2B4T Guide: Scaling Native 1.58-Bit LLMs",
        section "1. The BitLinear Operator": clip range [-128, 127] for the
-         8-bit codes; the dequantisation factor beta / gamma.
+         8-bit codes; the dequantisation factor beta / gamma;
+       section "2. Squared ReLU Activation": ReLU^2(x) = (max(0, x))^2
+         between the feed-forward projections (the page's module applies it
+         to the gate projection's output and feeds the result to the down
+         projection).
 
 Readings where the pages are silent or disagree (each one is listed with its
 reason in the design notes of the repository):
@@ -67,9 +71,12 @@ __all__ = [
     "pack_ternary",
     "unpack_ternary",
     "act_quant",
+    "act_quant_values",
+    "relu2_input",
     "matmul_i32",
     "rescale",
     "forward",
+    "forward_relu2",
 ]
 
 # Floor used for both scales (pages' code listings clamp(min=1e-5)).
@@ -286,6 +293,42 @@ def act_quant(x_bits: np.ndarray, bits: int = 8, a4_divide_form: bool = False):
     return q, s
 
 
+def act_quant_values(x: np.ndarray, bits: int = 8):
+    """The same per-token quantisation as ``act_quant`` on fp32 values that
+    need not be bf16 (the squared-ReLU feed-forward input):
+    s_m = Q / max(max_k |x_mk|, 1e-5), q = clip(rint(f32(x * s_m)), -Q-1, Q).
+    Returns (q int8 [M, K], s fp32 [M])."""
+    if bits not in QMAX:
+        raise ValueError("bits must be 8 or 4")
+    Q = QMAX[bits]
+    xf = np.asarray(x, dtype=np.float32)
+    if xf.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    a = np.max(np.abs(xf), axis=1) if xf.shape[1] else np.zeros(xf.shape[0], np.float32)
+    a_floor = np.maximum(a, EPS).astype(np.float32)
+    s = (np.float32(Q) / a_floor).astype(np.float32)
+    t = (xf * s[:, None]).astype(np.float32)
+    q = np.clip(np.rint(t), -Q - 1, Q).astype(np.int8)
+    return q, s
+
+
+# ---------------------------------------------------------------------------
+# [P3] section 2: squared ReLU between the feed-forward projections
+# ---------------------------------------------------------------------------
+
+def relu2_input(g_bits: np.ndarray, u_bits: np.ndarray | None = None) -> np.ndarray:
+    """Input of the down projection from the gate projection's bf16 output g:
+    h = max(0, g)^2 in fp32; with ``u_bits`` (the up projection's output, the
+    gated variant) h = f32(max(0, g)^2 * u).  For bf16 g and u both products
+    are exact in fp32 (8 + 8 and 16 + 8 significant bits), barring overflow."""
+    g = bf16_bits_to_f32(g_bits)
+    r = np.maximum(g, np.float32(0.0)).astype(np.float32)
+    h = (r * r).astype(np.float32)
+    if u_bits is not None:
+        h = (h * bf16_bits_to_f32(u_bits)).astype(np.float32)
+    return h
+
+
 # ---------------------------------------------------------------------------
 # [P2] eq. (3): integer matmul and rescale
 # ---------------------------------------------------------------------------
@@ -341,6 +384,28 @@ def forward(x_bits: np.ndarray, W: np.ndarray, bits: int = 8):
         "gamma": gamma,
         "codes": codes,
         "packed": pack_ternary(codes) if codes.shape[1] % 16 == 0 else None,
+        "q": q,
+        "s": s,
+        "acc": acc,
+        "y64": y64,
+        "y32": y32,
+        "Y": round_to_bf16_bits(y32),
+    }
+
+
+def forward_relu2(g_bits: np.ndarray, u_bits: np.ndarray | None, W: np.ndarray, bits: int = 8):
+    """Down projection of the squared-ReLU feed-forward block: BitLinear on
+    h = relu2_input(g, u).  Same dict as ``forward`` plus h."""
+    h = relu2_input(g_bits, u_bits)
+    gamma = absmean_scale(W)
+    codes = ternary_codes(W, gamma)
+    q, s = act_quant_values(h, bits)
+    acc = matmul_i32(q, codes)
+    y64, y32 = rescale(acc, gamma, s)
+    return {
+        "h": h,
+        "gamma": gamma,
+        "codes": codes,
         "q": q,
         "s": s,
         "acc": acc,

@@ -393,3 +393,71 @@ def test_zero_row_and_zero_weights():
     assert np.all(r["codes"] == 0)
     assert np.all(r["acc"] == 0)
     assert np.all(r["Y"] == 0)
+
+
+# ---------------------------------------------------------------------------
+# P3 section "2. Squared ReLU Activation": the down projection's input
+# ---------------------------------------------------------------------------
+
+def test_relu2_hand_cases():
+    # ReLU^2(x) = max(0, x)^2; gated: times the up output
+    g = to_bf16_bits_exact([[-3.0, -0.0, 0.5, 3.0, 1.5]])
+    u = to_bf16_bits_exact([[7.0, 2.0, -4.0, -1.5, 0.25]])
+    h = o.relu2_input(g)
+    assert h.dtype == np.float32
+    assert h.tolist() == [[0.0, 0.0, 0.25, 9.0, 2.25]]
+    hg = o.relu2_input(g, u)
+    assert hg.tolist() == [[0.0, 0.0, -1.0, -13.5, 0.5625]]
+
+
+def test_relu2_is_exact_for_bf16_inputs():
+    # bf16 has 8 significant bits: g^2 (16 bits) and g^2 * u (24 bits) are
+    # exact in fp32, so h equals the exact rational product
+    rng = np.random.default_rng(21)
+    vals = rng.standard_normal((4, 64)).astype(np.float32) * 3
+    ub = rng.standard_normal((4, 64)).astype(np.float32)
+    gb = (vals.view(np.uint32) >> 16).astype(np.uint16)
+    uu = (ub.view(np.uint32) >> 16).astype(np.uint16)
+    h = o.relu2_input(gb, uu)
+    g = gb.astype(np.uint32) << 16
+    u = uu.astype(np.uint32) << 16
+    for i in range(4):
+        for k in range(64):
+            gf = Fraction(float(np.uint32(g[i, k]).view(np.float32)))
+            uf = Fraction(float(np.uint32(u[i, k]).view(np.float32)))
+            exact = (max(gf, Fraction(0)) ** 2) * uf
+            assert Fraction(float(h[i, k])) == exact
+
+
+def test_act_quant_values_hand_case_and_agrees_on_bf16():
+    # h = [0.5, -2, 1]: a = 2, s = 63.5, h*s = [31.75, -127, 63.5] -> 32, -127, 64 (tie to even)
+    q, s = o.act_quant_values(np.array([[0.5, -2.0, 1.0]], np.float32))
+    assert s[0] == np.float32(63.5)
+    assert q.tolist() == [[32, -127, 64]]
+    # on bf16-representable values it is the (separately pinned) act_quant
+    rng = np.random.default_rng(5)
+    xb = (rng.standard_normal((6, 128)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    for bits in (8, 4):
+        q1, s1 = o.act_quant(xb, bits)
+        q2, s2 = o.act_quant_values(o.bf16_bits_to_f32(xb), bits)
+        assert np.array_equal(q1, q2) and np.array_equal(s1.view(np.uint32), s2.view(np.uint32))
+
+
+def test_forward_relu2_matches_dequantized_brute_force():
+    # y = sum_k c[n,k] * q[m,k] * gamma / s_m, against exact rationals
+    rng = np.random.default_rng(8)
+    M, K, N = 3, 64, 5
+    gb = (rng.standard_normal((M, K)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    out = o.forward_relu2(gb, None, W)
+    h = out["h"]
+    assert np.all(h >= 0) and np.any(h == 0)     # ReLU^2 is sparse and non-negative
+    for m in range(M):
+        a = max(Fraction(float(v)) for v in h[m])
+        for n in range(N):
+            acc = sum(int(out["codes"][n, k]) * int(out["q"][m, k]) for k in range(K))
+            assert acc == out["acc"][m, n]
+            exact = Fraction(acc) * Fraction(float(out["gamma"])) / Fraction(float(out["s"][m]))
+            assert abs(float(exact) - out["y64"][m, n]) <= 1e-12 * max(1.0, abs(float(exact)))
+        # s_m is 127 / max_k h, correctly rounded to fp32
+        assert out["s"][m] == o.round_rational_to_f32(127 * a.denominator, a.numerator)
