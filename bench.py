@@ -298,6 +298,51 @@ class GpuWorkload:
         for gi in range(len(self.groups)):
             self.run_group(gi, r)
 
+class FfnWorkload(GpuWorkload):
+    """The 2B decode feed-forward block as a chain: up and gate in one grouped
+    launch, then the down projection on max(0, gate)^2 * up formed and
+    quantised in the down kernel's prologue (its input is the previous
+    launch's output)."""
+
+    def __init__(self, rotations, seed=0, device="cuda"):
+        super().__init__("decode_2b", rotations, seed, device)
+        up, gate, down = self.layers
+        self.groups = [[0, 1], [2]]
+        self.bytes_per_step = (algorithmic_bytes(1, up["L"].K, up["L"].N)
+                               + algorithmic_bytes(1, gate["L"].K, gate["L"].N) - 2 * gate["L"].K
+                               + algorithmic_bytes(1, down["L"].K, down["L"].N) + 2 * down["L"].K)
+        self.launches_per_step = 2
+
+    def step(self, i):
+        from bitlinear_bl_forward_b200 import bl
+        r = i % self.rotations
+        self.run_group(0, r)
+        up, gate, down = self.layers
+        Wp, gamma = down["copies"][r]
+        bl.bl_forward_relu2(gate["Y"], up["Y"], Wp, gamma, down["L"].N, self.w.bits, out=down["Y"],
+                            workspace=down["ws"])
+
+
+def time_quantize_weights(N=28672, K=8192, reps=5):
+    """bl_quantize_weights on a 70B-class layer: GB/s of fp32 weights read
+    (offline step, not part of the forward metric)."""
+    import torch
+    from bitlinear_bl_forward_b200 import bl
+    W = torch.randn(N, K, device="cuda") * 0.01
+    Wp, g = bl.bl_quantize_weights(W)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        bl.bl_quantize_weights(W)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / reps
+    del W, Wp, g
+    torch.cuda.empty_cache()
+    return {"workload": "quantize_weights_70b", "N": N, "K": K, "ms": ms, "GB/s (fp32 W read)": N * K * 4 / ms / 1e6}
+
+
 def capture(wl, nsteps, start):
     import torch
     g = torch.cuda.CUDAGraph()
@@ -526,6 +571,19 @@ def secondary(args, ctx, peaks):
         out.append(ent)
         del wl
         torch.cuda.empty_cache()
+    if not args.secondary or "ffn_2b_decode" in args.secondary.split(","):
+        # the decode feed-forward chain (up+gate grouped, then down on the fused squared ReLU)
+        steps = 20000
+        wl = FfnWorkload(20)
+        ms, _ = time_workload(wl, steps, 3, ctx, sample_clocks=False)
+        gbs = wl.bytes_per_step * steps / (ms / 1e3) / 1e9
+        out.append({"workload": "ffn_2b_decode", "M": 1, "ms_per_step": ms / steps, "GB/s": gbs,
+                    "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps,
+                    "note": "down input = max(0, gate)^2 * up of the same step, formed in the down kernel"})
+        del wl
+        torch.cuda.empty_cache()
+    if not args.secondary or "quantize_weights_70b" in args.secondary.split(","):
+        out.append(time_quantize_weights())
     return out
 
 

@@ -40,6 +40,9 @@ SIGNATURES = {
     "bl_forward_noalloc": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p]),
     "bl_forward_grouped_workspace_bytes": (_sz, [_int, _p, _int]),
     "bl_forward_grouped": (_int, [_int, _p, _int, _p, _sz, _p]),
+    "bl_forward_relu2_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
+    "bl_forward_relu2": (_int, [_p, _p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
+    "bl_quant_act_relu2": (_int, [_p, _p, _i64, _i64, _int, _p, _p, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
@@ -222,6 +225,45 @@ def bl_forward_grouped(problems, bits: int = 8, outs=None, workspace: torch.Tens
     _check(lib().bl_forward_grouped(len(problems), arr, bits, ws.data_ptr() if ws is not None else None,
                                     ws.numel() if ws is not None else 0, _stream()), "bl_forward_grouped")
     return outs
+
+
+def bl_forward_relu2_workspace_bytes(M: int, K: int, N: int, bits: int = 8) -> int:
+    return int(lib().bl_forward_relu2_workspace_bytes(M, K, N, bits))
+
+
+def bl_forward_relu2(G: torch.Tensor, U: torch.Tensor | None, Wp: torch.Tensor, gamma: torch.Tensor, N: int,
+                     bits: int = 8, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Down projection of the squared-ReLU feed-forward: input max(0, G)^2
+    (times U when given), bf16 [M, K] each -> bf16 [M, N]."""
+    M, K = G.shape
+    pg_in = _dev(G, torch.bfloat16, "G")
+    pu = _dev(U, torch.bfloat16, "U") if U is not None else None
+    if U is not None and tuple(U.shape) != (M, K):
+        raise ValueError("U must have the shape of G")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=G.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    ws = workspace
+    if ws is None:
+        ws = _workspace(bl_forward_relu2_workspace_bytes(M, K, N, bits), G.device)
+    _check(lib().bl_forward_relu2(pg_in, pu, M, K, N, pw, pg, bits, py,
+                                  ws.data_ptr() if ws is not None else None,
+                                  ws.numel() if ws is not None else 0, _stream()), "bl_forward_relu2")
+    return Y
+
+
+def bl_quant_act_relu2(G: torch.Tensor, U: torch.Tensor | None, bits: int = 8):
+    """max(0, G)^2 (times U) quantised per token -> (int8 codes [M, K], scale fp32 [M])."""
+    M, K = G.shape
+    pg_in = _dev(G, torch.bfloat16, "G")
+    pu = _dev(U, torch.bfloat16, "U") if U is not None else None
+    Xq = torch.empty((M, K), dtype=torch.int8, device=G.device)
+    s = torch.empty(M, dtype=torch.float32, device=G.device)
+    _check(lib().bl_quant_act_relu2(pg_in, pu, M, K, bits, Xq.data_ptr(), s.data_ptr(), _stream()),
+           "bl_quant_act_relu2")
+    return Xq, s
 
 
 def bl_matmul_i32(Xq: torch.Tensor, Wp: torch.Tensor, N: int) -> torch.Tensor:

@@ -196,9 +196,9 @@ bl_status launch_gemv2_cpl(int cpl, const bl::G2Table& tab, int grid, int x_is_i
 template <int WPL>
 constexpr int g3_warps() { return BL_G3_WARPS; }
 
-template <int WPL>
+template <int WPL, bool RELU2>
 bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode, cudaStream_t stream) {
-  auto kern = bl::gemv3_kernel<WPL, g3_warps<WPL>()>;
+  auto kern = bl::gemv3_kernel<WPL, g3_warps<WPL>(), RELU2>;
   static std::atomic<uint64_t> done{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
@@ -232,9 +232,12 @@ bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int 
 // words of 16 weights per lane: K / 512 rounded up (K <= 8192)
 bl_status launch_gemv3_wpl(int wpl, const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode,
                            cudaStream_t stream) {
+  const bool relu2 = x_is_i8 == bl::kInRelu2 || x_is_i8 == bl::kInRelu2Gated;
   switch (wpl) {
 #define BL_G3_CASE(n) \
-  case n: return launch_gemv3_table<n>(tab, grid, x_is_i8, Q, out_mode, stream);
+  case n:                                                                                     \
+    return relu2 ? launch_gemv3_table<n, true>(tab, grid, x_is_i8, Q, out_mode, stream)       \
+                 : launch_gemv3_table<n, false>(tab, grid, x_is_i8, Q, out_mode, stream);
     BL_G3_CASE(1) BL_G3_CASE(2) BL_G3_CASE(3) BL_G3_CASE(4) BL_G3_CASE(5) BL_G3_CASE(6) BL_G3_CASE(7) BL_G3_CASE(8)
     BL_G3_CASE(9) BL_G3_CASE(10) BL_G3_CASE(11) BL_G3_CASE(12) BL_G3_CASE(13) BL_G3_CASE(14) BL_G3_CASE(15)
     BL_G3_CASE(16)
@@ -256,7 +259,7 @@ constexpr int kDecodeKernel = BL_DECODE_KERNEL;
 // problem gets CTAs in proportion to its weight bytes (at least one, at most
 // one per row), and the launch has exactly one CTA per SM when the rows allow.
 // Returns the grid size.
-int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms) {
+int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, const void* U) {
   std::memset(tab, 0, sizeof(*tab));
   double total = 0.0;
   int64_t rows = 0;
@@ -295,7 +298,7 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
   for (int i = 0; i < n; ++i) {
     const bl_linear& p = *probs[i];
     const int rows_per_cta = static_cast<int>((p.N + c[i] - 1) / c[i]);
-    tab->p[i] = bl::G2Problem{p.X, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
+    tab->p[i] = bl::G2Problem{p.X, U, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
                               rows_per_cta, grid, c[i]};
     grid += c[i];
   }
@@ -305,8 +308,10 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
 
 // Launch one-token problems that share a kernel variant (at most
 // kG2MaxProblems).
-bl_status launch_decode(const bl_linear* const* probs, int n, int x_is_i8, int Q, int out_mode,
-                        cudaStream_t stream) {
+// in_mode: bl::InMode of the token input; U: the up projection's output in
+// the gated squared-ReLU mode (shared by every problem of the call).
+bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q, int out_mode, cudaStream_t stream,
+                        const void* U = nullptr) {
   if (n <= 0) return BL_OK;
   const int sms = num_sms();
   bl::G2Table tab;
@@ -331,15 +336,15 @@ bl_status launch_decode(const bl_linear* const* probs, int n, int x_is_i8, int Q
       if (c < 1) c = 1;
       const int rows_per_cta = static_cast<int>((p.N + c - 1) / c);
       c = static_cast<int>((p.N + rows_per_cta - 1) / rows_per_cta);
-      tab.p[i] = bl::G2Problem{p.X, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N), rows_per_cta,
-                               grid, c};
+      tab.p[i] = bl::G2Problem{p.X, U, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
+                               rows_per_cta, grid, c};
       grid += c;
     }
     tab.count = n;
-    return launch_gemv2_cpl((maxK / 64 + 31) / 32, tab, grid, x_is_i8, Q, out_mode, stream);
+    return launch_gemv2_cpl((maxK / 64 + 31) / 32, tab, grid, in_mode, Q, out_mode, stream);
   }
-  const int grid = fill_decode_table(&tab, probs, n, sms);
-  return launch_gemv3_wpl((maxK + 511) / 512, tab, grid, x_is_i8, Q, out_mode, stream);
+  const int grid = fill_decode_table(&tab, probs, n, sms, U);
+  return launch_gemv3_wpl((maxK + 511) / 512, tab, grid, in_mode, Q, out_mode, stream);
 }
 
 // Single one-token problem.
@@ -844,6 +849,71 @@ bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, voi
     if (st != BL_OK) return st;
   }
   return BL_OK;
+}
+
+size_t relu2_ws_bytes(int64_t M, int64_t K) {
+  if (M == 1 && K <= 8192) return 0;   // the decode kernels quantise in their prologue
+  return align_up(static_cast<size_t>(M) * K, 256) + 2 * align_up(static_cast<size_t>(M) * 4, 256);
+}
+
+size_t bl_forward_relu2_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+  (void)bits;
+  if (check_shape_nk(N, K) != BL_OK || check_m(M, K) != BL_OK || M == 0) return 0;
+  return relu2_ws_bytes(M, K);
+}
+
+bl_status bl_quant_act_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int bits, int8_t* Xq,
+                             float* scale, cudaStream_t stream) {
+  if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
+  bl_status st = check_m(M, K);
+  if (st != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (M == 0) return BL_OK;
+  if (!G || !Xq || !scale) return BL_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(Xq) || (U && !aligned16(U))) return BL_ERR_ALIGNMENT;
+  bl::act_quant_relu2_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+      G, U, U != nullptr, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr);
+  return last_cuda();
+}
+
+bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
+                           const float* gamma, int bits, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (M == 0) return BL_OK;
+  if (!G || !Wp || !gamma || !Y) return BL_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(Wp) || (U && !aligned16(U))) return BL_ERR_ALIGNMENT;
+  const size_t need = relu2_ws_bytes(M, K);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+  }
+  const int Q = bits == 8 ? 127 : 7;
+  if (need == 0) {   // one token: squared ReLU and quantisation in the decode kernel's prologue
+    bl_linear p;
+    p.X = G;
+    p.M = 1;
+    p.K = K;
+    p.N = N;
+    p.Wp = Wp;
+    p.gamma = gamma;
+    p.Y = Y;
+    const bl_linear* pp = &p;
+    return launch_decode(&pp, 1, U ? bl::kInRelu2Gated : bl::kInRelu2, Q, bl::kOutBF16, stream, U);
+  }
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  int8_t* Xq = reinterpret_cast<int8_t*>(base);
+  float* s = reinterpret_cast<float*>(base + align_up(static_cast<size_t>(M) * K, 256));
+  int* R = reinterpret_cast<int*>(base + align_up(static_cast<size_t>(M) * K, 256) +
+                                  align_up(static_cast<size_t>(M) * 4, 256));
+  bl::act_quant_relu2_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+      G, U, U != nullptr, static_cast<int>(K), Q, Xq, s, R);
+  if ((st = last_cuda()) != BL_OK) return st;
+  return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16,
+                   0, stream);
 }
 
 bl_status bl_device_status(int clear, int* site) {

@@ -51,6 +51,47 @@ __device__ __forceinline__ uint2 quant8_bf16(uint4 v, float s, int Q, int& sum) 
   return make_uint2(lo, hi);
 }
 
+// Input modes of the token prologues: bf16 activations, int8 codes given
+// directly, or the squared-ReLU feed-forward input ("BitNet 2B4T Guide",
+// section "2. Squared ReLU Activation") h = max(0, g)^2 of the gate
+// projection's bf16 output g, optionally times the up projection's output u.
+enum InMode : int { kInBF16 = 0, kInI8 = 1, kInRelu2 = 2, kInRelu2Gated = 3 };
+
+// h for 8 consecutive elements (fp32; exact for bf16 g and u).
+__device__ __forceinline__ void relu2_8(uint4 g, uint4 u, bool gated, float (&h)[8]) {
+  const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+  const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float r0 = fmaxf(bf16_lo(gw[i]), 0.f), r1 = fmaxf(bf16_hi(gw[i]), 0.f);
+    h[2 * i] = __fmul_rn(r0, r0);
+    h[2 * i + 1] = __fmul_rn(r1, r1);
+    if (gated) {
+      h[2 * i] = __fmul_rn(h[2 * i], bf16_lo(uw[i]));
+      h[2 * i + 1] = __fmul_rn(h[2 * i + 1], bf16_hi(uw[i]));
+    }
+  }
+}
+
+__device__ __forceinline__ float absmax8_f32(const float (&h)[8]) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(h[i]));
+  return a;
+}
+
+// 8 fp32 values -> 8 codes (two 32-bit words) and their sum.
+__device__ __forceinline__ uint2 quant8_f32(const float (&h)[8], float s, int Q, int& sum) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = quant1(h[i], s, Q);
+  const uint32_t lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+  const uint32_t hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
+  return make_uint2(lo, hi);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -149,6 +190,55 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uin
   }
   for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
     qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
+  const int wsum = __reduce_add_sync(0xffffffffu, sum);
+  if (lane == 0) s_sum[warp] = wsum;
+  __syncthreads();
+  if (t == 0) {
+    int tot = 0;
+#pragma unroll
+    for (int w = 0; w < W; ++w) tot += s_sum[w];
+    if (s_out) s_out[m] = s;
+    if (R_out) R_out[m] = tot;
+  }
+}
+
+// Squared-ReLU feed-forward input, quantised per token: one CTA per row;
+// pass 1 takes the absmax of h over the row, pass 2 recomputes h (the row is
+// in L1/L2 by then) and writes the codes.  G, U: bf16 [M, K] (U only when
+// gated).
+__global__ void __launch_bounds__(kActRowThreads) act_quant_relu2_kernel(const uint16_t* __restrict__ G,
+                                                                         const uint16_t* __restrict__ U, int gated,
+                                                                         int K, int Q, int8_t* __restrict__ Xq,
+                                                                         float* __restrict__ s_out,
+                                                                         int* __restrict__ R_out) {
+  constexpr int W = kActRowThreads / 32;
+  __shared__ uint32_t s_max[W];
+  __shared__ int s_sum[W];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const size_t m = blockIdx.x;
+  const uint4* gr = reinterpret_cast<const uint4*>(G + m * K);
+  const uint4* ur = gated ? reinterpret_cast<const uint4*>(U + m * K) : nullptr;
+  const int nch = K >> 3;
+  float amax = 0.f;
+  for (int c = t; c < nch; c += kActRowThreads) {
+    float h[8];
+    relu2_8(__ldg(gr + c), gated ? __ldg(ur + c) : make_uint4(0, 0, 0, 0), gated != 0, h);
+    amax = fmaxf(amax, absmax8_f32(h));
+  }
+  const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+  if (lane == 0) s_max[warp] = wmax;
+  __syncthreads();
+  uint32_t bmax = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) bmax = max(bmax, s_max[w]);
+  const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
+  uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
+  int sum = 0;
+  for (int c = t; c < nch; c += kActRowThreads) {
+    float h[8];
+    relu2_8(__ldg(gr + c), gated ? __ldg(ur + c) : make_uint4(0, 0, 0, 0), gated != 0, h);
+    qr[c] = quant8_f32(h, s, Q, sum);
+  }
   const int wsum = __reduce_add_sync(0xffffffffu, sum);
   if (lane == 0) s_sum[warp] = wsum;
   __syncthreads();

@@ -499,6 +499,7 @@ __global__ void __launch_bounds__(THREADS, MINB)
 // decode): CTAs [cta_begin, next cta_begin) of the grid work on problem i.
 struct G2Problem {
   const void* X;
+  const void* U;      // squared-ReLU gated mode: the up projection's output (else unused)
   const uint8_t* Wp;
   const float* gamma;
   void* Y;
@@ -522,10 +523,11 @@ constexpr int kG2SmemBytes = kG2Stages * kG2StageBytes + 2048;
 
 template <int MT, int CPL>
 __global__ void __launch_bounds__(kG2Threads, 1)
-    gemv2_kernel(const __grid_constant__ G2Table tab, int x_is_i8, int Q, int out_mode, unsigned long long limit_ns) {
+    gemv2_kernel(const __grid_constant__ G2Table tab, int in_mode, int Q, int out_mode, unsigned long long limit_ns) {
   int pi = 0;
   while (pi + 1 < tab.count && static_cast<int>(blockIdx.x) >= tab.p[pi + 1].cta_begin) ++pi;
   const void* __restrict__ X = tab.p[pi].X;
+  const void* __restrict__ Up = tab.p[pi].U;
   const uint8_t* __restrict__ Wp = tab.p[pi].Wp;
   const float* __restrict__ gamma_p = tab.p[pi].gamma;
   void* __restrict__ Y = tab.p[pi].Y;
@@ -590,15 +592,19 @@ __global__ void __launch_bounds__(kG2Threads, 1)
   // ---------------- consumers: token quantisation ----------------
   constexpr int CT = kG2ConsumerWarps * 32;
   constexpr int U = (8192 / 8 + CT - 1) / CT;
+  const bool x_is_i8 = in_mode == kInI8;
+  const bool relu2 = in_mode == kInRelu2 || in_mode == kInRelu2Gated;
+  const bool gated = in_mode == kInRelu2Gated;
   const int nch = x_is_i8 ? (K >> 4) : (K >> 3);
-  uint4 xv[MT][U];
+  uint4 xv[MT][U], uv[MT][U];
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = threadIdx.x + CT * u;
-      xv[m][u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + static_cast<size_t>(m) * nch + c)
-                           : make_uint4(0, 0, 0, 0);
+      const size_t o = static_cast<size_t>(m) * nch + c;
+      xv[m][u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + o) : make_uint4(0, 0, 0, 0);
+      uv[m][u] = (gated && c < nch) ? __ldg(static_cast<const uint4*>(Up) + o) : make_uint4(0, 0, 0, 0);
     }
   const float gamma = (out_mode == kOutI32) ? 1.f : __ldg(gamma_p);
   int rsum[MT];
@@ -613,7 +619,15 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     for (int m = 0; m < MT; ++m) {
       float amax = 0.f;
 #pragma unroll
-      for (int u = 0; u < U; ++u) amax = fmaxf(amax, absmax8_bf16(xv[m][u]));
+      for (int u = 0; u < U; ++u) {
+        if (relu2) {
+          float h[8];
+          relu2_8(xv[m][u], uv[m][u], gated, h);
+          amax = fmaxf(amax, absmax8_f32(h));
+        } else {
+          amax = fmaxf(amax, absmax8_bf16(xv[m][u]));
+        }
+      }
       const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
       if (lane == 0) s_red_f[m][warp] = wmax;
     }
@@ -630,7 +644,17 @@ __global__ void __launch_bounds__(kG2Threads, 1)
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int c = threadIdx.x + CT * u;
-        if (c < nch) *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = quant8_bf16(xv[m][u], sc[m], Q, rsum[m]);
+        if (c < nch) {
+          uint2 qv;
+          if (relu2) {
+            float h[8];
+            relu2_8(xv[m][u], uv[m][u], gated, h);
+            qv = quant8_f32(h, sc[m], Q, rsum[m]);
+          } else {
+            qv = quant8_bf16(xv[m][u], sc[m], Q, rsum[m]);
+          }
+          *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = qv;
+        }
       }
     }
   } else {

@@ -110,13 +110,17 @@ __device__ __forceinline__ void g3_rows(const uint8_t* sbase, int rr, int rows, 
   }
 }
 
-template <int WPL, int CW>
+// RELU2: the token is the squared-ReLU feed-forward input (in_mode kInRelu2
+// or kInRelu2Gated); otherwise bf16 activations or int8 codes.  A template
+// parameter so that the plain path carries no code for it.
+template <int WPL, int CW, bool RELU2>
 __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
-    gemv3_kernel(const __grid_constant__ G2Table tab, int x_is_i8, int Q, int out_mode, unsigned long long limit_ns) {
+    gemv3_kernel(const __grid_constant__ G2Table tab, int in_mode, int Q, int out_mode, unsigned long long limit_ns) {
   constexpr bool ACT_SMEM = G3Cfg<WPL, CW>::kActSmem;
   int pi = 0;
   while (pi + 1 < tab.count && static_cast<int>(blockIdx.x) >= tab.p[pi + 1].cta_begin) ++pi;
   const void* __restrict__ X = tab.p[pi].X;
+  const void* __restrict__ Up = tab.p[pi].U;
   const uint8_t* __restrict__ Wp = tab.p[pi].Wp;
   const float* __restrict__ gamma_p = tab.p[pi].gamma;
   void* __restrict__ Y = tab.p[pi].Y;
@@ -195,12 +199,16 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
   pdl_wait();
   constexpr int CT = CW * 32;
   constexpr int U = (kG3MaxK / 8 + CT - 1) / CT;
+  const bool x_is_i8 = in_mode == kInI8;
+  constexpr bool relu2 = RELU2;
+  const bool gated = RELU2 && in_mode == kInRelu2Gated;
   const int nch = x_is_i8 ? (K >> 4) : (K >> 3);
-  uint4 xv[U];
+  uint4 xv[U], uv[RELU2 ? U : 1];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int c = threadIdx.x + CT * u;
     xv[u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + c) : make_uint4(0, 0, 0, 0);
+    if constexpr (RELU2) uv[u] = (gated && c < nch) ? __ldg(static_cast<const uint4*>(Up) + c) : make_uint4(0, 0, 0, 0);
   }
   const float gamma = (out_mode == kOutI32) ? 1.f : __ldg(gamma_p);
   int rsum = 0;
@@ -208,7 +216,15 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
   if (!x_is_i8) {
     float amax = 0.f;
 #pragma unroll
-    for (int u = 0; u < U; ++u) amax = fmaxf(amax, absmax8_bf16(xv[u]));
+    for (int u = 0; u < U; ++u) {
+      if constexpr (RELU2) {
+        float h[8];
+        relu2_8(xv[u], uv[u], gated, h);
+        amax = fmaxf(amax, absmax8_f32(h));
+      } else {
+        amax = fmaxf(amax, absmax8_bf16(xv[u]));
+      }
+    }
     const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
     if (lane == 0) s_red_f[warp] = wmax;
     named_bar_sync(1, CT);
@@ -222,7 +238,15 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = threadIdx.x + CT * u;
-      if (c < nch) *reinterpret_cast<uint2*>(&s_act[8 * c]) = quant8_bf16(xv[u], sc, Q, rsum);
+      if (c < nch) {
+        if constexpr (RELU2) {
+          float h[8];
+          relu2_8(xv[u], uv[u], gated, h);
+          *reinterpret_cast<uint2*>(&s_act[8 * c]) = quant8_f32(h, sc, Q, rsum);
+        } else {
+          *reinterpret_cast<uint2*>(&s_act[8 * c]) = quant8_bf16(xv[u], sc, Q, rsum);
+        }
+      }
     }
   } else {
 #pragma unroll

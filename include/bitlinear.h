@@ -206,6 +206,32 @@ BL_API size_t bl_forward_grouped_workspace_bytes(int count, const bl_linear* pro
 BL_API bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, void* workspace,
                                     size_t workspace_bytes, cudaStream_t stream);
 
+
+/*
+ * Squared-ReLU feed-forward: the down projection's input is formed from the
+ * gate projection's output ("BitNet 2B4T Guide: Scaling Native 1.58-Bit
+ * LLMs", section "2. Squared ReLU Activation", ReLU^2(x) = max(0, x)^2, and
+ * the page's feed-forward module, which feeds ReLU^2 of the gate projection
+ * to the down projection) and quantised in the same kernel:
+ *   h[m,k] = f32( max(0, G[m,k])^2 )                    (U == NULL)
+ *   h[m,k] = f32( f32(max(0, G[m,k])^2) * U[m,k] )      (gated, U != NULL)
+ * (exact for bf16 G and U), then exactly the per-token quantisation of
+ * bl_quant_act applied to the fp32 h, and the rest of bl_forward.
+ * G, U: bf16 bits [M, K], 16-byte aligned (U may be NULL).  Wp, gamma, Y and
+ * the workspace as in bl_forward (workspace: bl_forward_relu2_workspace_bytes,
+ * 0 when M == 1 and K <= 8192: the decode kernel forms h in its prologue).
+ * The ordering rule of bl_forward applies; G and U may be written by the
+ * preceding kernel of the stream (they are read after the dependency wait).
+ */
+BL_API size_t bl_forward_relu2_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+BL_API bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int64_t N,
+                                  const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+/* Test export: the quantisation step of bl_forward_relu2 alone (codes int8
+ * [M, K] and scales fp32 [M], as bl_quant_act). */
+BL_API bl_status bl_quant_act_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int bits, int8_t* Xq,
+                                    float* scale, cudaStream_t stream);
+
 /* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
 BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
 

@@ -151,3 +151,22 @@ def test_grouped_validation(L):
     assert L.bl_forward_grouped(2, arr, 8, None, 0, None) == WS
     assert L.bl_forward_grouped_workspace_bytes(2, arr, 8) >= 4 * 64
     assert L.bl_forward_grouped(0, arr, 8, None, 0, None) == OK
+
+
+def test_relu2_validation(L):
+    need = L.bl_forward_relu2_workspace_bytes(4, 64, 8, 8)
+    assert need >= 4 * 64
+    assert L.bl_forward_relu2_workspace_bytes(1, 2560, 6912, 8) == 0        # fused into the decode kernel
+    assert L.bl_forward_relu2_workspace_bytes(2, 2560, 6912, 8) > 0         # via the tensor-core path
+    assert L.bl_forward_relu2_workspace_bytes(1, 16384, 64, 8) > 0          # K beyond the decode kernels
+    args = (A, None, 4, 64, 8, A, A, 8, A, A, 1 << 20, None)
+    assert L.bl_forward_relu2(A, None, 4, 60, 8, A, A, 8, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_forward_relu2(None, None, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == INVALID
+    assert L.bl_forward_relu2(A, U, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == ALIGN     # misaligned U
+    assert L.bl_forward_relu2(A, None, 4, 64, 8, A, A, 3, A, A, 1 << 20, None) == UNSUP
+    assert L.bl_forward_relu2(A, None, 4, 64, 8, A, A, 8, A, None, 0, None) == WS
+    assert L.bl_forward_relu2(None, None, 0, 64, 8, None, None, 8, None, None, 0, None) == OK
+    assert L.bl_quant_act_relu2(A, None, 4, 65, 8, A, A, None) == SHAPE
+    assert L.bl_quant_act_relu2(A, A, 4, 64, 2, A, A, None) == UNSUP
+    assert L.bl_quant_act_relu2(A, U, 4, 64, 8, A, A, None) == ALIGN
+    assert len(args) == 12

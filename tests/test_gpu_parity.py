@@ -300,3 +300,58 @@ def test_grouped_mixed_shapes_fall_back_to_sequential():
     outs3 = bl.bl_forward_grouped(probs3)
     for a, b in zip(outs3, singles3):
         assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# squared-ReLU feed-forward input ("BitNet 2B4T Guide", section 2)
+# ---------------------------------------------------------------------------
+
+def relu2_inputs(M, K, N, seed):
+    G, W = random_case(M, K, N, seed=seed)
+    U, _ = random_case(M, K, 8, seed=seed + 7)
+    return G, U, W
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (3, 192), (16, 2560), (5, 6912), (2, 8192)])
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_quant_act_relu2_bit_exact(M, K, gated, bits):
+    G, U, _ = relu2_inputs(M, K, 8, seed=M * 31 + K)
+    h = o.relu2_input(G, U if gated else None)
+    q, s = o.act_quant_values(h, bits)
+    qd, sd = bl.bl_quant_act_relu2(x_to_dev(G), x_to_dev(U) if gated else None, bits)
+    assert np.array_equal(qd.cpu().numpy(), q)
+    assert np.array_equal(sd.cpu().numpy().view(np.uint32), s.view(np.uint32))
+
+
+RELU2_CASES = [(1, 2560, 700), (1, 6912, 2560), (1, 8192, 2100), (1, 8192, 8192), (1, 16384, 64),
+               (2, 320, 130), (3, 256, 512), (17, 320, 130), (130, 256, 300)]
+
+
+@pytest.mark.parametrize("M,K,N", RELU2_CASES)
+@pytest.mark.parametrize("gated", [False, True])
+def test_forward_relu2_parity(M, K, N, gated):
+    # one token: the decode kernels (resident for small layers, streaming for
+    # 8192 x 8192) form h in their prologue; otherwise the quantiser + GEMM
+    G, U, W = relu2_inputs(M, K, N, seed=M * 1000 + K + N)
+    ref = o.forward_relu2(G, U if gated else None, W)
+    Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+    Yd = bl.bl_forward_relu2(x_to_dev(G), x_to_dev(U) if gated else None, Wp, gd, N)
+    torch.cuda.synchronize()
+    d = bf16_ulp_distance(bf16_dev_to_bits(Yd), ref["Y"])
+    assert d.max() <= BF16_ULP_TOL, f"bf16 ulp distance {d.max()}"
+    # the same arithmetic as the oracle: almost every output is bit-identical
+    assert np.mean(d == 0) > 0.99
+
+
+def test_forward_relu2_bits4_and_zero_rows():
+    M, K, N = 4, 512, 96
+    G, U, W = relu2_inputs(M, K, N, seed=77)
+    G[1] = 0x8000          # -0.0 everywhere: relu^2 is all zero -> zero codes, Y = 0
+    G[2] = 0xBF80          # -1.0 everywhere: also all zero
+    for bits in (8, 4):
+        ref = o.forward_relu2(G, U, W, bits)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        Yd = bf16_dev_to_bits(bl.bl_forward_relu2(x_to_dev(G), x_to_dev(U), Wp, gd, N, bits))
+        assert bf16_ulp_distance(Yd, ref["Y"]).max() <= BF16_ULP_TOL
+        assert np.all(Yd[1] == 0) and np.all(Yd[2] == 0)
