@@ -72,11 +72,13 @@ __all__ = [
     "unpack_ternary",
     "act_quant",
     "act_quant_values",
+    "act_quant_per_tensor",
     "relu2_input",
     "matmul_i32",
     "rescale",
     "forward",
     "forward_relu2",
+    "forward_ex",
 ]
 
 # Floor used for both scales (pages' code listings clamp(min=1e-5)).
@@ -312,6 +314,24 @@ def act_quant_values(x: np.ndarray, bits: int = 8):
     return q, s
 
 
+def act_quant_per_tensor(x_bits: np.ndarray, bits: int = 8):
+    """The per-tensor variant ([P3] section "1. The BitLinear Operator"
+    quantises with one absmax over the whole activation tensor): a = max over
+    every |x|, s = Q / max(a, 1e-5) (fp32), q = clip(rint(f32(x * s)), -Q-1, Q).
+    Returns (q int8 [M, K], s fp32 [M], every entry the same scale)."""
+    if bits not in QMAX:
+        raise ValueError("bits must be 8 or 4")
+    Q = QMAX[bits]
+    x = bf16_bits_to_f32(x_bits)
+    if x.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    a = np.float32(np.max(np.abs(x))) if x.size else np.float32(0.0)
+    s1 = np.float32(np.float32(Q) / np.maximum(a, EPS))
+    t = (x * s1).astype(np.float32)
+    q = np.clip(np.rint(t), -Q - 1, Q).astype(np.int8)
+    return q, np.full(x.shape[0], s1, dtype=np.float32)
+
+
 # ---------------------------------------------------------------------------
 # [P3] section 2: squared ReLU between the feed-forward projections
 # ---------------------------------------------------------------------------
@@ -413,3 +433,22 @@ def forward_relu2(g_bits: np.ndarray, u_bits: np.ndarray | None, W: np.ndarray, 
         "y32": y32,
         "Y": round_to_bf16_bits(y32),
     }
+
+
+def forward_ex(x_bits: np.ndarray, W: np.ndarray, bits: int = 8, per_tensor: bool = False,
+               bias: np.ndarray | None = None):
+    """``forward`` with the two variants the pages print: per-tensor
+    activation scale ([P3] section 1) and an output bias added after the
+    rescale ([P2] BitLinear module, ``bias`` argument): y32 = f32(f32(f32(acc)
+    * f32(gamma / s_m)) + bias_n), y64 = acc * gamma / s_m + bias_n."""
+    gamma = absmean_scale(W)
+    codes = ternary_codes(W, gamma)
+    q, s = act_quant_per_tensor(x_bits, bits) if per_tensor else act_quant(x_bits, bits)
+    acc = matmul_i32(q, codes)
+    y64, y32 = rescale(acc, gamma, s)
+    if bias is not None:
+        b = np.asarray(bias, dtype=np.float32)
+        y64 = y64 + b.astype(np.float64)[None, :]
+        y32 = (y32 + b[None, :]).astype(np.float32)
+    return {"gamma": gamma, "codes": codes, "q": q, "s": s, "acc": acc, "y64": y64, "y32": y32,
+            "Y": round_to_bf16_bits(y32)}

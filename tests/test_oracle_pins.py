@@ -461,3 +461,45 @@ def test_forward_relu2_matches_dequantized_brute_force():
             assert abs(float(exact) - out["y64"][m, n]) <= 1e-12 * max(1.0, abs(float(exact)))
         # s_m is 127 / max_k h, correctly rounded to fp32
         assert out["s"][m] == o.round_rational_to_f32(127 * a.denominator, a.numerator)
+
+
+# ---------------------------------------------------------------------------
+# variants the pages print: per-tensor activation scale (P3 section 1) and bias
+# ---------------------------------------------------------------------------
+
+def test_act_quant_per_tensor_hand_case():
+    # rows [1, 2] and [4, -8]: a = 8 over the tensor, s = 127/8 = 15.875 (exact)
+    x = to_bf16_bits_exact([[1.0, 2.0], [4.0, -8.0]])
+    q, s = o.act_quant_per_tensor(x)
+    assert s.tolist() == [15.875, 15.875]
+    # 15.875 -> 16, 31.75 -> 32, 63.5 -> 64 (tie to even), -127
+    assert q.tolist() == [[16, 32], [64, -127]]
+
+
+def test_act_quant_per_tensor_reduces_to_per_token():
+    rng = np.random.default_rng(12)
+    x1 = (rng.standard_normal((1, 256)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    for bits in (8, 4):
+        assert np.array_equal(o.act_quant_per_tensor(x1, bits)[0], o.act_quant(x1, bits)[0])
+    # rows that share the same absmax: per-tensor equals per-token
+    x = rng.standard_normal((5, 128)).astype(np.float32)
+    x[:, 7] = 9.0
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    qa, sa = o.act_quant_per_tensor(xb)
+    qb, sb = o.act_quant(xb)
+    assert np.array_equal(qa, qb) and np.array_equal(sa, sb)
+    # otherwise every row uses the smallest per-token scale
+    xr = (rng.standard_normal((5, 128)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.all(o.act_quant_per_tensor(xr)[1] == o.act_quant(xr)[1].min())
+
+
+def test_forward_ex_bias_hand_case():
+    # the worked example (y32 = 143 * f32(gamma / s)) plus a bias of -0.25
+    ex = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    W = np.array([ex["W"]], np.float32)
+    x = to_bf16_bits_exact([ex["x"]])
+    plain = o.forward(x, W)
+    out = o.forward_ex(x, W, bias=np.array([-0.25], np.float32))
+    assert out["acc"][0, 0] == 143
+    assert out["y32"][0, 0] == np.float32(np.float32(plain["y32"][0, 0]) + np.float32(-0.25))
+    assert abs(out["y64"][0, 0] - (plain["y64"][0, 0] - 0.25)) < 1e-15
