@@ -43,6 +43,8 @@ SIGNATURES = {
     "bl_forward_relu2_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "bl_forward_relu2": (_int, [_p, _p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_quant_act_relu2": (_int, [_p, _p, _i64, _i64, _int, _p, _p, _p]),
+    "bl_forward_ex_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, ctypes.c_uint]),
+    "bl_forward_ex": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, ctypes.c_uint, _p, _p, _p, _sz, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
@@ -264,6 +266,34 @@ def bl_quant_act_relu2(G: torch.Tensor, U: torch.Tensor | None, bits: int = 8):
     _check(lib().bl_quant_act_relu2(pg_in, pu, M, K, bits, Xq.data_ptr(), s.data_ptr(), _stream()),
            "bl_quant_act_relu2")
     return Xq, s
+
+
+BL_ACT_PER_TENSOR = 1
+
+
+def bl_forward_ex_workspace_bytes(M: int, K: int, N: int, bits: int = 8, flags: int = 0) -> int:
+    return int(lib().bl_forward_ex_workspace_bytes(M, K, N, bits, flags))
+
+
+def bl_forward_ex(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8,
+                  per_tensor: bool = False, bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """bl_forward with the per-tensor activation scale and/or an fp32 bias [N]."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    pb = _dev(bias, torch.float32, "bias") if bias is not None else None
+    flags = BL_ACT_PER_TENSOR if per_tensor else 0
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    ws = workspace
+    if ws is None:
+        ws = _workspace(bl_forward_ex_workspace_bytes(M, K, N, bits, flags), X.device)
+    _check(lib().bl_forward_ex(px, M, K, N, pw, pg, bits, flags, pb, py,
+                               ws.data_ptr() if ws is not None else None,
+                               ws.numel() if ws is not None else 0, _stream()), "bl_forward_ex")
+    return Y
 
 
 def bl_matmul_i32(Xq: torch.Tensor, Wp: torch.Tensor, N: int) -> torch.Tensor:

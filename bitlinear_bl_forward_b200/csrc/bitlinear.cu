@@ -259,7 +259,8 @@ constexpr int kDecodeKernel = BL_DECODE_KERNEL;
 // problem gets CTAs in proportion to its weight bytes (at least one, at most
 // one per row), and the launch has exactly one CTA per SM when the rows allow.
 // Returns the grid size.
-int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, const void* U) {
+int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, const void* U,
+                      const float* bias) {
   std::memset(tab, 0, sizeof(*tab));
   double total = 0.0;
   int64_t rows = 0;
@@ -299,7 +300,7 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
     const bl_linear& p = *probs[i];
     const int rows_per_cta = static_cast<int>((p.N + c[i] - 1) / c[i]);
     tab->p[i] = bl::G2Problem{p.X, U, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
-                              rows_per_cta, grid, c[i]};
+                              rows_per_cta, grid, c[i], bias};
     grid += c[i];
   }
   tab->count = n;
@@ -311,7 +312,7 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
 // in_mode: bl::InMode of the token input; U: the up projection's output in
 // the gated squared-ReLU mode (shared by every problem of the call).
 bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q, int out_mode, cudaStream_t stream,
-                        const void* U = nullptr) {
+                        const void* U = nullptr, const float* bias = nullptr) {
   if (n <= 0) return BL_OK;
   const int sms = num_sms();
   bl::G2Table tab;
@@ -337,13 +338,13 @@ bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q
       const int rows_per_cta = static_cast<int>((p.N + c - 1) / c);
       c = static_cast<int>((p.N + rows_per_cta - 1) / rows_per_cta);
       tab.p[i] = bl::G2Problem{p.X, U, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
-                               rows_per_cta, grid, c};
+                               rows_per_cta, grid, c, bias};
       grid += c;
     }
     tab.count = n;
     return launch_gemv2_cpl((maxK / 64 + 31) / 32, tab, grid, in_mode, Q, out_mode, stream);
   }
-  const int grid = fill_decode_table(&tab, probs, n, sms, U);
+  const int grid = fill_decode_table(&tab, probs, n, sms, U, bias);
   return launch_gemv3_wpl((maxK + 511) / 512, tab, grid, in_mode, Q, out_mode, stream);
 }
 
@@ -395,7 +396,7 @@ bl_status launch_act_quant(const uint16_t* X, int m, int k, int Q, int8_t* Xq, f
   // measured: the CTA-per-row kernel also wins for long rows (K > 4096, where
   // a warp can no longer keep its row in registers and reads part of it twice)
   if (m < bl::kActRowsPerBlock * num_sms() || k > 32 * 8 * bl::kActCache) {
-    bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R);
+    bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, nullptr);
   } else {
     const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
     bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
@@ -429,7 +430,7 @@ bl_status launch_tc_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, 
 
 template <int BN, int EXPG>
 bl_status launch_tc2_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
-                       const float* gamma, void* Y, int out_mode, cudaStream_t stream) {
+                       const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias) {
   using C = bl::P2Cfg<BN>;
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(bl::tc_gemm_persistent_kernel<BN, EXPG>, C::kSmemBytes, &done)) return BL_ERR_CUDA;
@@ -443,7 +444,7 @@ bl_status launch_tc2_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp,
   const int ntiles = ((M + BN - 1) / BN) * ((N + bl::kTcRows - 1) / bl::kTcRows);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
   bl::tc_gemm_persistent_kernel<BN, EXPG><<<grid, bl::P2Warps<EXPG>::kThreads, C::kSmemBytes, stream>>>(
-      tmX, tmW, M, N, K, R, s, gamma, Y, out_mode, kWaitLimitNs);
+      tmX, tmW, M, N, K, R, s, gamma, Y, out_mode, bias, kWaitLimitNs);
   return last_cuda();
 }
 
@@ -474,7 +475,7 @@ int max_active_pairs(F* kernel, int threads, int smem) {
 }
 
 bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
-                         const float* gamma, void* Y, int out_mode, cudaStream_t stream) {
+                         const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias) {
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(bl::tc_gemm_pair_kernel, bl::kQSmemBytes, &done)) return BL_ERR_CUDA;
   CUtensorMap tmX, tmW;
@@ -521,7 +522,7 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
   cfg.numAttrs = 1;
   const unsigned long long lim = kWaitLimitNs;
   if (cudaLaunchKernelEx(&cfg, bl::tc_gemm_pair_kernel, tmX, tmW, tmY, M, N, K, R, s, gamma, Y, out_mode, tma_store,
-                         lim) != cudaSuccess)
+                         bias, lim) != cudaSuccess)
     return BL_ERR_CUDA;
   return last_cuda();
 }
@@ -534,14 +535,15 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
 #endif
 
 bl_status launch_tc(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
-                    const float* gamma, void* Y, int out_mode, int debug_flags, cudaStream_t stream) {
+                    const float* gamma, void* Y, int out_mode, int debug_flags, cudaStream_t stream,
+                    const float* bias = nullptr) {
   if (BL_TC_KERNEL == 0 && debug_flags == 0 && M > 64)
-    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
   if (BL_TC_KERNEL != 1 && debug_flags == 0) {
-    if (M <= 16) return launch_tc2_t<16, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
-    if (M <= 32) return launch_tc2_t<32, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
-    if (M <= 64) return launch_tc2_t<64, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
-    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream);
+    if (M <= 16) return launch_tc2_t<16, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
+    if (M <= 32) return launch_tc2_t<32, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
+    if (M <= 64) return launch_tc2_t<64, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
+    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
   }
   const unsigned long long lim = kWaitLimitNs;
   if (M <= 16) return launch_tc_t<16>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
@@ -914,6 +916,69 @@ bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int6
   if ((st = last_cuda()) != BL_OK) return st;
   return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16,
                    0, stream);
+}
+
+size_t ex_ws_bytes(int64_t M, int64_t K) {
+  if (M == 1 && K <= 8192) return 0;   // one token: the decode kernels, no workspace
+  return align_up(static_cast<size_t>(M) * K, 256) + 2 * align_up(static_cast<size_t>(M) * 4, 256) + 256;
+}
+
+size_t bl_forward_ex_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits, unsigned flags) {
+  (void)bits;
+  (void)flags;
+  if (check_shape_nk(N, K) != BL_OK || check_m(M, K) != BL_OK || M == 0) return 0;
+  return ex_ws_bytes(M, K);
+}
+
+bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
+                        int bits, unsigned flags, const float* bias, uint16_t* Y, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if ((flags & ~static_cast<unsigned>(BL_ACT_PER_TENSOR)) != 0u) return BL_ERR_UNSUPPORTED;
+  if (M == 0) return BL_OK;
+  if (!X || !Wp || !gamma || !Y) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wp) || (reinterpret_cast<uintptr_t>(bias) & 3u)) return BL_ERR_ALIGNMENT;
+  const size_t need = ex_ws_bytes(M, K);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+  }
+  const int Q = bits == 8 ? 127 : 7;
+  if (need == 0) {   // one token: per-tensor and per-token scales coincide
+    bl_linear p;
+    p.X = X;
+    p.M = 1;
+    p.K = K;
+    p.N = N;
+    p.Wp = Wp;
+    p.gamma = gamma;
+    p.Y = Y;
+    const bl_linear* pp = &p;
+    return launch_decode(&pp, 1, bl::kInBF16, Q, bl::kOutBF16, stream, nullptr, bias);
+  }
+  const int m = static_cast<int>(M), k = static_cast<int>(K);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const size_t codes = align_up(static_cast<size_t>(M) * K, 256), rows = align_up(static_cast<size_t>(M) * 4, 256);
+  int8_t* Xq = reinterpret_cast<int8_t*>(base);
+  float* s = reinterpret_cast<float*>(base + codes);
+  int* R = reinterpret_cast<int*>(base + codes + rows);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(base + codes + 2 * rows);
+  if (flags & BL_ACT_PER_TENSOR) {
+    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), stream) != cudaSuccess) return BL_ERR_CUDA;
+    const int64_t nch = static_cast<int64_t>(M) * K / 8;
+    int64_t blocks = (nch + 255) / 256;
+    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+    bl::act_absmax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, nch, amax);
+    if ((st = last_cuda()) != BL_OK) return st;
+    bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, amax);
+    if ((st = last_cuda()) != BL_OK) return st;
+  } else if ((st = launch_act_quant(X, m, k, Q, Xq, s, R, stream)) != BL_OK) {
+    return st;
+  }
+  return launch_tc(Xq, m, k, static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16, 0, stream, bias);
 }
 
 bl_status bl_device_status(int clear, int* site) {

@@ -154,7 +154,8 @@ constexpr int kActRowCache = 8;   // 16-byte chunks kept in registers per thread
 __global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uint16_t* __restrict__ X, int K, int Q,
                                                                        int8_t* __restrict__ Xq,
                                                                        float* __restrict__ s_out,
-                                                                       int* __restrict__ R_out) {
+                                                                       int* __restrict__ R_out,
+                                                                       const uint32_t* __restrict__ amax_all) {
   constexpr int W = kActRowThreads / 32;
   __shared__ uint32_t s_max[W];
   __shared__ int s_sum[W];
@@ -180,6 +181,7 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uin
   uint32_t bmax = 0;
 #pragma unroll
   for (int w = 0; w < W; ++w) bmax = max(bmax, s_max[w]);
+  if (amax_all) bmax = *amax_all;   // per-tensor mode: one absmax for every row
   const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
   uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
   int sum = 0;
@@ -200,6 +202,21 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uin
     if (s_out) s_out[m] = s;
     if (R_out) R_out[m] = tot;
   }
+}
+
+// Tensor-wide absmax of bf16 activations ("BitNet 2B4T Guide", section "1.
+// The BitLinear Operator", per-tensor form): non-negative floats order as
+// their bit patterns, so a max of the bits is the max of the values.
+// *amax_out must be zero before the launch.
+__global__ void __launch_bounds__(256) act_absmax_kernel(const uint16_t* __restrict__ X, int64_t nchunks,
+                                                        uint32_t* __restrict__ amax_out) {
+  const uint4* x4 = reinterpret_cast<const uint4*>(X);
+  float a = 0.f;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < nchunks;
+       c += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    a = fmaxf(a, absmax8_bf16(__ldg(x4 + c)));
+  const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_out, w);
 }
 
 // Squared-ReLU feed-forward input, quantised per token: one CTA per row;

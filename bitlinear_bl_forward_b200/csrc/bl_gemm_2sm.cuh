@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const int* __restrict__ Rg,
                         const float* __restrict__ sg, const float* __restrict__ gamma_p, void* __restrict__ Y,
-                        int out_mode, int tma_store, unsigned long long limit_ns) {
+                        int out_mode, int tma_store, const float* __restrict__ bias, unsigned long long limit_ns) {
   constexpr int S = kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!named_bar_and(3, 32 * kQEpiWarps, ok)) break;
       tc_fence_after();
       const int n = n0 + r;
+      const float bias_n = (bias && n < N) ? __ldg(bias + n) : 0.f;
       if (tma_store) {
         // bf16 tile of this warp, [BN tokens][32 rows], then one TMA store
         uint16_t* so = reinterpret_cast<uint16_t*>(sOut + (warp - kQFirstEpi) * kQStageOutBytes);
@@ -284,7 +285,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             const int a = static_cast<int>(v[t]) - sR[b * kQBN + c0 + t];
-            const float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
+            float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
+            if (bias) y = __fadd_rn(y, bias_n);
             so[(c0 - col0 + t) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
           }
         }
@@ -315,7 +317,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
               if (out_mode == kOutI32) {
                 static_cast<int*>(Y)[o] = a;
               } else {
-                const float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
+                float y = __fmul_rn(__int2float_rn(a), sF[b * kQBN + c0 + t]);
+                if (bias) y = __fadd_rn(y, bias_n);
                 if (out_mode == kOutF32)
                   static_cast<float*>(Y)[o] = y;
                 else

@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
     tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int M,
                               int N, int K, const int* __restrict__ Rg, const float* __restrict__ sg,
                               const float* __restrict__ gamma_p, void* __restrict__ Y, int out_mode,
-                              unsigned long long limit_ns) {
+                              const float* __restrict__ bias, unsigned long long limit_ns) {
   using C = P2Cfg<BN>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
       if (!named_bar_and(3, 128, ok)) break;
       tc_fence_after();
       const int n = n0 + r;
+      const float bias_n = (bias && n < N) ? __ldg(bias + n) : 0.f;
       constexpr int kChunk = BN < 32 ? BN : 32;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += kChunk) {
@@ -292,7 +293,8 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
               if (out_mode == kOutI32) {
                 static_cast<int*>(Y)[o] = a;
               } else {
-                const float y = __fmul_rn(__int2float_rn(a), sF[b * BN + c0 + t]);
+                float y = __fmul_rn(__int2float_rn(a), sF[b * BN + c0 + t]);
+                if (bias) y = __fadd_rn(y, bias_n);
                 if (out_mode == kOutF32)
                   static_cast<float*>(Y)[o] = y;
                 else

@@ -308,7 +308,8 @@ __device__ __forceinline__ void gemv1_accumulate(const uint4 (&w)[RT][CPL], cons
 // rescale, store.
 template <int MT, int RT>
 __device__ __forceinline__ void gemv1_finish(const int (&part)[RT][MT], int tile, int N, int lane, const int (&R)[MT],
-                                             const float (&f)[MT], void* __restrict__ Y, int out_mode) {
+                                             const float (&f)[MT], void* __restrict__ Y, int out_mode,
+                                             const float* __restrict__ bias = nullptr) {
 #pragma unroll
   for (int r = 0; r < RT; ++r)
 #pragma unroll
@@ -321,7 +322,8 @@ __device__ __forceinline__ void gemv1_finish(const int (&part)[RT][MT], int tile
         if (out_mode == kOutI32) {
           static_cast<int*>(Y)[o] = a;
         } else {
-          const float y = __fmul_rn(__int2float_rn(a), f[m]);
+          float y = __fmul_rn(__int2float_rn(a), f[m]);
+          if (bias) y = __fadd_rn(y, __ldg(bias + n));
           if (out_mode == kOutF32)
             static_cast<float*>(Y)[o] = y;
           else
@@ -508,6 +510,7 @@ struct G2Problem {
   int rows_per_cta;   // TMA-staged GEMV: CTA c takes rows [c*rows_per_cta, ...)
   int cta_begin;      // first CTA of this problem in the launch
   int ctas;           // decode kernel: CTA c takes rows [c*N/ctas, (c+1)*N/ctas)
+  const float* bias;  // optional fp32 [N] added after the rescale
 };
 constexpr int kG2MaxProblems = 8;
 struct G2Table {
@@ -722,7 +725,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
       }
       int part[1][MT];
       gemv1_accumulate<MT, CPL, 1>(w, act, KV, lane, part);
-      gemv1_finish<MT, 1>(part, row0 + rr, N, lane, R, f, Y, out_mode);
+      gemv1_finish<MT, 1>(part, row0 + rr, N, lane, R, f, Y, out_mode, tab.p[pi].bias);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);

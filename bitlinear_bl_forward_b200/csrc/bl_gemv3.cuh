@@ -53,7 +53,8 @@ struct G3Cfg {
 template <int RT, int WPL, bool ACT_SMEM>
 __device__ __forceinline__ void g3_rows(const uint8_t* sbase, int rr, int rows, int row_bytes, int words, int lane,
                                         const uint32_t (&act)[ACT_SMEM ? 1 : WPL][4], const uint8_t* s_act,
-                                        int row0, int R, float f, void* __restrict__ Y, int out_mode) {
+                                        int row0, int R, float f, void* __restrict__ Y, int out_mode,
+                                        const float* __restrict__ bias) {
   const uint32_t* p[RT];
   bool live[RT];
 #pragma unroll
@@ -100,7 +101,8 @@ __device__ __forceinline__ void g3_rows(const uint8_t* sbase, int rr, int rows, 
       if (out_mode == kOutI32) {
         static_cast<int*>(Y)[n] = v;
       } else {
-        const float y = __fmul_rn(__int2float_rn(v), f);
+        float y = __fmul_rn(__int2float_rn(v), f);
+        if (bias) y = __fadd_rn(y, __ldg(bias + n));
         if (out_mode == kOutF32)
           static_cast<float*>(Y)[n] = y;
         else
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
   const uint8_t* __restrict__ Wp = tab.p[pi].Wp;
   const float* __restrict__ gamma_p = tab.p[pi].gamma;
   void* __restrict__ Y = tab.p[pi].Y;
+  const float* __restrict__ bias = tab.p[pi].bias;
   const int K = tab.p[pi].K, N = tab.p[pi].N, ctas = tab.p[pi].ctas;
   const int cta = static_cast<int>(blockIdx.x) - tab.p[pi].cta_begin;
 
@@ -300,9 +303,9 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
     const uint8_t* sbase = g3_smem + s * kG3StageBytes;
     if (rows > CW) {   // some warp has two rows: take them together
       for (int rr = warp * 2; rr < rows; rr += CW * 2)
-        g3_rows<2, WPL, ACT_SMEM>(sbase, rr, rows, row_bytes, words, lane, act, s_act, row0, R, f, Y, out_mode);
+        g3_rows<2, WPL, ACT_SMEM>(sbase, rr, rows, row_bytes, words, lane, act, s_act, row0, R, f, Y, out_mode, bias);
     } else if (warp < rows) {
-      g3_rows<1, WPL, ACT_SMEM>(sbase, warp, rows, row_bytes, words, lane, act, s_act, row0, R, f, Y, out_mode);
+      g3_rows<1, WPL, ACT_SMEM>(sbase, warp, rows, row_bytes, words, lane, act, s_act, row0, R, f, Y, out_mode, bias);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);

@@ -232,6 +232,30 @@ BL_API bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t 
 BL_API bl_status bl_quant_act_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int bits, int8_t* Xq,
                                     float* scale, cudaStream_t stream);
 
+
+/*
+ * The variants the pages print, as one entry point:
+ *   BL_ACT_PER_TENSOR  one absmax over the whole activation tensor instead of
+ *                      one per token ("BitNet 2B4T Guide: Scaling Native
+ *                      1.58-Bit LLMs", section "1. The BitLinear Operator"):
+ *                      a = max over all |X|, s = Q / max(a, 1e-5) for every
+ *                      row, q = clamp(round_half_even(X * s), -Q-1, Q);
+ *   bias               optional fp32 [N] added after the rescale (the
+ *                      BitLinear module's bias argument, "BitNet b1.58: The
+ *                      1-Bit Ternary LLM Architecture Guide"):
+ *                      Y = bf16( f32( f32(f32(acc) * f32(gamma / s_m)) + bias[n] ) ).
+ * Otherwise exactly bl_forward.  flags: 0 or BL_ACT_PER_TENSOR (other bits
+ * return BL_ERR_UNSUPPORTED); bias may be NULL (4-byte aligned otherwise).
+ * workspace: bl_forward_ex_workspace_bytes (0 when M == 1 and K <= 8192).
+ * With M > 1 the tensor-core path runs for every M (the per-tensor absmax is
+ * one more kernel before the quantiser).
+ */
+#define BL_ACT_PER_TENSOR 1u
+BL_API size_t bl_forward_ex_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits, unsigned flags);
+BL_API bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
+                               const float* gamma, int bits, unsigned flags, const float* bias, uint16_t* Y,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
 BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
 

@@ -170,3 +170,14 @@ def test_relu2_validation(L):
     assert L.bl_quant_act_relu2(A, A, 4, 64, 2, A, A, None) == UNSUP
     assert L.bl_quant_act_relu2(A, U, 4, 64, 8, A, A, None) == ALIGN
     assert len(args) == 12
+
+
+def test_forward_ex_validation(L):
+    assert L.bl_forward_ex_workspace_bytes(1, 2560, 6912, 8, 1) == 0
+    assert L.bl_forward_ex_workspace_bytes(2, 2560, 6912, 8, 0) >= 2 * 2560
+    assert L.bl_forward_ex(A, 4, 64, 8, A, A, 8, 2, None, A, A, 1 << 20, None) == UNSUP      # unknown flag
+    assert L.bl_forward_ex(A, 4, 64, 8, A, A, 8, 1, A + 2, A, A, 1 << 20, None) == ALIGN    # bias not 4-byte aligned
+    assert L.bl_forward_ex(A, 4, 64, 8, A, A, 8, 1, None, A, None, 0, None) == WS
+    assert L.bl_forward_ex(None, 4, 64, 8, A, A, 8, 0, None, A, A, 1 << 20, None) == INVALID
+    assert L.bl_forward_ex(A, 4, 100, 8, A, A, 8, 0, None, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_forward_ex(None, 0, 64, 8, None, None, 8, 1, None, None, None, 0, None) == OK

@@ -355,3 +355,27 @@ def test_forward_relu2_bits4_and_zero_rows():
         Yd = bf16_dev_to_bits(bl.bl_forward_relu2(x_to_dev(G), x_to_dev(U), Wp, gd, N, bits))
         assert bf16_ulp_distance(Yd, ref["Y"]).max() <= BF16_ULP_TOL
         assert np.all(Yd[1] == 0) and np.all(Yd[2] == 0)
+
+
+# ---------------------------------------------------------------------------
+# per-tensor activation scale and output bias (bl_forward_ex)
+# ---------------------------------------------------------------------------
+
+EX_CASES = [(1, 2560, 700), (1, 8192, 8192), (1, 16384, 64), (2, 320, 130), (3, 256, 512), (17, 320, 130),
+            (130, 256, 300), (300, 1024, 700)]
+
+
+@pytest.mark.parametrize("M,K,N", EX_CASES)
+@pytest.mark.parametrize("per_tensor,with_bias", [(True, False), (False, True), (True, True)])
+def test_forward_ex_parity(M, K, N, per_tensor, with_bias):
+    X, W = random_case(M, K, N, seed=M * 7 + K + N)
+    bias = (np.random.default_rng(N).standard_normal(N) * 0.5).astype(np.float32) if with_bias else None
+    for bits in ((8, 4) if M in (3, 130) else (8,)):
+        ref = o.forward_ex(X, W, bits, per_tensor=per_tensor, bias=bias)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        Yd = bl.bl_forward_ex(x_to_dev(X), Wp, gd, N, bits, per_tensor=per_tensor,
+                              bias=torch.from_numpy(bias).cuda() if bias is not None else None)
+        torch.cuda.synchronize()
+        d = bf16_ulp_distance(bf16_dev_to_bits(Yd), ref["Y"])
+        assert d.max() <= BF16_ULP_TOL, f"bf16 ulp distance {d.max()}"
+        assert np.mean(d == 0) > 0.99
