@@ -397,25 +397,48 @@ def time_workload(wl, steps, warmup, dist_ctx, sample_clocks=True, chunk=None):
 
 def time_e2e(wl, steps, warmup, dist_ctx):
     """Same metric through the public API with host buffers: each step copies
-    every layer's input from pinned host memory, runs bl_forward and reads the
-    outputs back to pinned host memory."""
+    the step's inputs from pinned host memory in one transfer, runs the
+    library calls and reads all outputs back to pinned host memory in one
+    transfer (the layers' input and output tensors are views of one device
+    buffer each, 128-byte aligned)."""
     import torch
-    from bitlinear_bl_forward_b200 import bl
-    hx = {j: torch.from_numpy(d["xb"].view(np.int16)).view(torch.bfloat16).pin_memory()
-          for j, d in enumerate(wl.layers) if d["own_x"]}
-    hy = [torch.empty(tuple(d["Y"].shape), dtype=torch.bfloat16).pin_memory() for d in wl.layers]
-    h2d = sum(t.numel() * 2 for t in hx.values())
-    d2h = sum(t.numel() * 2 for t in hy)
+    own = [j for j, d in enumerate(wl.layers) if d["own_x"]]
+
+    def carve(shapes):
+        offs, n = [], 0
+        for shp in shapes:
+            offs.append(n)
+            n += (int(np.prod(shp)) + 63) // 64 * 64
+        return offs, n
+
+    in_offs, n_in = carve([tuple(wl.layers[j]["X"].shape) for j in own])
+    out_offs, n_out = carve([tuple(d["Y"].shape) for d in wl.layers])
+    dev_in = torch.zeros(n_in, dtype=torch.bfloat16, device="cuda")
+    dev_out = torch.empty(n_out, dtype=torch.bfloat16, device="cuda")
+    host_in = torch.zeros(n_in, dtype=torch.bfloat16).pin_memory()
+    host_out = torch.empty(n_out, dtype=torch.bfloat16).pin_memory()
+    for j, off in zip(own, in_offs):
+        d = wl.layers[j]
+        shp = tuple(d["X"].shape)
+        n = int(np.prod(shp))
+        host_in[off:off + n].copy_(torch.from_numpy(d["xb"].reshape(-1).view(np.int16)).view(torch.bfloat16))
+        view = dev_in[off:off + n].view(shp)
+        for dd in wl.layers:                       # every layer that reads this hidden state
+            if dd["X"] is d["X"] and dd is not d:
+                dd["X"] = view
+        d["X"] = view
+    for d, off in zip(wl.layers, out_offs):
+        shp = tuple(d["Y"].shape)
+        d["Y"] = dev_out[off:off + int(np.prod(shp))].view(shp)
+    h2d = sum(int(np.prod(tuple(wl.layers[j]["X"].shape))) * 2 for j in own)
+    d2h = sum(d["Y"].numel() * 2 for d in wl.layers)
 
     def one(i):
         r = i % wl.rotations
-        for gi, gr in enumerate(wl.groups):
-            for j in gr:
-                if j in hx:
-                    wl.layers[j]["X"].copy_(hx[j], non_blocking=True)
+        dev_in.copy_(host_in, non_blocking=True)
+        for gi in range(len(wl.groups)):
             wl.run_group(gi, r)
-            for j in gr:
-                hy[j].copy_(wl.layers[j]["Y"], non_blocking=True)
+        host_out.copy_(dev_out, non_blocking=True)
 
     for i in range(warmup):
         one(i)
