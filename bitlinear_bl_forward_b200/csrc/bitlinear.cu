@@ -634,7 +634,7 @@ static int absum_blocks(int64_t N, int64_t K) {
 
 size_t bl_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
   if (check_shape_nk(N, K) != BL_OK) return 0;
-  return static_cast<size_t>(absum_blocks(N, K)) * bl::kBins * sizeof(unsigned long long);
+  return static_cast<size_t>(bl::kAbsumTotals) * sizeof(unsigned long long);
 }
 
 bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gamma, void* workspace,
@@ -649,9 +649,11 @@ bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp,
   const int blocks = absum_blocks(N, K);
   auto* bins = static_cast<unsigned long long*>(workspace);
   const int64_t n = N * K;
+  if (cudaMemsetAsync(bins, 0, bl::kAbsumTotals * sizeof(unsigned long long), stream) != cudaSuccess)
+    return BL_ERR_CUDA;
   bl::weight_absum_bins_kernel<<<blocks, bl::kAbsumThreads, 0, stream>>>(W, n, bins);
   if ((st = last_cuda()) != BL_OK) return st;
-  bl::weight_gamma_kernel<<<1, 256, 0, stream>>>(bins, blocks, static_cast<uint64_t>(n), gamma);
+  bl::weight_gamma_kernel<<<1, 32, 0, stream>>>(bins, static_cast<uint64_t>(n), gamma);
   if ((st = last_cuda()) != BL_OK) return st;
   const int64_t nwords = n / 16;
   bl::weight_pack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(

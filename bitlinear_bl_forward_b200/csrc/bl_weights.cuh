@@ -26,55 +26,72 @@
 namespace bl {
 
 constexpr int kAbsumThreads = 256;
-constexpr int kAbsumWarps = kAbsumThreads / 32;
-constexpr int kBins = 256;   // bins 0..253: exponent groups, 255: non-finite count
+constexpr int kAbsumChunks = 9;     // |w| * 2^149 < 2^277: nine 32-bit positions (+ carry)
+constexpr int kAbsumTotals = 16;    // global accumulators: limbs 0..9, [15] = non-finite count
 
-// Pass 1: per-block exact bins of sum |W|.  out_bins: [gridDim.x][kBins].
+// Pass 1: the exact sum of |W| in units of 2^-149, as 32-bit limbs.
+// Every |w| is sig * 2^b * 2^-149 with sig < 2^24 and b = 0..253; a thread
+// adds the two 32-bit pieces of sig << (b % 32) to its own positional
+// accumulators b / 32 and b / 32 + 1 (private columns of a shared-memory
+// array: conflict-free whatever the exponents), the block sums them, carries
+// them into 32-bit limbs and adds those to total[0..9].  All additions are
+// exact integer additions (bounds: a thread sees < 2^23 elements, a block
+// < 2^31, so no accumulator can overflow), hence no dependence on the order.
+// total must be zero before the launch.
 __global__ void __launch_bounds__(kAbsumThreads) weight_absum_bins_kernel(const float* __restrict__ W, int64_t n,
-                                                                           unsigned long long* __restrict__ out_bins) {
-  __shared__ unsigned long long sb[kAbsumWarps][kBins];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kAbsumWarps * kBins; i += blockDim.x) (&sb[0][0])[i] = 0ull;
-  __syncthreads();
-
+                                                                           unsigned long long* __restrict__ total) {
+  __shared__ unsigned long long acc[kAbsumChunks + 1][kAbsumThreads];
+  __shared__ unsigned long long red[kAbsumChunks + 1];
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int c = 0; c <= kAbsumChunks; ++c) acc[c][tid] = 0ull;
+  if (tid <= kAbsumChunks) red[tid] = 0ull;
+  unsigned int nonfinite = 0;
   const int64_t n4 = n >> 2;   // n is a multiple of 64
   const float4* W4 = reinterpret_cast<const float4*>(W);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  // Every lane of the warp runs the same number of iterations so the
-  // warp-wide match/reduce below always sees a full warp.
-  const int64_t base0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
-  for (int64_t base = base0; base < n4; base += stride) {
-    const int64_t i = base + lane;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < n4) v = W4[i];
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n4; i += stride) {
+    const float4 v = __ldg(W4 + i);
     const float e4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const uint32_t u = __float_as_uint(e4[t]) & 0x7fffffffu;
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t u = __float_as_uint(e4[e]) & 0x7fffffffu;
       const uint32_t ex = u >> 23, fr = u & 0x7fffffu;
-      uint32_t bin, sig;
       if (ex == 255u) {
-        bin = 255u;
-        sig = 1u;
-      } else if (ex == 0u) {
-        bin = 0u;
-        sig = fr;
-      } else {
-        bin = ex - 1u;
-        sig = fr | 0x800000u;
+        ++nonfinite;
+        continue;
       }
-      // lanes that share a bin add their significands (< 32 * 2^24) first
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      const unsigned part = __reduce_add_sync(peers, sig);
-      if (lane == __ffs(peers) - 1) atomicAdd(&sb[warp][bin], static_cast<unsigned long long>(part));
+      // normal: (fr + 2^23) * 2^(ex - 150) = sig * 2^(ex - 1) * 2^-149; subnormal: fr * 2^-149
+      const uint32_t b = ex ? ex - 1u : 0u;
+      const uint32_t sig = ex ? (fr | 0x800000u) : fr;
+      const unsigned long long piece = static_cast<unsigned long long>(sig) << (b & 31u);
+      const uint32_t c = b >> 5;
+      acc[c][tid] += piece & 0xffffffffull;
+      acc[c + 1][tid] += piece >> 32;
     }
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
+  // column sums: warp w adds up chunk c = w, w + 8 over the 256 threads
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int c = warp; c <= kAbsumChunks; c += kAbsumThreads / 32) {
     unsigned long long t = 0;
+    for (int k = lane; k < kAbsumThreads; k += 32) t += acc[c][k];
 #pragma unroll
-    for (int w = 0; w < kAbsumWarps; ++w) t += sb[w][b];
-    out_bins[static_cast<int64_t>(blockIdx.x) * kBins + b] = t;
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) red[c] = t;
+  }
+  const unsigned int nf = __reduce_add_sync(0xffffffffu, nonfinite);
+  if (lane == 0 && nf) atomicAdd(&total[kAbsumTotals - 1], static_cast<unsigned long long>(nf));
+  __syncthreads();
+  if (tid == 0) {
+    unsigned long long carry = 0;
+    for (int c = 0; c <= kAbsumChunks; ++c) {
+      const unsigned long long t = red[c] + carry;   // red[c] < 2^63
+      const unsigned long long limb = t & 0xffffffffull;
+      carry = t >> 32;
+      if (limb) atomicAdd(&total[c], limb);
+    }
+    if (carry) atomicAdd(&total[kAbsumChunks + 1 < kAbsumTotals - 1 ? kAbsumChunks + 1 : 0], carry);
   }
 }
 
@@ -139,43 +156,24 @@ __device__ float round_ratio_to_f32(const uint32_t* S, int nlimbs, uint64_t D) {
   return __uint_as_float((static_cast<uint32_t>(E + 127) << 23) | (mant & 0x7fffffu));
 }
 
-// Pass 2: one block.  Sums the per-block bins and writes gamma.
-__global__ void __launch_bounds__(256) weight_gamma_kernel(const unsigned long long* __restrict__ bins, int nblocks,
-                                                           uint64_t count, float* __restrict__ gamma) {
-  __shared__ unsigned long long tot[kBins];
-  for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
-    unsigned long long t = 0;
-    for (int g = 0; g < nblocks; ++g) t += bins[static_cast<int64_t>(g) * kBins + b];
-    tot[b] = t;
-  }
-  __syncthreads();
+// Pass 2: one thread.  Turns the limb totals into gamma.
+__global__ void __launch_bounds__(32) weight_gamma_kernel(const unsigned long long* __restrict__ total, uint64_t count,
+                                                          float* __restrict__ gamma) {
   if (threadIdx.x != 0) return;
-  if (tot[255] != 0ull) {   // a non-finite weight
+  if (total[kAbsumTotals - 1] != 0ull) {   // a non-finite weight
     *gamma = __int_as_float(0x7fc00000);
     return;
   }
-  // S = sum_b tot[b] * 2^b, in units of 2^-149; tot[b] < 2^64, b <= 253
-  constexpr int kLimbs = 12;
+  // S = sum_c total[c] * 2^(32 c), in units of 2^-149; total[c] < 2^42
+  constexpr int kLimbs = 14;
   uint32_t S[kLimbs];
 #pragma unroll
   for (int i = 0; i < kLimbs; ++i) S[i] = 0;
-  for (int b = 0; b < 254; ++b) {
-    const unsigned long long v = tot[b];
-    if (!v) continue;
-    const int li = b >> 5, sh = b & 31;
-    // v << sh spans up to three limbs
-    uint32_t part[3];
-    part[0] = static_cast<uint32_t>(v << sh);
-    part[1] = static_cast<uint32_t>(sh ? (v >> (32 - sh)) : (v >> 32));
-    part[2] = static_cast<uint32_t>(sh ? (v >> (64 - sh)) : 0ull);
-    uint64_t carry = 0;
-    for (int k = li; k < kLimbs; ++k) {
-      const uint64_t add = (k - li < 3) ? part[k - li] : 0u;
-      const uint64_t s = static_cast<uint64_t>(S[k]) + add + carry;
-      S[k] = static_cast<uint32_t>(s);
-      carry = s >> 32;
-      if (k - li >= 2 && carry == 0) break;
-    }
+  unsigned long long carry = 0;
+  for (int c = 0; c < kLimbs; ++c) {
+    const unsigned long long t = (c < kAbsumTotals - 1 ? total[c] : 0ull) + carry;
+    S[c] = static_cast<uint32_t>(t);
+    carry = t >> 32;
   }
   const float mean = round_ratio_to_f32(S, kLimbs, count);
   *gamma = fmaxf(mean, 1e-5f);
