@@ -11,6 +11,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/bitlinear.h"
 #include "bl_act.cuh"
@@ -33,6 +34,15 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
 constexpr int kMaxDevices = 64;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// An NVTX range around each public call (visible in Nsight timelines; a
+// no-op unless a profiling tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bl_status check_shape_nk(int64_t N, int64_t K) {
@@ -639,6 +649,7 @@ size_t bl_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
 
 bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gamma, void* workspace,
                               size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quantize_weights");
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if (!W || !Wp || !gamma) return BL_ERR_INVALID_ARG;
@@ -662,6 +673,7 @@ bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp,
 }
 
 bl_status bl_unpack_weights(const uint8_t* Wp, int64_t N, int64_t K, int8_t* codes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_unpack_weights");
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if (!Wp || !codes) return BL_ERR_INVALID_ARG;
@@ -674,6 +686,7 @@ bl_status bl_unpack_weights(const uint8_t* Wp, int64_t N, int64_t K, int8_t* cod
 
 bl_status bl_quant_act(const uint16_t* X, int64_t M, int64_t K, int bits, int8_t* Xq, float* scale,
                        cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quant_act");
   if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
   bl_status st = check_m(M, K);
   if (st != BL_OK) return st;
@@ -693,11 +706,13 @@ size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
 
 bl_status bl_forward(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
                      int bits, uint16_t* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward");
   return forward_common(X, M, K, N, Wp, gamma, bits, Y, bl::kOutBF16, workspace, workspace_bytes, stream);
 }
 
 bl_status bl_forward_f32(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
                          int bits, float* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_f32");
   return forward_common(X, M, K, N, Wp, gamma, bits, Y, bl::kOutF32, workspace, workspace_bytes, stream);
 }
 
@@ -709,6 +724,7 @@ size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N) {
 
 bl_status bl_matmul_i32(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, int32_t* acc,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_matmul_i32");
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if ((st = check_m(M, K)) != BL_OK) return st;
@@ -804,6 +820,7 @@ size_t bl_forward_grouped_workspace_bytes(int count, const bl_linear* problems, 
 
 bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, void* workspace, size_t workspace_bytes,
                              cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_grouped");
   if (problems == nullptr) return BL_ERR_INVALID_ARG;
   if (count < 0 || count > bl::kG2MaxProblems) return BL_ERR_UNSUPPORTED;
   if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
@@ -868,6 +885,7 @@ size_t bl_forward_relu2_workspace_bytes(int64_t M, int64_t K, int64_t N, int bit
 
 bl_status bl_quant_act_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int bits, int8_t* Xq,
                              float* scale, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quant_act_relu2");
   if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
   bl_status st = check_m(M, K);
   if (st != BL_OK) return st;
@@ -883,6 +901,7 @@ bl_status bl_quant_act_relu2(const uint16_t* G, const uint16_t* U, int64_t M, in
 bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
                            const float* gamma, int bits, uint16_t* Y, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_relu2");
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if ((st = check_m(M, K)) != BL_OK) return st;
@@ -935,6 +954,7 @@ size_t bl_forward_ex_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits, 
 bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, const float* gamma,
                         int bits, unsigned flags, const float* bias, uint16_t* Y, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_ex");
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if ((st = check_m(M, K)) != BL_OK) return st;
