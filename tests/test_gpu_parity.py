@@ -124,6 +124,19 @@ def test_small_shapes(M, K, N, bits):
     check_forward(X, Wp, g, c, bits)
 
 
+# few weight-row tiles and long K (the one-SM GEMM with few tiles per launch)
+SPLIT_K = [(16, 6912, 2560), (5, 4096, 300), (33, 2560, 1000), (64, 8192, 700), (3, 1024, 64)]
+
+
+@pytest.mark.parametrize("M,K,N", SPLIT_K)
+def test_few_tiles_long_k(M, K, N):
+    X, W = random_case(M, K, N, seed=M * 100 + K + N)
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    Wp, gd = check_weights(W, g, c, o.pack_ternary(c))
+    check_forward(X, Wp, g, c, 8)
+
+
 def test_zero_inputs_and_degenerate_rows():
     M, K, N = 5, 128, 96
     X, W = random_case(M, K, N, seed=7)
@@ -325,7 +338,7 @@ def test_quant_act_relu2_bit_exact(M, K, gated, bits):
 
 
 RELU2_CASES = [(1, 2560, 700), (1, 6912, 2560), (1, 8192, 2100), (1, 8192, 8192), (1, 16384, 64),
-               (2, 320, 130), (3, 256, 512), (17, 320, 130), (130, 256, 300)]
+               (2, 320, 130), (3, 256, 512), (17, 320, 130), (130, 256, 300), (16, 4096, 300)]
 
 
 @pytest.mark.parametrize("M,K,N", RELU2_CASES)
@@ -362,7 +375,7 @@ def test_forward_relu2_bits4_and_zero_rows():
 # ---------------------------------------------------------------------------
 
 EX_CASES = [(1, 2560, 700), (1, 8192, 8192), (1, 16384, 64), (2, 320, 130), (3, 256, 512), (17, 320, 130),
-            (130, 256, 300), (300, 1024, 700)]
+            (130, 256, 300), (300, 1024, 700), (16, 4096, 300)]
 
 
 @pytest.mark.parametrize("M,K,N", EX_CASES)
