@@ -141,7 +141,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def oracle_step_fn(workload_name, row_fraction=1.0):
-    """Return (fn, bytes_per_call, description): fn() runs the oracle's forward
+    """Return (fn, bytes_per_call, ops_per_call, description): fn() runs the oracle's forward
     scope (activation quantisation, integer matmul, rescale, bf16 rounding)
     over every layer of the workload, restricted to the first
     ceil(row_fraction * N) output features of each layer."""
@@ -150,6 +150,7 @@ def oracle_step_fn(workload_name, row_fraction=1.0):
     w = WORKLOADS[workload_name]
     layers = []
     nbytes = 0
+    ops = 0
     for i, L in enumerate(w.layers):
         X, W = layer_inputs(w, i)
         n = max(1, int(math.ceil(row_fraction * L.N)))
@@ -157,7 +158,9 @@ def oracle_step_fn(workload_name, row_fraction=1.0):
         g = o.absmean_scale(W)
         c = o.ternary_codes(W, g)
         layers.append((X, g, c))
-        nbytes += algorithmic_bytes(w.M, L.K, n)
+        # an input shared with an earlier layer (same hidden state) is counted once, as on the GPU arm
+        nbytes += algorithmic_bytes(w.M, L.K, n) - (2 * w.M * L.K if L.x_layer >= 0 else 0)
+        ops += algorithmic_ops(w.M, L.K, n)
 
     def fn():
         for X, g, c in layers:
@@ -167,7 +170,7 @@ def oracle_step_fn(workload_name, row_fraction=1.0):
             o.round_to_bf16_bits(y32)
 
     desc = f"{workload_name}, first {row_fraction:.4g} of each layer's output rows"
-    return fn, nbytes, desc
+    return fn, nbytes, ops, desc
 
 
 def blas_threads():
@@ -182,7 +185,7 @@ def blas_threads():
 
 
 def cpu_baseline(workload_name, budget_s=10.0):
-    fn, nbytes, desc = oracle_step_fn(workload_name)
+    fn, nbytes, _ops, desc = oracle_step_fn(workload_name)
     fn()   # warm
     t0 = time.perf_counter()
     n = 0
@@ -203,29 +206,36 @@ def run_reference(args):
     name = args.workload
     K, W = args.steps, args.warmup
     # calibrate one full step, then size each step so the run stays within ~2 minutes
-    fn, nbytes, _ = oracle_step_fn(name)
+    fn, nbytes, ops, _ = oracle_step_fn(name)
     t0 = time.perf_counter()
     fn()
     t_full = time.perf_counter() - t0
     frac = min(1.0, 120.0 / max(1e-9, (K + W) * t_full))
     if frac < 1.0:
-        fn, nbytes, _ = oracle_step_fn(name, frac)
+        fn, nbytes, ops, _ = oracle_step_fn(name, frac)
     for _ in range(W):
         fn()
     t0 = time.perf_counter()
     for _ in range(K):
         fn()
     dt = time.perf_counter() - t0
-    value = nbytes * K / dt / 1e9
+    from bitlinear_bl_forward_b200.inputs import WORKLOADS
+    w = WORKLOADS[name]
+    decode = w.M <= 2
+    unit = "GB/s" if decode else "TOPS"
+    value = (nbytes * K / dt / 1e9) if decode else (ops * K / dt / 1e12)
     cores = blas_threads()
+    groups = [list(gr) for gr in w.groups] or [[i] for i in range(len(w.layers))]
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": K,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": K,
         "warmup": W, "ms_per_step": dt / K * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": name},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic (seeded; the oracle on the host cores)",
+        "config": {"workload": name, "M": w.M, "layers": [[L.name, L.K, L.N] for L in w.layers], "bits": w.bits,
+                   "calls_per_step": [[w.layers[j].name for j in gr] for gr in groups],
+                   "parallelism": "host cores (rank 0 only)"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": f"each step: {name}, fraction {frac:.4g} of each layer's output rows"},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
