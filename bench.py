@@ -466,18 +466,24 @@ def time_e2e(wl, steps, warmup, dist_ctx):
 
 
 class DistCtx:
-    def __init__(self, ngpus):
+    """One process per GPU (torchrun environment): barrier and max over ranks.
+    NCCL on GPUs; ``backend="gloo"`` runs the same logic on CPU processes."""
+
+    def __init__(self, ngpus, backend=None):
         import torch
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend or "nccl"
+        self.device = "cuda" if self.backend == "nccl" else "cpu"
         self.dist = None
-        torch.cuda.set_device(self.local)
+        if self.device == "cuda":
+            torch.cuda.set_device(self.local)
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"device_id": torch.device("cuda", self.local)} if self.device == "cuda" else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.dist = dist
 
     def barrier(self):
@@ -488,7 +494,7 @@ class DistCtx:
         if self.dist is None:
             return v
         import torch
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
 
@@ -496,6 +502,12 @@ class DistCtx:
         if self.dist is not None:
             self.dist.barrier()
             self.dist.destroy_process_group()
+
+
+def replica_value(work_per_rank, n_ranks, ms_max):
+    """Whole-job throughput of N independent replicas: every rank's work over
+    the slowest rank's time (weak scaling)."""
+    return n_ranks * work_per_rank / (ms_max / 1e3)
 
 
 def roofline_entry(kind, achieved, peak, unit, traffic):
@@ -525,10 +537,10 @@ def run_gpu(args):
     N = ctx.world
     sec = ms / 1e3
     if decode:
-        value = N * wl.bytes_per_step * K / sec / 1e9
+        value = replica_value(wl.bytes_per_step * K, N, ms) / 1e9
         unit = "GB/s"
     else:
-        value = N * wl.ops_per_step * K / sec / 1e12
+        value = replica_value(wl.ops_per_step * K, N, ms) / 1e12
         unit = "TOPS"
 
     # dominant kernel: on the decode path every launch of the step is the
