@@ -1,9 +1,12 @@
 // One-token BitLinear forward (decode), built for back-to-back launches.
 //
-// What it computes is the decode case of "BitNet b1.58" (The Era of 1-bit
-// LLMs), section 2 (absmean ternary weights, per-token absmax int8
-// activations) with the integer dot products of "bitnet.cpp" (Efficient Edge
-// Inference for Ternary LLMs), section 3: y = f32(f32(sum_k c*q) * f32(gamma/s)).
+// What it computes is the one-token case of the BitLinear forward of "BitNet
+// b1.58: The 1-Bit Ternary LLM Architecture Guide", section "The
+// Mathematical Formulation of BitLinear" (absmean ternary weights, eq. (1);
+// per-token absmax int8 activations, eq. (2); integer matmul and one rescale,
+// eq. (3)): y = f32(f32(sum_k c*q) * f32(gamma/s)), the sum taken exactly in
+// integers (each ternary weight adds, subtracts or skips an activation: the
+// same page, section "Why 1.58 Bits? The Power of Zero").
 //
 // The shape of the work: every weight byte is read once, the token is 5-16 KB,
 // and a whole decode layer is a few MB, i.e. well under a microsecond of HBM

@@ -316,7 +316,8 @@ def test_grouped_mixed_shapes_fall_back_to_sequential():
 
 
 # ---------------------------------------------------------------------------
-# squared-ReLU feed-forward input ("BitNet 2B4T Guide", section 2)
+# squared-ReLU feed-forward input ("BitNet 2B4T Guide: Scaling Native 1.58-Bit
+# LLMs", section "2. Squared ReLU Activation")
 # ---------------------------------------------------------------------------
 
 def relu2_inputs(M, K, N, seed):
