@@ -53,8 +53,9 @@ __device__ __forceinline__ uint2 quant8_bf16(uint4 v, float s, int Q, int& sum) 
 
 // Input modes of the token prologues: bf16 activations, int8 codes given
 // directly, or the squared-ReLU feed-forward input ("BitNet 2B4T Guide:
-// Scaling Native 1.58-Bit LLMs", section "2. Squared ReLU Activation") h = max(0, g)^2 of the gate
-// projection's bf16 output g, optionally times the up projection's output u.
+// Scaling Native 1.58-Bit LLMs", section "2. Squared ReLU Activation"):
+// h = max(0, g)^2 of the gate projection's bf16 output g, optionally times the
+// up projection's output u.
 enum InMode : int { kInBF16 = 0, kInI8 = 1, kInRelu2 = 2, kInRelu2Gated = 3 };
 
 // h for 8 consecutive elements (fp32; exact for bf16 g and u).
@@ -205,9 +206,9 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uin
 }
 
 // Tensor-wide absmax of bf16 activations ("BitNet 2B4T Guide: Scaling Native
-// 1.58-Bit LLMs", section "1. The BitLinear Operator", per-tensor form): non-negative floats order as
-// their bit patterns, so a max of the bits is the max of the values.
-// *amax_out must be zero before the launch.
+// 1.58-Bit LLMs", section "1. The BitLinear Operator", per-tensor form):
+// non-negative floats order as their bit patterns, so a max of the bits is the
+// max of the values.  *amax_out must be zero before the launch.
 __global__ void __launch_bounds__(256) act_absmax_kernel(const uint16_t* __restrict__ X, int64_t nchunks,
                                                         uint32_t* __restrict__ amax_out) {
   const uint4* x4 = reinterpret_cast<const uint4*>(X);
