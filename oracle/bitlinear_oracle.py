@@ -24,7 +24,10 @@ Sources (web pages, cited by title and section):
        section "2. Squared ReLU Activation": ReLU^2(x) = (max(0, x))^2
          between the feed-forward projections (the page's module applies it
          to the gate projection's output and feeds the result to the down
-         projection).
+         projection);
+       section "3. Sub-Layer Normalization (SubLN)" and the pipeline figure
+         of the same page: the activations pass through RMSNorm right
+         before the absmax quantisation.
 
 Readings where the pages are silent or disagree (each one is listed with its
 reason in the design notes of the repository):
@@ -49,6 +52,11 @@ reason in the design notes of the repository):
     and the fp32 value obtained with the pages' fp32 tensor arithmetic
     (f32(f32(acc) * f32(gamma / s_m))).  The bf16 output is the
     round-to-nearest-even bf16 of a value.
+
+  * RMSNorm (named, not defined, by the pages): ms = mean of the squares,
+    summed exactly and rounded once to fp32; r = sqrt(f32(ms + eps)); the
+    normalised value is bf16(f32(f32(x / r) * w)), every step an IEEE fp32
+    operation; the weight w (bf16 [K]) is optional.
 
 Array conventions: X is [M, K] (tokens x in-features) given as raw bf16 bit
 patterns (uint16); W is [N, K] fp32 (out-features x in-features, the
@@ -79,6 +87,9 @@ __all__ = [
     "forward",
     "forward_relu2",
     "forward_ex",
+    "exact_square_sum",
+    "rms_norm",
+    "forward_rmsnorm",
 ]
 
 # Floor used for both scales (pages' code listings clamp(min=1e-5)).
@@ -452,3 +463,86 @@ def forward_ex(x_bits: np.ndarray, W: np.ndarray, bits: int = 8, per_tensor: boo
         y32 = (y32 + b[None, :]).astype(np.float32)
     return {"gamma": gamma, "codes": codes, "q": q, "s": s, "acc": acc, "y64": y64, "y32": y32,
             "Y": round_to_bf16_bits(y32)}
+
+
+# ---------------------------------------------------------------------------
+# [P3] section "3. Sub-Layer Normalization (SubLN)": RMS normalisation of the
+# activations immediately before their absmax quantisation
+# ---------------------------------------------------------------------------
+
+def exact_square_sum(x_bits: np.ndarray) -> int:
+    """Exact value of sum_k x_k^2 over bf16 values, as an integer count of
+    2^-266 (the square of the smallest bf16 subnormal, 2^-133).
+
+    A finite bf16 with biased exponent e and 7-bit fraction f is
+    sig * 2^(max(e, 1) - 134) with sig = 128 + f for e > 0 and sig = f for
+    e = 0, so its square is sig^2 * 2^(2 max(e, 1) - 2) units.  Squares are
+    grouped by exponent (each group's significand sum is an integer below
+    2^53, exact in np.bincount's float64) and the groups are combined with
+    Python integers.
+    """
+    b = np.ascontiguousarray(x_bits, dtype=np.uint16).ravel().astype(np.int64)
+    e = (b >> 7) & 0xFF
+    f = b & 0x7F
+    if np.any(e == 255):
+        raise ValueError("non-finite activation")
+    if b.size >= (1 << 36):
+        raise ValueError("too many values for the exact sum")
+    sig = np.where(e > 0, f | 0x80, f)
+    sh = 2 * np.maximum(e, 1) - 2
+    groups = np.bincount(sh, weights=(sig * sig).astype(np.float64), minlength=510)
+    total = 0
+    for k in range(len(groups)):
+        if groups[k]:
+            total += int(groups[k]) << k
+    return total
+
+
+def rms_norm(x_bits: np.ndarray, weight_bits: np.ndarray | None = None, eps: float = 1e-5):
+    """RMSNorm of bf16 activations [M, K], per token, with an optional bf16
+    weight [K] ([P1] best-practice table, row "LayerNorm Preservation": the
+    normalisation parameters stay in bf16).
+
+    The pages name the operation (x_norm = RMSNorm(x) ahead of the absmax
+    step in [P3]'s pipeline figure) but fix no precision.  Reading:
+        ms  = fp32( (1/K) sum_k x_k^2 )      exact sum, rounded once
+        r   = sqrt( f32(ms + eps) )          fp32 square root (IEEE)
+        t   = f32(x / r)                     fp32 division (IEEE)
+        t   = f32(t * w_k)                   only with a weight
+        x_n = bf16(t)                        round to nearest even
+    x_n is what a bf16 model hands to the BitLinear layer, so the fused
+    operation equals ``forward`` applied to x_n.
+
+    Returns a dict: ms fp32 [M], r fp32 [M], xn bf16 bits [M, K].
+    """
+    x = bf16_bits_to_f32(x_bits)
+    if x.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    M, K = x.shape
+    if K == 0:
+        raise ValueError("K must be positive")
+    e32 = np.float32(eps)
+    if not (np.isfinite(e32) and e32 > 0):
+        raise ValueError("eps must be a positive finite fp32 value")
+    ms = np.empty(M, np.float32)
+    for m in range(M):
+        ms[m] = round_rational_to_f32(exact_square_sum(x_bits[m]), K << 266)
+    v = (ms + e32).astype(np.float32)
+    r = np.sqrt(v).astype(np.float32)
+    t = (x / r[:, None]).astype(np.float32)
+    if weight_bits is not None:
+        w = bf16_bits_to_f32(weight_bits)
+        if w.shape != (K,):
+            raise ValueError("weight must be [K]")
+        t = (t * w[None, :]).astype(np.float32)
+    return {"ms": ms, "r": r, "xn": round_to_bf16_bits(t)}
+
+
+def forward_rmsnorm(x_bits: np.ndarray, W: np.ndarray, weight_bits: np.ndarray | None = None,
+                    eps: float = 1e-5, bits: int = 8):
+    """BitLinear on the RMS-normalised activations: ``forward(rms_norm(x))``.
+    Same dict as ``forward`` plus ms, r and xn."""
+    nrm = rms_norm(x_bits, weight_bits, eps)
+    out = forward(nrm["xn"], W, bits)
+    out.update(nrm)
+    return out

@@ -503,3 +503,129 @@ def test_forward_ex_bias_hand_case():
     assert out["acc"][0, 0] == 143
     assert out["y32"][0, 0] == np.float32(np.float32(plain["y32"][0, 0]) + np.float32(-0.25))
     assert abs(out["y64"][0, 0] - (plain["y64"][0, 0] - 0.25)) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# P3 section "3. Sub-Layer Normalization (SubLN)": RMSNorm before the absmax
+# ---------------------------------------------------------------------------
+
+def _bf16_of(values):
+    """Round-to-nearest-even bf16 bit patterns, computed by torch (independent
+    of the oracle's own rounding helper)."""
+    t = torch.tensor(np.asarray(values, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_exact_square_sum_against_fractions():
+    rng = np.random.default_rng(41)
+    # every exponent class, subnormals and zeros included
+    bits = rng.integers(0, 0x7F80, size=700).astype(np.uint16)
+    bits[:40] = rng.integers(0, 0x80, size=40)          # subnormals and zero
+    bits[40:60] = 0
+    signs = rng.integers(0, 2, size=bits.size).astype(np.uint16) << 15
+    bits = bits | signs
+    vals = o.bf16_bits_to_f32(bits).astype(np.float64)
+    exact = sum((Fraction(float(v)) ** 2 for v in vals), Fraction(0))
+    assert Fraction(o.exact_square_sum(bits), 1 << 266) == exact
+
+
+def test_rms_norm_closed_form_rms_of_one_and_seven():
+    # half the entries 1, half -7: mean of squares (1 + 49) / 2 = 25, RMS 5
+    K = 64
+    x = to_bf16_bits_exact([1.0] * (K // 2) + [-7.0] * (K // 2))[None, :]
+    r = o.rms_norm(x, eps=1e-30)
+    assert r["ms"][0] == np.float32(25.0) and r["r"][0] == np.float32(5.0)
+    want = _bf16_of([1.0 / 5.0] * (K // 2) + [-7.0 / 5.0] * (K // 2))
+    assert np.array_equal(r["xn"][0], want)
+
+
+def test_rms_norm_unit_rows_map_to_themselves():
+    rng = np.random.default_rng(5)
+    x = to_bf16_bits_exact(rng.choice([-1.0, 1.0], size=(3, 256)))
+    r = o.rms_norm(x, eps=1e-30)
+    assert np.all(r["ms"] == 1.0) and np.all(r["r"] == 1.0)
+    assert np.array_equal(r["xn"], x)
+
+
+def test_rms_norm_power_of_two_scale_invariance():
+    # x -> 2^j x with eps -> 4^j eps scales ms by 4^j and r by 2^j exactly,
+    # so the normalised values do not move
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((4, 320)).astype(np.float32)
+    xb = _bf16_of(x)
+    base = o.rms_norm(xb, eps=2.0 ** -20)
+    for j in (-9, -1, 3, 12):
+        xs = _bf16_of(o.bf16_bits_to_f32(xb) * np.float32(2.0 ** j))
+        r = o.rms_norm(xs, eps=2.0 ** (-20 + 2 * j))
+        assert np.array_equal(r["ms"], (base["ms"] * np.float32(4.0 ** j)).astype(np.float32))
+        assert np.array_equal(r["r"], (base["r"] * np.float32(2.0 ** j)).astype(np.float32))
+        assert np.array_equal(r["xn"], base["xn"])
+
+
+def test_rms_norm_mean_of_squares_is_rounded_once_from_the_exact_sum():
+    # K = 128: 64 ones and one 2^-9 give sum 64 + 2^-18, mean 0.5 + 2^-25,
+    # exactly halfway between the fp32 neighbours 0.5 and 0.5 + 2^-24: ties
+    # to even -> 0.5.  One more entry 2^-60 puts the exact mean just above the
+    # midpoint -> 0.5 + 2^-24, which a float64 sum would miss.
+    K = 128
+    v = np.zeros(K, np.float32)
+    v[:64] = 1.0
+    v[64] = 2.0 ** -9
+    r = o.rms_norm(to_bf16_bits_exact(v)[None, :], eps=2.0 ** -40)
+    assert r["ms"][0] == np.float32(0.5)
+    v[65] = 2.0 ** -60
+    r = o.rms_norm(to_bf16_bits_exact(v)[None, :], eps=2.0 ** -40)
+    assert r["ms"][0] == np.float32(0.5 + 2.0 ** -24)
+    assert np.float32(np.sum(v.astype(np.float64) ** 2) / K) == np.float32(0.5)
+
+
+def test_rms_norm_weight():
+    rng = np.random.default_rng(7)
+    xb = _bf16_of(rng.standard_normal((2, 128)))
+    plain = o.rms_norm(xb, eps=1e-6)
+    two = o.rms_norm(xb, to_bf16_bits_exact(np.full(128, 2.0)), eps=1e-6)
+    assert np.array_equal(o.bf16_bits_to_f32(two["xn"]), 2.0 * o.bf16_bits_to_f32(plain["xn"]))
+    w = np.ones(128, np.float32)
+    w[::3] = 0.0
+    z = o.rms_norm(xb, to_bf16_bits_exact(w), eps=1e-6)
+    assert np.all(o.bf16_bits_to_f32(z["xn"])[:, ::3] == 0.0)
+    assert np.array_equal(z["xn"][:, 1::3], plain["xn"][:, 1::3])
+
+
+def test_rms_norm_against_float64_brute_force():
+    rng = np.random.default_rng(8)
+    M, K = 6, 448
+    x = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-8, 8, size=(M, 1)))).astype(np.float32)
+    x[:, rng.integers(0, K, 4)] *= 30.0
+    xb = _bf16_of(x)
+    wb = _bf16_of(rng.uniform(0.5, 1.5, size=K))
+    eps = 1e-5
+    r = o.rms_norm(xb, wb, eps=eps)
+    x64 = o.bf16_bits_to_f32(xb).astype(np.float64)
+    w64 = o.bf16_bits_to_f32(wb).astype(np.float64)
+    ref = x64 / np.sqrt(np.mean(x64 ** 2, axis=1, keepdims=True) + eps) * w64
+    got = o.bf16_bits_to_f32(r["xn"]).astype(np.float64)
+    ulp = np.ldexp(1.0, np.frexp(np.abs(ref))[1] - 8)   # one bf16 ulp at |ref|
+    assert np.all(np.abs(got - ref) <= ulp)
+
+
+def test_rms_norm_zero_row_and_bad_eps():
+    x = np.zeros((2, 64), np.uint16)
+    x[1, 5] = 0x3F80
+    r = o.rms_norm(x, eps=0.25)
+    assert r["ms"][0] == 0.0 and r["r"][0] == np.float32(0.5)
+    assert np.all(r["xn"][0] == 0)
+    # one entry 1 of 64: ms = 1/64, r = sqrt(1/64 + 0.25)
+    assert r["ms"][1] == np.float32(1.0 / 64.0)
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(ValueError):
+            o.rms_norm(x, eps=bad)
+
+
+def test_forward_rmsnorm_is_forward_on_the_normalised_input():
+    rng = np.random.default_rng(9)
+    xb = _bf16_of(rng.standard_normal((3, 128)) * 4.0)
+    W = rng.standard_normal((32, 128)).astype(np.float32)
+    got = o.forward_rmsnorm(xb, W, eps=1e-5, bits=4)
+    ref = o.forward(o.rms_norm(xb, eps=1e-5)["xn"], W, bits=4)
+    assert np.array_equal(got["Y"], ref["Y"]) and np.array_equal(got["q"], ref["q"])
