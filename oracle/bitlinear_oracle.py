@@ -139,8 +139,9 @@ def round_rational_to_f32(p: int, q: int) -> np.float32:
     if 2 * r > den or (2 * r == den and (m & 1)):
         m += 1
     # m * 2^-shift is the rounded value; a carry into the next binade
-    # (m == 2^24) is still exactly representable.
-    if e >= 127 and m >= (1 << 24):
+    # (m == 2^24) is still exactly representable.  A rounded value of 2^128
+    # or more overflows to infinity (IEEE round to nearest).
+    if e > 127 or (e == 127 and m >= (1 << 24)):
         return np.float32(np.inf)
     val = float(m) * 2.0 ** (-shift)   # exact in fp64: m < 2^25
     out = np.float32(val)

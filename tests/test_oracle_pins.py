@@ -629,3 +629,15 @@ def test_forward_rmsnorm_is_forward_on_the_normalised_input():
     got = o.forward_rmsnorm(xb, W, eps=1e-5, bits=4)
     ref = o.forward(o.rms_norm(xb, eps=1e-5)["xn"], W, bits=4)
     assert np.array_equal(got["Y"], ref["Y"]) and np.array_equal(got["q"], ref["q"])
+
+
+def test_round_rational_overflow_boundary():
+    # IEEE round to nearest: the largest fp32 is (2^24 - 1) 2^104; values
+    # from the midpoint (2^128 - 2^103) up round to infinity, below it to the
+    # largest fp32
+    fmax = np.finfo(np.float32).max
+    assert o.round_rational_to_f32((1 << 128) - (1 << 104), 1) == fmax
+    assert o.round_rational_to_f32((1 << 128) - (1 << 103) - 1, 1) == fmax
+    assert np.isinf(o.round_rational_to_f32((1 << 128) - (1 << 103), 1))
+    assert np.isinf(o.round_rational_to_f32(1 << 128, 1))
+    assert np.isinf(o.round_rational_to_f32(3 << 300, 7))
