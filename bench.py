@@ -333,6 +333,34 @@ class FfnWorkload(GpuWorkload):
                             workspace=down["ws"])
 
 
+class RmsWorkload(GpuWorkload):
+    """Every layer of a workload through bl_forward_rmsnorm: RMSNorm with a
+    bf16 weight [K], then the BitLinear forward, one call per layer (one
+    launch for a one-token layer, normalising quantiser + GEMM otherwise)."""
+
+    def __init__(self, name, rotations, seed=0, device="cuda"):
+        import torch
+        from bitlinear_bl_forward_b200 import bl
+        super().__init__(name, rotations, seed, device)
+        g = torch.Generator(device=device).manual_seed(seed + 99)
+        for d in self.layers:
+            L = d["L"]
+            d["nw"] = (torch.rand(L.K, generator=g, device=device) + 0.5).to(torch.bfloat16)
+            n = bl.bl_forward_rmsnorm_workspace_bytes(self.w.M, L.K, L.N, self.w.bits)
+            d["ws"] = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+        self.groups = [[i] for i in range(len(self.layers))]
+        self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N) + 2 * d["L"].K for d in self.layers)
+        self.launches_per_step = len(self.layers) * (1 if self.w.M == 1 else 2)
+
+    def step(self, i):
+        from bitlinear_bl_forward_b200 import bl
+        r = i % self.rotations
+        for d in self.layers:
+            Wp, gamma = d["copies"][r]
+            bl.bl_forward_rmsnorm(d["X"], Wp, gamma, d["L"].N, self.w.bits, norm_weight=d["nw"], eps=1e-5,
+                                  out=d["Y"], workspace=d["ws"])
+
+
 def time_quantize_weights(N=28672, K=8192, reps=5):
     """bl_quantize_weights on a 70B-class layer: GB/s of fp32 weights read
     (offline step, not part of the forward metric)."""
@@ -625,6 +653,25 @@ def secondary(args, ctx, peaks):
         out.append({"workload": "ffn_2b_decode", "M": 1, "ms_per_step": ms / steps, "GB/s": gbs,
                     "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps,
                     "note": "down input = max(0, gate)^2 * up of the same step, formed in the down kernel"})
+        del wl
+        torch.cuda.empty_cache()
+    for name, base, steps, rot in (("rmsnorm_decode_2b", "decode_2b", 20000, 20),
+                                   ("rmsnorm_prefill_2b", "prefill_2b", 300, 20)):
+        if args.secondary and name not in args.secondary.split(","):
+            continue
+        # the same layers with RMSNorm (bf16 weight) formed ahead of the quantiser
+        wl = RmsWorkload(base, rot)
+        ms, _ = time_workload(wl, steps, 3, ctx, sample_clocks=False)
+        sec = ms / 1e3
+        gbs = wl.bytes_per_step * steps / sec / 1e9
+        ent = {"workload": name, "M": wl.w.M, "ms_per_step": ms / steps, "GB/s": gbs,
+               "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps,
+               "note": "one bl_forward_rmsnorm call per layer (norm weight read counted)"}
+        if wl.w.M > 1:
+            tops = wl.ops_per_step * steps / sec / 1e12
+            ent["TOPS"] = tops
+            ent["tensor_frac"] = tops / (peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO)
+        out.append(ent)
         del wl
         torch.cuda.empty_cache()
     if not args.secondary or "quantize_weights_70b" in args.secondary.split(","):

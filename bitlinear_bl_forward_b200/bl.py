@@ -45,6 +45,9 @@ SIGNATURES = {
     "bl_quant_act_relu2": (_int, [_p, _p, _i64, _i64, _int, _p, _p, _p]),
     "bl_forward_ex_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, ctypes.c_uint]),
     "bl_forward_ex": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, ctypes.c_uint, _p, _p, _p, _sz, _p]),
+    "bl_forward_rmsnorm_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
+    "bl_forward_rmsnorm": (_int, [_p, _p, ctypes.c_float, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
+    "bl_quant_act_rmsnorm": (_int, [_p, _p, ctypes.c_float, _i64, _i64, _int, _p, _p, _p, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
@@ -294,6 +297,48 @@ def bl_forward_ex(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int
                                ws.data_ptr() if ws is not None else None,
                                ws.numel() if ws is not None else 0, _stream()), "bl_forward_ex")
     return Y
+
+
+def bl_forward_rmsnorm_workspace_bytes(M: int, K: int, N: int, bits: int = 8) -> int:
+    return int(lib().bl_forward_rmsnorm_workspace_bytes(M, K, N, bits))
+
+
+def bl_forward_rmsnorm(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8,
+                       norm_weight: torch.Tensor | None = None, eps: float = 1e-5,
+                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """bl_forward on RMSNorm(X) (optional bf16 weight [K]), formed in the same
+    kernels: bf16 [M, K] -> bf16 [M, N]."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pn = _dev(norm_weight, torch.bfloat16, "norm_weight") if norm_weight is not None else None
+    if norm_weight is not None and tuple(norm_weight.shape) != (K,):
+        raise ValueError("norm_weight must be [K]")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    ws = workspace
+    if ws is None:
+        ws = _workspace(bl_forward_rmsnorm_workspace_bytes(M, K, N, bits), X.device)
+    _check(lib().bl_forward_rmsnorm(px, pn, eps, M, K, N, pw, pg, bits, py,
+                                    ws.data_ptr() if ws is not None else None,
+                                    ws.numel() if ws is not None else 0, _stream()), "bl_forward_rmsnorm")
+    return Y
+
+
+def bl_quant_act_rmsnorm(X: torch.Tensor, bits: int = 8, norm_weight: torch.Tensor | None = None,
+                         eps: float = 1e-5):
+    """RMSNorm(X) quantised per token -> (int8 codes [M, K], scale fp32 [M],
+    mean of squares fp32 [M])."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pn = _dev(norm_weight, torch.bfloat16, "norm_weight") if norm_weight is not None else None
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    ms = torch.empty(M, dtype=torch.float32, device=X.device)
+    _check(lib().bl_quant_act_rmsnorm(px, pn, eps, M, K, bits, Xq.data_ptr(), s.data_ptr(), ms.data_ptr(),
+                                      _stream()), "bl_quant_act_rmsnorm")
+    return Xq, s, ms
 
 
 def bl_matmul_i32(Xq: torch.Tensor, Wp: torch.Tensor, N: int) -> torch.Tensor:

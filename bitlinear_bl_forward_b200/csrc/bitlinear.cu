@@ -7,6 +7,7 @@
 //               tcgen05 kind::i8 GEMM (weights expanded into tensor memory).
 #include <atomic>
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 
 #include <cuda.h>
@@ -206,9 +207,9 @@ bl_status launch_gemv2_cpl(int cpl, const bl::G2Table& tab, int grid, int x_is_i
 template <int WPL>
 constexpr int g3_warps() { return BL_G3_WARPS; }
 
-template <int WPL, bool RELU2>
+template <int WPL, int PRE>
 bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode, cudaStream_t stream) {
-  auto kern = bl::gemv3_kernel<WPL, g3_warps<WPL>(), RELU2>;
+  auto kern = bl::gemv3_kernel<WPL, g3_warps<WPL>(), PRE>;
   static std::atomic<uint64_t> done{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
@@ -242,12 +243,15 @@ bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int 
 // words of 16 weights per lane: K / 512 rounded up (K <= 8192)
 bl_status launch_gemv3_wpl(int wpl, const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode,
                            cudaStream_t stream) {
-  const bool relu2 = x_is_i8 == bl::kInRelu2 || x_is_i8 == bl::kInRelu2Gated;
+  const int pre = (x_is_i8 == bl::kInRelu2 || x_is_i8 == bl::kInRelu2Gated) ? bl::kG3Relu2
+                  : x_is_i8 == bl::kInRmsNorm                                ? bl::kG3Rms
+                                                                             : bl::kG3Plain;
   switch (wpl) {
-#define BL_G3_CASE(n) \
-  case n:                                                                                     \
-    return relu2 ? launch_gemv3_table<n, true>(tab, grid, x_is_i8, Q, out_mode, stream)       \
-                 : launch_gemv3_table<n, false>(tab, grid, x_is_i8, Q, out_mode, stream);
+#define BL_G3_CASE(n)                                                                    \
+  case n:                                                                                \
+    return pre == bl::kG3Relu2 ? launch_gemv3_table<n, bl::kG3Relu2>(tab, grid, x_is_i8, Q, out_mode, stream) \
+           : pre == bl::kG3Rms ? launch_gemv3_table<n, bl::kG3Rms>(tab, grid, x_is_i8, Q, out_mode, stream)   \
+                               : launch_gemv3_table<n, bl::kG3Plain>(tab, grid, x_is_i8, Q, out_mode, stream);
     BL_G3_CASE(1) BL_G3_CASE(2) BL_G3_CASE(3) BL_G3_CASE(4) BL_G3_CASE(5) BL_G3_CASE(6) BL_G3_CASE(7) BL_G3_CASE(8)
     BL_G3_CASE(9) BL_G3_CASE(10) BL_G3_CASE(11) BL_G3_CASE(12) BL_G3_CASE(13) BL_G3_CASE(14) BL_G3_CASE(15)
     BL_G3_CASE(16)
@@ -1001,6 +1005,85 @@ bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t N, cons
     return st;
   }
   return launch_tc(Xq, m, k, static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16, 0, stream, bias);
+}
+
+size_t rms_ws_bytes(int64_t M, int64_t K) {
+  return align_up(static_cast<size_t>(M) * K, 256) + 3 * align_up(static_cast<size_t>(M) * 4, 256);
+}
+
+size_t bl_forward_rmsnorm_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+  (void)bits;
+  if (check_shape_nk(N, K) != BL_OK || check_m(M, K) != BL_OK || M == 0) return 0;
+  return rms_ws_bytes(M, K);
+}
+
+bool rms_eps_ok(float eps) { return eps > 0.f && std::isfinite(eps); }
+
+bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
+                               int bits, int8_t* Xq, float* scale, float* mean_sq, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quant_act_rmsnorm");
+  if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
+  bl_status st = check_m(M, K);
+  if (st != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (!rms_eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!X || !Xq || !scale) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Xq) || (norm_weight && !aligned16(norm_weight)) ||
+      (reinterpret_cast<uintptr_t>(mean_sq) & 3u))
+    return BL_ERR_ALIGNMENT;
+  bl::act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+      X, norm_weight, eps, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr, mean_sq);
+  return last_cuda();
+}
+
+bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
+                             int64_t N, const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_rmsnorm");
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  if (!rms_eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!X || !Wp || !gamma || !Y) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wp) || (norm_weight && !aligned16(norm_weight))) return BL_ERR_ALIGNMENT;
+  const size_t need = rms_ws_bytes(M, K);
+  if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+  const int Q = bits == 8 ? 127 : 7;
+  const int sms = num_sms();
+  const double wbytes = static_cast<double>(N) * static_cast<double>(K) / 4.0;
+  if (M == 1 && K <= bl::kG3MaxK &&
+      wbytes <= static_cast<double>(sms) * bl::kG3Stages * bl::kG3StageBytes) {
+    // one token whose layer fits the resident decode kernel: RMSNorm,
+    // absmax and quantisation in its prologue (the workspace stays unused)
+    bl_linear p;
+    p.X = X;
+    p.M = 1;
+    p.K = K;
+    p.N = N;
+    p.Wp = Wp;
+    p.gamma = gamma;
+    p.Y = Y;
+    const bl_linear* pp = &p;
+    bl::G2Table tab;
+    const int grid = fill_decode_table(&tab, &pp, 1, sms, norm_weight, nullptr);
+    tab.p[0].eps = eps;
+    return launch_gemv3_wpl(static_cast<int>((K + 511) / 512), tab, grid, bl::kInRmsNorm, Q, bl::kOutBF16, stream);
+  }
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const size_t codes = align_up(static_cast<size_t>(M) * K, 256), rows = align_up(static_cast<size_t>(M) * 4, 256);
+  int8_t* Xq = reinterpret_cast<int8_t*>(base);
+  float* s = reinterpret_cast<float*>(base + codes);
+  int* R = reinterpret_cast<int*>(base + codes + rows);
+  float* ms = reinterpret_cast<float*>(base + codes + 2 * rows);
+  bl::act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+      X, norm_weight, eps, static_cast<int>(K), Q, Xq, s, R, ms);
+  if ((st = last_cuda()) != BL_OK) return st;
+  return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y,
+                   bl::kOutBF16, 0, stream);
 }
 
 bl_status bl_device_status(int clear, int* site) {

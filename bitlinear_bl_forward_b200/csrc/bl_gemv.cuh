@@ -501,7 +501,8 @@ __global__ void __launch_bounds__(THREADS, MINB)
 // decode): CTAs [cta_begin, next cta_begin) of the grid work on problem i.
 struct G2Problem {
   const void* X;
-  const void* U;      // squared-ReLU gated mode: the up projection's output (else unused)
+  const void* U;      // squared-ReLU gated mode: the up projection's output;
+                      // RMSNorm mode: the norm's bf16 weight [K] or null (else unused)
   const uint8_t* Wp;
   const float* gamma;
   void* Y;
@@ -511,6 +512,7 @@ struct G2Problem {
   int cta_begin;      // first CTA of this problem in the launch
   int ctas;           // decode kernel: CTA c takes rows [c*N/ctas, (c+1)*N/ctas)
   const float* bias;  // optional fp32 [N] added after the rescale
+  float eps;          // RMSNorm mode: added to the mean of squares
 };
 constexpr int kG2MaxProblems = 8;
 struct G2Table {

@@ -23,7 +23,8 @@
 //     into shared memory) BEFORE the dependency wait, i.e. while the previous
 //     launch is still running, and only the consumers wait for the token;
 //   * consumers: quantise the token (absmax per token, Q/max(a, eps), round to
-//     nearest even, clamp), keep it in registers, then for each weight row:
+//     nearest even, clamp; optionally after squared ReLU or RMSNorm, formed
+//     in the same prologue), keep it, then for each weight row:
 //     lane l takes the 32-bit words l, l+32, ... (16 weights each; balanced for
 //     every K that is a multiple of 64), four masked unsigned-by-signed dp4a
 //     per word (slice j of a word holds 4^j * (c+1) in each byte), exact fold
@@ -33,6 +34,7 @@
 
 #include "bl_act.cuh"
 #include "bl_gemv.cuh"
+#include "bl_norm.cuh"
 
 namespace bl {
 
@@ -41,6 +43,12 @@ constexpr int kG3StageBytes = 32768;
 constexpr int kG3MaxK = 8192;
 // dynamic shared memory: [3 x 32 KB weight ring][token codes, 8 KB]
 constexpr int kG3SmemBytes = kG3Stages * kG3StageBytes + kG3MaxK;
+
+// What the token prologue forms before the quantisation: nothing (bf16
+// activations or int8 codes), the squared-ReLU input, or the RMS-normalised
+// token.  A template parameter so that the plain path carries no code for
+// the others.
+enum G3Pre : int { kG3Plain = 0, kG3Relu2 = 1, kG3Rms = 2 };
 
 template <int WPL, int CW>
 struct G3Cfg {
@@ -115,13 +123,12 @@ __device__ __forceinline__ void g3_rows(const uint8_t* sbase, int rr, int rows, 
   }
 }
 
-// RELU2: the token is the squared-ReLU feed-forward input (in_mode kInRelu2
-// or kInRelu2Gated); otherwise bf16 activations or int8 codes.  A template
-// parameter so that the plain path carries no code for it.
-template <int WPL, int CW, bool RELU2>
+template <int WPL, int CW, int PRE>
 __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
     gemv3_kernel(const __grid_constant__ G2Table tab, int in_mode, int Q, int out_mode, unsigned long long limit_ns) {
   constexpr bool ACT_SMEM = G3Cfg<WPL, CW>::kActSmem;
+  constexpr bool RELU2 = PRE == kG3Relu2;
+  constexpr bool RMS = PRE == kG3Rms;
   int pi = 0;
   while (pi + 1 < tab.count && static_cast<int>(blockIdx.x) >= tab.p[pi + 1].cta_begin) ++pi;
   const void* __restrict__ X = tab.p[pi].X;
@@ -140,6 +147,9 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
   __shared__ __align__(16) int s_red_i[CW];
   __shared__ __align__(8) uint64_t full[kG3Stages], empty[kG3Stages];
   __shared__ int abort_flag;
+  __shared__ unsigned long long s_sq[RMS ? kSqLimbs : 1];
+  __shared__ uint32_t s_dig[RMS ? kSqLimbs : 1];
+  __shared__ float s_rms;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = K >> 4;
@@ -159,6 +169,9 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
     }
     abort_flag = 0;
     fence_mbar_init();
+  }
+  if constexpr (RMS) {
+    if (threadIdx.x < kSqLimbs) s_sq[threadIdx.x] = 0ull;
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -202,9 +215,19 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
   }
 
   // ---------------- consumers: the token (written by the preceding kernel) ----------------
-  pdl_wait();
   constexpr int CT = CW * 32;
   constexpr int U = (kG3MaxK / 8 + CT - 1) / CT;
+  // the norm's weight is a parameter like Wp: fetched before the wait
+  uint4 nw[RMS ? U : 1];
+  const bool has_nw = RMS && Up != nullptr;
+  if constexpr (RMS) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = threadIdx.x + CT * u;
+      nw[u] = (has_nw && c < (K >> 3)) ? __ldg(static_cast<const uint4*>(Up) + c) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  pdl_wait();
   const bool x_is_i8 = in_mode == kInI8;
   constexpr bool relu2 = RELU2;
   const bool gated = RELU2 && in_mode == kInRelu2Gated;
@@ -215,6 +238,30 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
     const int c = threadIdx.x + CT * u;
     xv[u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + c) : make_uint4(0, 0, 0, 0);
     if constexpr (RELU2) uv[u] = (gated && c < nch) ? __ldg(static_cast<const uint4*>(Up) + c) : make_uint4(0, 0, 0, 0);
+  }
+  if constexpr (RMS) {
+    // exact mean of squares (warp windows + shared limb counters), then
+    // x_n = bf16(x / sqrt(ms + eps) * w) in place of the token
+    int emax = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (threadIdx.x + CT * u < nch) emax = max(emax, sq_exp_max8(xv[u]));
+    const int Ew = max(static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax))), 1);
+    unsigned long long lo = 0ull, hi = 0ull;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (threadIdx.x + CT * u < nch) sq_add8(xv[u], Ew, lo, hi, s_sq);
+    sq_warp_flush(lo, hi, Ew, lane, s_sq);
+    named_bar_sync(1, CT);
+    if (threadIdx.x == 0) {
+      const float ms = sq_mean_f32(s_sq, s_dig, static_cast<uint32_t>(K));
+      s_rms = __fsqrt_rn(__fadd_rn(ms, tab.p[pi].eps));
+    }
+    named_bar_sync(1, CT);
+    const float r = s_rms;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (threadIdx.x + CT * u < nch) xv[u] = rms_apply8(xv[u], nw[u], has_nw, r);
   }
   const float gamma = (out_mode == kOutI32) ? 1.f : __ldg(gamma_p);
   int rsum = 0;

@@ -1,0 +1,267 @@
+// RMS normalisation of a token right before its absmax quantisation.
+//
+// "BitNet 2B4T Guide: Scaling Native 1.58-Bit LLMs", section "3. Sub-Layer
+// Normalization (SubLN)" and the page's pipeline figure: the activations are
+// normalised (x_norm = RMSNorm(x)) and then quantised with the per-token
+// absmax.  "BitNet a4.8 Guide: 4-Bit Activation 1-Bit LLMs", table "Best
+// Practices for Deploying BitNet a4.8 in Production", row "LayerNorm
+// Preservation": the normalisation parameters stay in bf16.
+//
+// The pages fix no precision; every step here has one exact result:
+//   ms  = fp32 round-to-nearest-even of (1/K) sum_k x_k^2, the sum EXACT,
+//   r   = __fsqrt_rn(__fadd_rn(ms, eps)),
+//   x_n = bf16_rn(__fmul_rn(__fdiv_rn(x, r), w_k))   (w: optional bf16 [K]),
+// so the result does not depend on how the sum is split between threads.
+//
+// Exact sum of squares.  A finite bf16 is sig * 2^(e' - 134) with e' =
+// max(e, 1) (e the biased exponent field) and sig < 256, so its square is
+// sig^2 * 2^(2e' - 268), a 16-bit integer at bit position P = 2e' + 96 of a
+// fixed-point number whose unit is 2^-364.  P runs from 98 to 604 and a sum
+// of up to 2^16 squares stays below 2^636: twenty 32-bit limbs.
+//   * Each warp anchors a 128-bit register accumulator at the largest
+//     exponent field among its values: its bit 0 sits at position 2 E_w and a
+//     square lands at bit 96 - 2 (E_w - e'), exactly, whenever that is >= 0.
+//     That covers every value within 2^48 of the warp's largest; the warp
+//     sums its 128-bit partials with shuffles (carries kept) and five lanes
+//     add the result, cut at 32-bit limb boundaries, into 64-bit limb
+//     counters in shared memory.
+//   * A square further down (a value below 2^-48 of the warp's largest) is
+//     added straight into the limb counter at its position.
+//   * Counters never overflow: a square's shifted value is < 2^47 and at most
+//     2^16 of them reach one counter (< 2^63); warp chunks add < 2^37.
+//   * One thread normalises the counters into 32-bit digits, divides by K
+//     digit by digit (a 64-bit multiply-high by ceil(2^64 / K) gives the
+//     exact quotient digit because every partial dividend is below 2^48 and
+//     K <= 2^16), and rounds to fp32 on the quotient's bits with the
+//     remainder as sticky: normal and subnormal results, ties to even,
+//     overflow to infinity.
+#pragma once
+
+#include "bl_act.cuh"
+
+namespace bl {
+
+constexpr int kSqLimbs = 20;            // 32-bit limbs of the fixed-point sum
+constexpr int kSqWindowShift = 96;      // bit of the warp anchor's square in its 128-bit window
+constexpr int kSqUnitExp = 364;         // unit of the fixed-point sum: 2^-364
+
+// Largest biased exponent field among 8 bf16 values.
+__device__ __forceinline__ int sq_exp_max8(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t e = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) e = max(e, max((w[i] >> 7) & 0xffu, (w[i] >> 23) & 0xffu));
+  return static_cast<int>(e);
+}
+
+// One bf16 square (b: the 16-bit pattern) into the warp window (lo, hi)
+// anchored at exponent field Ew, or into the shared limb counters.
+__device__ __forceinline__ void sq_add1(uint32_t b, int Ew, unsigned long long& lo, unsigned long long& hi,
+                                        unsigned long long* acc) {
+  const uint32_t e = (b >> 7) & 0xffu, f = b & 0x7fu;
+  const uint32_t sig = e ? (f | 0x80u) : f;
+  if (sig == 0u) return;
+  const int ei = e ? static_cast<int>(e) : 1;
+  const unsigned long long sq = static_cast<unsigned long long>(sig * sig);
+  const int sh = kSqWindowShift - 2 * (Ew - ei);
+  if (sh >= 0) {
+    unsigned long long a_lo, a_hi;
+    if (sh < 64) {
+      a_lo = sq << sh;
+      a_hi = sh > 48 ? (sq >> (64 - sh)) : 0ull;
+    } else {
+      a_lo = 0ull;
+      a_hi = sq << (sh - 64);
+    }
+    lo += a_lo;
+    hi += a_hi + (lo < a_lo ? 1ull : 0ull);
+  } else {
+    const int P = 2 * ei + kSqWindowShift;
+    atomicAdd(&acc[P >> 5], sq << (P & 31));
+  }
+}
+
+__device__ __forceinline__ void sq_add8(uint4 v, int Ew, unsigned long long& lo, unsigned long long& hi,
+                                        unsigned long long* acc) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sq_add1(w[i] & 0xffffu, Ew, lo, hi, acc);
+    sq_add1(w[i] >> 16, Ew, lo, hi, acc);
+  }
+}
+
+// Warp sum of the 128-bit windows (every lane holds the total afterwards),
+// then lanes 0..4 add it, shifted to its position 2 Ew and cut into 32-bit
+// limbs, to the counters.  All 32 lanes must call it with the same Ew.
+__device__ __forceinline__ void sq_warp_flush(unsigned long long lo, unsigned long long hi, int Ew, int lane,
+                                              unsigned long long* acc) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long olo = __shfl_xor_sync(0xffffffffu, lo, o);
+    const unsigned long long ohi = __shfl_xor_sync(0xffffffffu, hi, o);
+    lo += olo;
+    hi += ohi + (lo < olo ? 1ull : 0ull);
+  }
+  if (lane < 5) {
+    const int B = 2 * Ew;
+    const uint32_t w0 = static_cast<uint32_t>(lo), w1 = static_cast<uint32_t>(lo >> 32);
+    const uint32_t w2 = static_cast<uint32_t>(hi), w3 = static_cast<uint32_t>(hi >> 32);
+    const uint32_t cur = lane == 0 ? w0 : lane == 1 ? w1 : lane == 2 ? w2 : lane == 3 ? w3 : 0u;
+    const uint32_t prev = lane == 0 ? 0u : lane == 1 ? w0 : lane == 2 ? w1 : lane == 3 ? w2 : w3;
+    const uint32_t chunk = __funnelshift_l(prev, cur, static_cast<uint32_t>(B & 31));
+    if (chunk) atomicAdd(&acc[(B >> 5) + lane], static_cast<unsigned long long>(chunk));
+  }
+}
+
+// fp32 round-to-nearest-even of (sum * 2^-364) / K from the limb counters
+// (one thread; dig: kSqLimbs words of scratch).
+__device__ __noinline__ float sq_mean_f32(const unsigned long long* acc, uint32_t* dig, uint32_t K) {
+  unsigned long long carry = 0;
+  int h = -1;
+  for (int i = 0; i < kSqLimbs; ++i) {
+    const unsigned long long t = acc[i] + carry;
+    dig[i] = static_cast<uint32_t>(t);
+    carry = t >> 32;
+    if (dig[i]) h = i;
+  }
+  if (h < 0) return 0.f;
+  // quotient digits, in place, from the top; rem < K throughout
+  const unsigned long long inv = ~0ull / K + 1ull;   // ceil(2^64 / K), K >= 2
+  unsigned long long rem = 0;
+  for (int i = h; i >= 0; --i) {
+    const unsigned long long cur = (rem << 32) | dig[i];
+    const unsigned long long q = __umul64hi(cur, inv);
+    rem = cur - q * K;
+    dig[i] = static_cast<uint32_t>(q);
+  }
+  int hq = h;
+  while (hq > 0 && dig[hq] == 0u) --hq;
+  if (dig[hq] == 0u) return 0.f;
+  const int Lq = 32 * hq + 31 - __clz(dig[hq]);            // leading bit of the quotient
+  const int kSubLsb = kSqUnitExp - 149;                     // position of 2^-149
+  const int lsb = max(Lq - 23, kSubLsb);                    // last kept bit
+  if (lsb >= Lq + 2) return 0.f;                            // below half the smallest subnormal
+  const int width = Lq - lsb + 1;                           // kept bits, <= 24
+  unsigned long long win = dig[lsb >> 5];
+  if ((lsb >> 5) + 1 < kSqLimbs) win |= static_cast<unsigned long long>(dig[(lsb >> 5) + 1]) << 32;
+  const uint32_t kept0 = static_cast<uint32_t>((win >> (lsb & 31)) & ((1ull << width) - 1ull));
+  const int hp = lsb - 1;                                   // the half bit
+  const bool half = (dig[hp >> 5] >> (hp & 31)) & 1u;
+  bool sticky = rem != 0ull || (dig[hp >> 5] & ((1u << (hp & 31)) - 1u)) != 0u;
+  for (int j = 0; j < (hp >> 5) && !sticky; ++j) sticky = dig[j] != 0u;
+  const uint32_t kept = kept0 + ((half && (sticky || (kept0 & 1u))) ? 1u : 0u);
+  if (lsb > Lq - 23) return __uint_as_float(kept);          // subnormal (rounds up into 2^-126 exactly)
+  const int biased = Lq - kSqUnitExp + 127;
+  if (biased >= 255) return __uint_as_float(0x7f800000u);
+  return __uint_as_float((static_cast<uint32_t>(biased - 1) << 23) + kept);
+}
+
+// Normalise 8 bf16 values: bf16_rn(f32(f32(x / r) * w)), the weight optional.
+__device__ __forceinline__ uint4 rms_apply8(uint4 x, uint4 w, bool has_w, float r) {
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float lo = __fdiv_rn(bf16_lo(xs[i]), r), hi = __fdiv_rn(bf16_hi(xs[i]), r);
+    if (has_w) {
+      lo = __fmul_rn(lo, bf16_lo(ws[i]));
+      hi = __fmul_rn(hi, bf16_hi(ws[i]));
+    }
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    o[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// RMSNorm, then exactly act_quant_row_kernel's quantisation of the normalised
+// bf16 row: one CTA per token.  Wn: optional bf16 [K]; ms_out: optional fp32
+// [M] mean of squares.
+__global__ void __launch_bounds__(kActRowThreads) act_quant_rmsnorm_kernel(
+    const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wn, float eps, int K, int Q,
+    int8_t* __restrict__ Xq, float* __restrict__ s_out, int* __restrict__ R_out, float* __restrict__ ms_out) {
+  constexpr int W = kActRowThreads / 32;
+  __shared__ unsigned long long s_sq[kSqLimbs];
+  __shared__ uint32_t s_dig[kSqLimbs];
+  __shared__ float s_r;
+  __shared__ uint32_t s_max[W];
+  __shared__ int s_sum[W];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const size_t m = blockIdx.x;
+  if (t < kSqLimbs) s_sq[t] = 0ull;
+  const uint4* xr = reinterpret_cast<const uint4*>(X + m * K);
+  const uint4* wr = reinterpret_cast<const uint4*>(Wn);
+  const bool has_w = Wn != nullptr;
+  const int nch = K >> 3;
+  uint4 cache[kActRowCache];
+  int emax = 0;
+#pragma unroll
+  for (int i = 0; i < kActRowCache; ++i) {
+    const int c = t + kActRowThreads * i;
+    if (c < nch) {
+      cache[i] = __ldg(xr + c);
+      emax = max(emax, sq_exp_max8(cache[i]));
+    }
+  }
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+    emax = max(emax, sq_exp_max8(__ldg(xr + c)));
+  const int Ew = max(static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax))), 1);
+  __syncthreads();   // counters zeroed
+  unsigned long long lo = 0ull, hi = 0ull;
+#pragma unroll
+  for (int i = 0; i < kActRowCache; ++i) {
+    const int c = t + kActRowThreads * i;
+    if (c < nch) sq_add8(cache[i], Ew, lo, hi, s_sq);
+  }
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads) sq_add8(__ldg(xr + c), Ew, lo, hi, s_sq);
+  sq_warp_flush(lo, hi, Ew, lane, s_sq);
+  __syncthreads();
+  if (t == 0) {
+    const float ms = sq_mean_f32(s_sq, s_dig, static_cast<uint32_t>(K));
+    s_r = __fsqrt_rn(__fadd_rn(ms, eps));
+    if (ms_out) ms_out[m] = ms;
+  }
+  __syncthreads();
+  const float r = s_r;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kActRowCache; ++i) {
+    const int c = t + kActRowThreads * i;
+    if (c < nch) {
+      cache[i] = rms_apply8(cache[i], has_w ? __ldg(wr + c) : zero, has_w, r);
+      amax = fmaxf(amax, absmax8_bf16(cache[i]));
+    }
+  }
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+    amax = fmaxf(amax, absmax8_bf16(rms_apply8(__ldg(xr + c), has_w ? __ldg(wr + c) : zero, has_w, r)));
+  const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+  if (lane == 0) s_max[warp] = wmax;
+  __syncthreads();
+  uint32_t bmax = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) bmax = max(bmax, s_max[w]);
+  const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
+  uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kActRowCache; ++i) {
+    const int c = t + kActRowThreads * i;
+    if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+  }
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+    qr[c] = quant8_bf16(rms_apply8(__ldg(xr + c), has_w ? __ldg(wr + c) : zero, has_w, r), s, Q, sum);
+  const int wsum = __reduce_add_sync(0xffffffffu, sum);
+  if (lane == 0) s_sum[warp] = wsum;
+  __syncthreads();
+  if (t == 0) {
+    int tot = 0;
+#pragma unroll
+    for (int w = 0; w < W; ++w) tot += s_sum[w];
+    if (s_out) s_out[m] = s;
+    if (R_out) R_out[m] = tot;
+  }
+}
+
+}  // namespace bl

@@ -256,6 +256,42 @@ BL_API bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t 
                                const float* gamma, int bits, unsigned flags, const float* bias, uint16_t* Y,
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * RMSNorm ahead of the quantisation (SubLN: "BitNet 2B4T Guide: Scaling
+ * Native 1.58-Bit LLMs", section "3. Sub-Layer Normalization (SubLN)" and the
+ * page's pipeline figure, x_norm = RMSNorm(x) right before the absmax step;
+ * the norm's weight kept in bf16 per "BitNet a4.8 Guide: 4-Bit Activation
+ * 1-Bit LLMs", table "Best Practices for Deploying BitNet a4.8 in
+ * Production", row "LayerNorm Preservation").  Per token m:
+ *   ms_m   = fp32_rn( (1/K) sum_k X[m,k]^2 )      the sum exact, one rounding
+ *   r_m    = sqrt_rn( f32(ms_m + eps) )
+ *   Xn[m,k]= bf16_rn( f32( f32(X[m,k] / r_m) * w[k] ) )   (w == NULL: no product)
+ * then exactly bl_forward on Xn (per-token absmax, codes, ternary matmul,
+ * rescale).  The result is bit-identical to normalising into a bf16 tensor
+ * with these roundings and calling bl_forward on it; nothing is written
+ * between the steps except the int8 codes (M > 1).
+ * X: bf16 bits [M, K], 16-byte aligned.  norm_weight: bf16 bits [K] or NULL
+ * (16-byte aligned).  eps: positive and finite (else BL_ERR_INVALID_ARG).
+ * Wp, gamma, Y as in bl_forward.  workspace: at least
+ * bl_forward_rmsnorm_workspace_bytes(M, K, N, bits) bytes, 16-byte aligned,
+ * required for every M (one token whose layer fits the resident decode kernel
+ * forms everything in that kernel's prologue and leaves it untouched; other
+ * shapes write the codes and scales there and run the tensor-core GEMM).
+ * The ordering rule of bl_forward applies, and norm_weight counts as a
+ * parameter like Wp: one-token launches may read it before the dependency
+ * wait.  X may be written by the preceding kernel.
+ */
+BL_API size_t bl_forward_rmsnorm_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+BL_API bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
+                                    int64_t N, const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y,
+                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+/* Test export: the normalisation and quantisation step of bl_forward_rmsnorm
+ * alone: codes int8 [M, K] and scales fp32 [M] as bl_quant_act, and, when
+ * mean_sq is not NULL (4-byte aligned), ms_m fp32 [M]. */
+BL_API bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M,
+                                      int64_t K, int bits, int8_t* Xq, float* scale, float* mean_sq,
+                                      cudaStream_t stream);
+
 /* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
 BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
 

@@ -181,3 +181,26 @@ def test_forward_ex_validation(L):
     assert L.bl_forward_ex(None, 4, 64, 8, A, A, 8, 0, None, A, A, 1 << 20, None) == INVALID
     assert L.bl_forward_ex(A, 4, 100, 8, A, A, 8, 0, None, A, A, 1 << 20, None) == SHAPE
     assert L.bl_forward_ex(None, 0, 64, 8, None, None, 8, 1, None, None, None, 0, None) == OK
+
+
+def test_rmsnorm_validation(L):
+    # the workspace is required for every M (the fused one-token path leaves it unused)
+    assert L.bl_forward_rmsnorm_workspace_bytes(1, 2560, 6912, 8) >= 2560
+    assert L.bl_forward_rmsnorm_workspace_bytes(4, 64, 8, 8) >= 4 * 64
+    assert L.bl_forward_rmsnorm_workspace_bytes(4, 60, 8, 8) == 0
+    ok = (A, None, 1e-5, 4, 64, 8, A, A, 8, A, A, 1 << 20, None)
+    assert len(ok) == 13
+    assert L.bl_forward_rmsnorm(A, None, 1e-5, 4, 60, 8, A, A, 8, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_forward_rmsnorm(None, None, 1e-5, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == INVALID
+    assert L.bl_forward_rmsnorm(A, U, 1e-5, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == ALIGN   # misaligned weight
+    assert L.bl_forward_rmsnorm(A, None, 1e-5, 4, 64, 8, A, A, 5, A, A, 1 << 20, None) == UNSUP
+    assert L.bl_forward_rmsnorm(A, None, 1e-5, 1, 64, 8, A, A, 8, A, None, 0, None) == WS
+    for bad in (0.0, -1e-5, float("inf"), float("nan")):
+        assert L.bl_forward_rmsnorm(A, None, bad, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == INVALID
+        assert L.bl_quant_act_rmsnorm(A, None, bad, 4, 64, 8, A, A, None, None) == INVALID
+    assert L.bl_forward_rmsnorm(None, None, 1e-5, 0, 64, 8, None, None, 8, None, None, 0, None) == OK
+    assert L.bl_quant_act_rmsnorm(A, None, 1e-5, 4, 65, 8, A, A, None, None) == SHAPE
+    assert L.bl_quant_act_rmsnorm(A, None, 1e-5, 4, 64, 2, A, A, None, None) == UNSUP
+    assert L.bl_quant_act_rmsnorm(A, U, 1e-5, 4, 64, 8, A, A, None, None) == ALIGN
+    assert L.bl_quant_act_rmsnorm(A, None, 1e-5, 4, 64, 8, A, A, A + 2, None) == ALIGN       # mean_sq misaligned
+    assert L.bl_quant_act_rmsnorm(None, None, 1e-5, 4, 64, 8, A, A, None, None) == INVALID

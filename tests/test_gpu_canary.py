@@ -69,6 +69,11 @@ def test_forward_writes_stay_in_bounds(M, K, N):
     ws3 = Guarded((max(need3, 16),), torch.uint8)
     bl.bl_forward_relu2(x_to_dev(X), x_to_dev(X), Wp, g, N, out=Y3.t, workspace=ws3.t)
     assert Y3.intact() and ws3.intact()
+    Y4 = Guarded((M, N), torch.bfloat16)
+    ws4 = Guarded((bl.bl_forward_rmsnorm_workspace_bytes(M, K, N),), torch.uint8)
+    nw = torch.rand(K, device="cuda").to(torch.bfloat16)
+    bl.bl_forward_rmsnorm(x_to_dev(X), Wp, g, N, norm_weight=nw, out=Y4.t, workspace=ws4.t)
+    assert Y4.intact() and ws4.intact()
 
 
 def test_grouped_writes_stay_in_bounds():
@@ -96,6 +101,12 @@ def test_quantisers_write_in_bounds(M, K):
         bl.lib().bl_quant_act_relu2(x_to_dev(X).data_ptr(), None, M, K, bits, Xr.t.data_ptr(), sr.t.data_ptr(),
                                     torch.cuda.current_stream().cuda_stream)
         assert Xr.intact() and sr.intact()
+        Xn = Guarded((M, K), torch.int8)
+        sn = Guarded((M,), torch.float32)
+        ms = Guarded((M,), torch.float32)
+        bl.lib().bl_quant_act_rmsnorm(x_to_dev(X).data_ptr(), None, 1e-5, M, K, bits, Xn.t.data_ptr(),
+                                      sn.t.data_ptr(), ms.t.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert Xn.intact() and sn.intact() and ms.intact()
 
 
 @pytest.mark.parametrize("N,K", [(1, 64), (33, 192), (700, 2560), (130, 6912)])

@@ -393,3 +393,99 @@ def test_forward_ex_parity(M, K, N, per_tensor, with_bias):
         d = bf16_ulp_distance(bf16_dev_to_bits(Yd), ref["Y"])
         assert d.max() <= BF16_ULP_TOL, f"bf16 ulp distance {d.max()}"
         assert np.mean(d == 0) > 0.99
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm before the quantisation ("BitNet 2B4T Guide: Scaling Native 1.58-Bit
+# LLMs", section "3. Sub-Layer Normalization (SubLN)")
+# ---------------------------------------------------------------------------
+
+def norm_weight_bits(K, seed):
+    w = np.random.default_rng(seed).uniform(0.25, 2.0, size=K).astype(np.float32)
+    return (w.view(np.uint32) >> 16).astype(np.uint16)   # truncation: any bf16 will do
+
+
+def check_quant_rmsnorm(X, wb, eps, bits):
+    nrm = o.rms_norm(X, wb, eps)
+    q, s = o.act_quant(nrm["xn"], bits)
+    qd, sd, msd = bl.bl_quant_act_rmsnorm(x_to_dev(X), bits, x_to_dev(wb) if wb is not None else None, eps)
+    assert np.array_equal(msd.cpu().numpy().view(np.uint32), nrm["ms"].view(np.uint32))
+    assert np.array_equal(sd.cpu().numpy().view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(qd.cpu().numpy(), q)
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (3, 192), (16, 2560), (5, 6912), (2, 8192), (2, 20480), (1, 65536)])
+@pytest.mark.parametrize("with_weight", [False, True])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_quant_act_rmsnorm_bit_exact(M, K, with_weight, bits):
+    X, _ = random_case(M, K, 8, seed=M * 17 + K)
+    check_quant_rmsnorm(X, norm_weight_bits(K, K) if with_weight else None, 1e-5, bits)
+
+
+def test_quant_act_rmsnorm_hard_sums():
+    rng = np.random.default_rng(2024)
+    K = 2560
+    rows = []
+    rows.append(rng.integers(0, 0x7F80, K).astype(np.uint16))              # every exponent: many far terms
+    x = rng.standard_normal(K).astype(np.float32)
+    x[rng.integers(0, K, K // 3)] *= 1e-25                                 # a third far below the rest
+    rows.append((x.view(np.uint32) >> 16).astype(np.uint16))
+    rows.append(rng.integers(0x2000, 0x5F00, K).astype(np.uint16))         # 2^-63 .. 2^63: far terms, finite ms
+    rows.append(rng.integers(0x1A00, 0x2000, K).astype(np.uint16))         # 2^-75 .. 2^-63: subnormal ms
+    rows.append(rng.integers(0, 0x100, K).astype(np.uint16))               # bf16 subnormals: ms rounds to 0
+    big = np.zeros(K, np.uint16)
+    big[[3, 900]] = 0x7149                                                 # ~1e30: ms overflows to inf
+    rows.append(big)
+    rows.append(np.zeros(K, np.uint16))                                    # zero row
+    X = np.stack(rows) | (rng.integers(0, 2, (len(rows), K)).astype(np.uint16) << 15)
+    for eps in (1e-5, 1e-30):
+        check_quant_rmsnorm(X, None, eps, 8)
+    # an exact midpoint of two fp32 values (ties to even), and just above it
+    v = np.zeros((2, 128), np.float32)
+    v[:, :64] = 1.0
+    v[:, 64] = 2.0 ** -9
+    v[1, 65] = 2.0 ** -60
+    Xm = (v.view(np.uint32) >> 16).astype(np.uint16)
+    check_quant_rmsnorm(Xm, None, 2.0 ** -40, 8)
+    _, _, msd = bl.bl_quant_act_rmsnorm(x_to_dev(Xm), 8, None, 2.0 ** -40)
+    assert msd.cpu().numpy().tolist() == [0.5, 0.5 + 2.0 ** -24]
+
+
+RMS_CASES = [(1, 2560, 6912), (1, 6912, 2560), (1, 8192, 2100), (1, 8192, 8192), (1, 16384, 64),
+             (2, 320, 130), (17, 320, 130), (130, 256, 300), (16, 4096, 300)]
+
+
+@pytest.mark.parametrize("M,K,N", RMS_CASES)
+@pytest.mark.parametrize("with_weight", [False, True])
+def test_forward_rmsnorm_parity(M, K, N, with_weight):
+    # one token with a layer that fits the resident decode kernel: RMSNorm in
+    # its prologue; otherwise the normalising quantiser + the tensor-core GEMM
+    X, W = random_case(M, K, N, seed=M * 3 + K + N)
+    wb = norm_weight_bits(K, N) if with_weight else None
+    ref = o.forward_rmsnorm(X, W, wb, 1e-5)
+    Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+    Yd = bf16_dev_to_bits(bl.bl_forward_rmsnorm(x_to_dev(X), Wp, gd, N, norm_weight=x_to_dev(wb) if wb is not None
+                                                else None, eps=1e-5))
+    d = bf16_ulp_distance(Yd, ref["Y"])
+    assert d.max() <= BF16_ULP_TOL, f"bf16 ulp distance {d.max()}"
+    assert np.mean(d == 0) > 0.99
+    # and bit-identical to bl_forward on the oracle's normalised bf16 input
+    Y2 = bf16_dev_to_bits(bl.bl_forward(x_to_dev(ref["xn"]), Wp, gd, N))
+    assert np.array_equal(Yd, Y2)
+
+
+def test_forward_rmsnorm_bits4_zero_rows_and_back_to_back():
+    M, K, N = 1, 2560, 700
+    X, W = random_case(3, K, N, seed=99)
+    X[1] = 0
+    Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+    ws = torch.empty(bl.bl_forward_rmsnorm_workspace_bytes(M, K, N, 4), dtype=torch.uint8, device="cuda")
+    outs = []
+    for m in range(3):   # three decode launches back to back on one stream
+        outs.append(bl.bl_forward_rmsnorm(x_to_dev(X[m:m + 1]), Wp, gd, N, bits=4, workspace=ws))
+    torch.cuda.synchronize()
+    for m in range(3):
+        ref = o.forward_rmsnorm(X[m:m + 1], W, None, 1e-5, bits=4)
+        d = bf16_ulp_distance(bf16_dev_to_bits(outs[m]), ref["Y"])
+        assert d.max() <= BF16_ULP_TOL
+    assert np.all(bf16_dev_to_bits(outs[1]) == 0)
