@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
   __shared__ __align__(8) uint64_t full[kG3Stages], empty[kG3Stages];
   __shared__ int abort_flag;
   __shared__ unsigned long long s_sq[RMS ? kSqLimbs : 1];
+  __shared__ unsigned long long s_win[RMS ? 2 * CW : 1];
   __shared__ uint32_t s_dig[RMS ? kSqLimbs : 1];
   __shared__ float s_rms;
 
@@ -240,22 +241,36 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
     if constexpr (RELU2) uv[u] = (gated && c < nch) ? __ldg(static_cast<const uint4*>(Up) + c) : make_uint4(0, 0, 0, 0);
   }
   if constexpr (RMS) {
-    // exact mean of squares (warp windows + shared limb counters), then
+    // exact mean of squares (register windows anchored at the token's
+    // largest exponent, far squares in shared limb counters), then
     // x_n = bf16(x / sqrt(ms + eps) * w) in place of the token
     int emax = 0;
 #pragma unroll
     for (int u = 0; u < U; ++u)
       if (threadIdx.x + CT * u < nch) emax = max(emax, sq_exp_max8(xv[u]));
-    const int Ew = max(static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax))), 1);
+    const uint32_t wmax_e = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax));
+    if (lane == 0) s_red_f[warp] = wmax_e;
+    named_bar_sync(1, CT);
+    uint32_t eb = 1;
+#pragma unroll
+    for (int w = 0; w < CW; w += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(&s_red_f[w]);
+      eb = max(eb, max(max(v.x, v.y), max(v.z, v.w)));
+    }
+    const int E = static_cast<int>(eb);
     unsigned long long lo = 0ull, hi = 0ull;
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      if (threadIdx.x + CT * u < nch) sq_add8(xv[u], Ew, lo, hi, s_sq);
-    sq_warp_flush(lo, hi, Ew, lane, s_sq);
+      if (threadIdx.x + CT * u < nch) sq_add8(xv[u], E, lo, hi, s_sq);
+    sq_warp_sum(lo, hi);
+    if (lane == 0) {
+      s_win[2 * warp] = lo;
+      s_win[2 * warp + 1] = hi;
+    }
     named_bar_sync(1, CT);
-    if (threadIdx.x == 0) {
-      const float ms = sq_mean_f32(s_sq, s_dig, static_cast<uint32_t>(K));
-      s_rms = __fsqrt_rn(__fadd_rn(ms, tab.p[pi].eps));
+    if (warp == 0) {
+      const float ms = sq_block_mean(s_win, CW, E, s_sq, s_dig, static_cast<uint32_t>(K), lane);
+      if (lane == 0) s_rms = __fsqrt_rn(__fadd_rn(ms, tab.p[pi].eps));
     }
     named_bar_sync(1, CT);
     const float r = s_rms;

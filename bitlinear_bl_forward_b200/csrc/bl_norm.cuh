@@ -18,23 +18,32 @@
 // sig^2 * 2^(2e' - 268), a 16-bit integer at bit position P = 2e' + 96 of a
 // fixed-point number whose unit is 2^-364.  P runs from 98 to 604 and a sum
 // of up to 2^16 squares stays below 2^636: twenty 32-bit limbs.
-//   * Each warp anchors a 128-bit register accumulator at the largest
-//     exponent field among its values: its bit 0 sits at position 2 E_w and a
-//     square lands at bit 96 - 2 (E_w - e'), exactly, whenever that is >= 0.
-//     That covers every value within 2^48 of the warp's largest; the warp
-//     sums its 128-bit partials with shuffles (carries kept) and five lanes
-//     add the result, cut at 32-bit limb boundaries, into 64-bit limb
-//     counters in shared memory.
-//   * A square further down (a value below 2^-48 of the warp's largest) is
-//     added straight into the limb counter at its position.
-//   * Counters never overflow: a square's shifted value is < 2^47 and at most
-//     2^16 of them reach one counter (< 2^63); warp chunks add < 2^37.
-//   * One thread normalises the counters into 32-bit digits, divides by K
-//     digit by digit (a 64-bit multiply-high by ceil(2^64 / K) gives the
-//     exact quotient digit because every partial dividend is below 2^48 and
-//     K <= 2^16), and rounds to fp32 on the quotient's bits with the
-//     remainder as sticky: normal and subnormal results, ties to even,
-//     overflow to infinity.
+//   * The block first agrees on E, the largest exponent field of the token.
+//     Every thread then adds its squares into a 128-bit register window
+//     whose bit 0 sits at position 2E: a square lands at bit
+//     96 - 2 (E - e'), exactly, whenever that is >= 0, i.e. for every value
+//     within 2^48 of the token's largest.  Warps sum their windows with
+//     shuffles (carries kept), and one warp sums the warps' windows: all
+//     exact integer additions, so no atomics on this path.
+//   * A square further down (a value below 2^-48 of the largest) is added
+//     straight into 64-bit limb counters in shared memory at its position.
+//     Counters never overflow: such a value is < 2^47 and at most 2^16 of
+//     them reach one counter (< 2^63).
+//   * Rounding.  Without far squares the window W is the whole sum and
+//     ms = RN_f32(W * 2^(2E - 364) / K).  A double estimate
+//     q = (double(hi) 2^64 + double(lo)) / K * 2^(2E - 364) is within 2^-51
+//     relative of the exact value (three roundings of 2^-53 each plus an
+//     exact power-of-two scaling).  If q lies in the normal fp32 range and
+//     more than 2^-48 q away from both fp32 midpoints around RN_f32(q), no
+//     midpoint separates q from the exact value, so RN_f32(q) is the exact
+//     rounding.  Otherwise (a near-tie, far squares, the subnormal or
+//     overflow range) the window is folded into the limb counters and one
+//     thread takes the exact route: it normalises the counters into 32-bit
+//     digits, divides by K digit by digit (a 64-bit multiply-high by
+//     ceil(2^64 / K) gives the exact quotient digit because every partial
+//     dividend is below 2^48 and K <= 2^16), and rounds on the quotient's
+//     bits with the remainder as sticky: normal and subnormal results, ties
+//     to even, overflow to infinity.
 #pragma once
 
 #include "bl_act.cuh"
@@ -42,7 +51,7 @@
 namespace bl {
 
 constexpr int kSqLimbs = 20;            // 32-bit limbs of the fixed-point sum
-constexpr int kSqWindowShift = 96;      // bit of the warp anchor's square in its 128-bit window
+constexpr int kSqWindowShift = 96;      // bit of the anchor's square in the 128-bit window
 constexpr int kSqUnitExp = 364;         // unit of the fixed-point sum: 2^-364
 
 // Largest biased exponent field among 8 bf16 values.
@@ -54,16 +63,16 @@ __device__ __forceinline__ int sq_exp_max8(uint4 v) {
   return static_cast<int>(e);
 }
 
-// One bf16 square (b: the 16-bit pattern) into the warp window (lo, hi)
-// anchored at exponent field Ew, or into the shared limb counters.
-__device__ __forceinline__ void sq_add1(uint32_t b, int Ew, unsigned long long& lo, unsigned long long& hi,
+// One bf16 square (b: the 16-bit pattern) into the thread's window (lo, hi)
+// anchored at exponent field E, or into the shared limb counters.
+__device__ __forceinline__ void sq_add1(uint32_t b, int E, unsigned long long& lo, unsigned long long& hi,
                                         unsigned long long* acc) {
   const uint32_t e = (b >> 7) & 0xffu, f = b & 0x7fu;
   const uint32_t sig = e ? (f | 0x80u) : f;
   if (sig == 0u) return;
   const int ei = e ? static_cast<int>(e) : 1;
   const unsigned long long sq = static_cast<unsigned long long>(sig * sig);
-  const int sh = kSqWindowShift - 2 * (Ew - ei);
+  const int sh = kSqWindowShift - 2 * (E - ei);
   if (sh >= 0) {
     unsigned long long a_lo, a_hi;
     if (sh < 64) {
@@ -81,21 +90,18 @@ __device__ __forceinline__ void sq_add1(uint32_t b, int Ew, unsigned long long& 
   }
 }
 
-__device__ __forceinline__ void sq_add8(uint4 v, int Ew, unsigned long long& lo, unsigned long long& hi,
+__device__ __forceinline__ void sq_add8(uint4 v, int E, unsigned long long& lo, unsigned long long& hi,
                                         unsigned long long* acc) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    sq_add1(w[i] & 0xffffu, Ew, lo, hi, acc);
-    sq_add1(w[i] >> 16, Ew, lo, hi, acc);
+    sq_add1(w[i] & 0xffffu, E, lo, hi, acc);
+    sq_add1(w[i] >> 16, E, lo, hi, acc);
   }
 }
 
-// Warp sum of the 128-bit windows (every lane holds the total afterwards),
-// then lanes 0..4 add it, shifted to its position 2 Ew and cut into 32-bit
-// limbs, to the counters.  All 32 lanes must call it with the same Ew.
-__device__ __forceinline__ void sq_warp_flush(unsigned long long lo, unsigned long long hi, int Ew, int lane,
-                                              unsigned long long* acc) {
+// Warp sum of the 128-bit windows: every lane holds the total afterwards.
+__device__ __forceinline__ void sq_warp_sum(unsigned long long& lo, unsigned long long& hi) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const unsigned long long olo = __shfl_xor_sync(0xffffffffu, lo, o);
@@ -103,15 +109,22 @@ __device__ __forceinline__ void sq_warp_flush(unsigned long long lo, unsigned lo
     lo += olo;
     hi += ohi + (lo < olo ? 1ull : 0ull);
   }
+}
+
+// Add the window (lo, hi), whose bit 0 sits at position 2E, to the limb
+// counters: lane j (0..4) adds 32-bit chunk j.  One warp at a time, every
+// lane with the same window; the lanes' counters are distinct.
+__device__ __forceinline__ void sq_fold(unsigned long long lo, unsigned long long hi, int E, int lane,
+                                        unsigned long long* acc) {
   if (lane < 5) {
-    const int B = 2 * Ew;
+    const int B = 2 * E;
     const uint32_t w0 = static_cast<uint32_t>(lo), w1 = static_cast<uint32_t>(lo >> 32);
     const uint32_t w2 = static_cast<uint32_t>(hi), w3 = static_cast<uint32_t>(hi >> 32);
     const uint32_t cur = lane == 0 ? w0 : lane == 1 ? w1 : lane == 2 ? w2 : lane == 3 ? w3 : 0u;
     const uint32_t prev = lane == 0 ? 0u : lane == 1 ? w0 : lane == 2 ? w1 : lane == 3 ? w2 : w3;
-    const uint32_t chunk = __funnelshift_l(prev, cur, static_cast<uint32_t>(B & 31));
-    if (chunk) atomicAdd(&acc[(B >> 5) + lane], static_cast<unsigned long long>(chunk));
+    acc[(B >> 5) + lane] += __funnelshift_l(prev, cur, static_cast<uint32_t>(B & 31));
   }
+  __syncwarp();
 }
 
 // fp32 round-to-nearest-even of (sum * 2^-364) / K from the limb counters
@@ -157,6 +170,39 @@ __device__ __noinline__ float sq_mean_f32(const unsigned long long* acc, uint32_
   return __uint_as_float((static_cast<uint32_t>(biased - 1) << 23) + kept);
 }
 
+// The token's mean of squares, by one warp (all 32 lanes) once every
+// thread's far squares are in the counters and warp w's window is in
+// s_win[2w], s_win[2w + 1] (nw warps, anchored at E).  Returns ms on lane 0.
+__device__ __forceinline__ float sq_block_mean(const unsigned long long* s_win, int nw, int E,
+                                               unsigned long long* acc, uint32_t* dig, uint32_t K, int lane) {
+  unsigned long long lo = lane < nw ? s_win[2 * lane] : 0ull, hi = lane < nw ? s_win[2 * lane + 1] : 0ull;
+  sq_warp_sum(lo, hi);
+  const bool far = __ballot_sync(0xffffffffu, lane < kSqLimbs && acc[lane] != 0ull) != 0u;
+  float ms = 0.f;
+  int exact = far ? 1 : 0;
+  if (!far && lane == 0 && (lo | hi) != 0ull) {
+    const double D = fma(static_cast<double>(hi), 0x1p64, static_cast<double>(lo));
+    const double q = (D / static_cast<double>(K)) * __hiloint2double((2 * E - kSqUnitExp + 1023) << 20, 0);
+    exact = 1;
+    if (q >= 0x1p-126 && q < 0x1p127) {
+      const float f = __double2float_rn(q);
+      const double fd = f;
+      const double m_lo = 0.5 * (fd + static_cast<double>(__int_as_float(__float_as_int(f) - 1)));
+      const double m_hi = 0.5 * (fd + static_cast<double>(__int_as_float(__float_as_int(f) + 1)));
+      const double tol = q * 0x1p-48;
+      if (q - m_lo > tol && m_hi - q > tol) {
+        ms = f;
+        exact = 0;
+      }
+    }
+  }
+  if (__shfl_sync(0xffffffffu, exact, 0)) {
+    sq_fold(lo, hi, E, lane, acc);
+    if (lane == 0) ms = sq_mean_f32(acc, dig, K);
+  }
+  return ms;
+}
+
 // Normalise 8 bf16 values: bf16_rn(f32(f32(x / r) * w)), the weight optional.
 __device__ __forceinline__ uint4 rms_apply8(uint4 x, uint4 w, bool has_w, float r) {
   const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
@@ -183,6 +229,7 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_rmsnorm_kernel(
     int8_t* __restrict__ Xq, float* __restrict__ s_out, int* __restrict__ R_out, float* __restrict__ ms_out) {
   constexpr int W = kActRowThreads / 32;
   __shared__ unsigned long long s_sq[kSqLimbs];
+  __shared__ unsigned long long s_win[2 * W];
   __shared__ uint32_t s_dig[kSqLimbs];
   __shared__ float s_r;
   __shared__ uint32_t s_max[W];
@@ -206,21 +253,31 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_rmsnorm_kernel(
   }
   for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
     emax = max(emax, sq_exp_max8(__ldg(xr + c)));
-  const int Ew = max(static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax))), 1);
-  __syncthreads();   // counters zeroed
+  const uint32_t wmax_e = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax));
+  if (lane == 0) s_max[warp] = wmax_e;
+  __syncthreads();   // counters zeroed, per-warp exponents in
+  int E = 1;
+#pragma unroll
+  for (int w = 0; w < W; ++w) E = max(E, static_cast<int>(s_max[w]));
   unsigned long long lo = 0ull, hi = 0ull;
 #pragma unroll
   for (int i = 0; i < kActRowCache; ++i) {
     const int c = t + kActRowThreads * i;
-    if (c < nch) sq_add8(cache[i], Ew, lo, hi, s_sq);
+    if (c < nch) sq_add8(cache[i], E, lo, hi, s_sq);
   }
-  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads) sq_add8(__ldg(xr + c), Ew, lo, hi, s_sq);
-  sq_warp_flush(lo, hi, Ew, lane, s_sq);
+  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads) sq_add8(__ldg(xr + c), E, lo, hi, s_sq);
+  sq_warp_sum(lo, hi);
+  if (lane == 0) {
+    s_win[2 * warp] = lo;
+    s_win[2 * warp + 1] = hi;
+  }
   __syncthreads();
-  if (t == 0) {
-    const float ms = sq_mean_f32(s_sq, s_dig, static_cast<uint32_t>(K));
-    s_r = __fsqrt_rn(__fadd_rn(ms, eps));
-    if (ms_out) ms_out[m] = ms;
+  if (warp == 0) {
+    const float ms = sq_block_mean(s_win, W, E, s_sq, s_dig, static_cast<uint32_t>(K), lane);
+    if (lane == 0) {
+      s_r = __fsqrt_rn(__fadd_rn(ms, eps));
+      if (ms_out) ms_out[m] = ms;
+    }
   }
   __syncthreads();
   const float r = s_r;
