@@ -10,7 +10,11 @@
 //
 // Every rounding is explicit so results are bit-identical to an IEEE fp32
 // evaluation: __fdiv_rn for the scale, __fmul_rn for x * s (never fused),
-// __float2int_rn (round half to even) for the code.
+// then round half to even to an integer.  That last step adds 1.5 * 2^23:
+// for |v| < 2^22 the fp32 sum lies in [2^23, 2^24), where the spacing is 1,
+// so the round-to-nearest-even addition leaves 1.5 * 2^23 + rint(v) (the
+// constant is even, so ties go to even); |x * s| <= Q + 1 here.  Two
+// full-rate instructions instead of a float-to-int conversion.
 #pragma once
 
 #include "bl_common.cuh"
@@ -32,8 +36,12 @@ __device__ __forceinline__ float absmax8_bf16(uint4 v) {
   return a;
 }
 
+__device__ __forceinline__ int rint_small(float v) {
+  return __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
+}
+
 __device__ __forceinline__ uint32_t quant1(float x, float s, int Q) {
-  int q = __float2int_rn(__fmul_rn(x, s));
+  int q = rint_small(__fmul_rn(x, s));
   q = q < -Q - 1 ? -Q - 1 : (q > Q ? Q : q);
   return static_cast<uint32_t>(q) & 0xffu;
 }

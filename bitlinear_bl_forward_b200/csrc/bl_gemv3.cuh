@@ -244,20 +244,20 @@ __global__ void __launch_bounds__(G3Cfg<WPL, CW>::kThreads, 2)
     // exact mean of squares (register windows anchored at the token's
     // largest exponent, far squares in shared limb counters), then
     // x_n = bf16(x / sqrt(ms + eps) * w) in place of the token
-    int emax = 0;
+    float xmax = 0.f;
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      if (threadIdx.x + CT * u < nch) emax = max(emax, sq_exp_max8(xv[u]));
-    const uint32_t wmax_e = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax));
-    if (lane == 0) s_red_f[warp] = wmax_e;
+      if (threadIdx.x + CT * u < nch) xmax = fmaxf(xmax, absmax8_bf16(xv[u]));
+    const uint32_t wmax_x = __reduce_max_sync(0xffffffffu, __float_as_uint(xmax));
+    if (lane == 0) s_red_f[warp] = wmax_x;
     named_bar_sync(1, CT);
-    uint32_t eb = 1;
+    uint32_t xb = 0;
 #pragma unroll
     for (int w = 0; w < CW; w += 4) {
       const uint4 v = *reinterpret_cast<const uint4*>(&s_red_f[w]);
-      eb = max(eb, max(max(v.x, v.y), max(v.z, v.w)));
+      xb = max(xb, max(max(v.x, v.y), max(v.z, v.w)));
     }
-    const int E = static_cast<int>(eb);
+    const int E = sq_anchor(xb);
     unsigned long long lo = 0ull, hi = 0ull;
 #pragma unroll
     for (int u = 0; u < U; ++u)

@@ -54,34 +54,30 @@ constexpr int kSqLimbs = 20;            // 32-bit limbs of the fixed-point sum
 constexpr int kSqWindowShift = 96;      // bit of the anchor's square in the 128-bit window
 constexpr int kSqUnitExp = 364;         // unit of the fixed-point sum: 2^-364
 
-// Largest biased exponent field among 8 bf16 values.
-__device__ __forceinline__ int sq_exp_max8(uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t e = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) e = max(e, max((w[i] >> 7) & 0xffu, (w[i] >> 23) & 0xffu));
-  return static_cast<int>(e);
-}
+// Anchor exponent field of a token from its largest |x| (fp32 bits of a
+// bf16 value): the largest exponent field, at least 1.
+__device__ __forceinline__ int sq_anchor(uint32_t amax_bits) { return max(static_cast<int>(amax_bits >> 23), 1); }
 
 // One bf16 square (b: the 16-bit pattern) into the thread's window (lo, hi)
-// anchored at exponent field E, or into the shared limb counters.
+// anchored at exponent field E, or into the shared limb counters.  Squares of
+// values within 2^16 of the largest land in hi alone (bit 2 (e' - E) + 32 of
+// it, < 2^48 each): one 64-bit shift and add.
 __device__ __forceinline__ void sq_add1(uint32_t b, int E, unsigned long long& lo, unsigned long long& hi,
                                         unsigned long long* acc) {
-  const uint32_t e = (b >> 7) & 0xffu, f = b & 0x7fu;
-  const uint32_t sig = e ? (f | 0x80u) : f;
-  if (sig == 0u) return;
+  const uint32_t e = (b >> 7) & 0xffu;
+  const uint32_t sig = (b & 0x7fu) | (e ? 0x80u : 0u);
   const int ei = e ? static_cast<int>(e) : 1;
   const unsigned long long sq = static_cast<unsigned long long>(sig * sig);
-  const int sh = kSqWindowShift - 2 * (E - ei);
+  const int t = 2 * (ei - E) + kSqWindowShift - 64;
+  if (t >= 0) {
+    hi += sq << t;
+    return;
+  }
+  if (sq == 0ull) return;
+  const int sh = t + 64;
   if (sh >= 0) {
-    unsigned long long a_lo, a_hi;
-    if (sh < 64) {
-      a_lo = sq << sh;
-      a_hi = sh > 48 ? (sq >> (64 - sh)) : 0ull;
-    } else {
-      a_lo = 0ull;
-      a_hi = sq << (sh - 64);
-    }
+    const unsigned long long a_lo = sq << sh;
+    const unsigned long long a_hi = sh > 48 ? (sq >> (64 - sh)) : 0ull;
     lo += a_lo;
     hi += a_hi + (lo < a_lo ? 1ull : 0ull);
   } else {
@@ -242,23 +238,24 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_rmsnorm_kernel(
   const bool has_w = Wn != nullptr;
   const int nch = K >> 3;
   uint4 cache[kActRowCache];
-  int emax = 0;
+  float xmax = 0.f;
 #pragma unroll
   for (int i = 0; i < kActRowCache; ++i) {
     const int c = t + kActRowThreads * i;
     if (c < nch) {
       cache[i] = __ldg(xr + c);
-      emax = max(emax, sq_exp_max8(cache[i]));
+      xmax = fmaxf(xmax, absmax8_bf16(cache[i]));
     }
   }
   for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
-    emax = max(emax, sq_exp_max8(__ldg(xr + c)));
-  const uint32_t wmax_e = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(emax));
-  if (lane == 0) s_max[warp] = wmax_e;
-  __syncthreads();   // counters zeroed, per-warp exponents in
-  int E = 1;
+    xmax = fmaxf(xmax, absmax8_bf16(__ldg(xr + c)));
+  const uint32_t wmax_x = __reduce_max_sync(0xffffffffu, __float_as_uint(xmax));
+  if (lane == 0) s_max[warp] = wmax_x;
+  __syncthreads();   // counters zeroed, per-warp maxima in
+  uint32_t xb = 0;
 #pragma unroll
-  for (int w = 0; w < W; ++w) E = max(E, static_cast<int>(s_max[w]));
+  for (int w = 0; w < W; ++w) xb = max(xb, s_max[w]);
+  const int E = sq_anchor(xb);
   unsigned long long lo = 0ull, hi = 0ull;
 #pragma unroll
   for (int i = 0; i < kActRowCache; ++i) {
