@@ -78,6 +78,9 @@ __all__ = [
     "ternary_codes",
     "pack_ternary",
     "unpack_ternary",
+    "base3_row_bytes",
+    "pack_base3",
+    "unpack_base3",
     "act_quant",
     "act_quant_values",
     "act_quant_per_tensor",
@@ -273,6 +276,64 @@ def unpack_ternary(packed: np.ndarray, K: int) -> np.ndarray:
     if np.any(out == 3):
         raise ValueError("reserved 2-bit value 3 found")
     return (out.reshape(N, K) - 1).astype(np.int8)
+
+
+# ---------------------------------------------------------------------------
+# Base-3 storage: five ternary weights per byte ([P2] section "Why 1.58 Bits?
+# The Power of Zero": three states carry log2(3) ~ 1.58 bits; 3^5 = 243 states
+# fit in one byte, 1.6 bits a weight).  The pages fix only the density; the
+# layout is this library's:
+#   * a row of K weights is a run of little-endian 32-bit words padded to a
+#     multiple of four words (16 bytes); word g holds k = 20g .. 20g+19;
+#   * byte b (0..3) of word g holds the five digits d_L = code + 1 (L = 0..4)
+#     of the weights k = 20g + 4L + b; digits past the end of the row are 1
+#     (code 0);
+#   * the byte stores ceil(256 * v / 243) with v = sum_L d_L * 3^(4 - L), the
+#     base-3 number whose most significant digit is d_0.  (v is recovered
+#     exactly as floor(243 * byte / 256); the scaled form lets a decoder get
+#     the digits in order by repeated multiplication by 3.)
+# ---------------------------------------------------------------------------
+
+def base3_row_bytes(K: int) -> int:
+    """Bytes of one base-3 row of K weights (16-byte multiple)."""
+    words = -(-K // 20)
+    return 4 * (-(-words // 4) * 4)
+
+
+def pack_base3(codes: np.ndarray) -> np.ndarray:
+    """int8 codes [N, K] in {-1, 0, 1} -> base-3 bytes [N, base3_row_bytes(K)]."""
+    c = np.asarray(codes)
+    N, K = c.shape
+    d = c.astype(np.int64) + 1
+    if np.any((d < 0) | (d > 2)):
+        raise ValueError("codes must lie in {-1, 0, 1}")
+    rb = base3_row_bytes(K)
+    padded = np.ones((N, rb * 5), dtype=np.int64)        # digit 1 = code 0
+    padded[:, :K] = d
+    # word g, level L, byte b <-> k = 20g + 4L + b
+    digits = padded.reshape(N, rb // 4, 5, 4)              # [n, g, L, b]
+    v = np.zeros((N, rb // 4, 4), dtype=np.int64)
+    for L in range(5):
+        v += digits[:, :, L, :] * 3 ** (4 - L)
+    q = -((-256 * v) // 243)                               # ceil(256 v / 243)
+    return q.reshape(N, rb).astype(np.uint8)
+
+
+def unpack_base3(packed: np.ndarray, K: int) -> np.ndarray:
+    """Base-3 bytes [N, base3_row_bytes(K)] -> int8 codes [N, K] (inverse of
+    pack_base3: v = floor(243 * byte / 256), then its base-3 digits)."""
+    p = np.ascontiguousarray(packed, dtype=np.uint8).astype(np.int64)
+    N, rb = p.shape
+    if rb != base3_row_bytes(K):
+        raise ValueError("row length does not match K")
+    v = (243 * p) // 256
+    if np.any(v > 242):
+        raise ValueError("byte outside the 243 base-3 states")
+    v = v.reshape(N, rb // 4, 4)                           # [n, g, b]
+    digits = np.empty((N, rb // 4, 5, 4), dtype=np.int64)
+    for L in range(5):
+        digits[:, :, L, :] = (v // 3 ** (4 - L)) % 3
+    return (digits.reshape(N, rb * 5)[:, :K] - 1).astype(np.int8)
 
 
 # ---------------------------------------------------------------------------

@@ -238,6 +238,74 @@ def test_unpack_bytewise_definition():
 
 
 # ---------------------------------------------------------------------------
+# Base-3 storage (P2 "Why 1.58 Bits?": 3^5 = 243 states in a byte; the layout
+# is this library's)
+# ---------------------------------------------------------------------------
+
+def test_base3_layout_golden():
+    g = json.load(open(os.path.join(GOLDEN, "base3_layout.json")))
+    K = g["K"]
+    codes = np.zeros((1, K), np.int8)
+    for k, v in g["nonzero_codes"].items():
+        codes[0, int(k)] = v
+    packed = o.pack_base3(codes)
+    assert packed.tolist() == [g["packed_bytes"]]
+    assert np.array_equal(o.unpack_base3(packed, K), codes)
+
+
+def test_base3_every_byte_decodes_by_repeated_tripling():
+    # all 243 digit tuples: the stored bytes are distinct, and the digits come
+    # back in order from x -> 3x mod 256 (digit = floor(3x / 256)), a decode
+    # independent of the oracle's exact inverse floor(243 * byte / 256)
+    import itertools
+    seen = set()
+    for digits in itertools.product(range(3), repeat=5):
+        codes = np.zeros((1, 64), np.int8)
+        for L, d in enumerate(digits):
+            codes[0, 4 * L] = d - 1          # word 0, byte 0, level L
+        byte = int(o.pack_base3(codes)[0, 0])
+        assert 0 <= byte <= 255 and byte not in seen
+        seen.add(byte)
+        x = byte
+        got = []
+        for _ in range(5):
+            got.append((3 * x) >> 8)
+            x = (3 * x) & 0xFF
+        assert tuple(got) == digits, (digits, byte, got)
+    assert len(seen) == 243
+
+
+def test_base3_roundtrip_sizes_and_padding():
+    rng = np.random.default_rng(9)
+    for N, K in [(1, 64), (3, 192), (5, 2560), (2, 6912), (1, 8192)]:
+        c = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        p = o.pack_base3(c)
+        words = -(-K // 20)
+        assert p.shape == (N, 4 * (-(-words // 4) * 4)) and p.shape[1] % 16 == 0
+        assert p.shape[1] * 8 <= 1.61 * K + 128          # ~1.6 bits a weight
+        assert np.array_equal(o.unpack_base3(p, K), c)
+        # the same codes in both storages
+        assert np.array_equal(o.unpack_base3(p, K), o.unpack_ternary(o.pack_ternary(c), K))
+    # the all-zero row is the digit-1 byte everywhere, padding included
+    assert set(o.pack_base3(np.zeros((1, 8192), np.int8)).ravel().tolist()) == {128}
+
+
+def test_base3_bytewise_definition():
+    # decode one random row digit by digit from the layout definition (plain
+    # integer division of v, recovered from the byte by trying every v)
+    rng = np.random.default_rng(10)
+    K = 128
+    c = rng.integers(-1, 2, (1, K)).astype(np.int8)
+    p = o.pack_base3(c)[0]
+    inv = {-(-256 * v // 243): v for v in range(243)}
+    for k in range(K):
+        g, r = divmod(k, 20)
+        L, b = divmod(r, 4)
+        v = inv[int(p[4 * g + b])]
+        assert (v // 3 ** (4 - L)) % 3 - 1 == c[0, k]
+
+
+# ---------------------------------------------------------------------------
 # [P2] eq. (2), [P1] section 1: activation quantisation
 # ---------------------------------------------------------------------------
 
