@@ -37,6 +37,7 @@ if ROOT not in sys.path:
 
 METRIC = "BitLinear TOPS (prefill) and HBM GB/s (decode) vs roofline, 1×B200"
 INT8_NOMINAL_RATIO = 2.0   # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+DELAY_CYCLES = 400_000     # ~200 us at the 1965 MHz maximum SM clock
 
 
 # ---------------------------------------------------------------------------
@@ -78,7 +79,10 @@ def ncu_traffic(kernel_key):
             continue
         h = hashlib.sha256()
         for fn in kv["files"].split(","):
-            h.update(open(os.path.join(src, fn), "rb").read())
+            fp = os.path.join(src, fn)
+            if not os.path.exists(fp):    # the kernel's sources changed since the capture
+                return None
+            h.update(open(fp, "rb").read())
         if kv.get("src_sha") == h.hexdigest()[:16]:
             return float(kv["dram_bytes_per_launch"])
     return None
@@ -99,7 +103,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         time.sleep(0.25)
@@ -184,8 +188,7 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(workload_name, budget_s=10.0):
-    fn, nbytes, _ops, desc = oracle_step_fn(workload_name)
+def _time_oracle(fn, budget_s):
     fn()   # warm
     t0 = time.perf_counter()
     n = 0
@@ -194,9 +197,24 @@ def cpu_baseline(workload_name, budget_s=10.0):
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break
-    dt = time.perf_counter() - t0
-    return {"value": nbytes * n / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} full steps of {desc} in {dt:.1f} s (weight quantisation excluded)"}
+    return n, time.perf_counter() - t0
+
+
+def cpu_baseline(workload_name, budget_s=8.0):
+    """The oracle's forward scope on the host cores, twice: with the BLAS pool
+    (the oracle's float64 matmul) limited to one thread, and with all of it.
+    The oracle's quantisation and rescale are single-threaded numpy in both."""
+    from threadpoolctl import threadpool_limits
+    fn, nbytes, _ops, desc = oracle_step_fn(workload_name)
+    with threadpool_limits(limits=1, user_api="blas"):
+        n1, dt1 = _time_oracle(fn, budget_s)
+    n, dt = _time_oracle(fn, budget_s)
+    cores = blas_threads()
+    return {"value": nbytes * n / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} full steps of {desc} in {dt:.1f} s with {cores} BLAS threads (weight quantisation "
+                      f"excluded; the oracle's quantiser and rescale are single-threaded numpy)",
+            "single_thread": {"value": nbytes * n1 / dt1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"{n1} full steps in {dt1:.1f} s, BLAS limited to 1 thread"}}
 
 
 def run_reference(args):
@@ -248,17 +266,18 @@ class GpuWorkload:
     """Device buffers for one workload: R rotated copies of the packed weights
     of every layer, one bf16 input and output per layer, workspace."""
 
-    def __init__(self, name, rotations, seed=0, device="cuda"):
+    def __init__(self, name, rotations, seed=0, device="cuda", fmt="2bit"):
         import torch
         from bitlinear_bl_forward_b200 import bl
         from bitlinear_bl_forward_b200.inputs import WORKLOADS, make_activation
         self.w = WORKLOADS[name]
         self.name = name
+        self.fmt = fmt
         self.layers = []
         g = torch.Generator(device=device).manual_seed(seed)
         for i, L in enumerate(self.w.layers):
             Wf = torch.randn(L.N, L.K, generator=g, device=device, dtype=torch.float32) * self.w.w_std
-            Wp, gamma = bl.bl_quantize_weights(Wf)
+            Wp, gamma = (bl.bl_quantize_weights_b3 if fmt == "b3" else bl.bl_quantize_weights)(Wf)
             del Wf
             copies = [(Wp, gamma)] + [(Wp.clone(), gamma.clone()) for _ in range(rotations - 1)]
             if L.x_layer >= 0:          # reads the same hidden state as an earlier layer
@@ -286,6 +305,9 @@ class GpuWorkload:
         # activations shared by several layers are read (and counted) once
         self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N)
                                   - (0 if d["own_x"] else 2 * self.w.M * d["L"].K) for d in self.layers)
+        if fmt == "b3":   # the stored weight bytes are the base-3 rows
+            self.bytes_per_step += sum(bl.bl_packed_weight_bytes_b3(d["L"].N, d["L"].K) - d["L"].N * d["L"].K // 4
+                                       for d in self.layers)
         self.ops_per_step = sum(algorithmic_ops(self.w.M, d["L"].K, d["L"].N) for d in self.layers)
         # decode: one launch per call (a grouped call of decode problems is one launch);
         # otherwise activation quantisation + GEMM per layer
@@ -297,7 +319,10 @@ class GpuWorkload:
         if len(gr) == 1:
             d = self.layers[gr[0]]
             Wp, gamma = d["copies"][r]
-            bl.bl_forward(d["X"], Wp, gamma, d["L"].N, self.w.bits, out=d["Y"], workspace=d["ws"])
+            if self.fmt == "b3":
+                bl.bl_forward_b3(d["X"], Wp, gamma, d["L"].N, self.w.bits, out=d["Y"])
+            else:
+                bl.bl_forward(d["X"], Wp, gamma, d["L"].N, self.w.bits, out=d["Y"], workspace=d["ws"])
         else:
             ds = [self.layers[j] for j in gr]
             bl.bl_forward_grouped([(d["X"], *d["copies"][r], d["L"].N) for d in ds], self.w.bits,
@@ -419,6 +444,10 @@ def time_workload(wl, steps, warmup, dist_ctx, sample_clocks=True, chunk=None):
         sampler.__enter__()
     dist_ctx.barrier()
     torch.cuda.synchronize()
+    # a bounded device-side delay (~200 us of SM clock cycles) ahead of the
+    # start event: the host has queued the graph replays by the time the clock
+    # starts, so the timed region holds device work only, not graph submission
+    torch.cuda._sleep(DELAY_CYCLES)
     t0.record()
     for _ in range(steps // chunk):
         g_main.replay()
@@ -543,6 +572,34 @@ def roofline_entry(kind, achieved, peak, unit, traffic):
             "traffic": traffic}
 
 
+def i8_peak(peaks, n_mma=4096, reps=3):
+    """Measured dense kind::i8 peak: the library's tcgen05.mma probe on every
+    SM at once (M = 128, N = 256, K = 32 MMAs back to back).  Returns a dict
+    with TOPS (2 ops per multiply-accumulate) at the clock it ran, the rate per
+    SM per clock and that clock; falls back to 2 x the measured bf16 burst
+    GEMM when the probe cannot run."""
+    import torch
+    from bitlinear_bl_forward_b200 import bl
+    try:
+        best = None
+        for _ in range(reps):
+            out = bl.bl_probe_mma_i8(n_mma, 256)
+            torch.cuda.synchronize()
+            o = out.cpu().numpy().astype(np.float64)
+            if (o <= 0).any():
+                raise RuntimeError("probe wait gave up")
+            macs = 128.0 * 256 * 32 * n_mma
+            tops = 2 * macs * o.shape[0] / (o[:, 1].max() * 1e-9) / 1e12
+            ent = {"tops": tops, "mac_per_clk_per_sm": float(np.median(macs / o[:, 0])),
+                   "sm_ghz": float(np.median(o[:, 0] / o[:, 1])), "sms": int(o.shape[0]),
+                   "src": "measured tcgen05 kind::i8 probe (bl_probe_mma_i8)"}
+            if best is None or ent["tops"] > best["tops"]:
+                best = ent
+        return best
+    except Exception as e:   # report, then fall back to the bf16 burst figure
+        return {"tops": peaks["bf16_tflops"] * INT8_NOMINAL_RATIO, "src": f"2 x bf16 burst ({e})"}
+
+
 def run_gpu(args):
     import torch
     from bitlinear_bl_forward_b200 import build as blbuild
@@ -551,6 +608,7 @@ def run_gpu(args):
     bl.lib()
     ctx = DistCtx(args.gpus)
     peaks = load_peaks()
+    ipk = i8_peak(peaks)
     name = args.workload
     from bitlinear_bl_forward_b200.inputs import WORKLOADS
     w = WORKLOADS[name]
@@ -579,14 +637,13 @@ def run_gpu(args):
     per_rank_ms = ms
     if decode:
         achieved = wl.bytes_per_step * K / (per_rank_ms / 1e3) / 1e9
-        roof = roofline_entry("hbm", achieved, peaks["hbm_gbs"], "GB/s", ncu_traffic(f"gemv:{name}"))
+        roof = roofline_entry("hbm", achieved, peaks["hbm_gbs"], "GB/s", ncu_traffic(f"decode:{name}"))
     else:
         achieved = wl.ops_per_step * K / (per_rank_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO
-        roof = roofline_entry("tensor", achieved, peak, "TFLOP/s", ncu_traffic(f"tc:{name}"))
-    roof["peak_src"] = peaks["src"] + (" hbm copy" if decode else " bf16 sustained x2 (int8/bf16 nominal)")
-    roof["kernel"] = ("gemv3_kernel" if decode else
-                      ("tc_gemm_persistent_kernel" if w.M <= 64 else "tc_gemm_pair_kernel")
+        roof = roofline_entry("tensor", achieved, ipk["tops"], "TFLOP/s", ncu_traffic(f"tc:{name}"))
+    roof["peak_src"] = peaks["src"] + " hbm copy" if decode else ipk["src"]
+    roof["kernel"] = ("bl_decode_kernel" if decode else
+                      ("bl_mma_persistent_kernel" if w.M <= 64 else "bl_mma_pair_kernel")
                       + " (+ activation quantisation in the step)")
     roof["kernel_us_avg"] = per_rank_ms * 1e3 / launches
 
@@ -610,9 +667,10 @@ def run_gpu(args):
         "gpu_launches": K * wl.launches_per_step,
         "roofline": roof,
         "clocks": clocks,
+        "i8_peak": ipk,
     }
     if not args.no_secondary and ctx.world == 1:
-        line["secondary"] = secondary(args, ctx, peaks)
+        line["secondary"] = secondary(args, ctx, peaks, ipk)
     if ctx.rank == 0 and not args.no_cpu_baseline and ctx.world == 1:
         line["cpu_baseline"] = cpu_baseline(name, budget_s=args.cpu_seconds)
     ctx.close()
@@ -620,61 +678,79 @@ def run_gpu(args):
         print(json.dumps(line), flush=True)
 
 
-def secondary(args, ctx, peaks):
-    """Tensor-core workloads and the 70B decode layer, shorter runs."""
+def secondary(args, ctx, peaks, ipk):
+    """Tensor-core workloads, the 70B decode layer and the fused variants:
+    each timed region is about 0.3 s, with clocks sampled during it."""
     import torch
     out = []
-    for name, steps in (("prefill_2b", 300), ("layer_70b_m1", 3000), ("layer_70b_m16", 3000),
-                        ("layer_70b_m128", 2000), ("layer_70b_m2048", 200), ("a48", 300)):
-        if args.secondary and name not in args.secondary.split(","):
+    want = set(args.secondary.split(",")) if args.secondary else None
+    i8 = ipk["tops"]
+
+    def timed(wl, steps):
+        ms, clocks = time_workload(wl, steps, 3, ctx, sample_clocks=True)
+        return ms, clocks
+
+    for name, steps in (("prefill_2b", 2000), ("layer_70b_m1", 25000), ("layer_70b_m16", 10000),
+                        ("layer_70b_m128", 8000), ("layer_70b_m2048", 800), ("a48", 4000)):
+        if want and name not in want:
             continue
         from bitlinear_bl_forward_b200.inputs import WORKLOADS
         w = WORKLOADS[name]
         wbytes = sum(L.N * L.K // 4 for L in w.layers)
         rot = max(2, min(64, int(math.ceil(256e6 / wbytes))))
         wl = GpuWorkload(name, rot)
-        ms, _ = time_workload(wl, steps, 3, ctx, sample_clocks=False)
+        ms, clocks = timed(wl, steps)
         sec = ms / 1e3
         gbs = wl.bytes_per_step * steps / sec / 1e9
         tops = wl.ops_per_step * steps / sec / 1e12
-        ent = {"workload": name, "M": w.M, "ms_per_step": ms / steps, "GB/s": gbs, "TOPS": tops,
-               "hbm_frac": gbs / peaks["hbm_gbs"],
-               "tensor_frac": tops / (peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO),
-               "steps": steps}
-        out.append(ent)
+        out.append({"workload": name, "M": w.M, "ms_per_step": ms / steps, "GB/s": gbs, "TOPS": tops,
+                    "hbm_frac": gbs / peaks["hbm_gbs"], "tensor_frac": tops / i8, "steps": steps,
+                    "clocks": clocks})
         del wl
         torch.cuda.empty_cache()
-    if not args.secondary or "ffn_2b_decode" in args.secondary.split(","):
+    if not want or "layer_70b_m1_base3" in want:
+        # the same 70B-class one-token layer with base-3 weight storage (five
+        # weights a byte): compare ms_per_step with layer_70b_m1
+        wl = GpuWorkload("layer_70b_m1", 6, fmt="b3")
+        steps = 25000
+        ms, clocks = timed(wl, steps)
+        gbs = wl.bytes_per_step * steps / (ms / 1e3) / 1e9
+        out.append({"workload": "layer_70b_m1_base3", "M": 1, "ms_per_step": ms / steps, "GB/s": gbs,
+                    "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps, "clocks": clocks,
+                    "note": "GB/s of the base-3 bytes (1648 B a row instead of 2048); compare ms_per_step"})
+        del wl
+        torch.cuda.empty_cache()
+    if not want or "ffn_2b_decode" in want:
         # the decode feed-forward chain (up+gate grouped, then down on the fused squared ReLU)
-        steps = 20000
+        steps = 60000
         wl = FfnWorkload(20)
-        ms, _ = time_workload(wl, steps, 3, ctx, sample_clocks=False)
+        ms, clocks = timed(wl, steps)
         gbs = wl.bytes_per_step * steps / (ms / 1e3) / 1e9
         out.append({"workload": "ffn_2b_decode", "M": 1, "ms_per_step": ms / steps, "GB/s": gbs,
-                    "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps,
+                    "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps, "clocks": clocks,
                     "note": "down input = max(0, gate)^2 * up of the same step, formed in the down kernel"})
         del wl
         torch.cuda.empty_cache()
     for name, base, steps, rot in (("rmsnorm_decode_2b", "decode_2b", 20000, 20),
-                                   ("rmsnorm_prefill_2b", "prefill_2b", 300, 20)):
-        if args.secondary and name not in args.secondary.split(","):
+                                   ("rmsnorm_prefill_2b", "prefill_2b", 1200, 20)):
+        if want and name not in want:
             continue
         # the same layers with RMSNorm (bf16 weight) formed ahead of the quantiser
         wl = RmsWorkload(base, rot)
-        ms, _ = time_workload(wl, steps, 3, ctx, sample_clocks=False)
+        ms, clocks = timed(wl, steps)
         sec = ms / 1e3
         gbs = wl.bytes_per_step * steps / sec / 1e9
         ent = {"workload": name, "M": wl.w.M, "ms_per_step": ms / steps, "GB/s": gbs,
-               "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps,
+               "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps, "clocks": clocks,
                "note": "one bl_forward_rmsnorm call per layer (norm weight read counted)"}
         if wl.w.M > 1:
             tops = wl.ops_per_step * steps / sec / 1e12
             ent["TOPS"] = tops
-            ent["tensor_frac"] = tops / (peaks["bf16_tflops_sustained"] * INT8_NOMINAL_RATIO)
+            ent["tensor_frac"] = tops / i8
         out.append(ent)
         del wl
         torch.cuda.empty_cache()
-    if not args.secondary or "quantize_weights_70b" in args.secondary.split(","):
+    if not want or "quantize_weights_70b" in want:
         out.append(time_quantize_weights())
     return out
 
@@ -689,7 +765,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--secondary", default="", help="comma list restricting the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
     args = ap.parse_args()
     if args.impl == "reference":
         if args.steps is None:

@@ -52,6 +52,12 @@ SIGNATURES = {
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
     "bl_selftest_wait_timeout": (_int, [ctypes.c_ulonglong, _p, _p]),
+    "bl_probe_mma_i8": (_int, [_int, _int, _p, _int, _p]),
+    "bl_packed_weight_bytes_b3": (_sz, [_i64, _i64]),
+    "bl_quantize_weights_b3": (_int, [_p, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "bl_unpack_weights_b3": (_int, [_p, _i64, _i64, _p, _p]),
+    "bl_forward_b3": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p]),
+    "bl_matmul_i32_b3": (_int, [_p, _i64, _i64, _i64, _p, _p, _p]),
 }
 
 _lib = None
@@ -365,3 +371,65 @@ def bl_selftest_wait_timeout(limit_ns: int) -> torch.Tensor:
     out = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     _check(lib().bl_selftest_wait_timeout(limit_ns, out.data_ptr(), _stream()), "bl_selftest_wait_timeout")
     return out
+
+
+def bl_probe_mma_i8(n_mma: int, n_cols: int = 256, grid: int | None = None) -> torch.Tensor:
+    """tcgen05 kind::i8 rate probe: int64 [grid, 2] of (SM cycles, ns) per CTA
+    for n_mma MMAs of 128 x n_cols x 32 (one CTA per SM by default)."""
+    if grid is None:
+        grid = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    out = torch.zeros((grid, 2), dtype=torch.int64, device="cuda")
+    _check(lib().bl_probe_mma_i8(n_mma, n_cols, out.data_ptr(), grid, _stream()), "bl_probe_mma_i8")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# base-3 weight storage (five weights a byte)
+# ---------------------------------------------------------------------------
+
+def bl_packed_weight_bytes_b3(N: int, K: int) -> int:
+    return int(lib().bl_packed_weight_bytes_b3(N, K))
+
+
+def bl_quantize_weights_b3(W: torch.Tensor):
+    """fp32 [N, K] -> (base-3 uint8 [N, row bytes], gamma fp32 [1])."""
+    N, K = W.shape
+    pW = _dev(W, torch.float32, "W")
+    nb = bl_packed_weight_bytes_b3(N, K)
+    Wp3 = torch.empty((N, max(nb // max(N, 1), 1)), dtype=torch.uint8, device=W.device)
+    gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    ws = _workspace(int(lib().bl_quantize_weights_workspace_bytes(N, K)), W.device)
+    _check(lib().bl_quantize_weights_b3(pW, N, K, Wp3.data_ptr(), gamma.data_ptr(),
+                                        ws.data_ptr() if ws is not None else None,
+                                        ws.numel() if ws is not None else 0, _stream()), "bl_quantize_weights_b3")
+    return Wp3, gamma
+
+
+def bl_unpack_weights_b3(Wp3: torch.Tensor, N: int, K: int) -> torch.Tensor:
+    p = _dev(Wp3, torch.uint8, "Wp3")
+    codes = torch.empty((N, K), dtype=torch.int8, device=Wp3.device)
+    _check(lib().bl_unpack_weights_b3(p, N, K, codes.data_ptr(), _stream()), "bl_unpack_weights_b3")
+    return codes
+
+
+def bl_forward_b3(X: torch.Tensor, Wp3: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+    """One-token BitLinear forward on base-3 weights: bf16 [1, K] -> bf16 [1, N]."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pw = _dev(Wp3, torch.uint8, "Wp3")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    _check(lib().bl_forward_b3(px, M, K, N, pw, pg, bits, py, _stream()), "bl_forward_b3")
+    return Y
+
+
+def bl_matmul_i32_b3(Xq: torch.Tensor, Wp3: torch.Tensor, N: int) -> torch.Tensor:
+    """Exact int32 accumulators of one token's int8 codes x base-3 weights (test export)."""
+    M, K = Xq.shape
+    px = _dev(Xq, torch.int8, "Xq")
+    pw = _dev(Wp3, torch.uint8, "Wp3")
+    acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    _check(lib().bl_matmul_i32_b3(px, M, K, N, pw, acc.data_ptr(), _stream()), "bl_matmul_i32_b3")
+    return acc

@@ -17,11 +17,12 @@
 #include "../../include/bitlinear.h"
 #include "bl_act.cuh"
 #include "bl_common.cuh"
-#include "bl_gemm_tc.cuh"
+#include "bl_tc_common.cuh"
 #include "bl_gemm_tc2.cuh"
 #include "bl_gemm_2sm.cuh"
 #include "bl_gemv.cuh"
-#include "bl_gemv3.cuh"
+#include "bl_decode.cuh"
+#include "bl_probe.cuh"
 #include "bl_weights.cuh"
 
 namespace {
@@ -130,12 +131,12 @@ bl_status launch_gemv_t(const void* X, int x_is_i8, int M, int K, int N, const u
   static std::atomic<uint64_t> done{0};
   const int KL = static_cast<int>(align_up(static_cast<size_t>(K), 128));
   const int smem = MT * KL;
-  if (!ensure_smem(bl::gemv_kernel<MT, RT>, MT * static_cast<int>(kMaxK), &done)) return BL_ERR_CUDA;
+  if (!ensure_smem(bl::bl_decode_long_kernel<MT, RT>, MT * static_cast<int>(kMaxK), &done)) return BL_ERR_CUDA;
   const int ntiles = (N + RT - 1) / RT;
   int blocks = (ntiles + bl::kGemvWarps - 1) / bl::kGemvWarps;
   const int cap = 2 * num_sms();
   if (blocks > cap) blocks = cap;
-  bl::gemv_kernel<MT, RT><<<blocks, bl::kGemvThreads, smem, stream>>>(
+  bl::bl_decode_long_kernel<MT, RT><<<blocks, bl::kGemvThreads, smem, stream>>>(
       X, x_is_i8, M, K, N, reinterpret_cast<const uint4*>(Wp), gamma, Q, Y, out_mode);
   return last_cuda();
 }
@@ -163,61 +164,29 @@ bl_status launch_gemv1_t(const void* X, int x_is_i8, int K, int N, const uint8_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const uint4* wp4 = reinterpret_cast<const uint4*>(Wp);
-  if (cudaLaunchKernelEx(&cfg, bl::gemv1_kernel<MT, CPL, RT, D, THREADS, MINB>, X, x_is_i8, K, N, wp4, gamma, Q, Y,
+  if (cudaLaunchKernelEx(&cfg, bl::bl_decode_rows_kernel<MT, CPL, RT, D, THREADS, MINB>, X, x_is_i8, K, N, wp4, gamma, Q, Y,
                          out_mode, tiles_per_cta) != cudaSuccess)
     return BL_ERR_CUDA;
   return last_cuda();
 }
 
-template <int MT, int CPL>
-bl_status launch_gemv2_table(const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode, cudaStream_t stream) {
-  static std::atomic<uint64_t> done{0};
-  if (!ensure_smem(bl::gemv2_kernel<MT, CPL>, bl::kG2SmemBytes, &done)) return BL_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(bl::kG2Threads);
-  cfg.dynamicSmemBytes = bl::kG2SmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const unsigned long long lim = kWaitLimitNs;
-  if (cudaLaunchKernelEx(&cfg, bl::gemv2_kernel<MT, CPL>, tab, x_is_i8, Q, out_mode, lim) != cudaSuccess)
-    return BL_ERR_CUDA;
-  return last_cuda();
-}
+// ---------------------------------------------------------------------------
+// One-token problems: the decode kernel (bl_decode_kernel), resident or big
+// ring mode.
+// ---------------------------------------------------------------------------
 
-bl_status launch_gemv2_cpl(int cpl, const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode,
-                           cudaStream_t stream) {
-  switch (cpl) {
-    case 1: return launch_gemv2_table<1, 1>(tab, grid, x_is_i8, Q, out_mode, stream);
-    case 2: return launch_gemv2_table<1, 2>(tab, grid, x_is_i8, Q, out_mode, stream);
-    case 3: return launch_gemv2_table<1, 3>(tab, grid, x_is_i8, Q, out_mode, stream);
-    default: return launch_gemv2_table<1, 4>(tab, grid, x_is_i8, Q, out_mode, stream);
-  }
-}
-
-#ifndef BL_G3_WARPS
-#define BL_G3_WARPS 16
-#endif
-// consumer warps of the decode kernel (16: enough warps to hide shared-memory
-// and dp4a latency, and registers for two CTAs per SM)
-template <int WPL>
-constexpr int g3_warps() { return BL_G3_WARPS; }
-
-template <int WPL, int PRE>
-bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode, cudaStream_t stream) {
-  auto kern = bl::gemv3_kernel<WPL, g3_warps<WPL>(), PRE>;
+template <int A, int PRE, int FMT, int MODE>
+bl_status launch_dec_t(const bl::G2Table& tab, int grid, int in_mode, int Q, int out_mode, cudaStream_t stream) {
+  auto kern = bl::bl_decode_kernel<A, PRE, FMT, MODE>;
+  constexpr int smem = MODE == bl::kModeBig ? bl::kDecBigSmemBytes : bl::kDecSmemBytes;
   static std::atomic<uint64_t> done{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
   if (!(done.load(std::memory_order_acquire) & (uint64_t(1) << dev))) {
-    // two CTAs per SM (this launch's and the next one's) need the largest
-    // shared-memory carve-out
+    // resident mode: two CTAs per SM (this launch's and the next one's) need
+    // the largest shared-memory carve-out; big mode: one CTA takes most of it
     if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bl::kG3SmemBytes) != cudaSuccess ||
+                             smem) != cudaSuccess ||
         cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return BL_ERR_CUDA;
@@ -225,10 +194,10 @@ bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(bl::G3Cfg<WPL, g3_warps<WPL>()>::kThreads);
-  // the same footprint for every launch: a third CTA never fits on an SM,
-  // so two CTAs of one launch never share an SM
-  cfg.dynamicSmemBytes = bl::kG3SmemBytes;
+  cfg.blockDim = dim3(bl::kDecThreads);
+  // the same footprint for every launch: in resident mode a third CTA never
+  // fits on an SM, so two CTAs of one launch never share an SM
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -236,64 +205,151 @@ bl_status launch_gemv3_table(const bl::G2Table& tab, int grid, int x_is_i8, int 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const unsigned long long lim = kWaitLimitNs;
-  if (cudaLaunchKernelEx(&cfg, kern, tab, x_is_i8, Q, out_mode, lim) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, tab, in_mode, Q, out_mode, lim) != cudaSuccess) return BL_ERR_CUDA;
   return last_cuda();
 }
 
-// words of 16 weights per lane: K / 512 rounded up (K <= 8192)
-bl_status launch_gemv3_wpl(int wpl, const bl::G2Table& tab, int grid, int x_is_i8, int Q, int out_mode,
-                           cudaStream_t stream) {
-  const int pre = (x_is_i8 == bl::kInRelu2 || x_is_i8 == bl::kInRelu2Gated) ? bl::kG3Relu2
-                  : x_is_i8 == bl::kInRmsNorm                                ? bl::kG3Rms
-                                                                             : bl::kG3Plain;
-  switch (wpl) {
-#define BL_G3_CASE(n)                                                                    \
-  case n:                                                                                \
-    return pre == bl::kG3Relu2 ? launch_gemv3_table<n, bl::kG3Relu2>(tab, grid, x_is_i8, Q, out_mode, stream) \
-           : pre == bl::kG3Rms ? launch_gemv3_table<n, bl::kG3Rms>(tab, grid, x_is_i8, Q, out_mode, stream)   \
-                               : launch_gemv3_table<n, bl::kG3Plain>(tab, grid, x_is_i8, Q, out_mode, stream);
-    BL_G3_CASE(1) BL_G3_CASE(2) BL_G3_CASE(3) BL_G3_CASE(4) BL_G3_CASE(5) BL_G3_CASE(6) BL_G3_CASE(7) BL_G3_CASE(8)
-    BL_G3_CASE(9) BL_G3_CASE(10) BL_G3_CASE(11) BL_G3_CASE(12) BL_G3_CASE(13) BL_G3_CASE(14) BL_G3_CASE(15)
-    BL_G3_CASE(16)
-#undef BL_G3_CASE
-    default: return BL_ERR_UNSUPPORTED;
+template <int PRE>
+bl_status launch_dec_resident(int wplr, const bl::G2Table& tab, int grid, int in_mode, int Q, int out_mode,
+                              cudaStream_t stream) {
+  constexpr int F = bl::kFmt2Bit, M = bl::kModeResident;
+  switch (wplr) {
+    case 1: return launch_dec_t<1, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    case 2: return launch_dec_t<2, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    case 3: return launch_dec_t<3, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    case 4: return launch_dec_t<4, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    default: return launch_dec_t<5, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
   }
 }
 
-// Decode kernel selection (build-time, for experiments): 0 = by shape (one
-// token: the resident decode kernel when the layer's weights fit its ring on
-// every SM, the TMA-staged streaming GEMV otherwise), 1 = register-ring GEMV
-// only, 2 = the TMA-staged GEMV for every one-token layer.
-#ifndef BL_DECODE_KERNEL
-#define BL_DECODE_KERNEL 0
-#endif
-constexpr int kDecodeKernel = BL_DECODE_KERNEL;
-
-// Fill a launch table with one-token problems of one kernel variant: every
-// problem gets CTAs in proportion to its weight bytes (at least one, at most
-// one per row), and the launch has exactly one CTA per SM when the rows allow.
-// Returns the grid size.
-int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, const void* U,
-                      const float* bias) {
-  std::memset(tab, 0, sizeof(*tab));
-  double total = 0.0;
-  int64_t rows = 0;
-  for (int i = 0; i < n; ++i) {
-    total += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K);
-    rows += probs[i]->N;
+template <int PRE>
+bl_status launch_dec_big(int cpl, const bl::G2Table& tab, int grid, int in_mode, int Q, int out_mode,
+                         cudaStream_t stream) {
+  constexpr int F = bl::kFmt2Bit, M = bl::kModeBig;
+  switch (cpl) {
+    case 1: return launch_dec_t<1, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    case 2: return launch_dec_t<2, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    case 3: return launch_dec_t<3, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
+    default: return launch_dec_t<4, PRE, F, M>(tab, grid, in_mode, Q, out_mode, stream);
   }
-  const int target = static_cast<int>(rows < sms ? rows : sms);
+}
+
+// Words of 16 weights per lane for a row of K weights (resident mode).
+inline int dec_wpl(int64_t K) { return static_cast<int>((K + 511) / 512); }
+// 16-byte chunks per lane (big mode).
+inline int dec_cpl(int64_t K) { return static_cast<int>((K + 2047) / 2048); }
+
+// The register width A of one resident launch (words of codes a lane keeps,
+// <= 5): the words-per-lane class that holds the most weight bytes (5 if no
+// problem has K <= 2560), raised so that no row needs more than
+// kDecMaxSplit warps.  Longer rows are split across a team of warps.
+int dec_pick_wplr(const bl_linear* const* probs, int n) {
+  double bytes[bl::kDecRegMaxWpl + 1] = {};
+  int64_t max_words = 0;
+  for (int i = 0; i < n; ++i) {
+    const int w = dec_wpl(probs[i]->K);
+    if (w <= bl::kDecRegMaxWpl) bytes[w] += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K);
+    max_words = std::max<int64_t>(max_words, probs[i]->K / 16);
+  }
+  int best = bl::kDecRegMaxWpl;
+  double most = 0.0;
+  for (int w = 1; w <= bl::kDecRegMaxWpl; ++w)
+    if (bytes[w] > most) {
+      most = bytes[w];
+      best = w;
+    }
+  const int floor_a = static_cast<int>((max_words + 32 * bl::kDecMaxSplit - 1) / (32 * bl::kDecMaxSplit));
+  return std::max(best, floor_a);
+}
+
+// Warps that split one row of K weights at register width a (resident 2-bit).
+inline int dec_split(int64_t K, int a) { return static_cast<int>((K / 16 + 32 * a - 1) / (32 * a)); }
+
+// Bytes of one stored row.
+inline int dec_row_bytes(int64_t K, int fmt) {
+  return fmt == bl::kFmtBase3 ? 4 * bl::base3_row_words(static_cast<int>(K)) : static_cast<int>(K / 4);
+}
+
+// Rows a warp (team) takes at once.
+inline int dec_rt(int mode, int fmt) {
+  if (mode == bl::kModeBig) return bl::kDecBigRows;
+  return fmt == bl::kFmt2Bit ? bl::kDecRegRows : bl::kDecB3Rows;
+}
+
+// Estimated time of one CTA of a problem that gets `ctas` CTAs.  Resident
+// mode: rounds of row groups over the CTA's teams of warps times the cost of
+// a group (issue slots of one warp: per word a lane keeps, two shared loads,
+// eight masks and eight dp4a at half rate for the two rows; the rows'
+// reductions and stores; a team barrier when rows are split), plus a penalty
+// for bytes that do not fit the ring (fetched after the dependency wait).
+// Big mode: the weight bytes a CTA streams.
+double dec_cta_cost(int64_t N, int64_t K, int ctas, int a, int fmt, int mode) {
+  const int64_t rows = (N + ctas - 1) / ctas;
+  const double bytes = static_cast<double>(rows) * static_cast<double>(dec_row_bytes(K, fmt));
+  if (mode == bl::kModeBig) return bytes;
+  const int rt = dec_rt(mode, fmt);
+  const int64_t groups = (rows + rt - 1) / rt;
+  double group;
+  int teams;
+  if (fmt == bl::kFmtBase3) {
+    group = ((bl::base3_row_words(static_cast<int>(K)) + 31) / 32) * 140.0 + 70.0;
+    teams = bl::kDecWarps;
+  } else {
+    const int S = dec_split(K, a);
+    group = a * 26.0 + 40.0 + (S > 1 ? 60.0 : 0.0);
+    teams = bl::kDecWarps / S;
+  }
+  const int64_t rounds = (groups + teams - 1) / teams;
+  const double over = bytes > bl::kDecRingBytes ? (bytes - bl::kDecRingBytes) / 8.0 : 0.0;
+  return static_cast<double>(rounds) * group + over;
+}
+
+// Fill a launch table with one-token problems: CTAs are shared out so that
+// the slowest CTA (by the cost model above) is as fast as possible, and the
+// launch has exactly one CTA per SM when the rows allow.  Each problem's row
+// range per CTA is cut into whole-group chunks: in resident mode as few as
+// fit the ring without reuse when possible; in big mode one group per warp
+// per chunk.  Returns the grid size.
+int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, int mode, int a,
+                      const void* U, const float* bias, float eps, int fmt = bl::kFmt2Bit) {
+  std::memset(tab, 0, sizeof(*tab));
+  int64_t rows_total = 0;
+  for (int i = 0; i < n; ++i) rows_total += probs[i]->N;
+  const int target = static_cast<int>(rows_total < sms ? rows_total : sms);
+  // smallest CTA count of problem i whose cost is <= T
+  auto need = [&](int i, double T) {
+    const int64_t Nn = probs[i]->N;
+    int lo = 1, hi = static_cast<int>(Nn < target ? Nn : target);
+    if (dec_cta_cost(Nn, probs[i]->K, hi, a, fmt, mode) > T) return hi + 1;   // infeasible
+    while (lo < hi) {
+      const int mid = (lo + hi) / 2;
+      if (dec_cta_cost(Nn, probs[i]->K, mid, a, fmt, mode) <= T)
+        hi = mid;
+      else
+        lo = mid + 1;
+    }
+    return lo;
+  };
+  // the smallest makespan that fits the grid: binary search over the costs
+  double lo_t = 0.0, hi_t = 0.0;
+  for (int i = 0; i < n; ++i)
+    hi_t = std::max(hi_t, dec_cta_cost(probs[i]->N, probs[i]->K, 1, a, fmt, mode));
   int c[bl::kG2MaxProblems];
+  for (int it = 0; it < 60; ++it) {
+    const double mid = 0.5 * (lo_t + hi_t);
+    int sum = 0;
+    for (int i = 0; i < n; ++i) sum += need(i, mid);
+    if (sum <= target)
+      hi_t = mid;
+    else
+      lo_t = mid;
+  }
   int sum = 0;
   for (int i = 0; i < n; ++i) {
-    const double share = static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / total;
-    int v = static_cast<int>(share * target);
-    if (v < 1) v = 1;
-    if (v > probs[i]->N) v = static_cast<int>(probs[i]->N);
-    c[i] = v;
-    sum += v;
+    c[i] = need(i, hi_t);
+    sum += c[i];
   }
-  // hand out the remaining CTAs to the problems with the most bytes a CTA
+  // spare CTAs go to the problems with the most weight bytes per CTA
   while (sum < target) {
     int best = -1;
     double most = 0.0;
@@ -309,57 +365,82 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
     c[best] += 1;
     sum += 1;
   }
+  const int ring = mode == bl::kModeBig ? bl::kDecBigRingBytes : bl::kDecRingBytes;
+  const int chunk_max = mode == bl::kModeBig ? bl::kDecBigChunkMax : bl::kDecChunkMax;
   int grid = 0;
   for (int i = 0; i < n; ++i) {
     const bl_linear& p = *probs[i];
-    const int rows_per_cta = static_cast<int>((p.N + c[i] - 1) / c[i]);
-    tab->p[i] = bl::G2Problem{p.X, U, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
-                              rows_per_cta, grid, c[i], bias};
+    const int rb = dec_row_bytes(p.K, fmt);
+    const int rt = dec_rt(mode, fmt);
+    const int maxrows = static_cast<int>((p.N + c[i] - 1) / c[i]);
+    int cr = (chunk_max / rb) / rt * rt, slots = 0;
+    if (mode == bl::kModeBig) {
+      // one group per consumer warp per chunk
+      cr = std::min(cr, bl::kDecWarps * rt);
+      slots = std::min(bl::kDecMaxSlots, ring / (cr * rb));
+    } else {
+      const int cr_max = cr;
+      for (; cr >= rt; cr -= rt) {
+        slots = std::min(bl::kDecMaxSlots, ring / (cr * rb));
+        if ((maxrows + cr - 1) / cr <= slots) break;
+      }
+      if (cr < rt) {
+        cr = cr_max;
+        slots = std::min(bl::kDecMaxSlots, ring / (cr * rb));
+      }
+    }
+    bl::G2Problem& q = tab->p[i];
+    q.X = p.X;
+    q.U = U;
+    q.Wp = p.Wp;
+    q.gamma = p.gamma;
+    q.Y = p.Y;
+    q.K = static_cast<int>(p.K);
+    q.N = static_cast<int>(p.N);
+    q.rows_per_cta = static_cast<int>(p.N / c[i]);
+    q.rows_rem = static_cast<int>(p.N % c[i]);
+    q.cta_begin = grid;
+    q.ctas = c[i];
+    q.bias = bias;
+    q.eps = eps;
+    q.chunk_rows = cr;
+    q.slots = slots;
+    q.ksplit = (mode == bl::kModeResident && fmt == bl::kFmt2Bit) ? dec_split(p.K, a) : 1;
     grid += c[i];
   }
   tab->count = n;
   return grid;
 }
 
-// Launch one-token problems that share a kernel variant (at most
-// kG2MaxProblems).
-// in_mode: bl::InMode of the token input; U: the up projection's output in
-// the gated squared-ReLU mode (shared by every problem of the call).
+// Launch one-token problems (K <= 8192, at most kG2MaxProblems) in one kernel:
+// resident mode when the weights fit the rings of one CTA per SM, big mode
+// otherwise (RMSNorm is formed only in resident mode; callers check the fit).
+// in_mode: bl::InMode of the token input; U: the up projection's output in the
+// gated squared-ReLU mode, or the RMSNorm weight (shared by every problem of
+// the call); eps: the RMSNorm epsilon.
 bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q, int out_mode, cudaStream_t stream,
-                        const void* U = nullptr, const float* bias = nullptr) {
+                        const void* U = nullptr, const float* bias = nullptr, float eps = 0.f) {
   if (n <= 0) return BL_OK;
   const int sms = num_sms();
-  bl::G2Table tab;
-  int maxK = 64;
   double wbytes = 0.0;
+  int maxK = 64;
   for (int i = 0; i < n; ++i) {
-    if (probs[i]->K > maxK) maxK = static_cast<int>(probs[i]->K);
     wbytes += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / 4.0;
+    if (probs[i]->K > maxK) maxK = static_cast<int>(probs[i]->K);
   }
-  // layers whose weights do not fit the resident kernel's ring on every SM
-  // stream through the deeper TMA-staged GEMV instead
-  const bool streaming = wbytes > static_cast<double>(sms) * bl::kG3Stages * bl::kG3StageBytes;
-  if (kDecodeKernel == 2 || streaming) {
-    // the first TMA-staged GEMV: ceil(N / SMs) rows a CTA
-    std::memset(&tab, 0, sizeof(tab));
-    double total = 0.0;
-    for (int i = 0; i < n; ++i) total += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K);
-    int grid = 0;
-    for (int i = 0; i < n; ++i) {
-      const bl_linear& p = *probs[i];
-      int c = static_cast<int>(sms * (static_cast<double>(p.N) * static_cast<double>(p.K)) / total);
-      if (c < 1) c = 1;
-      const int rows_per_cta = static_cast<int>((p.N + c - 1) / c);
-      c = static_cast<int>((p.N + rows_per_cta - 1) / rows_per_cta);
-      tab.p[i] = bl::G2Problem{p.X, U, p.Wp, p.gamma, p.Y, static_cast<int>(p.K), static_cast<int>(p.N),
-                               rows_per_cta, grid, c, bias};
-      grid += c;
-    }
-    tab.count = n;
-    return launch_gemv2_cpl((maxK / 64 + 31) / 32, tab, grid, in_mode, Q, out_mode, stream);
+  const bool big = in_mode != bl::kInRmsNorm && wbytes > static_cast<double>(sms) * bl::kDecRingBytes;
+  const int mode = big ? bl::kModeBig : bl::kModeResident;
+  const int a = big ? dec_cpl(maxK) : dec_pick_wplr(probs, n);
+  bl::G2Table tab;
+  const int grid = fill_decode_table(&tab, probs, n, sms, mode, a, U, bias, eps);
+  const bool relu2 = in_mode == bl::kInRelu2 || in_mode == bl::kInRelu2Gated;
+  if (big) {
+    if (relu2) return launch_dec_big<bl::kDecRelu2>(a, tab, grid, in_mode, Q, out_mode, stream);
+    return launch_dec_big<bl::kDecPlain>(a, tab, grid, in_mode, Q, out_mode, stream);
   }
-  const int grid = fill_decode_table(&tab, probs, n, sms, U, bias);
-  return launch_gemv3_wpl((maxK + 511) / 512, tab, grid, in_mode, Q, out_mode, stream);
+  if (relu2) return launch_dec_resident<bl::kDecRelu2>(a, tab, grid, in_mode, Q, out_mode, stream);
+  if (in_mode == bl::kInRmsNorm) return launch_dec_resident<bl::kDecRms>(a, tab, grid, in_mode, Q, out_mode, stream);
+  return launch_dec_resident<bl::kDecPlain>(a, tab, grid, in_mode, Q, out_mode, stream);
 }
 
 // Single one-token problem.
@@ -377,25 +458,14 @@ bl_status launch_decode_one(const void* X, int x_is_i8, int K, int N, const uint
   return launch_decode(&pp, 1, x_is_i8, Q, out_mode, stream);
 }
 
+// One token with K <= 8192: the decode kernels; two tokens: the register-ring
+// GEMV; longer rows: the general GEMV.
 bl_status launch_gemv(const void* X, int x_is_i8, int M, int K, int N, const uint8_t* Wp, const float* gamma, int Q,
                       void* Y, int out_mode, cudaStream_t stream) {
-  const int cplx = (K / 64 + 31) / 32;
-  // one token: the TMA-staged kernel (measured at least as fast on every
-  // decode shape); two tokens: the register-ring kernel
-  const bool staged = (kDecodeKernel == 2) || (kDecodeKernel == 0 && M == 1);
-  (void)cplx;
-  if (staged && M == 1 && K <= 8192) return launch_decode_one(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
+  if (M == 1 && K <= bl::kDecMaxK) return launch_decode_one(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
   const int cpl = (K / 64 + 31) / 32;
   // one CTA of 16 warps per SM (room for the next kernel's CTA to start its
   // L2 prefetch alongside); D tiles of weights in flight per warp
-  if (M == 1 && K <= 8192) {
-    switch (cpl) {
-      case 1: return launch_gemv1_t<1, 1, 2, 4, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-      case 2: return launch_gemv1_t<1, 2, 1, 4, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-      case 3: return launch_gemv1_t<1, 3, 1, 3, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-      default: return launch_gemv1_t<1, 4, 1, 2, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
-    }
-  }
   if (M == 2 && K <= 4096) {
     if (cpl == 1) return launch_gemv1_t<2, 1, 2, 2, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
     return launch_gemv1_t<2, 2, 1, 2, 512, 1>(X, x_is_i8, K, N, Wp, gamma, Q, Y, out_mode, stream);
@@ -410,35 +480,11 @@ bl_status launch_act_quant(const uint16_t* X, int m, int k, int Q, int8_t* Xq, f
   // measured: the CTA-per-row kernel also wins for long rows (K > 4096, where
   // a warp can no longer keep its row in registers and reads part of it twice)
   if (m < bl::kActRowsPerBlock * num_sms() || k > 32 * 8 * bl::kActCache) {
-    bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, nullptr);
+    bl::bl_act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, nullptr);
   } else {
     const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
-    bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
+    bl::bl_act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
   }
-  return last_cuda();
-}
-
-#ifndef BL_P2_EXPG
-#define BL_P2_EXPG 1
-#endif
-
-template <int BN>
-bl_status launch_tc_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
-                      const float* gamma, void* Y, int out_mode, int debug_flags, unsigned long long limit_ns,
-                      cudaStream_t stream) {
-  using C = bl::TcCfg<BN>;
-  static std::atomic<uint64_t> done{0};
-  if (!ensure_smem(bl::tc_gemm_kernel<BN>, C::kSmemBytes, &done)) return BL_ERR_CUDA;
-  CUtensorMap tmX, tmW;
-  if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), BN, bl::kTcBK,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return BL_ERR_CUDA;
-  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kTcBK / 4,
-                    CU_TENSOR_MAP_SWIZZLE_32B))
-    return BL_ERR_CUDA;
-  const dim3 grid((N + bl::kTcRows - 1) / bl::kTcRows, (M + BN - 1) / BN);
-  bl::tc_gemm_kernel<BN><<<grid, bl::kTcThreads, C::kSmemBytes, stream>>>(tmX, tmW, M, N, K, R, s, gamma, Y, out_mode,
-                                                                         limit_ns, debug_flags);
   return last_cuda();
 }
 
@@ -447,7 +493,7 @@ bl_status launch_tc2_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp,
                        const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias) {
   using C = bl::P2Cfg<BN>;
   static std::atomic<uint64_t> done{0};
-  if (!ensure_smem(bl::tc_gemm_persistent_kernel<BN, EXPG>, C::kSmemBytes, &done)) return BL_ERR_CUDA;
+  if (!ensure_smem(bl::bl_mma_persistent_kernel<BN, EXPG>, C::kSmemBytes, &done)) return BL_ERR_CUDA;
   CUtensorMap tmX, tmW;
   if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), BN, bl::kTcBK,
                     CU_TENSOR_MAP_SWIZZLE_128B))
@@ -457,7 +503,7 @@ bl_status launch_tc2_t(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp,
     return BL_ERR_CUDA;
   const int ntiles = ((M + BN - 1) / BN) * ((N + bl::kTcRows - 1) / bl::kTcRows);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
-  bl::tc_gemm_persistent_kernel<BN, EXPG><<<grid, bl::P2Warps<EXPG>::kThreads, C::kSmemBytes, stream>>>(
+  bl::bl_mma_persistent_kernel<BN, EXPG><<<grid, bl::P2Warps<EXPG>::kThreads, C::kSmemBytes, stream>>>(
       tmX, tmW, M, N, K, R, s, gamma, Y, out_mode, bias, kWaitLimitNs);
   return last_cuda();
 }
@@ -491,13 +537,13 @@ int max_active_pairs(F* kernel, int threads, int smem) {
 bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
                          const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias) {
   static std::atomic<uint64_t> done{0};
-  if (!ensure_smem(bl::tc_gemm_pair_kernel, bl::kQSmemBytes, &done)) return BL_ERR_CUDA;
+  if (!ensure_smem(bl::bl_mma_pair_kernel, bl::kQSmemBytes, &done)) return BL_ERR_CUDA;
   CUtensorMap tmX, tmW;
   if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), bl::kQHalf, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BL_ERR_CUDA;
   if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kQBK / 4,
-                    bl::kQBK == 512 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+                    CU_TENSOR_MAP_SWIZZLE_128B))
     return BL_ERR_CUDA;
   // bf16 outputs leave through TMA stores when the rows are 16-byte aligned
   CUtensorMap tmY;
@@ -520,7 +566,7 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
   cudaLaunchConfig_t cfg = {};
   // a persistent grid must fit in one wave: not every SM can host half of a
   // two-SM cluster, so ask how many clusters are co-resident (once per device)
-  int npairs = max_active_pairs(bl::tc_gemm_pair_kernel, bl::kQThreads, bl::kQSmemBytes);
+  int npairs = max_active_pairs(bl::bl_mma_pair_kernel, bl::kQThreads, bl::kQSmemBytes);
   if (npairs <= 0) return BL_ERR_CUDA;
   if (npairs > ntiles) npairs = ntiles;
   cfg.gridDim = dim3(2 * npairs);
@@ -535,36 +581,20 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const unsigned long long lim = kWaitLimitNs;
-  if (cudaLaunchKernelEx(&cfg, bl::tc_gemm_pair_kernel, tmX, tmW, tmY, M, N, K, R, s, gamma, Y, out_mode, tma_store,
+  if (cudaLaunchKernelEx(&cfg, bl::bl_mma_pair_kernel, tmX, tmW, tmY, M, N, K, R, s, gamma, Y, out_mode, tma_store,
                          bias, lim) != cudaSuccess)
     return BL_ERR_CUDA;
   return last_cuda();
 }
 
-// Tensor-core kernel selection (build-time, for experiments): 0 = by shape
-// (CTA-pair kernel for M > 64, one-SM persistent kernel otherwise),
-// 1 = one-tile-per-CTA kernel.
-#ifndef BL_TC_KERNEL
-#define BL_TC_KERNEL 0
-#endif
-
+// Tensor-core GEMM by token count: the CTA-pair kernel for M > 64, the
+// one-SM persistent kernel (token tile 16, 32 or 64) otherwise.
 bl_status launch_tc(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
-                    const float* gamma, void* Y, int out_mode, int debug_flags, cudaStream_t stream,
-                    const float* bias = nullptr) {
-  if (BL_TC_KERNEL == 0 && debug_flags == 0 && M > 64)
-    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
-  if (BL_TC_KERNEL != 1 && debug_flags == 0) {
-    if (M <= 16) return launch_tc2_t<16, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
-    if (M <= 32) return launch_tc2_t<32, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
-    if (M <= 64) return launch_tc2_t<64, BL_P2_EXPG>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
-    return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
-  }
-  const unsigned long long lim = kWaitLimitNs;
-  if (M <= 16) return launch_tc_t<16>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
-  if (M <= 32) return launch_tc_t<32>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
-  if (M <= 64) return launch_tc_t<64>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
-  if (M <= 128) return launch_tc_t<128>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
-  return launch_tc_t<256>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, debug_flags, lim, stream);
+                    const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias = nullptr) {
+  if (M > 64) return launch_tc_pair(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
+  if (M <= 16) return launch_tc2_t<16, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
+  if (M <= 32) return launch_tc2_t<32, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
+  return launch_tc2_t<64, 1>(Xq, M, K, N, Wp, R, s, gamma, Y, out_mode, stream, bias);
 }
 
 struct FwdWs {
@@ -608,7 +638,7 @@ bl_status forward_common(const uint16_t* X, int64_t M, int64_t K, int64_t N, con
   if (M <= kGemvMaxM) return launch_gemv(X, 0, m, k, n, Wp, gamma, Q, Y, out_mode, stream);
   const FwdWs w = fwd_ws_split(ws, M, K);
   if ((st = launch_act_quant(X, m, k, Q, w.Xq, w.s, w.R, stream)) != BL_OK) return st;
-  return launch_tc(w.Xq, m, k, n, Wp, w.R, w.s, gamma, Y, out_mode, 0, stream);
+  return launch_tc(w.Xq, m, k, n, Wp, w.R, w.s, gamma, Y, out_mode, stream);
 }
 
 }  // namespace
@@ -666,12 +696,12 @@ bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp,
   const int64_t n = N * K;
   if (cudaMemsetAsync(bins, 0, bl::kAbsumTotals * sizeof(unsigned long long), stream) != cudaSuccess)
     return BL_ERR_CUDA;
-  bl::weight_absum_bins_kernel<<<blocks, bl::kAbsumThreads, 0, stream>>>(W, n, bins);
+  bl::bl_weight_absum_kernel<<<blocks, bl::kAbsumThreads, 0, stream>>>(W, n, bins);
   if ((st = last_cuda()) != BL_OK) return st;
-  bl::weight_gamma_kernel<<<1, 32, 0, stream>>>(bins, static_cast<uint64_t>(n), gamma);
+  bl::bl_weight_gamma_kernel<<<1, 32, 0, stream>>>(bins, static_cast<uint64_t>(n), gamma);
   if ((st = last_cuda()) != BL_OK) return st;
   const int64_t nwords = n / 16;
-  bl::weight_pack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
+  bl::bl_weight_pack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
       W, nwords, gamma, reinterpret_cast<uint32_t*>(Wp));
   return last_cuda();
 }
@@ -683,7 +713,7 @@ bl_status bl_unpack_weights(const uint8_t* Wp, int64_t N, int64_t K, int8_t* cod
   if (!Wp || !codes) return BL_ERR_INVALID_ARG;
   if (!aligned16(Wp) || !aligned16(codes)) return BL_ERR_ALIGNMENT;
   const int64_t nwords = N * K / 16;
-  bl::weight_unpack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
+  bl::bl_weight_unpack_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
       reinterpret_cast<const uint32_t*>(Wp), nwords, codes);
   return last_cuda();
 }
@@ -743,9 +773,9 @@ bl_status bl_matmul_i32(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const
   const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
   if (M <= kGemvMaxM) return launch_gemv(Xq, 1, m, k, n, Wp, nullptr, 0, acc, bl::kOutI32, stream);
   int* R = static_cast<int*>(workspace);
-  bl::act_rowsum_kernel<<<(m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock, 256, 0, stream>>>(Xq, m, k, R);
+  bl::bl_act_rowsum_kernel<<<(m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock, 256, 0, stream>>>(Xq, m, k, R);
   if ((st = last_cuda()) != BL_OK) return st;
-  return launch_tc(Xq, m, k, n, Wp, R, nullptr, nullptr, acc, bl::kOutI32, 0, stream);
+  return launch_tc(Xq, m, k, n, Wp, R, nullptr, nullptr, acc, bl::kOutI32, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -786,6 +816,7 @@ extern "C" {
 
 bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
                              const float* gamma, int bits, uint16_t* Y, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_noalloc");
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if ((st = check_m(M, K)) != BL_OK) return st;
@@ -803,10 +834,9 @@ bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N,
   int8_t* Xq = reinterpret_cast<int8_t*>(base);
   float* s = reinterpret_cast<float*>(base + kNoAllocCodeBytes);
   int* R = reinterpret_cast<int*>(base + kNoAllocCodeBytes + sizeof(float) * kNoAllocMaxM);
-  const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
-  bl::act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
-  if ((st = last_cuda()) != BL_OK) return st;
-  return launch_tc(Xq, m, k, n, Wp, R, s, gamma, Y, bl::kOutBF16, 0, stream);
+  // the same activation quantiser choice and GEMM as bl_forward
+  if ((st = launch_act_quant(X, m, k, Q, Xq, s, R, stream)) != BL_OK) return st;
+  return launch_tc(Xq, m, k, n, Wp, R, s, gamma, Y, bl::kOutBF16, stream);
 }
 
 size_t bl_forward_grouped_workspace_bytes(int count, const bl_linear* problems, int bits) {
@@ -846,24 +876,13 @@ bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, voi
     if (p.M != 1 || p.K > 8192) all_decode = false;
   }
   const int Q = bits == 8 ? 127 : 7;
-  if (all_decode && kDecodeKernel != 1) {
-    // one launch per kernel variant (words of 16 weights a lane, ceil(K / 512))
-    bool used[bl::kG2MaxProblems] = {};
-    for (int i = 0; i < count; ++i) {
-      if (used[i] || problems[i].M == 0) continue;
-      const int64_t key = kDecodeKernel == 2 ? 0 : (problems[i].K + 511) / 512;
-      const bl_linear* sel[bl::kG2MaxProblems];
-      int n = 0;
-      for (int j = i; j < count; ++j) {
-        const bl_linear& p = problems[j];
-        if (used[j] || p.M == 0 || (kDecodeKernel != 2 && (p.K + 511) / 512 != key)) continue;
-        used[j] = true;
-        sel[n++] = &p;
-      }
-      const bl_status st = launch_decode(sel, n, 0, Q, bl::kOutBF16, stream);
-      if (st != BL_OK) return st;
-    }
-    return BL_OK;
+  if (all_decode) {
+    // every one-token problem of the call in one launch (any mix of K)
+    const bl_linear* sel[bl::kG2MaxProblems];
+    int n = 0;
+    for (int i = 0; i < count; ++i)
+      if (problems[i].M != 0) sel[n++] = &problems[i];
+    return launch_decode(sel, n, bl::kInBF16, Q, bl::kOutBF16, stream);
   }
   // otherwise the problems run one after another on the stream (the
   // workspace is reused: stream order serialises them)
@@ -897,7 +916,7 @@ bl_status bl_quant_act_relu2(const uint16_t* G, const uint16_t* U, int64_t M, in
   if (M == 0) return BL_OK;
   if (!G || !Xq || !scale) return BL_ERR_INVALID_ARG;
   if (!aligned16(G) || !aligned16(Xq) || (U && !aligned16(U))) return BL_ERR_ALIGNMENT;
-  bl::act_quant_relu2_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+  bl::bl_act_quant_relu2_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
       G, U, U != nullptr, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr);
   return last_cuda();
 }
@@ -936,11 +955,11 @@ bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int6
   float* s = reinterpret_cast<float*>(base + align_up(static_cast<size_t>(M) * K, 256));
   int* R = reinterpret_cast<int*>(base + align_up(static_cast<size_t>(M) * K, 256) +
                                   align_up(static_cast<size_t>(M) * 4, 256));
-  bl::act_quant_relu2_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+  bl::bl_act_quant_relu2_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
       G, U, U != nullptr, static_cast<int>(K), Q, Xq, s, R);
   if ((st = last_cuda()) != BL_OK) return st;
   return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16,
-                   0, stream);
+                   stream);
 }
 
 size_t ex_ws_bytes(int64_t M, int64_t K) {
@@ -997,14 +1016,14 @@ bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t N, cons
     const int64_t nch = static_cast<int64_t>(M) * K / 8;
     int64_t blocks = (nch + 255) / 256;
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
-    bl::act_absmax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, nch, amax);
+    bl::bl_act_absmax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, nch, amax);
     if ((st = last_cuda()) != BL_OK) return st;
-    bl::act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, amax);
+    bl::bl_act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, amax);
     if ((st = last_cuda()) != BL_OK) return st;
   } else if ((st = launch_act_quant(X, m, k, Q, Xq, s, R, stream)) != BL_OK) {
     return st;
   }
-  return launch_tc(Xq, m, k, static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16, 0, stream, bias);
+  return launch_tc(Xq, m, k, static_cast<int>(N), Wp, R, s, gamma, Y, bl::kOutBF16, stream, bias);
 }
 
 size_t rms_ws_bytes(int64_t M, int64_t K) {
@@ -1032,7 +1051,7 @@ bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, f
   if (!aligned16(X) || !aligned16(Xq) || (norm_weight && !aligned16(norm_weight)) ||
       (reinterpret_cast<uintptr_t>(mean_sq) & 3u))
     return BL_ERR_ALIGNMENT;
-  bl::act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+  bl::bl_act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
       X, norm_weight, eps, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr, mean_sq);
   return last_cuda();
 }
@@ -1055,8 +1074,7 @@ bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, flo
   const int Q = bits == 8 ? 127 : 7;
   const int sms = num_sms();
   const double wbytes = static_cast<double>(N) * static_cast<double>(K) / 4.0;
-  if (M == 1 && K <= bl::kG3MaxK &&
-      wbytes <= static_cast<double>(sms) * bl::kG3Stages * bl::kG3StageBytes) {
+  if (M == 1 && K <= bl::kDecMaxK && wbytes <= static_cast<double>(sms) * bl::kDecRingBytes) {
     // one token whose layer fits the resident decode kernel: RMSNorm,
     // absmax and quantisation in its prologue (the workspace stays unused)
     bl_linear p;
@@ -1068,10 +1086,7 @@ bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, flo
     p.gamma = gamma;
     p.Y = Y;
     const bl_linear* pp = &p;
-    bl::G2Table tab;
-    const int grid = fill_decode_table(&tab, &pp, 1, sms, norm_weight, nullptr);
-    tab.p[0].eps = eps;
-    return launch_gemv3_wpl(static_cast<int>((K + 511) / 512), tab, grid, bl::kInRmsNorm, Q, bl::kOutBF16, stream);
+    return launch_decode(&pp, 1, bl::kInRmsNorm, Q, bl::kOutBF16, stream, norm_weight, nullptr, eps);
   }
   uint8_t* base = static_cast<uint8_t*>(workspace);
   const size_t codes = align_up(static_cast<size_t>(M) * K, 256), rows = align_up(static_cast<size_t>(M) * 4, 256);
@@ -1079,11 +1094,118 @@ bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, flo
   float* s = reinterpret_cast<float*>(base + codes);
   int* R = reinterpret_cast<int*>(base + codes + rows);
   float* ms = reinterpret_cast<float*>(base + codes + 2 * rows);
-  bl::act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+  bl::bl_act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
       X, norm_weight, eps, static_cast<int>(K), Q, Xq, s, R, ms);
   if ((st = last_cuda()) != BL_OK) return st;
   return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y,
-                   bl::kOutBF16, 0, stream);
+                   bl::kOutBF16, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Base-3 weight storage (five weights a byte; see bl_weights.cuh).
+// ---------------------------------------------------------------------------
+
+size_t bl_packed_weight_bytes_b3(int64_t N, int64_t K) {
+  if (check_shape_nk(N, K) != BL_OK) return 0;
+  return static_cast<size_t>(N) * 4u * static_cast<size_t>(bl::base3_row_words(static_cast<int>(K)));
+}
+
+bl_status bl_quantize_weights_b3(const float* W, int64_t N, int64_t K, uint8_t* Wp3, float* gamma, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quantize_weights_b3");
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if (N > INT32_MAX) return BL_ERR_SHAPE;
+  if (!W || !Wp3 || !gamma) return BL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wp3)) return BL_ERR_ALIGNMENT;
+  const size_t need = bl_quantize_weights_workspace_bytes(N, K);
+  if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
+  auto* bins = static_cast<unsigned long long*>(workspace);
+  const int64_t n = N * K;
+  if (cudaMemsetAsync(bins, 0, bl::kAbsumTotals * sizeof(unsigned long long), stream) != cudaSuccess)
+    return BL_ERR_CUDA;
+  bl::bl_weight_absum_kernel<<<absum_blocks(N, K), bl::kAbsumThreads, 0, stream>>>(W, n, bins);
+  if ((st = last_cuda()) != BL_OK) return st;
+  bl::bl_weight_gamma_kernel<<<1, 32, 0, stream>>>(bins, static_cast<uint64_t>(n), gamma);
+  if ((st = last_cuda()) != BL_OK) return st;
+  const int64_t nwords = N * bl::base3_row_words(static_cast<int>(K));
+  bl::bl_weight_pack3_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
+      W, static_cast<int>(N), static_cast<int>(K), gamma, reinterpret_cast<uint32_t*>(Wp3));
+  return last_cuda();
+}
+
+bl_status bl_unpack_weights_b3(const uint8_t* Wp3, int64_t N, int64_t K, int8_t* codes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_unpack_weights_b3");
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if (N > INT32_MAX) return BL_ERR_SHAPE;
+  if (!Wp3 || !codes) return BL_ERR_INVALID_ARG;
+  if (!aligned16(Wp3)) return BL_ERR_ALIGNMENT;
+  const int64_t nwords = N * bl::base3_row_words(static_cast<int>(K));
+  bl::bl_weight_unpack3_kernel<<<static_cast<unsigned>((nwords + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint32_t*>(Wp3), static_cast<int>(N), static_cast<int>(K), codes);
+  return last_cuda();
+}
+
+}  // extern "C"
+
+namespace {
+// One token on base-3 weights: the resident decode kernel in its base-3 form.
+bl_status forward_b3_common(const void* X, int in_mode, int64_t M, int64_t K, int64_t N, const uint8_t* Wp3,
+                            const float* gamma, int Q, void* Y, int out_mode, cudaStream_t stream) {
+  bl_status st = check_shape_nk(N, K);
+  if (st != BL_OK) return st;
+  if ((st = check_m(M, K)) != BL_OK) return st;
+  if (M == 0) return BL_OK;
+  if (M != 1 || K > bl::kDecMaxK || N > INT32_MAX) return BL_ERR_UNSUPPORTED;
+  if (!X || !Wp3 || !Y || (out_mode != bl::kOutI32 && !gamma)) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wp3)) return BL_ERR_ALIGNMENT;
+  bl_linear p;
+  p.X = static_cast<const uint16_t*>(X);
+  p.M = 1;
+  p.K = K;
+  p.N = N;
+  p.Wp = Wp3;
+  p.gamma = gamma;
+  p.Y = static_cast<uint16_t*>(Y);
+  const bl_linear* pp = &p;
+  const int sms = num_sms();
+  const bool big = static_cast<double>(N) * dec_row_bytes(K, bl::kFmtBase3) > static_cast<double>(sms) * bl::kDecRingBytes;
+  bl::G2Table tab;
+  const int mode = big ? bl::kModeBig : bl::kModeResident;
+  const int grid = fill_decode_table(&tab, &pp, 1, sms, mode, 0, nullptr, nullptr, 0.f, bl::kFmtBase3);
+  if (big)
+    return launch_dec_t<0, bl::kDecPlain, bl::kFmtBase3, bl::kModeBig>(tab, grid, in_mode, Q, out_mode, stream);
+  return launch_dec_t<0, bl::kDecPlain, bl::kFmtBase3, bl::kModeResident>(tab, grid, in_mode, Q, out_mode, stream);
+}
+}  // namespace
+
+extern "C" {
+
+bl_status bl_forward_b3(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp3, const float* gamma,
+                        int bits, uint16_t* Y, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_b3");
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  return forward_b3_common(X, bl::kInBF16, M, K, N, Wp3, gamma, bits == 8 ? 127 : 7, Y, bl::kOutBF16, stream);
+}
+
+bl_status bl_matmul_i32_b3(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const uint8_t* Wp3, int32_t* acc,
+                           cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_matmul_i32_b3");
+  return forward_b3_common(Xq, bl::kInI8, M, K, N, Wp3, nullptr, 0, acc, bl::kOutI32, stream);
+}
+
+// Throughput probe of tcgen05.mma kind::i8 (see bl_probe.cuh).
+bl_status bl_probe_mma_i8(int n_mma, int n_cols, unsigned long long* out, int grid, cudaStream_t stream) {
+  if (!out) return BL_ERR_INVALID_ARG;
+  if (n_mma <= 0 || n_mma > (1 << 22) || grid <= 0 || grid > 4096) return BL_ERR_SHAPE;
+  if (n_cols < 16 || n_cols > 256 || (n_cols % 16) != 0) return BL_ERR_SHAPE;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(bl::bl_probe_mma_i8_kernel, bl::kProbeSmemBytes, &done)) return BL_ERR_CUDA;
+  bl::bl_probe_mma_i8_kernel<<<grid, bl::kProbeThreads, bl::kProbeSmemBytes, stream>>>(n_mma, n_cols, out,
+                                                                                       kWaitLimitNs);
+  return last_cuda();
 }
 
 bl_status bl_device_status(int clear, int* site) {
@@ -1101,7 +1223,7 @@ bl_status bl_device_status(int clear, int* site) {
 bl_status bl_selftest_wait_timeout(unsigned long long limit_ns, int* waited_ok, cudaStream_t stream) {
   if (!waited_ok) return BL_ERR_INVALID_ARG;
   if (limit_ns > 10ull * kWaitLimitNs) return BL_ERR_INVALID_ARG;
-  bl::wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, waited_ok);
+  bl::bl_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, waited_ok);
   return last_cuda();
 }
 

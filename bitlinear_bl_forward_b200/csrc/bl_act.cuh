@@ -118,7 +118,7 @@ constexpr int kActCache = 16;         // 16-byte chunks kept in registers per la
 
 // X bf16 [M, K] -> Xq int8 [M, K], s[M] = Q / max(a, 1e-5), optional R[M] =
 // sum_k Xq[m, k] (used to undo the +1 offset of the stored weight codes).
-__global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restrict__ X, int M, int K, int Q,
+__global__ void __launch_bounds__(256) bl_act_quant_kernel(const uint16_t* __restrict__ X, int M, int K, int Q,
                                                         int8_t* __restrict__ Xq, float* __restrict__ s_out,
                                                         int* __restrict__ R_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,12 +156,12 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restri
 
 // The same quantisation with one CTA per token row, for few rows: the
 // absmax is a block reduction, so a row of K = 8192 costs four 16-byte loads
-// a thread instead of 32 a lane.  Bit-identical to act_quant_kernel (the max
+// a thread instead of 32 a lane.  Bit-identical to bl_act_quant_kernel (the max
 // and the integer sum do not depend on the order).
 constexpr int kActRowThreads = 256;
 constexpr int kActRowCache = 8;   // 16-byte chunks kept in registers per thread (K <= 16384)
 
-__global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uint16_t* __restrict__ X, int K, int Q,
+__global__ void __launch_bounds__(kActRowThreads) bl_act_quant_row_kernel(const uint16_t* __restrict__ X, int K, int Q,
                                                                        int8_t* __restrict__ Xq,
                                                                        float* __restrict__ s_out,
                                                                        int* __restrict__ R_out,
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_row_kernel(const uin
 // 1.58-Bit LLMs", section "1. The BitLinear Operator", per-tensor form):
 // non-negative floats order as their bit patterns, so a max of the bits is the
 // max of the values.  *amax_out must be zero before the launch.
-__global__ void __launch_bounds__(256) act_absmax_kernel(const uint16_t* __restrict__ X, int64_t nchunks,
+__global__ void __launch_bounds__(256) bl_act_absmax_kernel(const uint16_t* __restrict__ X, int64_t nchunks,
                                                         uint32_t* __restrict__ amax_out) {
   const uint4* x4 = reinterpret_cast<const uint4*>(X);
   float a = 0.f;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(256) act_absmax_kernel(const uint16_t* __restr
 // pass 1 takes the absmax of h over the row, pass 2 recomputes h (the row is
 // in L1/L2 by then) and writes the codes.  G, U: bf16 [M, K] (U only when
 // gated).
-__global__ void __launch_bounds__(kActRowThreads) act_quant_relu2_kernel(const uint16_t* __restrict__ G,
+__global__ void __launch_bounds__(kActRowThreads) bl_act_quant_relu2_kernel(const uint16_t* __restrict__ G,
                                                                          const uint16_t* __restrict__ U, int gated,
                                                                          int K, int Q, int8_t* __restrict__ Xq,
                                                                          float* __restrict__ s_out,
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kActRowThreads) act_quant_relu2_kernel(const u
 }
 
 // R[m] = sum_k Xq[m, k] for already-quantised int8 activations.
-__global__ void __launch_bounds__(256) act_rowsum_kernel(const int8_t* __restrict__ Xq, int M, int K,
+__global__ void __launch_bounds__(256) bl_act_rowsum_kernel(const int8_t* __restrict__ Xq, int M, int K,
                                                          int* __restrict__ R_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x * kActRowsPerBlock + warp;

@@ -33,7 +33,7 @@
 #include <cuda_bf16.h>
 
 #include "bl_common.cuh"
-#include "bl_gemm_tc.cuh"
+#include "bl_tc_common.cuh"
 #include "bl_gemv.cuh"
 
 namespace bl {
@@ -44,11 +44,8 @@ constexpr int kQExpGroups = 1;   // measured: a second group does not help
 constexpr int kQFirstEpi = 2 + 4 * kQExpGroups;
 constexpr int kQEpiWarps = 8;   // two per TMEM lane quadrant, each takes half of the tile's tokens
 constexpr int kQThreads = 32 * (kQFirstEpi + kQEpiWarps);
-#ifndef BL_Q_BK
-#define BL_Q_BK 512
-#endif
-constexpr int kQBK = BL_Q_BK;                   // K per pipeline stage: kQBK / 32 MMAs per hand-off
-constexpr int kQASlots = kQBK == 512 ? 2 : 4;   // TMEM: 2 x 128 accumulator + A slots = 512 columns
+constexpr int kQBK = 512;                       // K per pipeline stage: kQBK / 32 MMAs per hand-off
+constexpr int kQASlots = 2;                     // TMEM: 2 x 128 accumulator + 2 A slots = 512 columns
 constexpr int kQASlotCols = kQBK / 4;           // int8 codes, 4 per 32-bit column
 constexpr int kQBN = 128;                       // tokens per pair tile (MMA N)
 constexpr int kQHalf = kQBN / 2;                // token rows staged per CTA
@@ -56,9 +53,9 @@ constexpr int kQRows = 256;                     // weight rows per pair tile (MM
 constexpr int kQXBoxBytes = kQHalf * 128;       // one 128-byte-wide activation box (SW128)
 constexpr int kQXStageBytes = kQHalf * kQBK;    // 16 KB: kQBK / 128 boxes
 constexpr int kQWRowBytes = kQBK / 4;           // packed bytes of a weight row per stage
-constexpr int kQWStageBytes = kTcRows * kQWRowBytes;   // 64-byte rows (SW64) or 128-byte rows (SW128)
+constexpr int kQWStageBytes = kTcRows * kQWRowBytes;   // 128-byte rows (SW128)
 constexpr int kQStageBytes = kQXStageBytes + kQWStageBytes;
-constexpr int kQStages = kQBK == 512 ? 3 : 7;   // 144 KB / 168 KB
+constexpr int kQStages = 3;                    // 144 KB
 constexpr int kQEpiCols = kQBN / 2;             // tokens per epilogue warp
 constexpr int kQStageOutBytes = kQEpiCols * 32 * 2;  // bf16 [64 tokens][32 rows] per epilogue warp
 constexpr int kQAccCols = kQBN;
@@ -74,7 +71,7 @@ constexpr int kQEpiOffset = kQBarOffset + kQNumBars * 8 + 16;
 constexpr int kQSmemBytes = kQEpiOffset + 2 * kQBN * 8 + 1024;
 
 __global__ void __launch_bounds__(kQThreads, 1)
-    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+    bl_mma_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const int* __restrict__ Rg,
                         const float* __restrict__ sg, const float* __restrict__ gamma_p, void* __restrict__ Y,
                         int out_mode, int tma_store, const float* __restrict__ bias, unsigned long long limit_ns) {
@@ -83,7 +80,6 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem;
   uint8_t* sW = smem + S * kQXStageBytes;
-  static_assert(kQBK == 256 || kQBK == 512, "stage layout below assumes K = 256 or 512 per stage");
   static_assert(2 * kQAccCols + kQASlots * kQASlotCols <= kQTmemCols, "tensor memory budget");
   uint8_t* sOut = smem + kQOutOffset;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQBarOffset);
@@ -199,8 +195,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    // swizzle of the packed box: 16-byte chunk c of row r sits at chunk c ^ wsw
-    const uint32_t wsw = kQWRowBytes == 64 ? static_cast<uint32_t>((r >> 1) & 3) : static_cast<uint32_t>(r & 7);
+    // 128-byte swizzle of the packed box: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+    static_assert(kQWRowBytes == 128, "the packed box is 128-byte rows");
+    const uint32_t wsw = static_cast<uint32_t>(r & 7);
     uint32_t g = 0;
     bool stop = false;
     for (int tile = pair; tile < ntiles && !stop; tile += npairs) {

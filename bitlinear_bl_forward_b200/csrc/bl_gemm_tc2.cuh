@@ -1,6 +1,6 @@
 // Persistent tensor-core GEMM for few tokens (M <= 64).
 //
-// Same arithmetic as tc_gemm_kernel ("BitNet b1.58: The 1-Bit Ternary LLM
+// The BitLinear matmul and rescale ("BitNet b1.58: The 1-Bit Ternary LLM
 // Architecture Guide", section "The Mathematical Formulation of BitLinear",
 // eq. (3)): D[n, m] = sum_k u[n, k] * q[m, k] on tcgen05.mma kind::i8 with the
 // expanded weight codes u = c + 1 as the A operand in tensor memory and the
@@ -35,7 +35,7 @@
 #include <cuda_bf16.h>
 
 #include "bl_common.cuh"
-#include "bl_gemm_tc.cuh"
+#include "bl_tc_common.cuh"
 #include "bl_gemv.cuh"
 
 namespace bl {
@@ -76,7 +76,7 @@ struct P2Cfg {
 
 template <int BN, int EXPG>
 __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
-    tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int M,
+    bl_mma_persistent_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int M,
                               int N, int K, const int* __restrict__ Rg, const float* __restrict__ sg,
                               const float* __restrict__ gamma_p, void* __restrict__ Y, int out_mode,
                               const float* __restrict__ bias, unsigned long long limit_ns) {

@@ -75,7 +75,7 @@ __device__ __forceinline__ int block_reduce_sum_i(int v, int* scratch) {
 
 template <int MT, int RT>
 __global__ void __launch_bounds__(kGemvThreads, 2)
-    gemv_kernel(const void* __restrict__ X, int x_is_i8, int M, int K, int N, const uint4* __restrict__ Wp,
+    bl_decode_long_kernel(const void* __restrict__ X, int x_is_i8, int M, int K, int N, const uint4* __restrict__ Wp,
                 const float* __restrict__ gamma_p, int Q, void* __restrict__ Y, int out_mode) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float s_scale[MT];
@@ -335,7 +335,7 @@ __device__ __forceinline__ void gemv1_finish(const int (&part)[RT][MT], int tile
 
 template <int MT, int CPL, int RT, int D, int THREADS, int MINB>
 __global__ void __launch_bounds__(THREADS, MINB)
-    gemv1_kernel(const void* __restrict__ X, int x_is_i8, int K, int N, const uint4* __restrict__ Wp,
+    bl_decode_rows_kernel(const void* __restrict__ X, int x_is_i8, int K, int N, const uint4* __restrict__ Wp,
                  const float* __restrict__ gamma_p, int Q, void* __restrict__ Y, int out_mode, int tiles_per_cta) {
   constexpr int WARPS = THREADS / 32;
   __shared__ __align__(16) uint8_t s_act[MT][8192];
@@ -480,25 +480,10 @@ __global__ void __launch_bounds__(THREADS, MINB)
 
 
 // ---------------------------------------------------------------------------
-// Decode, large layers: the same arithmetic as gemv1_kernel, but the packed
-// weights reach the SM through a shared-memory ring filled by the TMA unit.
-//
-// Each CTA (one per SM) owns a contiguous row range, i.e. one contiguous byte
-// range.  Warp 16 is the producer: one thread cuts the range into stages of
-// whole rows (<= 32 KB) and issues one cp.async.bulk per stage onto the
-// stage's mbarrier, so up to kG2Stages x 32 KB are in flight per SM without
-// spending registers.  Warps 0-15 quantise the token (named barriers among
-// themselves, so the producer never waits on them), keep their lanes'
-// activation chunks in registers, and then consume stages: a warp takes rows
-// w, w+16, ... of the stage, its lanes read their 16-byte chunks of the row
-// from shared memory (consecutive lanes, consecutive addresses), accumulate
-// with the masked dp4a scheme, reduce with redux and store.  Each consumer
-// warp releases a stage with one arrive on its "empty" barrier.  All waits are
-// bounded; on a timeout the kernel records BL_ERR_TIMEOUT and unwinds, and
-// the producer waits for the copies it issued before the CTA exits.
+// Launch table of the one-token decode kernel (bl_decode.cuh): one launch can
+// serve several independent one-token problems; CTAs [cta_begin, cta_begin +
+// ctas) of the grid work on problem i.
 // ---------------------------------------------------------------------------
-// One launch can serve several independent one-token problems (grouped
-// decode): CTAs [cta_begin, next cta_begin) of the grid work on problem i.
 struct G2Problem {
   const void* X;
   const void* U;      // squared-ReLU gated mode: the up projection's output;
@@ -508,11 +493,15 @@ struct G2Problem {
   void* Y;
   int K;
   int N;
-  int rows_per_cta;   // TMA-staged GEMV: CTA c takes rows [c*rows_per_cta, ...)
+  int rows_per_cta;   // decode kernel: q = N / ctas; CTA c takes q + (c < rem) rows
   int cta_begin;      // first CTA of this problem in the launch
-  int ctas;           // decode kernel: CTA c takes rows [c*N/ctas, (c+1)*N/ctas)
+  int ctas;           // CTAs of this problem
+  int rows_rem;       // rem = N % ctas
   const float* bias;  // optional fp32 [N] added after the rescale
   float eps;          // RMSNorm mode: added to the mean of squares
+  int chunk_rows;     // decode kernel: rows per bulk copy (a multiple of the row group)
+  int slots;          // decode kernel: chunks the ring holds at once
+  int ksplit;         // decode kernel: warps that split one row (resident 2-bit rows)
 };
 constexpr int kG2MaxProblems = 8;
 struct G2Table {
@@ -520,217 +509,4 @@ struct G2Table {
   int count;
 };
 
-constexpr int kG2ConsumerWarps = 16;
-constexpr int kG2Threads = (kG2ConsumerWarps + 1) * 32;
-constexpr int kG2Stages = 6;
-constexpr int kG2StageBytes = 32 * 1024;
-constexpr int kG2SmemBytes = kG2Stages * kG2StageBytes + 2048;
-
-template <int MT, int CPL>
-__global__ void __launch_bounds__(kG2Threads, 1)
-    gemv2_kernel(const __grid_constant__ G2Table tab, int in_mode, int Q, int out_mode, unsigned long long limit_ns) {
-  int pi = 0;
-  while (pi + 1 < tab.count && static_cast<int>(blockIdx.x) >= tab.p[pi + 1].cta_begin) ++pi;
-  const void* __restrict__ X = tab.p[pi].X;
-  const void* __restrict__ Up = tab.p[pi].U;
-  const uint8_t* __restrict__ Wp = tab.p[pi].Wp;
-  const float* __restrict__ gamma_p = tab.p[pi].gamma;
-  void* __restrict__ Y = tab.p[pi].Y;
-  const int K = tab.p[pi].K, N = tab.p[pi].N, rows_per_cta = tab.p[pi].rows_per_cta;
-  const int cta = static_cast<int>(blockIdx.x) - tab.p[pi].cta_begin;
-  extern __shared__ __align__(128) uint8_t g2_smem[];
-  __shared__ __align__(16) uint8_t s_act[MT][8192];
-  __shared__ __align__(16) uint32_t s_red_f[MT][kG2ConsumerWarps];
-  __shared__ int s_red_i[MT][kG2ConsumerWarps];
-  __shared__ __align__(8) uint64_t full[kG2Stages], empty[kG2Stages];
-  __shared__ int abort_flag;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KV = K >> 6;
-  const size_t row_bytes = static_cast<size_t>(K) >> 2;
-  const int r0 = cta * rows_per_cta;
-  const int r1 = min(N, r0 + rows_per_cta);
-  const int stage_rows = kG2StageBytes / static_cast<int>(row_bytes);
-  const int nst = (r1 > r0) ? (r1 - r0 + stage_rows - 1) / stage_rows : 0;
-  volatile int* abort_v = &abort_flag;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kG2Stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kG2ConsumerWarps);
-    }
-    abort_flag = 0;
-    fence_mbar_init();
-    if (r1 > r0) {
-      const char* base = reinterpret_cast<const char*>(Wp) + static_cast<size_t>(r0) * row_bytes;
-      const size_t bytes = static_cast<size_t>(r1 - r0) * row_bytes;
-      for (size_t off = 0; off < bytes; off += kPrefetchChunk)
-        bulk_prefetch_l2(base + off, static_cast<uint32_t>(min(static_cast<size_t>(kPrefetchChunk), bytes - off)));
-    }
-  }
-  __syncthreads();
-  pdl_launch_dependents();
-  pdl_wait();
-
-  if (warp == kG2ConsumerWarps) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      int issued = 0;
-      for (int st = 0; st < nst; ++st) {
-        const int s = st % kG2Stages;
-        if (st >= kG2Stages && !mbar_wait(&empty[s], ((st / kG2Stages) & 1) ^ 1u, abort_v, limit_ns, 11)) break;
-        const int rows = min(stage_rows, r1 - (r0 + st * stage_rows));
-        const uint32_t bytes = static_cast<uint32_t>(rows * row_bytes);
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_load(g2_smem + s * kG2StageBytes,
-                  Wp + (static_cast<size_t>(r0) + static_cast<size_t>(st) * stage_rows) * row_bytes, bytes, &full[s]);
-        issued = st + 1;
-      }
-      for (int s = 0; s < kG2Stages && s < issued; ++s) {
-        const int last = s + kG2Stages * ((issued - 1 - s) / kG2Stages);
-        mbar_wait(&full[s], (last / kG2Stages) & 1, nullptr, limit_ns, 12);
-      }
-    }
-    return;
-  }
-
-  // ---------------- consumers: token quantisation ----------------
-  constexpr int CT = kG2ConsumerWarps * 32;
-  constexpr int U = (8192 / 8 + CT - 1) / CT;
-  const bool x_is_i8 = in_mode == kInI8;
-  const bool relu2 = in_mode == kInRelu2 || in_mode == kInRelu2Gated;
-  const bool gated = in_mode == kInRelu2Gated;
-  const int nch = x_is_i8 ? (K >> 4) : (K >> 3);
-  uint4 xv[MT][U], uv[MT][U];
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = threadIdx.x + CT * u;
-      const size_t o = static_cast<size_t>(m) * nch + c;
-      xv[m][u] = (c < nch) ? __ldg(static_cast<const uint4*>(X) + o) : make_uint4(0, 0, 0, 0);
-      uv[m][u] = (gated && c < nch) ? __ldg(static_cast<const uint4*>(Up) + o) : make_uint4(0, 0, 0, 0);
-    }
-  const float gamma = (out_mode == kOutI32) ? 1.f : __ldg(gamma_p);
-  int rsum[MT];
-  float sc[MT];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    rsum[m] = 0;
-    sc[m] = 1.f;
-  }
-  if (!x_is_i8) {
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      float amax = 0.f;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (relu2) {
-          float h[8];
-          relu2_8(xv[m][u], uv[m][u], gated, h);
-          amax = fmaxf(amax, absmax8_f32(h));
-        } else {
-          amax = fmaxf(amax, absmax8_bf16(xv[m][u]));
-        }
-      }
-      const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
-      if (lane == 0) s_red_f[m][warp] = wmax;
-    }
-    named_bar_sync(1, CT);
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      uint32_t bmax = 0;
-#pragma unroll
-      for (int w = 0; w < kG2ConsumerWarps; w += 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(&s_red_f[m][w]);
-        bmax = max(bmax, max(max(v.x, v.y), max(v.z, v.w)));
-      }
-      sc[m] = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = threadIdx.x + CT * u;
-        if (c < nch) {
-          uint2 qv;
-          if (relu2) {
-            float h[8];
-            relu2_8(xv[m][u], uv[m][u], gated, h);
-            qv = quant8_f32(h, sc[m], Q, rsum[m]);
-          } else {
-            qv = quant8_bf16(xv[m][u], sc[m], Q, rsum[m]);
-          }
-          *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = qv;
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = threadIdx.x + CT * u;
-        if (c < nch) {
-          const uint4 v = xv[m][u];
-          rsum[m] = __dp4a(static_cast<int>(v.x), 0x01010101, rsum[m]);
-          rsum[m] = __dp4a(static_cast<int>(v.y), 0x01010101, rsum[m]);
-          rsum[m] = __dp4a(static_cast<int>(v.z), 0x01010101, rsum[m]);
-          rsum[m] = __dp4a(static_cast<int>(v.w), 0x01010101, rsum[m]);
-          *reinterpret_cast<uint4*>(&s_act[m][act_swz(16u * c)]) = v;
-        }
-      }
-  }
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    const int ws = __reduce_add_sync(0xffffffffu, rsum[m]);
-    if (lane == 0) s_red_i[m][warp] = ws;
-  }
-  named_bar_sync(1, CT);
-  int R[MT];
-  float f[MT];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    R[m] = 0;
-#pragma unroll
-    for (int w = 0; w < kG2ConsumerWarps; ++w) R[m] += s_red_i[m][w];
-    f[m] = (x_is_i8 || out_mode == kOutI32) ? 0.f : __fdiv_rn(gamma, sc[m]);
-  }
-  uint32_t act[MT][CPL][16];
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const int c = lane + 32 * i;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (c < KV) v = *reinterpret_cast<const uint4*>(&s_act[m][act_swz(64u * c + 16u * g)]);
-        act[m][i][4 * g + 0] = v.x;
-        act[m][i][4 * g + 1] = v.y;
-        act[m][i][4 * g + 2] = v.z;
-        act[m][i][4 * g + 3] = v.w;
-      }
-    }
-
-  // ---------------- consumers: stream the stages ----------------
-  for (int st = 0; st < nst; ++st) {
-    const int s = st % kG2Stages;
-    const bool ok = mbar_wait(&full[s], (st / kG2Stages) & 1, abort_v, limit_ns, 13);
-    if (!__all_sync(0xffffffffu, ok)) break;
-    const int row0 = r0 + st * stage_rows;
-    const int rows = min(stage_rows, r1 - row0);
-    const uint8_t* sbase = g2_smem + s * kG2StageBytes;
-    for (int rr = warp; rr < rows; rr += kG2ConsumerWarps) {
-      uint4 w[1][CPL];
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        const int c = lane + 32 * i;
-        w[0][i] = (c < KV) ? *reinterpret_cast<const uint4*>(sbase + rr * row_bytes + 16 * c) : make_uint4(0, 0, 0, 0);
-      }
-      int part[1][MT];
-      gemv1_accumulate<MT, CPL, 1>(w, act, KV, lane, part);
-      gemv1_finish<MT, 1>(part, row0 + rr, N, lane, R, f, Y, out_mode, tab.p[pi].bias);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-  }
-}
 }  // namespace bl

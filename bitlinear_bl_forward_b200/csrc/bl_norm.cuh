@@ -217,10 +217,10 @@ __device__ __forceinline__ uint4 rms_apply8(uint4 x, uint4 w, bool has_w, float 
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// RMSNorm, then exactly act_quant_row_kernel's quantisation of the normalised
+// RMSNorm, then exactly bl_act_quant_row_kernel's quantisation of the normalised
 // bf16 row: one CTA per token.  Wn: optional bf16 [K]; ms_out: optional fp32
 // [M] mean of squares.
-__global__ void __launch_bounds__(kActRowThreads) act_quant_rmsnorm_kernel(
+__global__ void __launch_bounds__(kActRowThreads) bl_act_quant_rmsnorm_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wn, float eps, int K, int Q,
     int8_t* __restrict__ Xq, float* __restrict__ s_out, int* __restrict__ R_out, float* __restrict__ ms_out) {
   constexpr int W = kActRowThreads / 32;

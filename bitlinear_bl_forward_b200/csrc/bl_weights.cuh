@@ -38,7 +38,7 @@ constexpr int kAbsumTotals = 16;    // global accumulators: limbs 0..9, [15] = n
 // exact integer additions (bounds: a thread sees < 2^23 elements, a block
 // < 2^31, so no accumulator can overflow), hence no dependence on the order.
 // total must be zero before the launch.
-__global__ void __launch_bounds__(kAbsumThreads) weight_absum_bins_kernel(const float* __restrict__ W, int64_t n,
+__global__ void __launch_bounds__(kAbsumThreads) bl_weight_absum_kernel(const float* __restrict__ W, int64_t n,
                                                                            unsigned long long* __restrict__ total) {
   __shared__ unsigned long long acc[kAbsumChunks + 1][kAbsumThreads];
   __shared__ unsigned long long red[kAbsumChunks + 1];
@@ -157,7 +157,7 @@ __device__ float round_ratio_to_f32(const uint32_t* S, int nlimbs, uint64_t D) {
 }
 
 // Pass 2: one thread.  Turns the limb totals into gamma.
-__global__ void __launch_bounds__(32) weight_gamma_kernel(const unsigned long long* __restrict__ total, uint64_t count,
+__global__ void __launch_bounds__(32) bl_weight_gamma_kernel(const unsigned long long* __restrict__ total, uint64_t count,
                                                           float* __restrict__ gamma) {
   if (threadIdx.x != 0) return;
   if (total[kAbsumTotals - 1] != 0ull) {   // a non-finite weight
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(32) weight_gamma_kernel(const unsigned long lo
 }
 
 // Pass 3: ternary codes and packing, one thread per 32-bit output word.
-__global__ void __launch_bounds__(256) weight_pack_kernel(const float* __restrict__ W, int64_t nwords,
+__global__ void __launch_bounds__(256) bl_weight_pack_kernel(const float* __restrict__ W, int64_t nwords,
                                                           const float* __restrict__ gamma_p,
                                                           uint32_t* __restrict__ Wp) {
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(const float* __restric
 }
 
 // Packed words -> int8 codes, one thread per word (16 codes, one uint4 out).
-__global__ void __launch_bounds__(256) weight_unpack_kernel(const uint32_t* __restrict__ Wp, int64_t nwords,
+__global__ void __launch_bounds__(256) bl_weight_unpack_kernel(const uint32_t* __restrict__ Wp, int64_t nwords,
                                                             int8_t* __restrict__ codes) {
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= nwords) return;
@@ -217,6 +217,71 @@ __global__ void __launch_bounds__(256) weight_unpack_kernel(const uint32_t* __re
     out[j] = ((u | 0x80808080u) - 0x01010101u) ^ 0x80808080u;
   }
   reinterpret_cast<uint4*>(codes)[g] = make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Base-3 storage: five ternary weights per byte (3^5 = 243 states fit in a
+// byte: "BitNet b1.58: The 1-Bit Ternary LLM Architecture Guide", section
+// "Why 1.58 Bits? The Power of Zero", log2(3) ~ 1.58 bits a weight).  Layout
+// (this library's): a row is base3 words padded to a multiple of four (16
+// bytes); byte b of little-endian word g holds the digits d_L = code + 1 of
+// weights k = 20g + 4L + b (L = 0..4, digits past the row end are 1) as
+// ceil(256 * v / 243), v = sum_L d_L 3^(4-L).  Level L of the four bytes of a
+// word is then four consecutive weights, and a decoder gets the levels in
+// order by tripling each byte (digit = (3x) >> 8, next x = 3x mod 256).
+// ---------------------------------------------------------------------------
+
+__host__ __device__ constexpr int base3_row_words(int K) { return ((K + 19) / 20 + 3) / 4 * 4; }
+
+// One thread per output word: 20 weights -> four bytes.
+__global__ void __launch_bounds__(256) bl_weight_pack3_kernel(const float* __restrict__ W, int N, int K,
+                                                           const float* __restrict__ gamma_p,
+                                                           uint32_t* __restrict__ Wp3) {
+  const int rw = base3_row_words(K);
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(N) * rw) return;
+  const int n = static_cast<int>(idx / rw), g = static_cast<int>(idx % rw);
+  const float gamma = *gamma_p;
+  const float* row = W + static_cast<size_t>(n) * K;
+  uint32_t word = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    int v = 0;
+#pragma unroll
+    for (int L = 0; L < 5; ++L) {
+      const int k = 20 * g + 4 * L + b;
+      int d = 1;   // padding: code 0
+      if (k < K) {
+        int c = __float2int_rn(__fdiv_rn(__ldg(row + k), gamma));
+        c = c < -1 ? -1 : (c > 1 ? 1 : c);
+        d = c + 1;
+      }
+      v = 3 * v + d;
+    }
+    word |= static_cast<uint32_t>((256 * v + 242) / 243) << (8 * b);
+  }
+  Wp3[idx] = word;
+}
+
+// Base-3 words -> int8 codes [N, K], one thread per word (up to 20 codes).
+__global__ void __launch_bounds__(256) bl_weight_unpack3_kernel(const uint32_t* __restrict__ Wp3, int N, int K,
+                                                             int8_t* __restrict__ codes) {
+  const int rw = base3_row_words(K);
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(N) * rw) return;
+  const int n = static_cast<int>(idx / rw), g = static_cast<int>(idx % rw);
+  const uint32_t w = Wp3[idx];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    uint32_t x = (w >> (8 * b)) & 0xffu;
+#pragma unroll
+    for (int L = 0; L < 5; ++L) {
+      const uint32_t t = 3u * x;
+      const int k = 20 * g + 4 * L + b;
+      if (k < K) codes[static_cast<size_t>(n) * K + k] = static_cast<int8_t>(static_cast<int>(t >> 8) - 1);
+      x = t & 0xffu;
+    }
+  }
 }
 
 }  // namespace bl

@@ -46,7 +46,7 @@ class Workload:
     outlier_mult: float = 1.0
     bits: int = 8
     note: str = ""
-    groups: tuple = ()          # layers a step runs in one grouped call, e.g. ((0, 1), (2,))
+    groups: tuple = ()          # layers a step runs in one grouped call, e.g. ((0, 1, 2),)
 
     def outliers_for(self, K: int) -> int:
         if isinstance(self.n_outliers, str) and self.n_outliers.endswith("%"):
@@ -62,7 +62,7 @@ WORKLOADS = {
     # up and gate project the same hidden state; down reads its own input
     "decode_2b": Workload("decode_2b", 1,
                           (Layer("up", 2560, 6912), Layer("gate", 2560, 6912, x_layer=0), Layer("down", 6912, 2560)),
-                          0.02, "outliers", "1%", 10.0, 8, "2B-class decode GEMV, batch 1", ((0, 1), (2,))),
+                          0.02, "outliers", "1%", 10.0, 8, "2B-class decode GEMV, batch 1", ((0, 1, 2),)),
     "prefill_2b": Workload("prefill_2b", 4096,
                            (Layer("up", 2560, 6912), Layer("down", 6912, 2560)),
                            0.02, "outliers", "1%", 10.0, 8, "2B-class prefill GEMM, 4096 tokens"),

@@ -2,8 +2,11 @@
  * libbitlinear -- BitNet b1.58 BitLinear forward on NVIDIA B200 (sm_100a).
  *
  * C ABI.  Every pointer argument that names a tensor is a DEVICE pointer that
- * the caller allocated and owns; the library allocates no device memory of its
- * own except one 4-byte status word (see bl_device_status).  Every compute
+ * the caller allocated and owns.  The library allocates no device memory at
+ * run time; its only device memory of its own is static: one 4-byte status
+ * word (see bl_device_status) and the 16 MiB + 64 KiB scratch array of
+ * bl_forward_noalloc, both present on every GPU that loads the library until
+ * the process exits.  Every compute
  * call is asynchronous on the given CUDA stream (0 = legacy default stream)
  * and returns a bl_status:
  *   - arguments are validated on the host before anything is launched; a
@@ -137,8 +140,8 @@ BL_API size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bi
  * bytes, 16-byte aligned (may be null when that is 0).
  * Ordering: the kernels are launched with programmatic dependent launch.  They
  * read X (and the workspace) only after the preceding kernel on the stream has
- * completed, but a one-token launch may fetch Wp before that, while the
- * preceding kernel still runs: Wp must not be written by the kernel launched
+ * completed, but a one-token launch may fetch Wp and gamma before that, while
+ * the preceding kernel still runs: neither may be written by the kernel launched
  * immediately before on the same stream if that kernel triggers its dependents
  * early (this library's forward kernels do; bl_quantize_weights and ordinary
  * kernels do not, and a dependent launch after them starts only once they
@@ -181,14 +184,15 @@ BL_API bl_status bl_forward_noalloc(const uint16_t* X, int64_t M, int64_t K, int
 
 /*
  * Grouped forward: up to 8 independent BitLinear problems in one call, e.g.
- * the up and gate projections of a feed-forward block (same X, two weight
- * tensors) or several requests' layers.  Each problem is exactly one
- * bl_forward (same formulas, same rounding, bit-identical results).  When
- * every problem has M == 1 and K <= 8192, the problems with the same
- * ceil(K / 512) share one decode kernel launch (its CTAs are shared out in
- * proportion to each problem's weight bytes), so the fixed cost of a launch is
- * paid once per such set; otherwise the problems run one after another on the
- * stream.  The ordering rule of bl_forward applies to every Wp.
+ * the up, gate and down projections of a feed-forward block at one decode
+ * step, or several requests' layers.  Each problem is exactly one bl_forward
+ * (same formulas, same rounding, bit-identical results).  When every problem
+ * has M == 1 and K <= 8192, all of them share one decode kernel launch,
+ * whatever their K (the launch's CTAs are shared out by an estimate of each
+ * problem's work), so the fixed cost of a launch is paid once per call;
+ * otherwise the problems run one after another on the stream.  The problems
+ * are independent: no problem's X may be another problem's Y.  The ordering
+ * rule of bl_forward applies to every Wp and gamma.
  * workspace: >= bl_forward_grouped_workspace_bytes(count, problems, bits)
  * (the largest per-problem bl_forward workspace; 0 for an all-decode group).
  * count > 8 returns BL_ERR_UNSUPPORTED; problems with M == 0 are skipped.
@@ -302,6 +306,58 @@ BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
  */
 BL_API bl_status bl_matmul_i32(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const uint8_t* Wp, int32_t* acc,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Base-3 weight storage: five ternary weights per byte, 1.6 bits a weight
+ * ("BitNet b1.58: The 1-Bit Ternary LLM Architecture Guide", section "Why 1.58
+ * Bits? The Power of Zero": a ternary weight carries log2(3) ~ 1.58 bits, and
+ * 3^5 = 243 states fit in one byte), i.e. 20% fewer weight bytes than the
+ * 2-bit storage for the same codes.  Layout (this library's): a row of K
+ * weights is 4 * ceil(ceil(K / 20) / 4) bytes (16-byte multiple) of
+ * little-endian 32-bit words; byte b of word g holds the digits
+ * d_L = code + 1 of the weights k = 20g + 4L + b (L = 0..4; digits past the
+ * end of the row are 1) as ceil(256 * v / 243) with v = sum_L d_L * 3^(4-L).
+ * The codes and gamma are exactly those of bl_quantize_weights.
+ * ------------------------------------------------------------------------- */
+
+/* N * 4 * ceil(ceil(K / 20) / 4) (0 for an invalid shape). */
+BL_API size_t bl_packed_weight_bytes_b3(int64_t N, int64_t K);
+
+/* [b1.58] eq. (1) as bl_quantize_weights, stored in base 3.  Wp3:
+ * bl_packed_weight_bytes_b3(N, K) bytes, 16-byte aligned; workspace as for
+ * bl_quantize_weights (bl_quantize_weights_workspace_bytes). */
+BL_API bl_status bl_quantize_weights_b3(const float* W, int64_t N, int64_t K, uint8_t* Wp3, float* gamma,
+                                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Base-3 weights -> int8 codes [N, K].  For tests and inspection. */
+BL_API bl_status bl_unpack_weights_b3(const uint8_t* Wp3, int64_t N, int64_t K, int8_t* codes, cudaStream_t stream);
+
+/* bl_forward on base-3 weights, for one token (M == 1, K <= 8192; other
+ * shapes return BL_ERR_UNSUPPORTED, M == 0 is a no-op): the same formulas and
+ * roundings, so Y is bit-identical to bl_forward on the 2-bit storage of the
+ * same codes.  The decode kernel decodes five weights a byte.  No workspace.
+ * The ordering rule of bl_forward applies to Wp3 and gamma. */
+BL_API bl_status bl_forward_b3(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* Wp3,
+                               const float* gamma, int bits, uint16_t* Y, cudaStream_t stream);
+
+/* [b1.58] eq. (3) without the rescale on base-3 weights and int8 codes Xq
+ * (M == 1): exact int32 acc [N].  For tests. */
+BL_API bl_status bl_matmul_i32_b3(const int8_t* Xq, int64_t M, int64_t K, int64_t N, const uint8_t* Wp3,
+                                  int32_t* acc, cudaStream_t stream);
+
+/*
+ * Throughput probe of the tensor-core instruction the prefill GEMMs run on
+ * (tcgen05.mma kind::i8, A in tensor memory, B in shared memory).  No
+ * counterpart on the pages: it measures the peak that the GEMMs' tensor-pipe
+ * fraction is quoted against.  grid CTAs (one per SM when grid <= the SM
+ * count) each issue n_mma MMAs of M = 128, N = n_cols, K = 32 into one
+ * accumulator and write, to out[2*i] and out[2*i+1] (device, 2*grid values),
+ * the SM clock cycles and nanoseconds the issue-to-completion took (0 and 0 if
+ * the bounded wait gave up).  Rate per SM = 128 * n_cols * 32 * n_mma / cycles
+ * multiply-accumulates per clock.  n_mma in [1, 2^22], n_cols a multiple of
+ * 16 in [16, 256], grid in [1, 4096] (else BL_ERR_SHAPE).
+ */
+BL_API bl_status bl_probe_mma_i8(int n_mma, int n_cols, unsigned long long* out, int grid, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Device status.

@@ -204,3 +204,30 @@ def test_rmsnorm_validation(L):
     assert L.bl_quant_act_rmsnorm(A, U, 1e-5, 4, 64, 8, A, A, None, None) == ALIGN
     assert L.bl_quant_act_rmsnorm(A, None, 1e-5, 4, 64, 8, A, A, A + 2, None) == ALIGN       # mean_sq misaligned
     assert L.bl_quant_act_rmsnorm(None, None, 1e-5, 4, 64, 8, A, A, None, None) == INVALID
+
+
+def test_base3_host_checks(L):
+    # sizes: 4 * ceil(ceil(K / 20) / 4) bytes a row
+    assert L.bl_packed_weight_bytes_b3(1, 64) == 16
+    assert L.bl_packed_weight_bytes_b3(6912, 2560) == 6912 * 512
+    assert L.bl_packed_weight_bytes_b3(28672, 8192) == 28672 * 1648
+    assert L.bl_packed_weight_bytes_b3(4, 100) == 0                    # bad shape
+    # one token only; K <= 8192; rejected before any launch
+    assert L.bl_forward_b3(A, 2, 2560, 8, A, A, 8, A, None) == UNSUP
+    assert L.bl_forward_b3(A, 1, 16384, 8, A, A, 8, A, None) == UNSUP
+    assert L.bl_forward_b3(A, 1, 2560, 8, A, A, 5, A, None) == UNSUP     # bits
+    assert L.bl_forward_b3(A, 1, 100, 8, A, A, 8, A, None) == SHAPE
+    assert L.bl_forward_b3(None, 1, 2560, 8, A, A, 8, A, None) == INVALID
+    assert L.bl_forward_b3(U, 1, 2560, 8, A, A, 8, A, None) == ALIGN
+    assert L.bl_forward_b3(A, 0, 2560, 8, A, A, 8, A, None) == OK         # M == 0: no-op
+    assert L.bl_matmul_i32_b3(A, 2, 2560, 8, A, A, None) == UNSUP
+    assert L.bl_quantize_weights_b3(A, 8, 100, A, A, A, 1 << 12, None) == SHAPE
+    assert L.bl_quantize_weights_b3(A, 8, 64, A, A, A, 0, None) == WS
+    assert L.bl_unpack_weights_b3(U, 8, 64, A, None) == ALIGN
+
+
+def test_probe_host_checks(L):
+    assert L.bl_probe_mma_i8(0, 256, A, 148, None) == SHAPE
+    assert L.bl_probe_mma_i8(16, 8, A, 148, None) == SHAPE
+    assert L.bl_probe_mma_i8(16, 264, A, 148, None) == SHAPE
+    assert L.bl_probe_mma_i8(16, 256, None, 148, None) == INVALID

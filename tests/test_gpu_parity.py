@@ -264,26 +264,62 @@ def test_workload_a48():
 # grouped forward
 # ---------------------------------------------------------------------------
 
+def oracle_bf16(x_bits, codes, g, bits=8):
+    q, s = o.act_quant(x_bits, bits)
+    return o.round_to_bf16_bits(o.rescale(o.matmul_i32(q, codes), g, s)[1])
+
+
 def test_grouped_decode_matches_single_calls_and_oracle():
-    # up and gate of the 2B decode layer share X: one grouped launch
+    # the 2B decode step in one launch: up and gate share X (K = 2560), down
+    # reads its own input (K = 6912)
     w = WORKLOADS["decode_2b"]
-    X, _ = layer_inputs(w, 0)
-    Xd = x_to_dev(X)
     probs, refs = [], []
-    for i in (0, 1):
+    xs = {}
+    for i, L in enumerate(w.layers):
+        X, _ = layer_inputs(w, i)
+        key = L.x_layer if L.x_layer >= 0 else i
+        if key not in xs:
+            xs[key] = x_to_dev(X)
+        Xd = xs[key]
         W, g, c, p = oracle_weights(("decode_2b", i))
         Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
         N = W.shape[0]
         probs.append((Xd, Wp, gd, N))
-        refs.append(bl.bl_forward(Xd, Wp, gd, N))
-        q, s = o.act_quant(X, 8)
-        Y = o.round_to_bf16_bits(o.rescale(o.matmul_i32(q, c), g, s)[1])
-        refs[-1] = (refs[-1], Y)
+        refs.append((bl.bl_forward(Xd, Wp, gd, N), oracle_bf16(X, c, g)))
     outs = bl.bl_forward_grouped(probs)
     torch.cuda.synchronize()
     for Yg, (Ys, Yo) in zip(outs, refs):
         assert torch.equal(Yg, Ys)
         assert bf16_ulp_distance(bf16_dev_to_bits(Yg), Yo).max() <= BF16_ULP_TOL
+    # the same group twice more in a row, outputs reused (back-to-back launches)
+    for _ in range(2):
+        bl.bl_forward_grouped(probs, outs=outs)
+    torch.cuda.synchronize()
+    for Yg, (Ys, _) in zip(outs, refs):
+        assert torch.equal(Yg, Ys)
+
+
+def test_grouped_decode_mixed_k_one_launch():
+    # eight one-token problems of eight different K in one launch: one register
+    # width class, the rest on the shared-memory path; ragged row counts
+    # (including one row, fewer rows than CTAs, and rows that do not fill a
+    # row group), bits 8 and 4
+    shapes = [(64, 7), (512, 1), (1536, 999), (2560, 6912), (3072, 130), (4096, 2049), (6912, 2560), (8192, 3)]
+    for bits in (8, 4):
+        probs, cases = [], []
+        for j, (K, N) in enumerate(shapes):
+            X, W = random_case(1, K, N, seed=500 + j + 10 * bits)
+            g = o.absmean_scale(W)
+            c = o.ternary_codes(W, g)
+            Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+            probs.append((x_to_dev(X), Wp, gd, N))
+            cases.append((X, c, g))
+        singles = [bl.bl_forward(Xd, Wp, gd, N, bits) for (Xd, Wp, gd, N) in probs]
+        outs = bl.bl_forward_grouped(probs, bits)
+        torch.cuda.synchronize()
+        for (X, c, g), a, b in zip(cases, outs, singles):
+            assert torch.equal(a, b)
+            assert bf16_ulp_distance(bf16_dev_to_bits(a), oracle_bf16(X, c, g, bits)).max() <= BF16_ULP_TOL
 
 
 def test_grouped_mixed_shapes_fall_back_to_sequential():
@@ -299,7 +335,7 @@ def test_grouped_mixed_shapes_fall_back_to_sequential():
     torch.cuda.synchronize()
     for a, b in zip(outs, singles):
         assert torch.equal(a, b)
-    # all-decode group of different K (one launch per kernel variant)
+    # all-decode group of different K (one launch)
     probs2 = [probs[0], probs[2]]
     outs2 = bl.bl_forward_grouped(probs2)
     assert torch.equal(outs2[0], singles[0]) and torch.equal(outs2[1], singles[2])
