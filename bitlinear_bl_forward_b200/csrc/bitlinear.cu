@@ -280,7 +280,7 @@ inline int dec_rt(int mode, int fmt) {
 // mode: rounds of row groups over the CTA's teams of warps times the cost of
 // a group (issue slots of one warp: per word a lane keeps, two shared loads,
 // eight masks and eight dp4a at half rate for the two rows; the rows'
-// reductions and stores; a team barrier when rows are split), plus a penalty
+// reductions and stores; shared adds when rows are split), plus a penalty
 // for bytes that do not fit the ring (fetched after the dependency wait).
 // Big mode: the weight bytes a CTA streams.
 double dec_cta_cost(int64_t N, int64_t K, int ctas, int a, int fmt, int mode) {
@@ -296,7 +296,7 @@ double dec_cta_cost(int64_t N, int64_t K, int ctas, int a, int fmt, int mode) {
     teams = bl::kDecWarps;
   } else {
     const int S = dec_split(K, a);
-    group = a * 26.0 + 40.0 + (S > 1 ? 60.0 : 0.0);
+    group = a * 26.0 + 40.0 + (S > 1 ? 10.0 : 0.0);
     teams = bl::kDecWarps / S;
   }
   const int64_t rounds = (groups + teams - 1) / teams;
@@ -374,6 +374,8 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
     const int rt = dec_rt(mode, fmt);
     const int maxrows = static_cast<int>((p.N + c[i] - 1) / c[i]);
     int cr = (chunk_max / rb) / rt * rt, slots = 0;
+    if (mode == bl::kModeResident && fmt == bl::kFmt2Bit && dec_split(p.K, a) > 1)
+      cr = std::min(cr, bl::kDecSplitRows / rt * rt);   // split rows: the chunk's totals in shared memory
     if (mode == bl::kModeBig) {
       // one group per consumer warp per chunk
       cr = std::min(cr, bl::kDecWarps * rt);

@@ -83,8 +83,10 @@ enum DecMode : int { kModeResident = 0, kModeBig = 1 };
 constexpr int kDecRegRows = 2;     // 2-bit rows, token codes in registers
 constexpr int kDecB3Rows = 4;      // base-3 rows, resident mode
 constexpr int kDecBigRows = 2;     // big mode (both formats)
-// Largest team of warps that splits one long row (resident 2-bit rows).
+// Largest team of warps that splits one long row (resident 2-bit rows), and
+// the most rows a chunk of split rows may hold (the rows' shared totals).
 constexpr int kDecMaxSplit = 8;
+constexpr int kDecSplitRows = 256;
 
 template <int FMT, int MODE>
 __host__ __device__ constexpr int dec_group_rows() {
@@ -558,25 +560,49 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
   // ---------------- consumers: row groups, chunk by chunk ----------------
   // group g holds rows [g*RT, g*RT + RT) of this CTA's range and goes to team
   // g % teams; chunks hold a multiple of RT rows, so a group never straddles
-  // two.  A team of S > 1 warps agrees on every chunk wait (a timeout unwinds
-  // the whole team together), and per group its parts' row totals meet in
-  // shared memory (double-buffered: one team barrier a group).
+  // two.  Rows split across a team (S > 1): each part adds its row totals
+  // into shared row sums (integer adds, in any order) and the consumers store
+  // the rows after meeting once at the end, when the CTA has at most
+  // kDecSplitRows rows; otherwise once per chunk (chunks of split rows hold
+  // at most kDecSplitRows rows), with the chunk waits agreed CTA-wide so a
+  // timeout unwinds every consumer together.
   constexpr int RT = dec_group_rows<FMT, MODE>();
-  __shared__ int s_part[2][kDecWarps][RT];
+  __shared__ int s_rowsum[2][kDecSplitRows];
   const bool active = team < teams;
+  const bool once = rows <= kDecSplitRows;   // split rows: one final store pass
+  if (S > 1) {
+    for (int t = threadIdx.x; t < 2 * kDecSplitRows; t += CT) (&s_rowsum[0][0])[t] = 0;
+    named_bar_sync(1, CT);
+  }
   auto walk = [&](auto out_tag) {
     constexpr int OUT = decltype(out_tag)::value;
     int g = team;
-    int buf = 0;
     int s = 0, ph = 0;   // ring slot and phase parity of chunk c
+    // The previous group's row totals wait here (lane r: row r) and are
+    // stored after the next group's dot products are issued: the warp
+    // reductions and the store's dependent chain then overlap the next
+    // group's work instead of stalling the warp.
+    int pend_t = 0, pend_row = 0, pend_n = 0;   // pend_n: live rows (0: none)
+    int* pend_rs = nullptr;
+    auto flush = [&]() {
+      if (lane < pend_n) {
+        if (S == 1)
+          dec_put<OUT>(pend_t, r0 + pend_row + lane, f, Y, bias, out_mode);
+        else
+          atomicAdd(pend_rs + lane, pend_t);
+      }
+    };
     for (int c = 0; c < nch; ++c) {
       bool ok = mbar_wait(&full[s], ph, abort_v, limit_ns, 23);
       ok = __all_sync(0xffffffffu, ok);
-      if (S > 1 && active) ok = named_bar_and(2 + team, 32 * S, ok);
+      if (S > 1 && !once) ok = named_bar_and(1, CT, ok);
       if (!ok) break;
       const int c0 = c * CR;
       const int cend = min(c0 + CR, rows);
       const uint8_t* sbase = dec_smem + s * chunk_bytes;
+      // split rows: row r of the CTA at rs[r - rbase]
+      int* rs = once ? &s_rowsum[0][0] : s_rowsum[c & 1];
+      const int rbase = once ? 0 : c0;
       if (active) {
         for (; g * RT < cend; g += teams) {
           const int lr = g * RT;
@@ -590,19 +616,24 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
           } else {
             dec_dot_reg<RT, AW>(rowp, row_bytes, nlive, word0, lane, act, neg_r, pt);
           }
-          if (S == 1) {
-            dec_store<RT, OUT>(pt, r0 + lr, nlive, lane, f, Y, bias, out_mode);
-          } else {
-            const int t = dec_warp_totals<RT>(pt, lane);
-            if (lane < RT) s_part[buf][warp][lane] = t;
-            named_bar_sync(2 + team, 32 * S);
-            if (part == 0 && lane < nlive) {
-              int tot = 0;
-              for (int q = 0; q < S; ++q) tot += s_part[buf][warp + q][lane];
-              dec_put<OUT>(tot, r0 + lr + lane, f, Y, bias, out_mode);
-            }
-            buf ^= 1;
-          }
+          const int t = dec_warp_totals<RT>(pt, lane);
+          flush();
+          pend_t = t;
+          pend_row = lr;
+          pend_n = nlive;
+          pend_rs = rs + (lr - rbase);
+        }
+      }
+      if (S > 1 && !once) {
+        // every part of the chunk's rows has added its totals: store them,
+        // and clear the buffer for chunk c + 2 (its adds follow the next
+        // chunk's agreement barrier)
+        flush();
+        pend_n = 0;
+        named_bar_sync(1, CT);
+        for (int t = threadIdx.x; t < cend - c0; t += CT) {
+          dec_put<OUT>(rs[t], r0 + c0 + t, f, Y, bias, out_mode);
+          rs[t] = 0;
         }
       }
       __syncwarp();
@@ -612,11 +643,19 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
         ph ^= 1;
       }
     }
+    flush();
+    if (S > 1 && once) {
+      // every consumer leaves the loop (a bounded wait that gives up ends it
+      // too), so all of them reach this barrier; a stalled CTA stores
+      // nothing (its status word records the timeout)
+      const bool all_ok = named_bar_and(1, CT, !*abort_v);
+      if (all_ok)
+        for (int t = threadIdx.x; t < rows; t += CT) dec_put<OUT>(s_rowsum[0][t], r0 + t, f, Y, bias, out_mode);
+    }
   };
-  if (out_mode == kOutBF16)
-    walk(std::integral_constant<int, kOutBF16>{});
-  else
-    walk(std::integral_constant<int, kOutAny>{});
+  // one copy of the loop for every output type: a smaller kernel runs faster
+  // here than one specialised for bf16 (instruction fetch)
+  walk(std::integral_constant<int, kOutAny>{});
 }
 
 }  // namespace bl
