@@ -53,6 +53,7 @@ SIGNATURES = {
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
     "bl_selftest_wait_timeout": (_int, [ctypes.c_ulonglong, _p, _p]),
     "bl_probe_mma_i8": (_int, [_int, _int, _p, _int, _p]),
+    "bl_probe_mma_i8_pair": (_int, [_int, _int, _p, _int, _p]),
     "bl_packed_weight_bytes_b3": (_sz, [_i64, _i64]),
     "bl_quantize_weights_b3": (_int, [_p, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_unpack_weights_b3": (_int, [_p, _i64, _i64, _p, _p]),
@@ -433,3 +434,13 @@ def bl_matmul_i32_b3(Xq: torch.Tensor, Wp3: torch.Tensor, N: int) -> torch.Tenso
     acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
     _check(lib().bl_matmul_i32_b3(px, M, K, N, pw, acc.data_ptr(), _stream()), "bl_matmul_i32_b3")
     return acc
+
+
+def bl_probe_mma_i8_pair(n_mma: int, n_cols: int = 128, grid: int | None = None) -> torch.Tensor:
+    """CTA-pair (cta_group::2) kind::i8 rate probe: int64 [grid, 2] of (SM
+    cycles, ns) per CTA for n_mma MMAs of 256 x n_cols x 32 over each pair."""
+    if grid is None:
+        grid = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count // 2 * 2
+    out = torch.zeros((grid, 2), dtype=torch.int64, device="cuda")
+    _check(lib().bl_probe_mma_i8_pair(n_mma, n_cols, out.data_ptr(), grid, _stream()), "bl_probe_mma_i8_pair")
+    return out

@@ -1210,6 +1210,30 @@ bl_status bl_probe_mma_i8(int n_mma, int n_cols, unsigned long long* out, int gr
   return last_cuda();
 }
 
+bl_status bl_probe_mma_i8_pair(int n_mma, int n_cols, unsigned long long* out, int grid, cudaStream_t stream) {
+  if (!out) return BL_ERR_INVALID_ARG;
+  if (n_mma <= 0 || n_mma > (1 << 22) || grid <= 0 || grid > 4096 || (grid % 2) != 0) return BL_ERR_SHAPE;
+  if (n_cols < 32 || n_cols > 256 || (n_cols % 32) != 0) return BL_ERR_SHAPE;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(bl::bl_probe_mma_i8_pair_kernel, bl::kProbeSmemBytes, &done)) return BL_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(bl::kProbeThreads);
+  cfg.dynamicSmemBytes = bl::kProbeSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const unsigned long long lim = kWaitLimitNs;
+  if (cudaLaunchKernelEx(&cfg, bl::bl_probe_mma_i8_pair_kernel, n_mma, n_cols, out, lim) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return last_cuda();
+}
+
 bl_status bl_device_status(int clear, int* site) {
   if (cudaDeviceSynchronize() != cudaSuccess) return BL_ERR_CUDA;
   unsigned int v = 0;

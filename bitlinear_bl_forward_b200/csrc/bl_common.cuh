@@ -342,6 +342,185 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// Sixteen tcgen05.mma kind::i8 (cta_group::2) of one K = 512 pipeline stage
+// in one asm block.  MMA k (k = 0..15) reads A at tensor-memory column
+// a0 + 8k and B through the shared-memory descriptor {dlo + boff(k), dhi},
+// boff(k) = (k / 4) * BOX16 + 2 (k % 4) in the 16-byte units of the
+// descriptor's start-address field (the sum cannot carry out of it for
+// shared-memory addresses); the first MMA accumulates when acc0 != 0, the
+// others always.  The issuing thread does nothing else between the MMAs: its
+// instruction count per MMA bounds the MMA rate.
+template <int BOX16>
+__device__ __forceinline__ void mma_i8_stage16_pair(uint32_t d_tmem, uint32_t a0, uint32_t dlo, uint32_t dhi, uint32_t idesc,
+                                                uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b64 d;\n\t.reg .b32 a, lo;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "setp.eq.b32 q, %5, %5;\n\t"
+      "mov.b64 d, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], d, %4, p;\n\t"
+      "add.u32 a, %1, 8;\n\t"
+      "add.u32 lo, %2, %6;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 16;\n\t"
+      "add.u32 lo, %2, %7;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 24;\n\t"
+      "add.u32 lo, %2, %8;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 32;\n\t"
+      "add.u32 lo, %2, %9;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 40;\n\t"
+      "add.u32 lo, %2, %10;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 48;\n\t"
+      "add.u32 lo, %2, %11;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 56;\n\t"
+      "add.u32 lo, %2, %12;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 64;\n\t"
+      "add.u32 lo, %2, %13;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 72;\n\t"
+      "add.u32 lo, %2, %14;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 80;\n\t"
+      "add.u32 lo, %2, %15;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 88;\n\t"
+      "add.u32 lo, %2, %16;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 96;\n\t"
+      "add.u32 lo, %2, %17;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 104;\n\t"
+      "add.u32 lo, %2, %18;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 112;\n\t"
+      "add.u32 lo, %2, %19;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 120;\n\t"
+      "add.u32 lo, %2, %20;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a0), "r"(dlo), "r"(dhi),
+         "r"(idesc), "r"(acc0), "n"((1 / 4) * BOX16 + 2 * (1 % 4)),
+         "n"((2 / 4) * BOX16 + 2 * (2 % 4)), "n"((3 / 4) * BOX16 + 2 * (3 % 4)), "n"((4 / 4) * BOX16 + 2 * (4 % 4)), "n"((5 / 4) * BOX16 + 2 * (5 % 4)),
+         "n"((6 / 4) * BOX16 + 2 * (6 % 4)), "n"((7 / 4) * BOX16 + 2 * (7 % 4)), "n"((8 / 4) * BOX16 + 2 * (8 % 4)), "n"((9 / 4) * BOX16 + 2 * (9 % 4)),
+         "n"((10 / 4) * BOX16 + 2 * (10 % 4)), "n"((11 / 4) * BOX16 + 2 * (11 % 4)), "n"((12 / 4) * BOX16 + 2 * (12 % 4)), "n"((13 / 4) * BOX16 + 2 * (13 % 4)),
+         "n"((14 / 4) * BOX16 + 2 * (14 % 4)), "n"((15 / 4) * BOX16 + 2 * (15 % 4))
+      : "memory");
+}
+
+// Sixteen tcgen05.mma kind::i8 (cta_group::1) of one K = 512 pipeline stage
+// in one asm block.  MMA k (k = 0..15) reads A at tensor-memory column
+// a0 + 8k and B through the shared-memory descriptor {dlo + boff(k), dhi},
+// boff(k) = (k / 4) * BOX16 + 2 (k % 4) in the 16-byte units of the
+// descriptor's start-address field (the sum cannot carry out of it for
+// shared-memory addresses); the first MMA accumulates when acc0 != 0, the
+// others always.  The issuing thread does nothing else between the MMAs: its
+// instruction count per MMA bounds the MMA rate.
+template <int BOX16>
+__device__ __forceinline__ void mma_i8_stage16(uint32_t d_tmem, uint32_t a0, uint32_t dlo, uint32_t dhi, uint32_t idesc,
+                                                uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b64 d;\n\t.reg .b32 a, lo;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "setp.eq.b32 q, %5, %5;\n\t"
+      "mov.b64 d, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], d, %4, p;\n\t"
+      "add.u32 a, %1, 8;\n\t"
+      "add.u32 lo, %2, %6;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 16;\n\t"
+      "add.u32 lo, %2, %7;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 24;\n\t"
+      "add.u32 lo, %2, %8;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 32;\n\t"
+      "add.u32 lo, %2, %9;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 40;\n\t"
+      "add.u32 lo, %2, %10;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 48;\n\t"
+      "add.u32 lo, %2, %11;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 56;\n\t"
+      "add.u32 lo, %2, %12;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 64;\n\t"
+      "add.u32 lo, %2, %13;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 72;\n\t"
+      "add.u32 lo, %2, %14;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 80;\n\t"
+      "add.u32 lo, %2, %15;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 88;\n\t"
+      "add.u32 lo, %2, %16;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 96;\n\t"
+      "add.u32 lo, %2, %17;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 104;\n\t"
+      "add.u32 lo, %2, %18;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 112;\n\t"
+      "add.u32 lo, %2, %19;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "add.u32 a, %1, 120;\n\t"
+      "add.u32 lo, %2, %20;\n\t"
+      "mov.b64 d, {lo, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [a], d, %4, q;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a0), "r"(dlo), "r"(dhi),
+         "r"(idesc), "r"(acc0), "n"((1 / 4) * BOX16 + 2 * (1 % 4)),
+         "n"((2 / 4) * BOX16 + 2 * (2 % 4)), "n"((3 / 4) * BOX16 + 2 * (3 % 4)), "n"((4 / 4) * BOX16 + 2 * (4 % 4)), "n"((5 / 4) * BOX16 + 2 * (5 % 4)),
+         "n"((6 / 4) * BOX16 + 2 * (6 % 4)), "n"((7 / 4) * BOX16 + 2 * (7 % 4)), "n"((8 / 4) * BOX16 + 2 * (8 % 4)), "n"((9 / 4) * BOX16 + 2 * (9 % 4)),
+         "n"((10 / 4) * BOX16 + 2 * (10 % 4)), "n"((11 / 4) * BOX16 + 2 * (11 % 4)), "n"((12 / 4) * BOX16 + 2 * (12 % 4)), "n"((13 / 4) * BOX16 + 2 * (13 % 4)),
+         "n"((14 / 4) * BOX16 + 2 * (14 % 4)), "n"((15 / 4) * BOX16 + 2 * (15 % 4))
+      : "memory");
+}
+
+// The constant high word and the start-address low word of a 128-byte-swizzled
+// K-major descriptor (smem_desc_k_sw128 split in two).
+constexpr uint32_t kDescSw128Hi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_sw128_lo(uint32_t smem_addr) { return ((smem_addr >> 4) & 0x3FFFu) | (1u << 16); }
+
 // Instruction descriptor: kind::i8, s8 x s8 -> s32, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4)                                   // D format: s32

@@ -173,13 +173,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
             break;
           }
           tc_fence_after();
+          // the stage's 16 MMAs (K = 32 each) from one asm block: MMA k reads
+          // A column 8k of the slot and token box k / 4, bytes 32 (k % 4)
+          static_assert(kQBK == 512, "one stage is sixteen MMAs");
           const uint32_t xs = smem_u32(sX + s * kQXStageBytes);
-#pragma unroll
-          for (int kk = 0; kk < kQBK / 32; ++kk) {
-            const uint32_t a_tmem = tmem + kQACol + kQASlotCols * t + 8 * kk;
-            const uint32_t b_addr = xs + (kk >> 2) * kQXBoxBytes + 32 * (kk & 3);
-            mma_i8_ts_pair(d_tmem, a_tmem, smem_desc_k_sw128(b_addr), idesc, (ks | kk) != 0 ? 1u : 0u);
-          }
+          mma_i8_stage16_pair<kQXBoxBytes / 16>(d_tmem, tmem + kQACol + kQASlotCols * t, desc_sw128_lo(xs),
+                                                kDescSw128Hi, idesc, ks != 0 ? 1u : 0u);
           tc_commit_pair(&done[s], 3);
         }
         if (stop) break;

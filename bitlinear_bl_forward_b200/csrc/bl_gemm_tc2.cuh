@@ -177,14 +177,12 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          // the stage's 16 MMAs (K = 32 each) from one asm block: MMA k reads
+          // A column 8k of the slot and token box k / 4, bytes 32 (k % 4)
+          static_assert(kP2Sub * (kTcBK / 32) == 16, "one stage is sixteen MMAs");
           const uint32_t xs = smem_u32(sX + s * C::kXStageBytes);
-          const uint32_t as = tmem + C::kACol + kP2ASlotCols * t;
-#pragma unroll
-          for (int j = 0; j < kP2Sub; ++j)
-#pragma unroll
-            for (int kk = 0; kk < kTcBK / 32; ++kk)
-              mma_i8_ts(d_tmem, as + 32 * j + 8 * kk, smem_desc_k_sw128(xs + j * C::kXSubBytes + 32 * kk), idesc,
-                        (ks | j | kk) != 0 ? 1u : 0u);
+          mma_i8_stage16<C::kXSubBytes / 16>(d_tmem, tmem + C::kACol + kP2ASlotCols * t, desc_sw128_lo(xs),
+                                             kDescSw128Hi, idesc, ks != 0 ? 1u : 0u);
           // one commit frees both the smem stage (producer) and, three stages
           // later, the tensor-memory slot (expanders wait on the same phase)
           tc_commit(&empty[s]);

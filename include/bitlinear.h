@@ -358,6 +358,12 @@ BL_API bl_status bl_matmul_i32_b3(const int8_t* Xq, int64_t M, int64_t K, int64_
  * 16 in [16, 256], grid in [1, 4096] (else BL_ERR_SHAPE).
  */
 BL_API bl_status bl_probe_mma_i8(int n_mma, int n_cols, unsigned long long* out, int grid, cudaStream_t stream);
+/* The CTA-pair form of the probe (tcgen05.mma cta_group::2, clusters of two
+ * CTAs, M = 256 over the pair, N = n_cols with half of B in each CTA): the
+ * pair's leader issues the MMAs; every CTA writes its cycles and nanoseconds
+ * as above.  Rate per SM = 128 * n_cols * 32 * n_mma / cycles.  grid even,
+ * n_cols a multiple of 32 in [32, 256] (else BL_ERR_SHAPE). */
+BL_API bl_status bl_probe_mma_i8_pair(int n_mma, int n_cols, unsigned long long* out, int grid, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Device status.

@@ -231,3 +231,9 @@ def test_probe_host_checks(L):
     assert L.bl_probe_mma_i8(16, 8, A, 148, None) == SHAPE
     assert L.bl_probe_mma_i8(16, 264, A, 148, None) == SHAPE
     assert L.bl_probe_mma_i8(16, 256, None, 148, None) == INVALID
+
+
+def test_probe_pair_host_checks(L):
+    assert L.bl_probe_mma_i8_pair(16, 128, A, 147, None) == SHAPE     # odd grid
+    assert L.bl_probe_mma_i8_pair(16, 16, A, 148, None) == SHAPE      # n_cols % 32
+    assert L.bl_probe_mma_i8_pair(16, 128, None, 148, None) == INVALID
