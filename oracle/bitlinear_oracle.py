@@ -84,6 +84,8 @@ __all__ = [
     "act_quant",
     "act_quant_values",
     "act_quant_per_tensor",
+    "pack_int4",
+    "unpack_int4",
     "relu2_input",
     "matmul_i32",
     "rescale",
@@ -408,6 +410,33 @@ def act_quant_per_tensor(x_bits: np.ndarray, bits: int = 8):
 # ---------------------------------------------------------------------------
 # [P3] section 2: squared ReLU between the feed-forward projections
 # ---------------------------------------------------------------------------
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """4-bit activation codes int8 [M, K] in [-8, 7] -> packed uint8 [M, K/2]
+    ([P1] "Step 4: Verification and Benchmarking Test Harness" counts the 4-bit
+    activations at half a byte each).  The layout is this library's: byte j of
+    row m holds code 2j in its low nibble and code 2j + 1 in its high nibble,
+    each as a 4-bit two's-complement number."""
+    c = np.asarray(q, dtype=np.int64)
+    M, K = c.shape
+    if K % 2:
+        raise ValueError("K must be even")
+    if np.any((c < -8) | (c > 7)):
+        raise ValueError("codes must lie in [-8, 7]")
+    nib = c & 0xF
+    return (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed: np.ndarray, K: int) -> np.ndarray:
+    """Inverse of pack_int4: packed uint8 [M, K/2] -> int8 codes [M, K]."""
+    p = np.asarray(packed, dtype=np.int64)
+    M = p.shape[0]
+    out = np.empty((M, K), dtype=np.int64)
+    lo, hi = p & 0xF, (p >> 4) & 0xF
+    out[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return out.astype(np.int8)
+
 
 def relu2_input(g_bits: np.ndarray, u_bits: np.ndarray | None = None) -> np.ndarray:
     """Input of the down projection from the gate projection's bf16 output g:

@@ -306,6 +306,44 @@ def test_base3_bytewise_definition():
 
 
 # ---------------------------------------------------------------------------
+# Packed 4-bit activations (P1 Step 4: n // 2 bytes; the nibble order is this
+# library's)
+# ---------------------------------------------------------------------------
+
+def test_int4_layout_golden():
+    g = json.load(open(os.path.join(GOLDEN, "int4_layout.json")))
+    q = np.array([g["codes"]], dtype=np.int8)
+    p = o.pack_int4(q)
+    assert p.tolist() == [g["packed_bytes"]]
+    assert np.array_equal(o.unpack_int4(p, q.shape[1]), q)
+
+
+def test_int4_nibble_by_nibble_and_roundtrip():
+    rng = np.random.default_rng(11)
+    for M, K in [(1, 64), (3, 4096), (5, 8192)]:
+        q = rng.integers(-8, 8, (M, K)).astype(np.int8)
+        p = o.pack_int4(q)
+        assert p.shape == (M, K // 2) and p.nbytes * 2 == q.size
+        assert np.array_equal(o.unpack_int4(p, K), q)
+        # nibble by nibble with explicit sign extension
+        for m, k in [(0, 0), (0, 1), (M - 1, K - 1), (M - 1, K - 2)]:
+            nib = (int(p[m, k // 2]) >> (4 * (k % 2))) & 0xF
+            assert (nib - 16 if nib & 8 else nib) == q[m, k]
+    with pytest.raises(ValueError):
+        o.pack_int4(np.array([[8, 0]], dtype=np.int8))
+
+
+def test_int4_of_the_a48_quantiser_output():
+    # the a4.8 quantiser's codes (Q = 7) fit the nibbles and survive packing
+    from bitlinear_bl_forward_b200.inputs import WORKLOADS, layer_inputs
+    w = WORKLOADS["a48"]
+    X, _ = layer_inputs(w, 0, M=4)
+    q, _ = o.act_quant(X, 4)
+    assert q.min() >= -8 and q.max() <= 7
+    assert np.array_equal(o.unpack_int4(o.pack_int4(q), q.shape[1]), q)
+
+
+# ---------------------------------------------------------------------------
 # [P2] eq. (2), [P1] section 1: activation quantisation
 # ---------------------------------------------------------------------------
 
