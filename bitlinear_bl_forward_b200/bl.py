@@ -34,6 +34,7 @@ SIGNATURES = {
     "bl_quantize_weights": (_int, [_p, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_unpack_weights": (_int, [_p, _i64, _i64, _p, _p]),
     "bl_quant_act": (_int, [_p, _i64, _i64, _int, _p, _p, _p]),
+    "bl_quant_act_packed4": (_int, [_p, _i64, _i64, _p, _p, _p]),
     "bl_forward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "bl_forward": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_forward_f32": (_int, [_p, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
@@ -155,6 +156,16 @@ def bl_quant_act(X: torch.Tensor, bits: int = 8):
     s = torch.empty(M, dtype=torch.float32, device=X.device)
     _check(lib().bl_quant_act(px, M, K, bits, Xq.data_ptr(), s.data_ptr(), _stream()), "bl_quant_act")
     return Xq, s
+
+
+def bl_quant_act_packed4(X: torch.Tensor):
+    """bf16 [M, K] -> (4-bit codes packed two a byte uint8 [M, K/2], scale fp32 [M])."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    Xq4 = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    _check(lib().bl_quant_act_packed4(px, M, K, Xq4.data_ptr(), s.data_ptr(), _stream()), "bl_quant_act_packed4")
+    return Xq4, s
 
 
 def bl_forward_workspace_bytes(M: int, K: int, N: int, bits: int = 8) -> int:

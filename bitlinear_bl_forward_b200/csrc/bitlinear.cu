@@ -482,7 +482,7 @@ bl_status launch_act_quant(const uint16_t* X, int m, int k, int Q, int8_t* Xq, f
   // measured: the CTA-per-row kernel also wins for long rows (K > 4096, where
   // a warp can no longer keep its row in registers and reads part of it twice)
   if (m < bl::kActRowsPerBlock * num_sms() || k > 32 * 8 * bl::kActCache) {
-    bl::bl_act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, nullptr);
+    bl::bl_act_quant_row_kernel<false><<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, nullptr);
   } else {
     const int blocks = (m + bl::kActRowsPerBlock - 1) / bl::kActRowsPerBlock;
     bl::bl_act_quant_kernel<<<blocks, 256, 0, stream>>>(X, m, k, Q, Xq, s, R);
@@ -536,35 +536,57 @@ int max_active_pairs(F* kernel, int threads, int smem) {
   return n;
 }
 
-bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
-                         const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias) {
+// One weight tensor of a tensor-core launch.
+struct TcProb {
+  const uint8_t* Wp;
+  const float* gamma;
+  void* Y;
+  int N;
+  const float* bias;
+};
+
+// The CTA-pair GEMM over one or two problems that share the quantised
+// activations Xq [M, K] (its tiles run over both weight tensors).
+bl_status launch_tc_pair_multi(const int8_t* Xq, int M, int K, const TcProb* probs, int count, const int* R,
+                               const float* s, int out_mode, cudaStream_t stream) {
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(bl::bl_mma_pair_kernel, bl::kQSmemBytes, &done)) return BL_ERR_CUDA;
-  CUtensorMap tmX, tmW;
+  CUtensorMap tmX;
   if (!encode_u8_2d(&tmX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), bl::kQHalf, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return BL_ERR_CUDA;
-  if (!encode_u8_2d(&tmW, Wp, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTcRows, bl::kQBK / 4,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return BL_ERR_CUDA;
-  // bf16 outputs leave through TMA stores when the rows are 16-byte aligned
-  CUtensorMap tmY;
-  std::memset(&tmY, 0, sizeof(tmY));
-  int tma_store = 0;
-  if (out_mode == bl::kOutBF16 && (N % 8) == 0 && (reinterpret_cast<uintptr_t>(Y) & 15u) == 0) {
-    EncodeTiledFn enc = get_encode();
-    if (!enc) return BL_ERR_CUDA;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(bl::kQEpiCols)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-        CUDA_SUCCESS)
+  bl::QProblems P;
+  std::memset(&P, 0, sizeof(P));
+  P.count = count;
+  int ntn = 0;
+  for (int w = 0; w < count; ++w) {
+    const TcProb& q = probs[w];
+    bl::QOut& O = P.p[w];
+    if (!encode_u8_2d(&O.tmW, q.Wp, static_cast<uint64_t>(q.N), static_cast<uint64_t>(K / 4), bl::kTcRows,
+                      bl::kQBK / 4, CU_TENSOR_MAP_SWIZZLE_128B))
       return BL_ERR_CUDA;
-    tma_store = 1;
+    // bf16 outputs leave through TMA stores when the rows are 16-byte aligned
+    if (out_mode == bl::kOutBF16 && (q.N % 8) == 0 && (reinterpret_cast<uintptr_t>(q.Y) & 15u) == 0) {
+      EncodeTiledFn enc = get_encode();
+      if (!enc) return BL_ERR_CUDA;
+      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(q.N), static_cast<cuuint64_t>(M)};
+      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(q.N) * 2};
+      const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(bl::kQEpiCols)};
+      const cuuint32_t estr[2] = {1, 1};
+      if (enc(&O.tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.Y, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return BL_ERR_CUDA;
+      O.tma_store = 1;
+    }
+    O.gamma = q.gamma;
+    O.Y = q.Y;
+    O.bias = q.bias;
+    O.N = q.N;
+    O.ntn = (q.N + bl::kQRows - 1) / bl::kQRows;
+    ntn += O.ntn;
   }
-  const int ntiles = ((M + bl::kQBN - 1) / bl::kQBN) * ((N + bl::kQRows - 1) / bl::kQRows);
+  const int ntiles = ((M + bl::kQBN - 1) / bl::kQBN) * ntn;
   cudaLaunchConfig_t cfg = {};
   // a persistent grid must fit in one wave: not every SM can host half of a
   // two-SM cluster, so ask how many clusters are co-resident (once per device)
@@ -583,10 +605,15 @@ bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* W
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const unsigned long long lim = kWaitLimitNs;
-  if (cudaLaunchKernelEx(&cfg, bl::bl_mma_pair_kernel, tmX, tmW, tmY, M, N, K, R, s, gamma, Y, out_mode, tma_store,
-                         bias, lim) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, bl::bl_mma_pair_kernel, tmX, P, M, K, R, s, out_mode, lim) != cudaSuccess)
     return BL_ERR_CUDA;
   return last_cuda();
+}
+
+bl_status launch_tc_pair(const int8_t* Xq, int M, int K, int N, const uint8_t* Wp, const int* R, const float* s,
+                         const float* gamma, void* Y, int out_mode, cudaStream_t stream, const float* bias) {
+  const TcProb p{Wp, gamma, Y, N, bias};
+  return launch_tc_pair_multi(Xq, M, K, &p, 1, R, s, out_mode, stream);
 }
 
 // Tensor-core GEMM by token count: the CTA-pair kernel for M > 64, the
@@ -732,6 +759,20 @@ bl_status bl_quant_act(const uint16_t* X, int64_t M, int64_t K, int bits, int8_t
   if (!aligned16(X) || !aligned16(Xq)) return BL_ERR_ALIGNMENT;
   return launch_act_quant(X, static_cast<int>(M), static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr,
                           stream);
+}
+
+bl_status bl_quant_act_packed4(const uint16_t* X, int64_t M, int64_t K, uint8_t* Xq4, float* scale,
+                               cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quant_act_packed4");
+  if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
+  bl_status st = check_m(M, K);
+  if (st != BL_OK) return st;
+  if (M == 0) return BL_OK;
+  if (!X || !Xq4 || !scale) return BL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Xq4)) return BL_ERR_ALIGNMENT;
+  bl::bl_act_quant_row_kernel<true><<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
+      X, static_cast<int>(K), 7, reinterpret_cast<int8_t*>(Xq4), scale, nullptr, nullptr);
+  return last_cuda();
 }
 
 size_t bl_forward_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
@@ -887,11 +928,39 @@ bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, voi
     return launch_decode(sel, n, bl::kInBF16, Q, bl::kOutBF16, stream);
   }
   // otherwise the problems run one after another on the stream (the
-  // workspace is reused: stream order serialises them)
+  // workspace is reused: stream order serialises them); two problems with
+  // more than two tokens that read the same X (same pointer, M and K, e.g.
+  // the up and gate projections) share one activation quantisation and, for
+  // M > 64, one tensor-core launch over both weight tensors
+  bool done_p[bl::kG2MaxProblems] = {};
   for (int i = 0; i < count; ++i) {
+    if (done_p[i]) continue;
     const bl_linear& p = problems[i];
-    const bl_status st =
-        forward_common(p.X, p.M, p.K, p.N, p.Wp, p.gamma, bits, p.Y, bl::kOutBF16, workspace, workspace_bytes, stream);
+    int j = -1;
+    if (p.M > kGemvMaxM)
+      for (int k = i + 1; k < count && j < 0; ++k)
+        if (!done_p[k] && problems[k].X == p.X && problems[k].M == p.M && problems[k].K == p.K) j = k;
+    if (j < 0) {
+      const bl_status st = forward_common(p.X, p.M, p.K, p.N, p.Wp, p.gamma, bits, p.Y, bl::kOutBF16, workspace,
+                                          workspace_bytes, stream);
+      if (st != BL_OK) return st;
+      continue;
+    }
+    done_p[j] = true;
+    const bl_linear& p2 = problems[j];
+    const int m = static_cast<int>(p.M), k = static_cast<int>(p.K);
+    const FwdWs w = fwd_ws_split(workspace, p.M, p.K);
+    bl_status st = launch_act_quant(p.X, m, k, Q, w.Xq, w.s, w.R, stream);
+    if (st != BL_OK) return st;
+    if (p.M > 64) {
+      const TcProb tp[2] = {{p.Wp, p.gamma, p.Y, static_cast<int>(p.N), nullptr},
+                            {p2.Wp, p2.gamma, p2.Y, static_cast<int>(p2.N), nullptr}};
+      st = launch_tc_pair_multi(w.Xq, m, k, tp, 2, w.R, w.s, bl::kOutBF16, stream);
+    } else {
+      st = launch_tc(w.Xq, m, k, static_cast<int>(p.N), p.Wp, w.R, w.s, p.gamma, p.Y, bl::kOutBF16, stream);
+      if (st == BL_OK)
+        st = launch_tc(w.Xq, m, k, static_cast<int>(p2.N), p2.Wp, w.R, w.s, p2.gamma, p2.Y, bl::kOutBF16, stream);
+    }
     if (st != BL_OK) return st;
   }
   return BL_OK;
@@ -1020,7 +1089,7 @@ bl_status bl_forward_ex(const uint16_t* X, int64_t M, int64_t K, int64_t N, cons
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
     bl::bl_act_absmax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, nch, amax);
     if ((st = last_cuda()) != BL_OK) return st;
-    bl::bl_act_quant_row_kernel<<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, amax);
+    bl::bl_act_quant_row_kernel<false><<<m, bl::kActRowThreads, 0, stream>>>(X, k, Q, Xq, s, R, amax);
     if ((st = last_cuda()) != BL_OK) return st;
   } else if ((st = launch_act_quant(X, m, k, Q, Xq, s, R, stream)) != BL_OK) {
     return st;

@@ -161,6 +161,16 @@ __global__ void __launch_bounds__(256) bl_act_quant_kernel(const uint16_t* __res
 constexpr int kActRowThreads = 256;
 constexpr int kActRowCache = 8;   // 16-byte chunks kept in registers per thread (K <= 16384)
 
+// Eight int8 codes in [-8, 7] (two words) -> eight two's-complement nibbles
+// in one word: code 2j in the low nibble of byte j, code 2j + 1 in its high
+// nibble.
+__device__ __forceinline__ uint32_t pack_nibbles8(uint2 q) {
+  const uint32_t lo = q.x & 0x0f0f0f0fu, hi = q.y & 0x0f0f0f0fu;
+  const uint32_t a = lo | (lo >> 4), b = hi | (hi >> 4);   // bytes 0 and 2 hold code pairs
+  return __byte_perm(a, b, 0x6420);
+}
+
+template <bool PACK4 = false>
 __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_row_kernel(const uint16_t* __restrict__ X, int K, int Q,
                                                                        int8_t* __restrict__ Xq,
                                                                        float* __restrict__ s_out,
@@ -193,15 +203,27 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_row_kernel(const 
   for (int w = 0; w < W; ++w) bmax = max(bmax, s_max[w]);
   if (amax_all) bmax = *amax_all;   // per-tensor mode: one absmax for every row
   const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(__uint_as_float(bmax), 1e-5f));
-  uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
   int sum = 0;
+  if constexpr (PACK4) {
+    // 4-bit codes, two a byte: row m is K / 2 bytes
+    uint32_t* qr = reinterpret_cast<uint32_t*>(Xq + m * (K / 2));
 #pragma unroll
-  for (int i = 0; i < kActRowCache; ++i) {
-    const int c = t + kActRowThreads * i;
-    if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+    for (int i = 0; i < kActRowCache; ++i) {
+      const int c = t + kActRowThreads * i;
+      if (c < nch) qr[c] = pack_nibbles8(quant8_bf16(cache[i], s, Q, sum));
+    }
+    for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+      qr[c] = pack_nibbles8(quant8_bf16(__ldg(xr + c), s, Q, sum));
+  } else {
+    uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
+#pragma unroll
+    for (int i = 0; i < kActRowCache; ++i) {
+      const int c = t + kActRowThreads * i;
+      if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+    }
+    for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+      qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
   }
-  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
-    qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
   const int wsum = __reduce_add_sync(0xffffffffu, sum);
   if (lane == 0) s_sum[warp] = wsum;
   __syncthreads();

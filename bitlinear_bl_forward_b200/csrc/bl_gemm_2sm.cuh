@@ -70,11 +70,30 @@ constexpr int kQNumBars = 2 * kQStages + kQASlots + 5;
 constexpr int kQEpiOffset = kQBarOffset + kQNumBars * 8 + 16;
 constexpr int kQSmemBytes = kQEpiOffset + 2 * kQBN * 8 + 1024;
 
+// One weight tensor of a launch.  A launch serves one or two problems that
+// share the quantised activations (e.g. the up and gate projections of a
+// feed-forward block): its tiles run over the weight rows of problem 0 then
+// of problem 1, so every activation tile is quantised once and each tile of
+// either weight tensor is computed by the same pipeline.
+struct QOut {
+  CUtensorMap tmW;      // packed weights [N, K/4] (128-byte swizzle boxes)
+  CUtensorMap tmY;      // bf16 output [M, N] (TMA stores), when tma_store
+  const float* gamma;   // device fp32
+  void* Y;              // output [M, N]
+  const float* bias;    // optional fp32 [N]
+  int N;
+  int tma_store;
+  int ntn;              // weight-row tiles: ceil(N / 256)
+};
+struct QProblems {
+  QOut p[2];
+  int count;
+};
+
 __global__ void __launch_bounds__(kQThreads, 1)
-    bl_mma_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                        const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const int* __restrict__ Rg,
-                        const float* __restrict__ sg, const float* __restrict__ gamma_p, void* __restrict__ Y,
-                        int out_mode, int tma_store, const float* __restrict__ bias, unsigned long long limit_ns) {
+    bl_mma_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ QProblems P, int M, int K,
+                        const int* __restrict__ Rg, const float* __restrict__ sg, int out_mode,
+                        unsigned long long limit_ns) {
   constexpr int S = kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -98,7 +117,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nk = (K + kQBK - 1) / kQBK;
   const int mt = (M + kQBN - 1) / kQBN;
-  const int ntiles = mt * ((N + kQRows - 1) / kQRows);
+  const int ntn0 = P.p[0].ntn;
+  const int ntiles = mt * (ntn0 + (P.count > 1 ? P.p[1].ntn : 0));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -127,12 +147,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
       prefetch_tmap(&tmX);
-      prefetch_tmap(&tmW);
+      prefetch_tmap(&P.p[0].tmW);
+      if (P.count > 1) prefetch_tmap(&P.p[1].tmW);
       uint32_t g = 0;
       bool stop = false;
       for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
         const int m0 = (tile % mt) * kQBN + static_cast<int>(rank) * kQHalf;
-        const int n0 = (tile / mt) * kQRows + static_cast<int>(rank) * kTcRows;
+        const int nt = tile / mt, w = nt >= ntn0 ? 1 : 0;
+        const int n0 = (nt - (w ? ntn0 : 0)) * kQRows + static_cast<int>(rank) * kTcRows;
+        const CUtensorMap* tmW = &P.p[w].tmW;
         for (int ks = 0; ks < nk; ++ks, ++g) {
           const int s = g % S;
           if (g >= static_cast<uint32_t>(S) &&
@@ -144,7 +167,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
           for (int bx = 0; bx < kQBK / 128; ++bx)
             tma_load_2d(sX + s * kQXStageBytes + bx * kQXBoxBytes, &tmX, ks * kQBK + bx * 128, m0, &full[s]);
-          tma_load_2d(sW + s * kQWStageBytes, &tmW, ks * (kQBK / 4), n0, &full[s]);
+          tma_load_2d(sW + s * kQWStageBytes, tmW, ks * (kQBK / 4), n0, &full[s]);
         }
       }
       const uint32_t issued = g;
@@ -157,7 +180,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
     // ---------------- MMA issuer (leader only) ----------------
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_i8(kQRows, kQBN);
-      uint32_t g = 0;
+      // ring positions kept as counters: this thread's instruction count
+      // bounds the MMA rate
+      const uint32_t dlo0 = desc_sw128_lo(smem_u32(sX));
+      int s = 0, t = 0;
+      uint32_t tph = 0;   // phase parity of afull[t]
       int i = 0;
       bool stop = false;
       for (int tile = pair; tile < ntiles && !stop; tile += npairs, ++i) {
@@ -165,10 +192,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (i >= 2 && !mbar_wait_cluster(&accempty[b], ((i >> 1) & 1) ^ 1u, abort_flag, limit_ns, kSiteAcc)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + b * kQAccCols;
-        for (int ks = 0; ks < nk; ++ks, ++g) {
-          const int s = g % S;
-          const int t = g % kQASlots;
-          if (!mbar_wait_cluster(&afull[t], (g / kQASlots) & 1, abort_flag, limit_ns, kSiteMmaExfull)) {
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait_cluster(&afull[t], tph, abort_flag, limit_ns, kSiteMmaExfull)) {
             stop = true;
             break;
           }
@@ -176,10 +201,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
           // the stage's 16 MMAs (K = 32 each) from one asm block: MMA k reads
           // A column 8k of the slot and token box k / 4, bytes 32 (k % 4)
           static_assert(kQBK == 512, "one stage is sixteen MMAs");
-          const uint32_t xs = smem_u32(sX + s * kQXStageBytes);
-          mma_i8_stage16_pair<kQXBoxBytes / 16>(d_tmem, tmem + kQACol + kQASlotCols * t, desc_sw128_lo(xs),
-                                                kDescSw128Hi, idesc, ks != 0 ? 1u : 0u);
+          mma_i8_stage16_pair<kQXBoxBytes / 16>(d_tmem, tmem + kQACol + kQASlotCols * t,
+                                                dlo0 + s * (kQXStageBytes / 16), kDescSw128Hi, idesc,
+                                                ks != 0 ? 1u : 0u);
           tc_commit_pair(&done[s], 3);
+          if (++s == S) s = 0;
+          if (++t == kQASlots) {
+            t = 0;
+            tph ^= 1u;
+          }
         }
         if (stop) break;
         tc_commit_pair(&accfull[b], 3);
@@ -243,12 +273,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int et = threadIdx.x - 32 * kQFirstEpi;
     const int col0 = ((warp - kQFirstEpi) >> 2) * kQEpiCols;   // this warp's half of the tokens
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const float gamma = (out_mode == kOutI32) ? 1.f : *gamma_p;
+    const float gamma0 = (out_mode == kOutI32) ? 1.f : *P.p[0].gamma;
+    const float gamma1 = (out_mode == kOutI32 || P.count < 2) ? 1.f : *P.p[1].gamma;
     int i = 0;
     for (int tile = pair; tile < ntiles; tile += npairs, ++i) {
       const int b = i & 1;
       const int m0 = (tile % mt) * kQBN;
-      const int n0 = (tile / mt) * kQRows + static_cast<int>(rank) * kTcRows;
+      const int nt = tile / mt, w = nt >= ntn0 ? 1 : 0;
+      const int n0 = (nt - (w ? ntn0 : 0)) * kQRows + static_cast<int>(rank) * kTcRows;
+      const QOut& O = P.p[w];
+      const int N = O.N;
+      void* __restrict__ Y = O.Y;
+      const float* __restrict__ bias = O.bias;
+      const float gamma = w ? gamma1 : gamma0;
       for (int j = et; j < kQBN; j += 32 * kQEpiWarps) {
         const int m = m0 + j;
         int rv = 0;
@@ -268,7 +305,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       tc_fence_after();
       const int n = n0 + r;
       const float bias_n = (bias && n < N) ? __ldg(bias + n) : 0.f;
-      if (tma_store) {
+      if (O.tma_store) {
         // bf16 tile of this warp, [BN tokens][32 rows], then one TMA store
         uint16_t* so = reinterpret_cast<uint16_t*>(sOut + (warp - kQFirstEpi) * kQStageOutBytes);
         if (lane == 0) bulk_wait_group_read0();   // the previous store has read the buffer
@@ -291,7 +328,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && m0 + col0 < M) {   // (a box starting past the last token writes nothing)
-          tma_store_2d(&tmY, n0 + q * 32, m0 + col0, so);
+          tma_store_2d(&O.tmY, n0 + q * 32, m0 + col0, so);
           bulk_commit_group();
         }
         __syncwarp();

@@ -161,7 +161,11 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = idesc_i8(kTcRows, BN);
-      uint32_t g = 0;
+      // ring positions kept as counters: this thread's instruction count
+      // bounds the MMA rate
+      const uint32_t dlo0 = desc_sw128_lo(smem_u32(sX));
+      int s = 0, t = 0;
+      uint32_t tph = 0;   // phase parity of afull[t]
       int i = 0;
       bool stop = false;
       for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x, ++i) {
@@ -169,10 +173,8 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
         if (i >= 2 && !mbar_wait(&accempty[b], ((i >> 1) & 1) ^ 1u, abort_flag, limit_ns, kSiteAcc)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + b * C::kAccCols;
-        for (int ks = 0; ks < nk; ++ks, ++g) {   // g counts stages
-          const int s = g % S;
-          const int t = g % kP2ASlots;
-          if (!mbar_wait(&afull[t], (g / kP2ASlots) & 1, abort_flag, limit_ns, kSiteMmaExfull)) {
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait(&afull[t], tph, abort_flag, limit_ns, kSiteMmaExfull)) {
             stop = true;
             break;
           }
@@ -180,12 +182,17 @@ __global__ void __launch_bounds__(P2Warps<EXPG>::kThreads, 1)
           // the stage's 16 MMAs (K = 32 each) from one asm block: MMA k reads
           // A column 8k of the slot and token box k / 4, bytes 32 (k % 4)
           static_assert(kP2Sub * (kTcBK / 32) == 16, "one stage is sixteen MMAs");
-          const uint32_t xs = smem_u32(sX + s * C::kXStageBytes);
-          mma_i8_stage16<C::kXSubBytes / 16>(d_tmem, tmem + C::kACol + kP2ASlotCols * t, desc_sw128_lo(xs),
-                                             kDescSw128Hi, idesc, ks != 0 ? 1u : 0u);
+          mma_i8_stage16<C::kXSubBytes / 16>(d_tmem, tmem + C::kACol + kP2ASlotCols * t,
+                                             dlo0 + s * (C::kXStageBytes / 16), kDescSw128Hi, idesc,
+                                             ks != 0 ? 1u : 0u);
           // one commit frees both the smem stage (producer) and, three stages
           // later, the tensor-memory slot (expanders wait on the same phase)
           tc_commit(&empty[s]);
+          if (++s == S) s = 0;
+          if (++t == kP2ASlots) {
+            t = 0;
+            tph ^= 1u;
+          }
         }
         if (stop) break;
         tc_commit(&accfull[b]);

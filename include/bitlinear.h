@@ -119,6 +119,18 @@ BL_API bl_status bl_unpack_weights(const uint8_t* Wp, int64_t N, int64_t K, int8
 BL_API bl_status bl_quant_act(const uint16_t* X, int64_t M, int64_t K, int bits, int8_t* Xq, float* scale,
                        cudaStream_t stream);
 
+/*
+ * The 4-bit mode of bl_quant_act with the codes packed two a byte ("BitNet
+ * a4.8 Guide: 4-Bit Activation 1-Bit LLMs", section "Step 4: Verification and
+ * Benchmarking Test Harness": 4-bit activations take n / 2 bytes): the same
+ * per-token codes as bl_quant_act(bits = 4) (Q = 7, range [-8, 7]), stored as
+ * two's-complement nibbles, code 2j of a row in the low nibble of byte j and
+ * code 2j + 1 in its high nibble.  Xq4: [M, K/2] bytes, 16-byte aligned.
+ * scale: fp32 [M], receives s_m.  M == 0 is a no-op.
+ */
+BL_API bl_status bl_quant_act_packed4(const uint16_t* X, int64_t M, int64_t K, uint8_t* Xq4, float* scale,
+                                      cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Forward.
  * ------------------------------------------------------------------------- */

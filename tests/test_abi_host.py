@@ -237,3 +237,11 @@ def test_probe_pair_host_checks(L):
     assert L.bl_probe_mma_i8_pair(16, 128, A, 147, None) == SHAPE     # odd grid
     assert L.bl_probe_mma_i8_pair(16, 16, A, 148, None) == SHAPE      # n_cols % 32
     assert L.bl_probe_mma_i8_pair(16, 128, None, 148, None) == INVALID
+
+
+def test_quant_act_packed4_host_checks(L):
+    assert L.bl_quant_act_packed4(A, 4, 100, A, A, None) == SHAPE
+    assert L.bl_quant_act_packed4(A, -1, 64, A, A, None) == SHAPE
+    assert L.bl_quant_act_packed4(None, 4, 64, A, A, None) == INVALID
+    assert L.bl_quant_act_packed4(A, 4, 64, U, A, None) == ALIGN
+    assert L.bl_quant_act_packed4(A, 0, 64, A, A, None) == OK

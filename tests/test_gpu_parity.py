@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from bitlinear_bl_forward_b200 import bl
-from bitlinear_bl_forward_b200.inputs import WORKLOADS, layer_inputs, random_case
+from bitlinear_bl_forward_b200.inputs import WORKLOADS, layer_inputs, make_weight, random_case
 from oracle import bitlinear_oracle as o
 from tests.gpu_helpers import (BF16_ULP_TOL, F32_REL_TOL, bf16_dev_to_bits, bf16_ulp_distance, rel_err,
                                x_to_dev)
@@ -351,6 +351,60 @@ def test_grouped_mixed_shapes_fall_back_to_sequential():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("M,K,N1,N2", [(3, 512, 300, 129), (64, 1024, 520, 256), (65, 512, 130, 1000),
+                                        (130, 2560, 1000, 264), (257, 640, 6912, 8), (300, 256, 7, 2049)])
+def test_grouped_shared_input_pair(M, K, N1, N2):
+    # two projections of one X (the up and gate shape) share the activation
+    # quantisation and, past 64 tokens, one tensor-core launch over both
+    # weight tensors; a third problem with its own X sits between them; ragged
+    # M and N, N not a multiple of 8 (plain epilogue stores) and of 256 (a
+    # partial last tile in either weight tensor)
+    X, W1 = random_case(M, K, N1, seed=700 + M)
+    _, W2 = random_case(M, K, N2, seed=800 + M)
+    X3, W3 = random_case(M, K, 96, seed=900 + M)
+    Xd = x_to_dev(X)
+    probs, cases = [], []
+    for Xh, Xt, W in ((X, Xd, W1), (X3, x_to_dev(X3), W3), (X, Xd, W2)):
+        g = o.absmean_scale(W)
+        c = o.ternary_codes(W, g)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        probs.append((Xt, Wp, gd, W.shape[0]))
+        cases.append((Xh, c, g))
+    for bits in (8, 4):
+        singles = [bl.bl_forward(Xt, Wp, gd, N, bits) for (Xt, Wp, gd, N) in probs]
+        outs = bl.bl_forward_grouped(probs, bits)
+        outs = bl.bl_forward_grouped(probs, bits, outs=outs)   # twice in a row, outputs reused
+        torch.cuda.synchronize()
+        for (Xh, c, g), a, b in zip(cases, outs, singles):
+            assert torch.equal(a, b)
+            assert bf16_ulp_distance(bf16_dev_to_bits(a), oracle_bf16(Xh, c, g, bits)).max() <= BF16_ULP_TOL
+
+
+def test_grouped_shared_input_pair_prefill_full_size():
+    # the 2B prefill up and gate projections (4096 tokens, K = 2560, N = 6912
+    # each) in one tensor-core launch: equal to two single calls everywhere,
+    # and to the oracle on sampled rows
+    w = WORKLOADS["prefill_2b"]
+    X, _ = layer_inputs(w, 0)
+    Xd = x_to_dev(X)
+    probs, cases = [], []
+    W_up, _, _, _ = oracle_weights(("prefill_2b", 0))
+    for W in (W_up, make_weight(W_up.shape[0], W_up.shape[1], 0.02, 4321)):
+        g = o.absmean_scale(W)
+        c = o.ternary_codes(W, g)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        probs.append((Xd, Wp, gd, W.shape[0]))
+        cases.append((c, g))
+    singles = [bl.bl_forward(Xd, Wp, gd, N) for (_, Wp, gd, N) in probs]
+    outs = bl.bl_forward_grouped(probs)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(7).choice(X.shape[0], 24, replace=False))
+    for (c, g), a, b in zip(cases, outs, singles):
+        assert torch.equal(a, b)
+        ref = oracle_bf16(X[rows], c, g)
+        assert bf16_ulp_distance(bf16_dev_to_bits(a[torch.from_numpy(rows).cuda()]), ref).max() <= BF16_ULP_TOL
+
+
 # ---------------------------------------------------------------------------
 # squared-ReLU feed-forward input ("BitNet 2B4T Guide: Scaling Native 1.58-Bit
 # LLMs", section "2. Squared ReLU Activation")
@@ -525,3 +579,28 @@ def test_forward_rmsnorm_bits4_zero_rows_and_back_to_back():
         d = bf16_ulp_distance(bf16_dev_to_bits(outs[m]), ref["Y"])
         assert d.max() <= BF16_ULP_TOL
     assert np.all(bf16_dev_to_bits(outs[1]) == 0)
+
+
+# ---------------------------------------------------------------------------
+# packed 4-bit activations ("BitNet a4.8 Guide: 4-Bit Activation 1-Bit LLMs",
+# section "Step 4: Verification and Benchmarking Test Harness")
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K", [(1, 64), (3, 4096), (7, 8192), (2, 65536)])
+def test_quant_act_packed4_bit_exact(M, K):
+    X, _ = random_case(M, K, 8, seed=700 + M + K, x_kind="relu2")
+    q, s = o.act_quant(X, 4)
+    p4, sd = bl.bl_quant_act_packed4(x_to_dev(X))
+    assert np.array_equal(p4.cpu().numpy(), o.pack_int4(q))
+    assert np.array_equal(sd.cpu().numpy().view(np.uint32), s.view(np.uint32))
+
+
+def test_quant_act_packed4_a48_full_size():
+    w = WORKLOADS["a48"]
+    X, _ = layer_inputs(w, 0)
+    q, s = o.act_quant(X, 4)
+    p4, sd = bl.bl_quant_act_packed4(x_to_dev(X))
+    assert np.array_equal(p4.cpu().numpy(), o.pack_int4(q))
+    # the same codes as the one-byte-a-code quantiser
+    qd, _ = bl.bl_quant_act(x_to_dev(X), 4)
+    assert np.array_equal(o.unpack_int4(p4.cpu().numpy(), X.shape[1]), qd.cpu().numpy())
