@@ -57,6 +57,11 @@ reason in the design notes of the repository):
     summed exactly and rounded once to fp32; r = sqrt(f32(ms + eps)); the
     normalised value is bf16(f32(f32(x / r) * w)), every step an IEEE fp32
     operation; the weight w (bf16 [K]) is optional.
+  * LayerNorm (the code listings' non-affine layer_norm over the feature
+    axis, whose eps the pages leave at the library default 1e-5):
+    mu = mean of x, the sum exact and rounded once to fp32; var = the
+    biased (1/K) variance of x, exact and rounded once; r = sqrt(f32(var +
+    eps)); the normalised value is bf16(f32(f32(x - mu) / r)).
 
 Array conventions: X is [M, K] (tokens x in-features) given as raw bf16 bit
 patterns (uint16); W is [N, K] fp32 (out-features x in-features, the
@@ -95,6 +100,9 @@ __all__ = [
     "exact_square_sum",
     "rms_norm",
     "forward_rmsnorm",
+    "exact_sum",
+    "layer_norm",
+    "forward_layernorm",
 ]
 
 # Floor used for both scales (pages' code listings clamp(min=1e-5)).
@@ -636,4 +644,90 @@ def forward_rmsnorm(x_bits: np.ndarray, W: np.ndarray, weight_bits: np.ndarray |
     nrm = rms_norm(x_bits, weight_bits, eps)
     out = forward(nrm["xn"], W, bits)
     out.update(nrm)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# [P2] "BitLinear" code listing (forward step 1) and [P3]'s BitLinear module:
+# a LayerNorm without affine parameters over the feature axis, immediately
+# before the absmax quantisation
+# ---------------------------------------------------------------------------
+
+def exact_sum(x_bits: np.ndarray) -> int:
+    """Exact value of sum_k x_k over bf16 values, as a signed integer count
+    of 2^-133 (the smallest bf16 subnormal).
+
+    x = (-1)^s sig * 2^(max(e, 1) - 1) units, with sig as in
+    ``exact_square_sum``; values are grouped by exponent (a group's signed
+    significand sum is an integer below 2^53 in magnitude, exact in float64)
+    and the groups are combined with Python integers.
+    """
+    b = np.ascontiguousarray(x_bits, dtype=np.uint16).ravel().astype(np.int64)
+    e = (b >> 7) & 0xFF
+    f = b & 0x7F
+    if np.any(e == 255):
+        raise ValueError("non-finite activation")
+    if b.size >= (1 << 36):
+        raise ValueError("too many values for the exact sum")
+    sig = np.where(e > 0, f | 0x80, f)
+    sig = np.where((b >> 15) & 1, -sig, sig)
+    sh = np.maximum(e, 1) - 1
+    groups = np.bincount(sh, weights=sig.astype(np.float64), minlength=254)
+    total = 0
+    for k in range(len(groups)):
+        if groups[k]:
+            total += int(groups[k]) << k
+    return total
+
+
+def layer_norm(x_bits: np.ndarray, eps: float = 1e-5):
+    """Non-affine LayerNorm of bf16 activations [M, K], per token.
+
+    The listings normalise with the library's layer_norm and no weight or
+    bias; the pages fix no precision.  Reading (every rounding named):
+        mu  = fp32( (1/K) sum_k x_k )                  exact sum, rounded once
+        var = fp32( (1/K) sum_k (x_k - (1/K) sum_j x_j)^2 )
+              the biased variance, exact, rounded once
+        r   = sqrt( f32(var + eps) )                   fp32 square root (IEEE)
+        d   = f32(x - mu)                              fp32 subtraction
+        t   = f32(d / r)                               fp32 division (IEEE)
+        x_n = bf16(t)                                  round to nearest even
+    The exact variance is formed as (K * sum x^2 - (sum x)^2) / K^2 from the
+    two exact sums.
+
+    Returns a dict: mean fp32 [M], var fp32 [M], r fp32 [M], t fp32 [M, K],
+    xn bf16 bits [M, K].
+    """
+    x = bf16_bits_to_f32(x_bits)
+    if x.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    M, K = x.shape
+    if K == 0:
+        raise ValueError("K must be positive")
+    e32 = np.float32(eps)
+    if not (np.isfinite(e32) and e32 > 0):
+        raise ValueError("eps must be a positive finite fp32 value")
+    mean = np.empty(M, np.float32)
+    var = np.empty(M, np.float32)
+    for m in range(M):
+        s1 = exact_sum(x_bits[m])          # units 2^-133
+        s2 = exact_square_sum(x_bits[m])   # units 2^-266
+        mu = round_rational_to_f32(abs(s1), K << 133)
+        mean[m] = -mu if s1 < 0 else mu
+        num = K * s2 - s1 * s1             # K^2 var, units 2^-266; >= 0
+        var[m] = round_rational_to_f32(num, (K * K) << 266)
+    v = (var + e32).astype(np.float32)
+    r = np.sqrt(v).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        d = (x - mean[:, None]).astype(np.float32)
+        t = (d / r[:, None]).astype(np.float32)
+    return {"mean": mean, "var": var, "r": r, "t": t, "xn": round_to_bf16_bits(t)}
+
+
+def forward_layernorm(x_bits: np.ndarray, W: np.ndarray, eps: float = 1e-5, bits: int = 8):
+    """BitLinear on the layer-normalised activations: ``forward(layer_norm(x))``.
+    Same dict as ``forward`` plus mean, var, r and xn."""
+    nrm = layer_norm(x_bits, eps)
+    out = forward(nrm["xn"], W, bits)
+    out.update({k: nrm[k] for k in ("mean", "var", "r", "xn")})
     return out

@@ -747,3 +747,142 @@ def test_round_rational_overflow_boundary():
     assert np.isinf(o.round_rational_to_f32((1 << 128) - (1 << 103), 1))
     assert np.isinf(o.round_rational_to_f32(1 << 128, 1))
     assert np.isinf(o.round_rational_to_f32(3 << 300, 7))
+
+
+# ---------------------------------------------------------------------------
+# LayerNorm (non-affine) ahead of the quantiser: "BitNet b1.58: The 1-Bit
+# Ternary LLM Architecture Guide", BitLinear code listing, forward step 1
+# ---------------------------------------------------------------------------
+
+def _f32_round_signed(fr: Fraction) -> np.float32:
+    """fp32 round-to-nearest-even of a rational (symmetric in the sign)."""
+    v = o.round_rational_to_f32(abs(fr.numerator), fr.denominator)
+    return np.float32(-v) if fr < 0 else v
+
+
+def test_layer_norm_hand_worked_golden():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "layernorm_example.json")) as f:
+        g = json.load(f)
+    xb = to_bf16_bits_exact(np.asarray(g["x"], np.float32))
+    r = o.layer_norm(xb, eps=g["eps"])
+    assert np.array_equal(r["mean"], np.asarray(g["mean"], np.float32))
+    assert np.array_equal(r["var"], np.asarray(g["var"], np.float32))
+    assert np.array_equal(r["xn"], np.asarray(g["xn_bf16_bits"], np.uint16))
+
+
+def test_exact_sum_against_fractions():
+    rng = np.random.default_rng(42)
+    bits = rng.integers(0, 0x7F80, size=900).astype(np.uint16)
+    bits[:50] = rng.integers(0, 0x80, size=50)          # subnormals and zero
+    bits[50:70] = 0
+    bits |= rng.integers(0, 2, size=bits.size).astype(np.uint16) << 15
+    vals = o.bf16_bits_to_f32(bits).astype(np.float64)
+    exact = sum((Fraction(float(v)) for v in vals), Fraction(0))
+    assert Fraction(o.exact_sum(bits), 1 << 133) == exact
+    # cancellation to exactly zero across the whole exponent range
+    both = np.concatenate([bits, bits ^ np.uint16(0x8000)])
+    assert o.exact_sum(both) == 0
+
+
+def test_layer_norm_against_two_pass_fractions():
+    # textbook two-pass definition in exact rationals: mu = sum/K, var =
+    # sum (x - mu)^2 / K; then every fp32 step rounded from its exact value
+    rng = np.random.default_rng(43)
+    for K in (2, 3, 5, 16, 64):
+        x = (rng.standard_normal((3, K)) * np.exp(rng.uniform(-6, 6, size=(3, 1))) + rng.uniform(-4, 4, (3, 1)))
+        xb = _bf16_of(x)
+        eps = 1e-5
+        r = o.layer_norm(xb, eps=eps)
+        xs = o.bf16_bits_to_f32(xb)
+        for m in range(3):
+            fr = [Fraction(float(v)) for v in xs[m]]
+            mu = sum(fr, Fraction(0)) / K
+            var = sum(((v - mu) ** 2 for v in fr), Fraction(0)) / K
+            assert r["mean"][m] == _f32_round_signed(mu)
+            assert r["var"][m] == o.round_rational_to_f32(var.numerator, var.denominator)
+            v32 = _f32_round_signed(Fraction(float(r["var"][m])) + Fraction(float(np.float32(eps))))
+            r32 = np.float32(math.sqrt(float(v32)))   # IEEE sqrt of a double holding an fp32, then rounded
+            assert r["r"][m] == r32
+            for k in range(K):
+                d = _f32_round_signed(fr[k] - Fraction(float(r["mean"][m])))
+                t = _f32_round_signed(Fraction(float(d)) / Fraction(float(r32)))
+                assert r["t"][m, k] == t
+
+
+def test_layer_norm_mean_rounds_once_ties_to_even():
+    # K = 64: 64 and 2^-18 sum to 64 + 2^-18, mean 1 + 2^-24, halfway between
+    # 1 and 1 + 2^-23: ties to even -> 1.  64 + 2^-17 + 2^-18 gives mean
+    # 1 + 3 2^-24, halfway between 1 + 2^-23 and 1 + 2^-22: even -> 1 + 2^-22.
+    # One more entry 2^-100 lifts the first case just above its midpoint
+    # (-> 1 + 2^-23), which a float64 sum would not see.
+    v = np.zeros(64, np.float32)
+    v[0], v[1] = 64.0, 2.0 ** -18
+    assert o.layer_norm(to_bf16_bits_exact(v)[None, :])["mean"][0] == np.float32(1.0)
+    v[2] = 2.0 ** -100
+    assert o.layer_norm(to_bf16_bits_exact(v)[None, :])["mean"][0] == np.float32(1.0 + 2.0 ** -23)
+    assert np.float32(np.sum(v.astype(np.float64)) / 64) == np.float32(1.0)
+    v[1], v[2] = 2.0 ** -17, 2.0 ** -18
+    assert o.layer_norm(to_bf16_bits_exact(v)[None, :])["mean"][0] == np.float32(1.0 + 2.0 ** -22)
+    # negative mirror image
+    assert o.layer_norm(to_bf16_bits_exact(-v)[None, :])["mean"][0] == np.float32(-1.0 - 2.0 ** -22)
+
+
+def test_layer_norm_constant_and_zero_rows():
+    x = to_bf16_bits_exact(np.array([[3.5] * 128, [0.0] * 128, [-2.0 ** 100] * 128], np.float32))
+    r = o.layer_norm(x, eps=0.25)
+    assert np.array_equal(r["var"], np.zeros(3, np.float32))
+    assert r["mean"][0] == np.float32(3.5) and r["mean"][1] == 0.0
+    assert r["mean"][2] == o.bf16_bits_to_f32(x[2:3, 0])[0]
+    assert np.all(r["r"] == np.float32(0.5)) and np.all(r["xn"] == 0)
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(ValueError):
+            o.layer_norm(x, eps=bad)
+
+
+def test_layer_norm_power_of_two_scale_and_integer_shift():
+    rng = np.random.default_rng(44)
+    xb = _bf16_of(rng.standard_normal((4, 320)))
+    base = o.layer_norm(xb, eps=2.0 ** -20)
+    for j in (-9, -1, 3, 12):
+        xs = _bf16_of(o.bf16_bits_to_f32(xb) * np.float32(2.0 ** j))
+        r = o.layer_norm(xs, eps=2.0 ** (-20 + 2 * j))
+        assert np.array_equal(r["mean"], (base["mean"] * np.float32(2.0 ** j)).astype(np.float32))
+        assert np.array_equal(r["var"], (base["var"] * np.float32(4.0 ** j)).astype(np.float32))
+        assert np.array_equal(r["xn"], base["xn"])
+    # integers in [-100, 100] shifted by 64 stay exact in bf16: the exact
+    # variance does not move
+    xi = rng.integers(-100, 101, size=(3, 192)).astype(np.float32)
+    a, b = o.layer_norm(to_bf16_bits_exact(xi)), o.layer_norm(to_bf16_bits_exact(xi + 64.0))
+    assert np.array_equal(a["var"], b["var"])
+
+
+def test_layer_norm_against_torch_float64():
+    # the library's layer_norm in float64 on the same bf16 inputs (biased
+    # variance, eps inside the square root); the oracle's fp32 steps stay
+    # within a few fp32 roundings of it
+    rng = np.random.default_rng(45)
+    M, K = 6, 448
+    x = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-8, 8, size=(M, 1)))
+         + rng.uniform(-3, 3, size=(M, 1)) * np.exp(rng.uniform(-8, 8, size=(M, 1))))
+    x[:, rng.integers(0, K, 4)] *= 30.0
+    xb = _bf16_of(x)
+    eps = 1e-5
+    r = o.layer_norm(xb, eps=eps)
+    x64 = torch.from_numpy(o.bf16_bits_to_f32(xb).astype(np.float64))
+    ref = torch.nn.functional.layer_norm(x64, (K,), eps=float(np.float32(eps))).numpy()
+    mu = np.abs(r["mean"].astype(np.float64))[:, None]
+    rr = r["r"].astype(np.float64)[:, None]
+    tol = 4 * 2.0 ** -24 * ((np.abs(x64.numpy()) + mu) / rr + np.abs(ref))
+    assert np.all(np.abs(r["t"].astype(np.float64) - ref) <= tol)
+    # the unbiased (1/(K-1)) variance is measurably different
+    unb = (x64.numpy() - x64.numpy().mean(1, keepdims=True)) / np.sqrt(x64.numpy().var(1, ddof=1, keepdims=True) + eps)
+    assert np.any(np.abs(r["t"].astype(np.float64) - unb) > tol)
+
+
+def test_forward_layernorm_is_forward_on_the_normalised_input():
+    rng = np.random.default_rng(46)
+    xb = _bf16_of(rng.standard_normal((3, 128)) * 4.0 + 2.0)
+    W = rng.standard_normal((32, 128)).astype(np.float32)
+    got = o.forward_layernorm(xb, W, eps=1e-5, bits=4)
+    ref = o.forward(o.layer_norm(xb, eps=1e-5)["xn"], W, bits=4)
+    assert np.array_equal(got["Y"], ref["Y"]) and np.array_equal(got["q"], ref["q"])
