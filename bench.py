@@ -358,32 +358,55 @@ class FfnWorkload(GpuWorkload):
                             workspace=down["ws"])
 
 
-class RmsWorkload(GpuWorkload):
-    """Every layer of a workload through bl_forward_rmsnorm: RMSNorm with a
-    bf16 weight [K], then the BitLinear forward, one call per layer (one
-    launch for a one-token layer, normalising quantiser + GEMM otherwise)."""
+class NormWorkload(GpuWorkload):
+    """Every layer of a workload with a normalisation ahead of its quantiser:
+    RMSNorm with a bf16 weight [K] per layer, or LayerNorm without parameters.
+    One-token steps issue one bl_forward_norm_grouped call over all layers
+    (one launch); otherwise one bl_forward_rmsnorm / bl_forward_layernorm call
+    per layer (normalising quantiser + GEMM)."""
 
-    def __init__(self, name, rotations, seed=0, device="cuda"):
+    def __init__(self, name, rotations, norm, seed=0, device="cuda"):
         import torch
         from bitlinear_bl_forward_b200 import bl
         super().__init__(name, rotations, seed, device)
+        self.norm = norm
         g = torch.Generator(device=device).manual_seed(seed + 99)
         for d in self.layers:
             L = d["L"]
-            d["nw"] = (torch.rand(L.K, generator=g, device=device) + 0.5).to(torch.bfloat16)
+            d["nw"] = ((torch.rand(L.K, generator=g, device=device) + 0.5).to(torch.bfloat16)
+                       if norm == bl.BL_NORM_RMS else None)
             n = bl.bl_forward_rmsnorm_workspace_bytes(self.w.M, L.K, L.N, self.w.bits)
             d["ws"] = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
-        self.groups = [[i] for i in range(len(self.layers))]
-        self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N) + 2 * d["L"].K for d in self.layers)
-        self.launches_per_step = len(self.layers) * (1 if self.w.M == 1 else 2)
+        self.one_call = self.w.M == 1
+        if self.one_call:
+            probs = [(d["X"], *d["copies"][0], d["L"].N) for d in self.layers]
+            n = bl.bl_forward_norm_grouped_workspace_bytes(probs, self.w.bits)
+            self.gws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+            self.groups = [list(range(len(self.layers)))]
+        else:
+            self.groups = [[i] for i in range(len(self.layers))]
+        # every layer normalises its own copy of the input: a shared X is read per layer
+        self.bytes_per_step = sum(algorithmic_bytes(self.w.M, d["L"].K, d["L"].N)
+                                  + (2 * d["L"].K if norm == bl.BL_NORM_RMS else 0) for d in self.layers)
+        self.launches_per_step = 1 if self.one_call else 2 * len(self.layers)
 
     def step(self, i):
         from bitlinear_bl_forward_b200 import bl
         r = i % self.rotations
+        if self.one_call:
+            bl.bl_forward_norm_grouped([(d["X"], *d["copies"][r], d["L"].N) for d in self.layers], self.norm,
+                                       [d["nw"] for d in self.layers] if self.norm == bl.BL_NORM_RMS else None,
+                                       eps=1e-5, bits=self.w.bits, outs=[d["Y"] for d in self.layers],
+                                       workspace=self.gws)
+            return
         for d in self.layers:
             Wp, gamma = d["copies"][r]
-            bl.bl_forward_rmsnorm(d["X"], Wp, gamma, d["L"].N, self.w.bits, norm_weight=d["nw"], eps=1e-5,
-                                  out=d["Y"], workspace=d["ws"])
+            if self.norm == bl.BL_NORM_RMS:
+                bl.bl_forward_rmsnorm(d["X"], Wp, gamma, d["L"].N, self.w.bits, norm_weight=d["nw"], eps=1e-5,
+                                      out=d["Y"], workspace=d["ws"])
+            else:
+                bl.bl_forward_layernorm(d["X"], Wp, gamma, d["L"].N, self.w.bits, eps=1e-5, out=d["Y"],
+                                        workspace=d["ws"])
 
 
 def time_quantize_weights(N=28672, K=8192, reps=5):
@@ -690,6 +713,9 @@ def secondary(args, ctx, peaks, ipk):
         ms, clocks = time_workload(wl, steps, 3, ctx, sample_clocks=True)
         return ms, clocks
 
+    def nsteps(n):
+        return args.secondary_steps or n
+
     for name, steps in (("prefill_2b", 2000), ("layer_70b_m1", 25000), ("layer_70b_m16", 10000),
                         ("layer_70b_m128", 8000), ("layer_70b_m2048", 800), ("a48", 4000)):
         if want and name not in want:
@@ -699,6 +725,7 @@ def secondary(args, ctx, peaks, ipk):
         wbytes = sum(L.N * L.K // 4 for L in w.layers)
         rot = max(2, min(64, int(math.ceil(256e6 / wbytes))))
         wl = GpuWorkload(name, rot)
+        steps = nsteps(steps)
         ms, clocks = timed(wl, steps)
         sec = ms / 1e3
         gbs = wl.bytes_per_step * steps / sec / 1e9
@@ -712,7 +739,7 @@ def secondary(args, ctx, peaks, ipk):
         # the same 70B-class one-token layer with base-3 weight storage (five
         # weights a byte): compare ms_per_step with layer_70b_m1
         wl = GpuWorkload("layer_70b_m1", 6, fmt="b3")
-        steps = 25000
+        steps = nsteps(25000)
         ms, clocks = timed(wl, steps)
         gbs = wl.bytes_per_step * steps / (ms / 1e3) / 1e9
         out.append({"workload": "layer_70b_m1_base3", "M": 1, "ms_per_step": ms / steps, "GB/s": gbs,
@@ -722,7 +749,7 @@ def secondary(args, ctx, peaks, ipk):
         torch.cuda.empty_cache()
     if not want or "ffn_2b_decode" in want:
         # the decode feed-forward chain (up+gate grouped, then down on the fused squared ReLU)
-        steps = 60000
+        steps = nsteps(60000)
         wl = FfnWorkload(20)
         ms, clocks = timed(wl, steps)
         gbs = wl.bytes_per_step * steps / (ms / 1e3) / 1e9
@@ -731,18 +758,42 @@ def secondary(args, ctx, peaks, ipk):
                     "note": "down input = max(0, gate)^2 * up of the same step, formed in the down kernel"})
         del wl
         torch.cuda.empty_cache()
-    for name, base, steps, rot in (("rmsnorm_decode_2b", "decode_2b", 20000, 20),
-                                   ("rmsnorm_prefill_2b", "prefill_2b", 1200, 20)):
+    if not want or "ffn_prefill_2b" in want:
+        # up and gate of one 4096-token hidden state: one grouped call (one
+        # activation quantisation, one tensor-core launch over both weight
+        # tensors) against two single calls on the same buffers
+        steps = nsteps(2000)
+        res = {}
+        for mode in ("grouped", "two_calls"):
+            wl = GpuWorkload("ffn_prefill_2b", 16)
+            if mode == "two_calls":
+                wl.groups = [[0], [1]]
+            ms, clocks = timed(wl, steps)
+            res[mode] = (ms / steps, clocks, wl.ops_per_step, wl.bytes_per_step)
+            del wl
+            torch.cuda.empty_cache()
+        ms1, clocks, ops, nbytes = res["grouped"]
+        tops = ops / (ms1 / 1e3) / 1e12
+        out.append({"workload": "ffn_prefill_2b", "M": 4096, "ms_per_step": ms1, "TOPS": tops,
+                    "tensor_frac": tops / i8, "GB/s": nbytes / (ms1 / 1e3) / 1e9,
+                    "two_calls_ms_per_step": res["two_calls"][0], "steps": steps, "clocks": clocks,
+                    "note": "up+gate sharing X in one grouped call vs two bl_forward calls"})
+    for name, base, norm, steps, rot in (("rmsnorm_decode_2b", "decode_2b", 0, 20000, 20),
+                                         ("rmsnorm_prefill_2b", "prefill_2b", 0, 1200, 20),
+                                         ("layernorm_decode_2b", "decode_2b", 1, 20000, 20),
+                                         ("layernorm_prefill_2b", "prefill_2b", 1, 1200, 20)):
         if want and name not in want:
             continue
-        # the same layers with RMSNorm (bf16 weight) formed ahead of the quantiser
-        wl = RmsWorkload(base, rot)
+        # the same layers with RMSNorm (bf16 weight) or LayerNorm formed ahead of the quantiser
+        wl = NormWorkload(base, rot, norm)
+        steps = nsteps(steps)
         ms, clocks = timed(wl, steps)
         sec = ms / 1e3
         gbs = wl.bytes_per_step * steps / sec / 1e9
         ent = {"workload": name, "M": wl.w.M, "ms_per_step": ms / steps, "GB/s": gbs,
                "hbm_frac": gbs / peaks["hbm_gbs"], "steps": steps, "clocks": clocks,
-               "note": "one bl_forward_rmsnorm call per layer (norm weight read counted)"}
+               "note": ("one bl_forward_norm_grouped call over the three layers (one launch)" if wl.w.M == 1 else
+                        "one normalised forward call per layer") + ("; norm weight read counted" if norm == 0 else "")}
         if wl.w.M > 1:
             tops = wl.ops_per_step * steps / sec / 1e12
             ent["TOPS"] = tops
@@ -764,6 +815,8 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--secondary", default="", help="comma list restricting the secondary workloads")
+    ap.add_argument("--secondary-steps", type=int, default=0,
+                    help="timed steps of every secondary line (default: each line's own, about 0.3 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
     args = ap.parse_args()

@@ -49,6 +49,11 @@ SIGNATURES = {
     "bl_forward_rmsnorm_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "bl_forward_rmsnorm": (_int, [_p, _p, ctypes.c_float, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_quant_act_rmsnorm": (_int, [_p, _p, ctypes.c_float, _i64, _i64, _int, _p, _p, _p, _p]),
+    "bl_forward_layernorm_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
+    "bl_forward_layernorm": (_int, [_p, ctypes.c_float, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
+    "bl_quant_act_layernorm": (_int, [_p, ctypes.c_float, _i64, _i64, _int, _p, _p, _p, _p, _p]),
+    "bl_forward_norm_grouped_workspace_bytes": (_sz, [_int, _p, _int]),
+    "bl_forward_norm_grouped": (_int, [_int, _p, _int, _p, ctypes.c_float, _int, _p, _sz, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_matmul_i32": (_int, [_p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_device_status": (_int, [_int, ctypes.POINTER(_int)]),
@@ -357,6 +362,82 @@ def bl_quant_act_rmsnorm(X: torch.Tensor, bits: int = 8, norm_weight: torch.Tens
     _check(lib().bl_quant_act_rmsnorm(px, pn, eps, M, K, bits, Xq.data_ptr(), s.data_ptr(), ms.data_ptr(),
                                       _stream()), "bl_quant_act_rmsnorm")
     return Xq, s, ms
+
+
+BL_NORM_RMS = 0
+BL_NORM_LAYER = 1
+
+
+def bl_forward_layernorm_workspace_bytes(M: int, K: int, N: int, bits: int = 8) -> int:
+    return int(lib().bl_forward_layernorm_workspace_bytes(M, K, N, bits))
+
+
+def bl_forward_layernorm(X: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int, bits: int = 8,
+                         eps: float = 1e-5, out: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """bl_forward on LayerNorm(X) (no affine parameters), formed in the same
+    kernels: bf16 [M, K] -> bf16 [M, N]."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    pw = _dev(Wp, torch.uint8, "Wp")
+    pg = _dev(gamma, torch.float32, "gamma")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    py = _dev(Y, torch.bfloat16, "out")
+    ws = workspace
+    if ws is None:
+        ws = _workspace(bl_forward_layernorm_workspace_bytes(M, K, N, bits), X.device)
+    _check(lib().bl_forward_layernorm(px, eps, M, K, N, pw, pg, bits, py,
+                                      ws.data_ptr() if ws is not None else None,
+                                      ws.numel() if ws is not None else 0, _stream()), "bl_forward_layernorm")
+    return Y
+
+
+def bl_quant_act_layernorm(X: torch.Tensor, bits: int = 8, eps: float = 1e-5):
+    """LayerNorm(X) quantised per token -> (int8 codes [M, K], scale fp32 [M],
+    mean fp32 [M], variance fp32 [M])."""
+    M, K = X.shape
+    px = _dev(X, torch.bfloat16, "X")
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    mu = torch.empty(M, dtype=torch.float32, device=X.device)
+    var = torch.empty(M, dtype=torch.float32, device=X.device)
+    _check(lib().bl_quant_act_layernorm(px, eps, M, K, bits, Xq.data_ptr(), s.data_ptr(), mu.data_ptr(),
+                                        var.data_ptr(), _stream()), "bl_quant_act_layernorm")
+    return Xq, s, mu, var
+
+
+def bl_forward_norm_grouped_workspace_bytes(problems, bits: int = 8) -> int:
+    """problems: list of (X, Wp, gamma, N)."""
+    outs = [torch.empty((X.shape[0], N), dtype=torch.bfloat16, device=X.device) for (X, _, _, N) in problems]
+    arr = _grouped_structs(problems, outs)
+    return int(lib().bl_forward_norm_grouped_workspace_bytes(len(problems), arr, bits))
+
+
+def bl_forward_norm_grouped(problems, norm: int, norm_weights=None, eps: float = 1e-5, bits: int = 8, outs=None,
+                            workspace: torch.Tensor | None = None):
+    """Several normalised BitLinear forwards in one call (problems: list of
+    (X bf16 [M, K], Wp, gamma, N); norm BL_NORM_RMS with optional per-problem
+    bf16 weights, or BL_NORM_LAYER); returns the list of bf16 outputs."""
+    if outs is None:
+        outs = [torch.empty((X.shape[0], N), dtype=torch.bfloat16, device=X.device) for (X, _, _, N) in problems]
+    arr = _grouped_structs(problems, outs)
+    wa = None
+    if norm_weights is not None:
+        ptrs = []
+        for (X, _, _, _), w in zip(problems, norm_weights):
+            if w is not None and tuple(w.shape) != (X.shape[1],):
+                raise ValueError("norm weight must be [K]")
+            ptrs.append(_dev(w, torch.bfloat16, "norm_weight") if w is not None else None)
+        wa = (ctypes.c_void_p * len(ptrs))(*ptrs)
+    ws = workspace
+    if ws is None:
+        need = int(lib().bl_forward_norm_grouped_workspace_bytes(len(problems), arr, bits))
+        ws = _workspace(need, problems[0][0].device if problems else "cuda")
+    _check(lib().bl_forward_norm_grouped(len(problems), arr, norm, wa, eps, bits,
+                                         ws.data_ptr() if ws is not None else None,
+                                         ws.numel() if ws is not None else 0, _stream()),
+           "bl_forward_norm_grouped")
+    return outs
 
 
 def bl_matmul_i32(Xq: torch.Tensor, Wp: torch.Tensor, N: int) -> torch.Tensor:

@@ -311,7 +311,7 @@ double dec_cta_cost(int64_t N, int64_t K, int ctas, int a, int fmt, int mode) {
 // fit the ring without reuse when possible; in big mode one group per warp
 // per chunk.  Returns the grid size.
 int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, int mode, int a,
-                      const void* U, const float* bias, float eps, int fmt = bl::kFmt2Bit) {
+                      const void* const* Us, const float* bias, float eps, int fmt = bl::kFmt2Bit) {
   std::memset(tab, 0, sizeof(*tab));
   int64_t rows_total = 0;
   for (int i = 0; i < n; ++i) rows_total += probs[i]->N;
@@ -393,7 +393,7 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
     }
     bl::G2Problem& q = tab->p[i];
     q.X = p.X;
-    q.U = U;
+    q.U = Us ? Us[i] : nullptr;
     q.Wp = p.Wp;
     q.gamma = p.gamma;
     q.Y = p.Y;
@@ -416,12 +416,12 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
 
 // Launch one-token problems (K <= 8192, at most kG2MaxProblems) in one kernel:
 // resident mode when the weights fit the rings of one CTA per SM, big mode
-// otherwise (RMSNorm is formed only in resident mode; callers check the fit).
-// in_mode: bl::InMode of the token input; U: the up projection's output in the
-// gated squared-ReLU mode, or the RMSNorm weight (shared by every problem of
-// the call); eps: the RMSNorm epsilon.
+// otherwise (the normalising prologues exist only in resident mode; callers
+// check the fit).  in_mode: bl::InMode of the token input; Us: per problem,
+// the up projection's output in the gated squared-ReLU mode or the RMSNorm
+// weight (NULL array: none); eps: the normalisation epsilon.
 bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q, int out_mode, cudaStream_t stream,
-                        const void* U = nullptr, const float* bias = nullptr, float eps = 0.f) {
+                        const void* const* Us = nullptr, const float* bias = nullptr, float eps = 0.f) {
   if (n <= 0) return BL_OK;
   const int sms = num_sms();
   double wbytes = 0.0;
@@ -430,11 +430,12 @@ bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q
     wbytes += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / 4.0;
     if (probs[i]->K > maxK) maxK = static_cast<int>(probs[i]->K);
   }
-  const bool big = in_mode != bl::kInRmsNorm && wbytes > static_cast<double>(sms) * bl::kDecRingBytes;
+  const bool norm = in_mode == bl::kInRmsNorm || in_mode == bl::kInLayerNorm;
+  const bool big = !norm && wbytes > static_cast<double>(sms) * bl::kDecRingBytes;
   const int mode = big ? bl::kModeBig : bl::kModeResident;
   const int a = big ? dec_cpl(maxK) : dec_pick_wplr(probs, n);
   bl::G2Table tab;
-  const int grid = fill_decode_table(&tab, probs, n, sms, mode, a, U, bias, eps);
+  const int grid = fill_decode_table(&tab, probs, n, sms, mode, a, Us, bias, eps);
   const bool relu2 = in_mode == bl::kInRelu2 || in_mode == bl::kInRelu2Gated;
   if (big) {
     if (relu2) return launch_dec_big<bl::kDecRelu2>(a, tab, grid, in_mode, Q, out_mode, stream);
@@ -442,6 +443,7 @@ bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q
   }
   if (relu2) return launch_dec_resident<bl::kDecRelu2>(a, tab, grid, in_mode, Q, out_mode, stream);
   if (in_mode == bl::kInRmsNorm) return launch_dec_resident<bl::kDecRms>(a, tab, grid, in_mode, Q, out_mode, stream);
+  if (in_mode == bl::kInLayerNorm) return launch_dec_resident<bl::kDecLn>(a, tab, grid, in_mode, Q, out_mode, stream);
   return launch_dec_resident<bl::kDecPlain>(a, tab, grid, in_mode, Q, out_mode, stream);
 }
 
@@ -1019,7 +1021,8 @@ bl_status bl_forward_relu2(const uint16_t* G, const uint16_t* U, int64_t M, int6
     p.gamma = gamma;
     p.Y = Y;
     const bl_linear* pp = &p;
-    return launch_decode(&pp, 1, U ? bl::kInRelu2Gated : bl::kInRelu2, Q, bl::kOutBF16, stream, U);
+    const void* us[1] = {U};
+    return launch_decode(&pp, 1, U ? bl::kInRelu2Gated : bl::kInRelu2, Q, bl::kOutBF16, stream, us);
   }
   uint8_t* base = static_cast<uint8_t*>(workspace);
   int8_t* Xq = reinterpret_cast<int8_t*>(base);
@@ -1107,11 +1110,72 @@ size_t bl_forward_rmsnorm_workspace_bytes(int64_t M, int64_t K, int64_t N, int b
   return rms_ws_bytes(M, K);
 }
 
+size_t bl_forward_layernorm_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+  return bl_forward_rmsnorm_workspace_bytes(M, K, N, bits);
+}
+
 bool rms_eps_ok(float eps) { return eps > 0.f && std::isfinite(eps); }
 
-bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
-                               int bits, int8_t* Xq, float* scale, float* mean_sq, cudaStream_t stream) {
-  const NvtxRange nvtx_range("bl_quant_act_rmsnorm");
+// The normalising quantiser (one CTA per token): RMSNorm with an optional
+// weight, or LayerNorm.  st0: ms (RMSNorm) or mean (LayerNorm); st1: var.
+bl_status launch_norm_quant(int norm, const uint16_t* X, const uint16_t* w, float eps, int m, int k, int Q,
+                            int8_t* Xq, float* s, int* R, float* st0, float* st1, cudaStream_t stream) {
+  if (norm == BL_NORM_LAYER)
+    bl::bl_act_quant_norm_kernel<bl::kNormLayer><<<static_cast<unsigned>(m), bl::kActRowThreads, 0, stream>>>(
+        X, nullptr, eps, k, Q, Xq, s, R, st0, st1);
+  else
+    bl::bl_act_quant_norm_kernel<bl::kNormRms><<<static_cast<unsigned>(m), bl::kActRowThreads, 0, stream>>>(
+        X, w, eps, k, Q, Xq, s, R, st0, nullptr);
+  return last_cuda();
+}
+
+// Whether one-token problems go through one resident decode launch with the
+// normalising prologue (K <= 8192 each, all weights within the SMs' rings).
+bool norm_decode_fits(const bl_linear* const* probs, int n) {
+  double wbytes = 0.0;
+  for (int i = 0; i < n; ++i) {
+    if (probs[i]->M != 1 || probs[i]->K > bl::kDecMaxK) return false;
+    wbytes += static_cast<double>(probs[i]->N) * static_cast<double>(probs[i]->K) / 4.0;
+  }
+  return wbytes <= static_cast<double>(num_sms()) * bl::kDecRingBytes;
+}
+
+// One normalised BitLinear forward (arguments validated by the caller).
+bl_status forward_norm(int norm, const uint16_t* X, const uint16_t* w, float eps, int64_t M, int64_t K, int64_t N,
+                       const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y, void* workspace,
+                       cudaStream_t stream) {
+  const int Q = bits == 8 ? 127 : 7;
+  bl_linear p;
+  p.X = X;
+  p.M = M;
+  p.K = K;
+  p.N = N;
+  p.Wp = Wp;
+  p.gamma = gamma;
+  p.Y = Y;
+  const bl_linear* pp = &p;
+  if (norm_decode_fits(&pp, 1)) {
+    // one token whose layer fits the resident decode kernel: normalisation,
+    // absmax and quantisation in its prologue (the workspace stays unused)
+    const void* us[1] = {w};
+    return launch_decode(&pp, 1, norm == BL_NORM_LAYER ? bl::kInLayerNorm : bl::kInRmsNorm, Q, bl::kOutBF16, stream,
+                         us, nullptr, eps);
+  }
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const size_t codes = align_up(static_cast<size_t>(M) * K, 256), rows = align_up(static_cast<size_t>(M) * 4, 256);
+  int8_t* Xq = reinterpret_cast<int8_t*>(base);
+  float* s = reinterpret_cast<float*>(base + codes);
+  int* R = reinterpret_cast<int*>(base + codes + rows);
+  bl_status st = launch_norm_quant(norm, X, w, eps, static_cast<int>(M), static_cast<int>(K), Q, Xq, s, R, nullptr,
+                                   nullptr, stream);
+  if (st != BL_OK) return st;
+  return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y,
+                   bl::kOutBF16, stream);
+}
+
+// Shared validation of the normalising quantiser exports.
+bl_status check_norm_quant(const uint16_t* X, const uint16_t* w, float eps, int64_t M, int64_t K, int bits,
+                           const int8_t* Xq, const float* scale, const float* st0, const float* st1) {
   if (K <= 0 || (K % 64) != 0 || K > kMaxK) return BL_ERR_SHAPE;
   bl_status st = check_m(M, K);
   if (st != BL_OK) return st;
@@ -1119,18 +1183,34 @@ bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, f
   if (!rms_eps_ok(eps)) return BL_ERR_INVALID_ARG;
   if (M == 0) return BL_OK;
   if (!X || !Xq || !scale) return BL_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(Xq) || (norm_weight && !aligned16(norm_weight)) ||
-      (reinterpret_cast<uintptr_t>(mean_sq) & 3u))
+  if (!aligned16(X) || !aligned16(Xq) || (w && !aligned16(w)) || (reinterpret_cast<uintptr_t>(st0) & 3u) ||
+      (reinterpret_cast<uintptr_t>(st1) & 3u))
     return BL_ERR_ALIGNMENT;
-  bl::bl_act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
-      X, norm_weight, eps, static_cast<int>(K), bits == 8 ? 127 : 7, Xq, scale, nullptr, mean_sq);
-  return last_cuda();
+  return BL_OK;
 }
 
-bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
-                             int64_t N, const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y,
-                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  const NvtxRange nvtx_range("bl_forward_rmsnorm");
+bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
+                               int bits, int8_t* Xq, float* scale, float* mean_sq, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quant_act_rmsnorm");
+  const bl_status st = check_norm_quant(X, norm_weight, eps, M, K, bits, Xq, scale, mean_sq, nullptr);
+  if (st != BL_OK || M == 0) return st;
+  return launch_norm_quant(BL_NORM_RMS, X, norm_weight, eps, static_cast<int>(M), static_cast<int>(K),
+                           bits == 8 ? 127 : 7, Xq, scale, nullptr, mean_sq, nullptr, stream);
+}
+
+bl_status bl_quant_act_layernorm(const uint16_t* X, float eps, int64_t M, int64_t K, int bits, int8_t* Xq,
+                                 float* scale, float* mean, float* var, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_quant_act_layernorm");
+  const bl_status st = check_norm_quant(X, nullptr, eps, M, K, bits, Xq, scale, mean, var);
+  if (st != BL_OK || M == 0) return st;
+  return launch_norm_quant(BL_NORM_LAYER, X, nullptr, eps, static_cast<int>(M), static_cast<int>(K),
+                           bits == 8 ? 127 : 7, Xq, scale, nullptr, mean, var, stream);
+}
+
+// Shared validation of one normalised forward problem.
+bl_status check_norm_forward(const uint16_t* X, const uint16_t* w, float eps, int64_t M, int64_t K, int64_t N,
+                             const uint8_t* Wp, const float* gamma, int bits, const uint16_t* Y, const void* workspace,
+                             size_t workspace_bytes) {
   bl_status st = check_shape_nk(N, K);
   if (st != BL_OK) return st;
   if ((st = check_m(M, K)) != BL_OK) return st;
@@ -1138,38 +1218,80 @@ bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, flo
   if (!rms_eps_ok(eps)) return BL_ERR_INVALID_ARG;
   if (M == 0) return BL_OK;
   if (!X || !Wp || !gamma || !Y) return BL_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(Wp) || (norm_weight && !aligned16(norm_weight))) return BL_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned16(Wp) || (w && !aligned16(w))) return BL_ERR_ALIGNMENT;
   const size_t need = rms_ws_bytes(M, K);
   if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return BL_ERR_ALIGNMENT;
-  const int Q = bits == 8 ? 127 : 7;
-  const int sms = num_sms();
-  const double wbytes = static_cast<double>(N) * static_cast<double>(K) / 4.0;
-  if (M == 1 && K <= bl::kDecMaxK && wbytes <= static_cast<double>(sms) * bl::kDecRingBytes) {
-    // one token whose layer fits the resident decode kernel: RMSNorm,
-    // absmax and quantisation in its prologue (the workspace stays unused)
-    bl_linear p;
-    p.X = X;
-    p.M = 1;
-    p.K = K;
-    p.N = N;
-    p.Wp = Wp;
-    p.gamma = gamma;
-    p.Y = Y;
-    const bl_linear* pp = &p;
-    return launch_decode(&pp, 1, bl::kInRmsNorm, Q, bl::kOutBF16, stream, norm_weight, nullptr, eps);
+  return BL_OK;
+}
+
+bl_status bl_forward_rmsnorm(const uint16_t* X, const uint16_t* norm_weight, float eps, int64_t M, int64_t K,
+                             int64_t N, const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_rmsnorm");
+  const bl_status st =
+      check_norm_forward(X, norm_weight, eps, M, K, N, Wp, gamma, bits, Y, workspace, workspace_bytes);
+  if (st != BL_OK || M == 0) return st;
+  return forward_norm(BL_NORM_RMS, X, norm_weight, eps, M, K, N, Wp, gamma, bits, Y, workspace, stream);
+}
+
+bl_status bl_forward_layernorm(const uint16_t* X, float eps, int64_t M, int64_t K, int64_t N, const uint8_t* Wp,
+                               const float* gamma, int bits, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_layernorm");
+  const bl_status st = check_norm_forward(X, nullptr, eps, M, K, N, Wp, gamma, bits, Y, workspace, workspace_bytes);
+  if (st != BL_OK || M == 0) return st;
+  return forward_norm(BL_NORM_LAYER, X, nullptr, eps, M, K, N, Wp, gamma, bits, Y, workspace, stream);
+}
+
+size_t bl_forward_norm_grouped_workspace_bytes(int count, const bl_linear* problems, int bits) {
+  (void)bits;
+  if (!problems || count < 0 || count > bl::kG2MaxProblems) return 0;
+  size_t need = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    if (check_shape_nk(p.N, p.K) != BL_OK || check_m(p.M, p.K) != BL_OK) return 0;
+    if (p.M != 0) need = std::max(need, rms_ws_bytes(p.M, p.K));
   }
-  uint8_t* base = static_cast<uint8_t*>(workspace);
-  const size_t codes = align_up(static_cast<size_t>(M) * K, 256), rows = align_up(static_cast<size_t>(M) * 4, 256);
-  int8_t* Xq = reinterpret_cast<int8_t*>(base);
-  float* s = reinterpret_cast<float*>(base + codes);
-  int* R = reinterpret_cast<int*>(base + codes + rows);
-  float* ms = reinterpret_cast<float*>(base + codes + 2 * rows);
-  bl::bl_act_quant_rmsnorm_kernel<<<static_cast<unsigned>(M), bl::kActRowThreads, 0, stream>>>(
-      X, norm_weight, eps, static_cast<int>(K), Q, Xq, s, R, ms);
-  if ((st = last_cuda()) != BL_OK) return st;
-  return launch_tc(Xq, static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), Wp, R, s, gamma, Y,
-                   bl::kOutBF16, stream);
+  return need;
+}
+
+bl_status bl_forward_norm_grouped(int count, const bl_linear* problems, int norm, const uint16_t* const* norm_weights,
+                                  float eps, int bits, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_norm_grouped");
+  if (problems == nullptr) return BL_ERR_INVALID_ARG;
+  if (count < 0 || count > bl::kG2MaxProblems) return BL_ERR_UNSUPPORTED;
+  if (norm != BL_NORM_RMS && norm != BL_NORM_LAYER) return BL_ERR_UNSUPPORTED;
+  if (norm == BL_NORM_LAYER && norm_weights != nullptr) return BL_ERR_INVALID_ARG;
+  // validate everything before launching anything
+  const bl_linear* sel[bl::kG2MaxProblems];
+  const void* us[bl::kG2MaxProblems];
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    const uint16_t* w = norm_weights ? norm_weights[i] : nullptr;
+    const bl_status st = check_norm_forward(static_cast<const uint16_t*>(p.X), w, eps, p.M, p.K, p.N, p.Wp, p.gamma,
+                                            bits, static_cast<const uint16_t*>(p.Y), workspace, workspace_bytes);
+    if (st != BL_OK) return st;
+    if (p.M == 0) continue;
+    sel[n] = &p;
+    us[n++] = w;
+  }
+  if (n == 0) return BL_OK;
+  if (norm_decode_fits(sel, n)) {
+    // every one-token problem of the call in one launch, each CTA normalising
+    // its own problem's token
+    return launch_decode(sel, n, norm == BL_NORM_LAYER ? bl::kInLayerNorm : bl::kInRmsNorm, bits == 8 ? 127 : 7,
+                         bl::kOutBF16, stream, us, nullptr, eps);
+  }
+  for (int i = 0; i < n; ++i) {
+    const bl_linear& p = *sel[i];
+    const bl_status st = forward_norm(norm, static_cast<const uint16_t*>(p.X), static_cast<const uint16_t*>(us[i]),
+                                      eps, p.M, p.K, p.N, p.Wp, p.gamma, bits, static_cast<uint16_t*>(p.Y), workspace,
+                                      stream);
+    if (st != BL_OK) return st;
+  }
+  return BL_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -64,8 +64,10 @@ __device__ __forceinline__ uint2 quant8_bf16(uint4 v, float s, int Q, int& sum) 
 // Scaling Native 1.58-Bit LLMs", section "2. Squared ReLU Activation"):
 // h = max(0, g)^2 of the gate projection's bf16 output g, optionally times the
 // up projection's output u, or bf16 activations RMS-normalised first (the
-// same page, section "3. Sub-Layer Normalization (SubLN)").
-enum InMode : int { kInBF16 = 0, kInI8 = 1, kInRelu2 = 2, kInRelu2Gated = 3, kInRmsNorm = 4 };
+// same page, section "3. Sub-Layer Normalization (SubLN)") or
+// layer-normalised first ("BitNet b1.58: The 1-Bit Ternary LLM Architecture
+// Guide", BitLinear code listing).
+enum InMode : int { kInBF16 = 0, kInI8 = 1, kInRelu2 = 2, kInRelu2Gated = 3, kInRmsNorm = 4, kInLayerNorm = 5 };
 
 // h for 8 consecutive elements (fp32; exact for bf16 g and u).
 __device__ __forceinline__ void relu2_8(uint4 g, uint4 u, bool gated, float (&h)[8]) {

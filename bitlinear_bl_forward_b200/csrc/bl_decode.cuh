@@ -70,10 +70,10 @@ constexpr int kDecBigSmemBytes = kDecBigRingBytes + kDecActBytes;
 constexpr int kDecBigMaxCpl = kDecMaxK / 2048;       // 16-byte chunks a lane
 
 // What the token prologue forms before the quantisation: nothing (bf16
-// activations or int8 codes), the squared-ReLU input, or the RMS-normalised
-// token.  A template parameter so that the plain path carries no code for
-// the others.
-enum DecPre : int { kDecPlain = 0, kDecRelu2 = 1, kDecRms = 2 };
+// activations or int8 codes), the squared-ReLU input, or the RMS- or
+// layer-normalised token.  A template parameter so that the plain path
+// carries no code for the others.
+enum DecPre : int { kDecPlain = 0, kDecRelu2 = 1, kDecRms = 2, kDecLn = 3 };
 // Weight storage: 2 bits a weight, or base 3 (five weights a byte, see
 // bl_weights.cuh).
 enum DecFmt : int { kFmt2Bit = 0, kFmtBase3 = 1 };
@@ -307,6 +307,8 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
   constexpr int CW = kDecWarps;
   constexpr bool RELU2 = PRE == kDecRelu2;
   constexpr bool RMS = PRE == kDecRms;
+  constexpr bool LN = PRE == kDecLn;
+  constexpr bool NORM = RMS || LN;
   constexpr bool B3 = FMT == kFmtBase3;
   constexpr bool BIG = MODE == kModeBig;
   constexpr int RING = BIG ? kDecBigRingBytes : kDecRingBytes;
@@ -335,10 +337,12 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
   __shared__ __align__(16) uint32_t s_red_f[CW];
   __shared__ __align__(8) uint64_t full[kDecMaxSlots], empty[kDecMaxSlots];
   __shared__ int abort_flag;
-  __shared__ unsigned long long s_sq[RMS ? kSqLimbs : 1];
-  __shared__ unsigned long long s_win[RMS ? 2 * CW : 1];
+  __shared__ unsigned long long s_sq[NORM ? kSqLimbs : 1];
+  __shared__ unsigned long long s_win[NORM ? 2 * CW : 1];
   __shared__ uint32_t s_dig[RMS ? kSqLimbs : 1];
-  __shared__ float s_rms;
+  __shared__ unsigned long long s_s1[LN ? kS1Limbs : 1];
+  __shared__ long long s_w1[LN ? CW : 1];
+  __shared__ float s_rms, s_mu;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = B3 ? base3_row_words(K) : (K >> 4);   // 32-bit words of a row
@@ -355,8 +359,11 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
     abort_flag = 0;
     fence_mbar_init();
   }
-  if constexpr (RMS) {
+  if constexpr (NORM) {
     if (threadIdx.x < kSqLimbs) s_sq[threadIdx.x] = 0ull;
+  }
+  if constexpr (LN) {
+    if (threadIdx.x < kS1Limbs) s_s1[threadIdx.x] = 0ull;
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -429,10 +436,11 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
     xv[u] = (c < nchx) ? __ldg(static_cast<const uint4*>(X) + c) : make_uint4(0, 0, 0, 0);
     if constexpr (RELU2) uv[u] = (gated && c < nchx) ? __ldg(static_cast<const uint4*>(Up) + c) : make_uint4(0, 0, 0, 0);
   }
-  if constexpr (RMS) {
-    // exact mean of squares (register windows anchored at the token's
-    // largest exponent, far squares in shared limb counters), then
-    // x_n = bf16(x / sqrt(ms + eps) * w) in place of the token
+  if constexpr (NORM) {
+    // exact mean of squares (RMSNorm) or exact mean and variance
+    // (LayerNorm): register windows anchored at the token's largest
+    // exponent, far values in shared limb counters; then the normalised
+    // bf16 token in place of the input
     float xmax = 0.f;
 #pragma unroll
     for (int u = 0; u < U; ++u)
@@ -448,24 +456,52 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
     }
     const int E = sq_anchor(xb);
     unsigned long long lo = 0ull, hi = 0ull;
+    long long w1 = 0ll;
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (threadIdx.x + CT * u < nchx) sq_add8(xv[u], E, lo, hi, s_sq);
+    for (int u = 0; u < U; ++u) {
+      if (threadIdx.x + CT * u < nchx) {
+        if constexpr (LN)
+          ln_add8(xv[u], E, w1, lo, hi, s_s1, s_sq);
+        else
+          sq_add8(xv[u], E, lo, hi, s_sq);
+      }
+    }
     sq_warp_sum(lo, hi);
+    if constexpr (LN) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) w1 += __shfl_xor_sync(0xffffffffu, w1, o);
+    }
     if (lane == 0) {
       s_win[2 * warp] = lo;
       s_win[2 * warp + 1] = hi;
+      if constexpr (LN) s_w1[warp] = w1;
     }
     named_bar_sync(1, CT);
     if (warp == 0) {
-      const float ms = sq_block_mean(s_win, CW, E, s_sq, s_dig, static_cast<uint32_t>(K), lane);
-      if (lane == 0) s_rms = __fsqrt_rn(__fadd_rn(ms, tab.p[pi].eps));
+      if constexpr (LN) {
+        float mu, var;
+        ln_block_stats(s_w1, s_win, CW, E, s_s1, s_sq, static_cast<uint32_t>(K), lane, mu, var);
+        if (lane == 0) {
+          s_mu = mu;
+          s_rms = __fsqrt_rn(__fadd_rn(var, tab.p[pi].eps));
+        }
+      } else {
+        const float ms = sq_block_mean(s_win, CW, E, s_sq, s_dig, static_cast<uint32_t>(K), lane);
+        if (lane == 0) s_rms = __fsqrt_rn(__fadd_rn(ms, tab.p[pi].eps));
+      }
     }
     named_bar_sync(1, CT);
     const float r = s_rms;
+    if constexpr (LN) {
+      const float mu = s_mu;
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (threadIdx.x + CT * u < nchx) xv[u] = rms_apply8(xv[u], nw[u], has_nw, r);
+      for (int u = 0; u < U; ++u)
+        if (threadIdx.x + CT * u < nchx) xv[u] = ln_apply8(xv[u], mu, r);
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (threadIdx.x + CT * u < nchx) xv[u] = rms_apply8(xv[u], nw[u], has_nw, r);
+    }
   }
   float sc = 1.f;
   if (!x_is_i8) {

@@ -76,6 +76,9 @@ WORKLOADS = {
                                 "70B-class layer, M=2048"),
     "a48": Workload("a48", 2048, (Layer("proj", 4096, 11008),), 0.02, "relu2", 0, 1.0, 4,
                     "a4.8 mode: 4-bit activations, 2048x4096 -> 11008"),
+    # the 2B prefill feed-forward input side: up and gate of one hidden state
+    "ffn_prefill_2b": Workload("ffn_prefill_2b", 4096, (Layer("up", 2560, 6912), Layer("gate", 2560, 6912, x_layer=0)),
+                               0.02, "outliers", "1%", 10.0, 8, "2B-class up+gate prefill, 4096 tokens", ((0, 1),)),
 }
 
 

@@ -308,6 +308,53 @@ BL_API bl_status bl_quant_act_rmsnorm(const uint16_t* X, const uint16_t* norm_we
                                       int64_t K, int bits, int8_t* Xq, float* scale, float* mean_sq,
                                       cudaStream_t stream);
 
+/*
+ * LayerNorm ahead of the quantisation, without affine parameters ("BitNet
+ * b1.58: The 1-Bit Ternary LLM Architecture Guide", BitLinear code listing,
+ * forward step 1: a layer_norm over the feature axis before the activation
+ * quantiser; the "BitNet 2B4T Guide: Scaling Native 1.58-Bit LLMs" BitLinear
+ * module, a LayerNorm with its affine parameters off).  Per token m:
+ *   mu_m   = fp32_rn( (1/K) sum_k X[m,k] )              the sum exact
+ *   var_m  = fp32_rn( (1/K) sum_k (X[m,k] - (1/K) sum_j X[m,j])^2 )
+ *            the biased variance, exact, one rounding
+ *   r_m    = sqrt_rn( f32(var_m + eps) )
+ *   Xn[m,k]= bf16_rn( f32( f32(X[m,k] - mu_m) / r_m ) )
+ * then exactly bl_forward on Xn.  Arguments, workspace
+ * (bl_forward_layernorm_workspace_bytes), errors and ordering as in
+ * bl_forward_rmsnorm (there is no weight).
+ */
+BL_API size_t bl_forward_layernorm_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+BL_API bl_status bl_forward_layernorm(const uint16_t* X, float eps, int64_t M, int64_t K, int64_t N,
+                                      const uint8_t* Wp, const float* gamma, int bits, uint16_t* Y, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream);
+/* Test export: the normalisation and quantisation step of bl_forward_layernorm
+ * alone: codes and scales as bl_quant_act and, when not NULL (4-byte
+ * aligned), mu_m and var_m fp32 [M]. */
+BL_API bl_status bl_quant_act_layernorm(const uint16_t* X, float eps, int64_t M, int64_t K, int bits, int8_t* Xq,
+                                        float* scale, float* mean, float* var, cudaStream_t stream);
+
+/*
+ * Several normalised BitLinear forwards in one call: each problem i is
+ * bl_forward_rmsnorm (norm == BL_NORM_RMS, weight norm_weights[i], which may
+ * be NULL, or norm_weights == NULL for none) or bl_forward_layernorm (norm ==
+ * BL_NORM_LAYER, norm_weights must be NULL) of its own X, with one eps.
+ * When every non-empty problem has one token, K <= 8192, and all weights fit
+ * the resident decode kernel's rings (sum N*K/4 <= SMs * 96 KiB), the whole
+ * group is ONE launch in which every CTA normalises its own problem's token;
+ * otherwise the problems run one after another.  At most 8 problems; no
+ * problem's X may be another's Y.  workspace: at least
+ * bl_forward_norm_grouped_workspace_bytes(count, problems, bits) bytes,
+ * 16-byte aligned, reused by the problems in stream order.  Errors as in
+ * bl_forward_rmsnorm; BL_ERR_UNSUPPORTED for another norm or more than 8
+ * problems.  Nothing is launched unless every problem is valid.
+ */
+#define BL_NORM_RMS 0
+#define BL_NORM_LAYER 1
+BL_API size_t bl_forward_norm_grouped_workspace_bytes(int count, const bl_linear* problems, int bits);
+BL_API bl_status bl_forward_norm_grouped(int count, const bl_linear* problems, int norm,
+                                         const uint16_t* const* norm_weights, float eps, int bits, void* workspace,
+                                         size_t workspace_bytes, cudaStream_t stream);
+
 /* Device workspace bytes bl_matmul_i32 needs (0 when M <= 2). */
 BL_API size_t bl_matmul_i32_workspace_bytes(int64_t M, int64_t K, int64_t N);
 

@@ -23,6 +23,18 @@ int main(void) {
                          (const float*)0x10000, 8, (uint16_t*)0x10000, (void*)0x10000, 1 << 20,
                          (cudaStream_t)0) != BL_ERR_INVALID_ARG)
     bad |= 64;
+  /* LayerNorm: eps must be positive; the grouped form takes no weights */
+  if (bl_forward_layernorm((const uint16_t*)0x10000, -1.0f, 1, 64, 8, (const uint8_t*)0x10000, (const float*)0x10000,
+                           8, (uint16_t*)0x10000, (void*)0x10000, 1 << 20, (cudaStream_t)0) != BL_ERR_INVALID_ARG)
+    bad |= 128;
+  {
+    bl_linear p = {(const uint16_t*)0x10000, 1, 64, 8, (const uint8_t*)0x10000, (const float*)0x10000,
+                   (uint16_t*)0x10000};
+    const uint16_t* w[1] = {(const uint16_t*)0x10000};
+    if (bl_forward_norm_grouped(1, &p, BL_NORM_LAYER, w, 1e-5f, 8, (void*)0x10000, 1 << 20, (cudaStream_t)0) !=
+        BL_ERR_INVALID_ARG)
+      bad |= 256;
+  }
   printf("c abi check: %s (%d)\n", bad ? "FAILED" : "ok", bad);
   return bad ? 1 : 0;
 }

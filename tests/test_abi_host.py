@@ -206,6 +206,48 @@ def test_rmsnorm_validation(L):
     assert L.bl_quant_act_rmsnorm(None, None, 1e-5, 4, 64, 8, A, A, None, None) == INVALID
 
 
+def test_layernorm_validation(L):
+    assert L.bl_forward_layernorm_workspace_bytes(1, 2560, 6912, 8) == L.bl_forward_rmsnorm_workspace_bytes(1, 2560, 6912, 8)
+    assert L.bl_forward_layernorm_workspace_bytes(4, 60, 8, 8) == 0
+    assert L.bl_forward_layernorm(A, 1e-5, 4, 60, 8, A, A, 8, A, A, 1 << 20, None) == SHAPE
+    assert L.bl_forward_layernorm(None, 1e-5, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == INVALID
+    assert L.bl_forward_layernorm(U, 1e-5, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == ALIGN
+    assert L.bl_forward_layernorm(A, 1e-5, 4, 64, 8, A, A, 5, A, A, 1 << 20, None) == UNSUP
+    assert L.bl_forward_layernorm(A, 1e-5, 1, 64, 8, A, A, 8, A, None, 0, None) == WS
+    for bad in (0.0, -1e-5, float("inf"), float("nan")):
+        assert L.bl_forward_layernorm(A, bad, 4, 64, 8, A, A, 8, A, A, 1 << 20, None) == INVALID
+        assert L.bl_quant_act_layernorm(A, bad, 4, 64, 8, A, A, None, None, None) == INVALID
+    assert L.bl_forward_layernorm(None, 1e-5, 0, 64, 8, None, None, 8, None, None, 0, None) == OK
+    assert L.bl_quant_act_layernorm(A, 1e-5, 4, 65, 8, A, A, None, None, None) == SHAPE
+    assert L.bl_quant_act_layernorm(A, 1e-5, 4, 64, 2, A, A, None, None, None) == UNSUP
+    assert L.bl_quant_act_layernorm(A, 1e-5, 4, 64, 8, A, A, A + 2, None, None) == ALIGN    # mean misaligned
+    assert L.bl_quant_act_layernorm(A, 1e-5, 4, 64, 8, A, A, None, A + 1, None) == ALIGN    # var misaligned
+    assert L.bl_quant_act_layernorm(None, 1e-5, 4, 64, 8, A, A, None, None, None) == INVALID
+
+
+def test_norm_grouped_validation(L):
+    import ctypes
+    from bitlinear_bl_forward_b200.bl import BLLinear
+    arr = (BLLinear * 9)()
+    for i in range(9):
+        arr[i] = BLLinear(A, 1, 256, 64, A, A, A)
+    ws = L.bl_forward_norm_grouped_workspace_bytes(3, arr, 8)
+    assert ws >= 256
+    assert L.bl_forward_norm_grouped_workspace_bytes(9, arr, 8) == 0
+    assert L.bl_forward_norm_grouped(9, arr, 0, None, 1e-5, 8, A, 1 << 20, None) == UNSUP     # > 8 problems
+    assert L.bl_forward_norm_grouped(3, arr, 2, None, 1e-5, 8, A, 1 << 20, None) == UNSUP     # unknown norm
+    w = (ctypes.c_void_p * 3)(A, A, A)
+    assert L.bl_forward_norm_grouped(3, arr, 1, w, 1e-5, 8, A, 1 << 20, None) == INVALID      # LayerNorm has no weight
+    assert L.bl_forward_norm_grouped(3, arr, 0, None, 0.0, 8, A, 1 << 20, None) == INVALID    # eps
+    assert L.bl_forward_norm_grouped(3, arr, 0, None, 1e-5, 8, None, 0, None) == WS
+    assert L.bl_forward_norm_grouped(3, None, 0, None, 1e-5, 8, A, 1 << 20, None) == INVALID
+    wu = (ctypes.c_void_p * 3)(A, U, A)
+    assert L.bl_forward_norm_grouped(3, arr, 0, wu, 1e-5, 8, A, 1 << 20, None) == ALIGN       # misaligned weight
+    arr[2] = BLLinear(A, 1, 100, 64, A, A, A)
+    assert L.bl_forward_norm_grouped(3, arr, 1, None, 1e-5, 8, A, 1 << 20, None) == SHAPE     # bad third problem
+    assert L.bl_forward_norm_grouped(0, arr, 1, None, 1e-5, 8, None, 0, None) == OK
+
+
 def test_base3_host_checks(L):
     # sizes: 4 * ceil(ceil(K / 20) / 4) bytes a row
     assert L.bl_packed_weight_bytes_b3(1, 64) == 16

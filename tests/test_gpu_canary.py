@@ -74,6 +74,10 @@ def test_forward_writes_stay_in_bounds(M, K, N):
     nw = torch.rand(K, device="cuda").to(torch.bfloat16)
     bl.bl_forward_rmsnorm(x_to_dev(X), Wp, g, N, norm_weight=nw, out=Y4.t, workspace=ws4.t)
     assert Y4.intact() and ws4.intact()
+    Y5 = Guarded((M, N), torch.bfloat16)
+    ws5 = Guarded((bl.bl_forward_layernorm_workspace_bytes(M, K, N),), torch.uint8)
+    bl.bl_forward_layernorm(x_to_dev(X), Wp, g, N, out=Y5.t, workspace=ws5.t)
+    assert Y5.intact() and ws5.intact()
 
 
 def test_grouped_writes_stay_in_bounds():
@@ -85,6 +89,12 @@ def test_grouped_writes_stay_in_bounds():
         outs.append(Guarded((1, N), torch.bfloat16))
     bl.bl_forward_grouped(probs, outs=[o.t for o in outs])
     assert all(o.intact() for o in outs)
+    for norm in (bl.BL_NORM_RMS, bl.BL_NORM_LAYER):
+        outs = [Guarded((1, N), torch.bfloat16) for (_, _, _, N) in probs]
+        nws = [torch.rand(X.shape[1], device="cuda").to(torch.bfloat16) for (X, _, _, _) in probs] \
+            if norm == bl.BL_NORM_RMS else None
+        bl.bl_forward_norm_grouped(probs, norm, nws, outs=[o.t for o in outs])
+        assert all(o.intact() for o in outs)
 
 
 @pytest.mark.parametrize("M,K", [(1, 64), (5, 192), (9, 6912), (3, 16384)])
@@ -107,6 +117,13 @@ def test_quantisers_write_in_bounds(M, K):
         bl.lib().bl_quant_act_rmsnorm(x_to_dev(X).data_ptr(), None, 1e-5, M, K, bits, Xn.t.data_ptr(),
                                       sn.t.data_ptr(), ms.t.data_ptr(), torch.cuda.current_stream().cuda_stream)
         assert Xn.intact() and sn.intact() and ms.intact()
+        Xl = Guarded((M, K), torch.int8)
+        sl = Guarded((M,), torch.float32)
+        mu = Guarded((M,), torch.float32)
+        var = Guarded((M,), torch.float32)
+        bl.lib().bl_quant_act_layernorm(x_to_dev(X).data_ptr(), 1e-5, M, K, bits, Xl.t.data_ptr(), sl.t.data_ptr(),
+                                        mu.t.data_ptr(), var.t.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert Xl.intact() and sl.intact() and mu.intact() and var.intact()
 
 
 @pytest.mark.parametrize("N,K", [(1, 64), (33, 192), (700, 2560), (130, 6912)])

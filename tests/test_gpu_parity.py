@@ -582,6 +582,141 @@ def test_forward_rmsnorm_bits4_zero_rows_and_back_to_back():
 
 
 # ---------------------------------------------------------------------------
+# LayerNorm before the quantisation ("BitNet b1.58: The 1-Bit Ternary LLM
+# Architecture Guide", BitLinear code listing, forward step 1)
+# ---------------------------------------------------------------------------
+
+def bf16_bits_of(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def check_quant_layernorm(X, eps, bits):
+    nrm = o.layer_norm(X, eps)
+    q, s = o.act_quant(nrm["xn"], bits)
+    qd, sd, mud, vard = bl.bl_quant_act_layernorm(x_to_dev(X), bits, eps)
+    assert np.array_equal(mud.cpu().numpy().view(np.uint32), nrm["mean"].view(np.uint32))
+    assert np.array_equal(vard.cpu().numpy().view(np.uint32), nrm["var"].view(np.uint32))
+    assert np.array_equal(sd.cpu().numpy().view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(qd.cpu().numpy(), q)
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (3, 192), (16, 2560), (5, 6912), (2, 8192), (2, 20480), (1, 65536)])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_quant_act_layernorm_bit_exact(M, K, bits):
+    # per-row offsets make the mean matter next to the spread
+    X, _ = random_case(M, K, 8, seed=M * 19 + K)
+    off = np.random.default_rng(K + M).uniform(-6, 6, size=(M, 1))
+    X = bf16_bits_of(o.bf16_bits_to_f32(X) + off)
+    check_quant_layernorm(X, 1e-5, bits)
+
+
+def test_quant_act_layernorm_hard_sums():
+    rng = np.random.default_rng(2025)
+    K = 2560
+    rows = []
+    rows.append(rng.integers(0, 0x7F80, K).astype(np.uint16))              # every exponent: far terms
+    x = rng.standard_normal(K).astype(np.float32) + 3.0
+    x[rng.integers(0, K, K // 3)] *= 1e-25                                 # a third far below the rest
+    rows.append((x.view(np.uint32) >> 16).astype(np.uint16))
+    rows.append(rng.integers(0x2000, 0x5F00, K).astype(np.uint16))         # 2^-63 .. 2^63
+    rows.append(rng.integers(0x1A00, 0x2000, K).astype(np.uint16))         # 2^-75 .. 2^-63: subnormal var
+    rows.append(rng.integers(0, 0x100, K).astype(np.uint16))               # bf16 subnormals: subnormal mean
+    big = np.zeros(K, np.uint16)
+    big[[3, 900]] = 0x7149                                                 # ~1e30: var overflows to inf
+    rows.append(big)
+    rows.append(np.zeros(K, np.uint16))                                    # zero row
+    rows.append(np.full(K, 0x4060, np.uint16))                             # constant 3.5: var 0
+    near = np.full(K, 0x4060, np.uint16)
+    near[7] = 0x4061                                                       # one value one step away
+    rows.append(near)
+    X = np.stack(rows)
+    X[:5] |= (rng.integers(0, 2, (5, K)).astype(np.uint16) << 15)
+    for eps in (1e-5, 1e-30):
+        check_quant_layernorm(X, eps, 8)
+    # exact fp32 midpoints of the mean (ties to even), and just above one
+    v = np.zeros((3, 128), np.float32)
+    v[:, 0] = v[:, 1] = 64.0
+    v[:2, 2] = 2.0 ** -17                                                  # sum 128 + 2^-17, K = 128:
+    #                                                                        mean 1 + 2^-24, a tie -> 1
+    v[1, 3] = 2.0 ** -100                                                  # just above -> 1 + 2^-23
+    v[2, 2], v[2, 3] = 2.0 ** -16, 2.0 ** -17                              # mean 1 + 3 2^-24: tie -> 1 + 2^-22
+    Xm = (v.view(np.uint32) >> 16).astype(np.uint16)
+    check_quant_layernorm(Xm, 2.0 ** -40, 8)
+    _, _, mud, _ = bl.bl_quant_act_layernorm(x_to_dev(Xm), 8, 2.0 ** -40)
+    assert mud.cpu().numpy().tolist() == [1.0, 1.0 + 2.0 ** -23, 1.0 + 2.0 ** -22]
+
+
+@pytest.mark.parametrize("M,K,N", RMS_CASES)
+def test_forward_layernorm_parity(M, K, N):
+    # one token with a layer that fits the resident decode kernel: LayerNorm
+    # in its prologue; otherwise the normalising quantiser + the tensor-core GEMM
+    X, W = random_case(M, K, N, seed=M * 5 + K + N)
+    X = bf16_bits_of(o.bf16_bits_to_f32(X) + np.float32(1.5))
+    ref = o.forward_layernorm(X, W, 1e-5)
+    Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+    Yd = bf16_dev_to_bits(bl.bl_forward_layernorm(x_to_dev(X), Wp, gd, N, eps=1e-5))
+    d = bf16_ulp_distance(Yd, ref["Y"])
+    assert d.max() <= BF16_ULP_TOL, f"bf16 ulp distance {d.max()}"
+    assert np.mean(d == 0) > 0.99
+    Y2 = bf16_dev_to_bits(bl.bl_forward(x_to_dev(ref["xn"]), Wp, gd, N))
+    assert np.array_equal(Yd, Y2)
+
+
+@pytest.mark.parametrize("norm", ["rms", "layer"])
+def test_norm_grouped_decode_one_launch(norm):
+    # the 2B decode step with a normalisation ahead of every projection, one
+    # launch: up and gate read the same X, down its own; RMSNorm weights
+    # differ per problem; bits 8 and 4
+    w = WORKLOADS["decode_2b"]
+    probs, cases, nws = [], [], []
+    xs = {}
+    for i, L in enumerate(w.layers):
+        X, _ = layer_inputs(w, i)
+        key = L.x_layer if L.x_layer >= 0 else i
+        if key not in xs:
+            xs[key] = (X, x_to_dev(X))
+        Xh, Xd = xs[key]
+        W, g, c, _ = oracle_weights(("decode_2b", i))
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        probs.append((Xd, Wp, gd, W.shape[0]))
+        wb = norm_weight_bits(L.K, 31 + i) if norm == "rms" else None
+        nws.append(x_to_dev(wb) if wb is not None else None)
+        cases.append((Xh, W, wb))
+    kind = bl.BL_NORM_RMS if norm == "rms" else bl.BL_NORM_LAYER
+    for bits in (8, 4):
+        if norm == "rms":
+            singles = [bl.bl_forward_rmsnorm(Xd, Wp, gd, N, bits, norm_weight=nw) for (Xd, Wp, gd, N), nw in
+                       zip(probs, nws)]
+        else:
+            singles = [bl.bl_forward_layernorm(Xd, Wp, gd, N, bits) for (Xd, Wp, gd, N) in probs]
+        outs = bl.bl_forward_norm_grouped(probs, kind, nws if norm == "rms" else None, bits=bits)
+        outs = bl.bl_forward_norm_grouped(probs, kind, nws if norm == "rms" else None, bits=bits, outs=outs)
+        torch.cuda.synchronize()
+        for (Xh, W, wb), a, b in zip(cases, outs, singles):
+            assert torch.equal(a, b)
+            ref = o.forward_rmsnorm(Xh, W, wb, 1e-5, bits) if norm == "rms" else o.forward_layernorm(Xh, W, 1e-5, bits)
+            assert bf16_ulp_distance(bf16_dev_to_bits(a), ref["Y"]).max() <= BF16_ULP_TOL
+
+
+def test_norm_grouped_sequential_shapes():
+    # problems that do not fit one decode launch (several tokens, long rows)
+    cases = [(3, 256, 300), (1, 16384, 64), (1, 2560, 700), (0, 64, 8), (130, 512, 264)]
+    for kind in (bl.BL_NORM_RMS, bl.BL_NORM_LAYER):
+        probs, singles = [], []
+        for j, (M, K, N) in enumerate(cases):
+            X, W = random_case(M, K, N, seed=600 + j)
+            Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+            Xd = x_to_dev(X) if M > 0 else torch.zeros((0, K), dtype=torch.bfloat16, device="cuda")
+            probs.append((Xd, Wp, gd, N))
+            singles.append(bl.bl_forward_rmsnorm(Xd, Wp, gd, N) if kind == bl.BL_NORM_RMS
+                           else bl.bl_forward_layernorm(Xd, Wp, gd, N))
+        outs = bl.bl_forward_norm_grouped(probs, kind)
+        torch.cuda.synchronize()
+        for a, b in zip(outs, singles):
+            assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
 # packed 4-bit activations ("BitNet a4.8 Guide: 4-Bit Activation 1-Bit LLMs",
 # section "Step 4: Verification and Benchmarking Test Harness")
 # ---------------------------------------------------------------------------
