@@ -455,17 +455,15 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
       xb = max(xb, max(max(v.x, v.y), max(v.z, v.w)));
     }
     const int E = sq_anchor(xb);
+    const float thr = norm_thr(E);
     unsigned long long lo = 0ull, hi = 0ull;
     long long w1 = 0ll;
+    double p1 = 0.0, p2 = 0.0;
+    static_assert(8 * U <= kNormFlush, "one flush per thread");
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (threadIdx.x + CT * u < nchx) {
-        if constexpr (LN)
-          ln_add8(xv[u], E, w1, lo, hi, s_s1, s_sq);
-        else
-          sq_add8(xv[u], E, lo, hi, s_sq);
-      }
-    }
+    for (int u = 0; u < U; ++u)
+      if (threadIdx.x + CT * u < nchx) norm_add8<LN>(xv[u], E, thr, p1, p2, w1, lo, hi, s_s1, s_sq);
+    norm_flush<LN>(E, p1, p2, w1, hi);
     sq_warp_sum(lo, hi);
     if constexpr (LN) {
 #pragma unroll

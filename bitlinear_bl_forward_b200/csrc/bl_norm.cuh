@@ -86,16 +86,6 @@ __device__ __forceinline__ void sq_add1(uint32_t b, int E, unsigned long long& l
   }
 }
 
-__device__ __forceinline__ void sq_add8(uint4 v, int E, unsigned long long& lo, unsigned long long& hi,
-                                        unsigned long long* acc) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    sq_add1(w[i] & 0xffffu, E, lo, hi, acc);
-    sq_add1(w[i] >> 16, E, lo, hi, acc);
-  }
-}
-
 // Warp sum of the 128-bit windows: every lane holds the total afterwards.
 __device__ __forceinline__ void sq_warp_sum(unsigned long long& lo, unsigned long long& hi) {
 #pragma unroll
@@ -267,17 +257,55 @@ __device__ __forceinline__ void s1_add1(uint32_t b, int E, long long& w1, unsign
   atomicAdd(&acc1[P >> 5], static_cast<unsigned long long>(v * (1ll << (P & 31))));
 }
 
-// Eight bf16 values into both windows (sum and sum of squares).
-__device__ __forceinline__ void ln_add8(uint4 v, int E, long long& w1, unsigned long long& lo, unsigned long long& hi,
-                                        unsigned long long* acc1, unsigned long long* acc2) {
+// ---------------------------------------------------------------------------
+// Per-thread accumulation.  A value x of exponent field e' >= max(E - 16, 1)
+// (|x| >= norm_thr(E)) goes into fp64 partial sums p1 = sum x (LayerNorm)
+// and p2 = sum x^2, which are exact: such an x is a multiple of
+// u1 = 2^(E - 150) below 2^(E - 126), so x is below 2^24 u1 and x^2 a multiple
+// of u2 = 2^(2E - 300) below 2^48 u2; up to kNormFlush values keep both sums
+// below 2^53 units.  norm_flush then moves them, exactly, into the integer
+// windows: p1 / u1 is an integer, times 2^22 in the window's unit
+// 2^(E - 172); p2 / u2 is an integer in units of 2^64 of the squares'
+// window (its high word).  Values further down (and zeros) take
+// s1_add1 / sq_add1.
+// ---------------------------------------------------------------------------
+
+constexpr int kNormFlush = 32;          // values between two flushes at most
+
+__device__ __forceinline__ float norm_thr(int E) { return __uint_as_float(static_cast<uint32_t>(max(E - 16, 1)) << 23); }
+
+// Eight bf16 values into the accumulators (p1, w1 and acc1: LayerNorm only).
+template <bool LN>
+__device__ __forceinline__ void norm_add8(uint4 v, int E, float thr, double& p1, double& p2, long long& w1,
+                                          unsigned long long& lo, unsigned long long& hi, unsigned long long* acc1,
+                                          unsigned long long* acc2) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    s1_add1(w[i] & 0xffffu, E, w1, acc1);
-    s1_add1(w[i] >> 16, E, w1, acc1);
-    sq_add1(w[i] & 0xffffu, E, lo, hi, acc2);
-    sq_add1(w[i] >> 16, E, lo, hi, acc2);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t xu = (i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16);   // fp32 bits of the value
+    if (fabsf(__uint_as_float(xu)) >= thr) {
+      // the fp64 value from the fp32 bits of a normal number (exact)
+      const double xd = __hiloint2double(static_cast<int>((xu & 0x80000000u) | (((xu & 0x7fffffffu) >> 3) + 0x38000000u)), 0);
+      if constexpr (LN) p1 += xd;
+      p2 = fma(xd, xd, p2);
+    } else {
+      if constexpr (LN) s1_add1(xu >> 16, E, w1, acc1);
+      sq_add1(xu >> 16, E, lo, hi, acc2);
+    }
   }
+}
+
+// Move the fp64 partial sums into the integer windows (exact) and reset them.
+template <bool LN>
+__device__ __forceinline__ void norm_flush(int E, double& p1, double& p2, long long& w1, unsigned long long& hi) {
+  if constexpr (LN) {
+    const double s1 = __hiloint2double((150 - E + 1023) << 20, 0);        // 1 / u1
+    w1 += __double2ll_rn(p1 * s1) * (1ll << 22);
+    p1 = 0.0;
+  }
+  const double s2 = __hiloint2double((300 - 2 * E + 1023) << 20, 0);      // 1 / u2
+  hi += __double2ull_rn(p2 * s2);
+  p2 = 0.0;
 }
 
 // Exact route (one thread): mu and var from the counters.
@@ -454,8 +482,10 @@ enum NormKind : int { kNormRms = 0, kNormLayer = 1 };
 // quantisation of the normalised bf16 row: one CTA per token.  st0: optional
 // fp32 [M] mean of squares (RMSNorm) or mean (LayerNorm); st1: optional fp32
 // [M] variance (LayerNorm).
+constexpr int kNormCache = 4;   // 16-byte chunks a thread keeps in registers (K <= 8192)
+
 template <int NORM>
-__global__ void __launch_bounds__(kActRowThreads) bl_act_quant_norm_kernel(
+__global__ void __launch_bounds__(kActRowThreads, 4) bl_act_quant_norm_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wn, float eps, int K, int Q,
     int8_t* __restrict__ Xq, float* __restrict__ s_out, int* __restrict__ R_out, float* __restrict__ st0,
     float* __restrict__ st1) {
@@ -479,17 +509,17 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_norm_kernel(
   const uint4* wr = reinterpret_cast<const uint4*>(Wn);
   const bool has_w = !LN && Wn != nullptr;
   const int nch = K >> 3;
-  uint4 cache[kActRowCache];
+  uint4 cache[kNormCache];
   float xmax = 0.f;
 #pragma unroll
-  for (int i = 0; i < kActRowCache; ++i) {
+  for (int i = 0; i < kNormCache; ++i) {
     const int c = t + kActRowThreads * i;
     if (c < nch) {
       cache[i] = __ldg(xr + c);
       xmax = fmaxf(xmax, absmax8_bf16(cache[i]));
     }
   }
-  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+  for (int c = t + kActRowThreads * kNormCache; c < nch; c += kActRowThreads)
     xmax = fmaxf(xmax, absmax8_bf16(__ldg(xr + c)));
   const uint32_t wmax_x = __reduce_max_sync(0xffffffffu, __float_as_uint(xmax));
   if (lane == 0) s_max[warp] = wmax_x;
@@ -498,24 +528,26 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_norm_kernel(
 #pragma unroll
   for (int w = 0; w < W; ++w) xb = max(xb, s_max[w]);
   const int E = sq_anchor(xb);
+  const float thr = norm_thr(E);
   unsigned long long lo = 0ull, hi = 0ull;
   long long w1 = 0ll;
+  double p1 = 0.0, p2 = 0.0;
+  static_assert(kNormFlush % 8 == 0 && kNormCache % (kNormFlush / 8) == 0, "flush on chunk boundaries");
 #pragma unroll
-  for (int i = 0; i < kActRowCache; ++i) {
+  for (int i = 0; i < kNormCache; ++i) {
     const int c = t + kActRowThreads * i;
-    if (c < nch) {
-      if constexpr (LN)
-        ln_add8(cache[i], E, w1, lo, hi, s_s1, s_sq);
-      else
-        sq_add8(cache[i], E, lo, hi, s_sq);
+    if (c < nch) norm_add8<LN>(cache[i], E, thr, p1, p2, w1, lo, hi, s_s1, s_sq);
+    if ((i + 1) % (kNormFlush / 8) == 0) norm_flush<LN>(E, p1, p2, w1, hi);
+  }
+  int nf = 0;
+  for (int c = t + kActRowThreads * kNormCache; c < nch; c += kActRowThreads) {
+    norm_add8<LN>(__ldg(xr + c), E, thr, p1, p2, w1, lo, hi, s_s1, s_sq);
+    if (++nf == kNormFlush / 8) {
+      norm_flush<LN>(E, p1, p2, w1, hi);
+      nf = 0;
     }
   }
-  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads) {
-    if constexpr (LN)
-      ln_add8(__ldg(xr + c), E, w1, lo, hi, s_s1, s_sq);
-    else
-      sq_add8(__ldg(xr + c), E, lo, hi, s_sq);
-  }
+  norm_flush<LN>(E, p1, p2, w1, hi);
   sq_warp_sum(lo, hi);
   if constexpr (LN) {
 #pragma unroll
@@ -557,14 +589,14 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_norm_kernel(
   };
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < kActRowCache; ++i) {
+  for (int i = 0; i < kNormCache; ++i) {
     const int c = t + kActRowThreads * i;
     if (c < nch) {
       cache[i] = apply(cache[i], c);
       amax = fmaxf(amax, absmax8_bf16(cache[i]));
     }
   }
-  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+  for (int c = t + kActRowThreads * kNormCache; c < nch; c += kActRowThreads)
     amax = fmaxf(amax, absmax8_bf16(apply(__ldg(xr + c), c)));
   const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
   if (lane == 0) s_max[warp] = wmax;
@@ -576,11 +608,11 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_norm_kernel(
   uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
   int sum = 0;
 #pragma unroll
-  for (int i = 0; i < kActRowCache; ++i) {
+  for (int i = 0; i < kNormCache; ++i) {
     const int c = t + kActRowThreads * i;
     if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
   }
-  for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
+  for (int c = t + kActRowThreads * kNormCache; c < nch; c += kActRowThreads)
     qr[c] = quant8_bf16(apply(__ldg(xr + c), c), s, Q, sum);
   const int wsum = __reduce_add_sync(0xffffffffu, sum);
   if (lane == 0) s_sum[warp] = wsum;
