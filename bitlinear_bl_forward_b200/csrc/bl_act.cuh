@@ -24,36 +24,34 @@ namespace bl {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-__device__ __forceinline__ float absmax8_bf16(uint4 v) {
-  float a = fabsf(bf16_lo(v.x));
-  a = fmaxf(a, fabsf(bf16_hi(v.x)));
-  a = fmaxf(a, fabsf(bf16_lo(v.y)));
-  a = fmaxf(a, fabsf(bf16_hi(v.y)));
-  a = fmaxf(a, fabsf(bf16_lo(v.z)));
-  a = fmaxf(a, fabsf(bf16_hi(v.z)));
-  a = fmaxf(a, fabsf(bf16_lo(v.w)));
-  a = fmaxf(a, fabsf(bf16_hi(v.w)));
-  return a;
+// max |x| of 8 bf16 as a pair of 16-bit magnitudes (non-negative bf16 bit
+// patterns order like their values): accumulate with __vmaxu2, convert once
+// with absmax2_f32.
+__device__ __forceinline__ uint32_t absmax2_bf16x8(uint4 v) {
+  constexpr uint32_t m = 0x7fff7fffu;
+  return __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+}
+__device__ __forceinline__ float absmax2_f32(uint32_t a2) { return __uint_as_float(max(a2 & 0xffffu, a2 >> 16) << 16); }
+__device__ __forceinline__ float absmax8_bf16(uint4 v) { return absmax2_f32(absmax2_bf16x8(v)); }
+
+// Four codes q = rint(x * s) (fp32 product, round half to even) as the bytes
+// of one word.  x * s + 1.5 * 2^23 lies in [2^23, 2^24), where the spacing
+// is 1, so its bit pattern is 0x4B400000 + rint(x * s) and its low byte is
+// the code.  No clamp is needed: with a = max|x| and s = RN(Q / max(a, eps)),
+// |x * s| <= Q (1 + 2^-24), whose fp32 rounding is at most one ulp above Q
+// (Q = 7 or 127), so |q| <= Q and -Q-1 is never reached.
+__device__ __forceinline__ uint32_t codes4(float a, float b, float c, float d, float s) {
+  const uint32_t qa = __float_as_uint(__fadd_rn(__fmul_rn(a, s), 12582912.0f));
+  const uint32_t qb = __float_as_uint(__fadd_rn(__fmul_rn(b, s), 12582912.0f));
+  const uint32_t qc = __float_as_uint(__fadd_rn(__fmul_rn(c, s), 12582912.0f));
+  const uint32_t qd = __float_as_uint(__fadd_rn(__fmul_rn(d, s), 12582912.0f));
+  return __byte_perm(__byte_perm(qa, qb, 0x0040), __byte_perm(qc, qd, 0x0040), 0x5410);
 }
 
-__device__ __forceinline__ int rint_small(float v) {
-  return __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
-}
-
-__device__ __forceinline__ uint32_t quant1(float x, float s, int Q) {
-  int q = rint_small(__fmul_rn(x, s));
-  q = q < -Q - 1 ? -Q - 1 : (q > Q ? Q : q);
-  return static_cast<uint32_t>(q) & 0xffu;
-}
-
-// 8 bf16 -> 8 int8 codes (as two 32-bit words) and their sum.
-__device__ __forceinline__ uint2 quant8_bf16(uint4 v, float s, int Q, int& sum) {
-  const uint32_t b0 = quant1(bf16_lo(v.x), s, Q), b1 = quant1(bf16_hi(v.x), s, Q);
-  const uint32_t b2 = quant1(bf16_lo(v.y), s, Q), b3 = quant1(bf16_hi(v.y), s, Q);
-  const uint32_t b4 = quant1(bf16_lo(v.z), s, Q), b5 = quant1(bf16_hi(v.z), s, Q);
-  const uint32_t b6 = quant1(bf16_lo(v.w), s, Q), b7 = quant1(bf16_hi(v.w), s, Q);
-  const uint32_t lo = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-  const uint32_t hi = b4 | (b5 << 8) | (b6 << 16) | (b7 << 24);
+// 8 bf16 -> 8 int8 codes (two 32-bit words), their sum added to `sum`.
+__device__ __forceinline__ uint2 quant8_bf16(uint4 v, float s, int& sum) {
+  const uint32_t lo = codes4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), s);
+  const uint32_t hi = codes4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w), s);
   sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
   sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
   return make_uint2(lo, hi);
@@ -92,13 +90,9 @@ __device__ __forceinline__ float absmax8_f32(const float (&h)[8]) {
   return a;
 }
 
-// 8 fp32 values -> 8 codes (two 32-bit words) and their sum.
-__device__ __forceinline__ uint2 quant8_f32(const float (&h)[8], float s, int Q, int& sum) {
-  uint32_t b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) b[i] = quant1(h[i], s, Q);
-  const uint32_t lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  const uint32_t hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+// 8 fp32 values -> 8 codes (two 32-bit words), their sum added to `sum`.
+__device__ __forceinline__ uint2 quant8_f32(const float (&h)[8], float s, int& sum) {
+  const uint32_t lo = codes4(h[0], h[1], h[2], h[3], s), hi = codes4(h[4], h[5], h[6], h[7], s);
   sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
   sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
   return make_uint2(lo, hi);
@@ -129,26 +123,26 @@ __global__ void __launch_bounds__(256) bl_act_quant_kernel(const uint16_t* __res
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
   const int nch = K >> 3;
   uint4 cache[kActCache];
-  float amax = 0.f;
+  uint32_t a2 = 0u;
 #pragma unroll
   for (int i = 0; i < kActCache; ++i) {
     const int c = lane + 32 * i;
     if (c < nch) {
       cache[i] = __ldg(xr + c);
-      amax = fmaxf(amax, absmax8_bf16(cache[i]));
+      a2 = __vmaxu2(a2, absmax2_bf16x8(cache[i]));
     }
   }
-  for (int c = lane + 32 * kActCache; c < nch; c += 32) amax = fmaxf(amax, absmax8_bf16(__ldg(xr + c)));
-  amax = warp_max(amax);
+  for (int c = lane + 32 * kActCache; c < nch; c += 32) a2 = __vmaxu2(a2, absmax2_bf16x8(__ldg(xr + c)));
+  const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(absmax2_f32(a2))));
   const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(amax, 1e-5f));
   uint2* qr = reinterpret_cast<uint2*>(Xq + static_cast<size_t>(m) * K);
   int sum = 0;
 #pragma unroll
   for (int i = 0; i < kActCache; ++i) {
     const int c = lane + 32 * i;
-    if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+    if (c < nch) qr[c] = quant8_bf16(cache[i], s, sum);
   }
-  for (int c = lane + 32 * kActCache; c < nch; c += 32) qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
+  for (int c = lane + 32 * kActCache; c < nch; c += 32) qr[c] = quant8_bf16(__ldg(xr + c), s, sum);
   sum = warp_sum(sum);
   if (lane == 0) {
     if (s_out) s_out[m] = s;
@@ -186,18 +180,18 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_row_kernel(const 
   const uint4* xr = reinterpret_cast<const uint4*>(X + m * K);
   const int nch = K >> 3;
   uint4 cache[kActRowCache];
-  float amax = 0.f;
+  uint32_t a2 = 0u;
 #pragma unroll
   for (int i = 0; i < kActRowCache; ++i) {
     const int c = t + kActRowThreads * i;
     if (c < nch) {
       cache[i] = __ldg(xr + c);
-      amax = fmaxf(amax, absmax8_bf16(cache[i]));
+      a2 = __vmaxu2(a2, absmax2_bf16x8(cache[i]));
     }
   }
   for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
-    amax = fmaxf(amax, absmax8_bf16(__ldg(xr + c)));
-  const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    a2 = __vmaxu2(a2, absmax2_bf16x8(__ldg(xr + c)));
+  const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(absmax2_f32(a2)));
   if (lane == 0) s_max[warp] = wmax;
   __syncthreads();
   uint32_t bmax = 0;
@@ -212,19 +206,19 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_row_kernel(const 
 #pragma unroll
     for (int i = 0; i < kActRowCache; ++i) {
       const int c = t + kActRowThreads * i;
-      if (c < nch) qr[c] = pack_nibbles8(quant8_bf16(cache[i], s, Q, sum));
+      if (c < nch) qr[c] = pack_nibbles8(quant8_bf16(cache[i], s, sum));
     }
     for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
-      qr[c] = pack_nibbles8(quant8_bf16(__ldg(xr + c), s, Q, sum));
+      qr[c] = pack_nibbles8(quant8_bf16(__ldg(xr + c), s, sum));
   } else {
     uint2* qr = reinterpret_cast<uint2*>(Xq + m * K);
 #pragma unroll
     for (int i = 0; i < kActRowCache; ++i) {
       const int c = t + kActRowThreads * i;
-      if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+      if (c < nch) qr[c] = quant8_bf16(cache[i], s, sum);
     }
     for (int c = t + kActRowThreads * kActRowCache; c < nch; c += kActRowThreads)
-      qr[c] = quant8_bf16(__ldg(xr + c), s, Q, sum);
+      qr[c] = quant8_bf16(__ldg(xr + c), s, sum);
   }
   const int wsum = __reduce_add_sync(0xffffffffu, sum);
   if (lane == 0) s_sum[warp] = wsum;
@@ -288,7 +282,7 @@ __global__ void __launch_bounds__(kActRowThreads) bl_act_quant_relu2_kernel(cons
   for (int c = t; c < nch; c += kActRowThreads) {
     float h[8];
     relu2_8(__ldg(gr + c), gated ? __ldg(ur + c) : make_uint4(0, 0, 0, 0), gated != 0, h);
-    qr[c] = quant8_f32(h, s, Q, sum);
+    qr[c] = quant8_f32(h, s, sum);
   }
   const int wsum = __reduce_add_sync(0xffffffffu, sum);
   if (lane == 0) s_sum[warp] = wsum;

@@ -101,34 +101,14 @@ constexpr int kOutAny = -1;
 // token quantisation helpers
 // ---------------------------------------------------------------------------
 
-// max |x| of 8 bf16 as a pair of 16-bit magnitudes (non-negative bf16 bit
-// patterns order like their values).
-__device__ __forceinline__ uint32_t dec_absmax2(uint4 v) {
-  constexpr uint32_t m = 0x7fff7fffu;
-  return __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
-}
-
-// Four codes q = rint(x * s) (fp32 product, round half to even) as the bytes
-// of one word.  x * s + 1.5 * 2^23 lies in [2^23, 2^24), where the spacing
-// is 1, so its bit pattern is 0x4B400000 + rint(x * s) and its low byte is
-// the code.  No clamp is needed: with a = max|x| and s = RN(Q / max(a, eps)),
-// |x * s| <= Q (1 + 2^-24), whose fp32 rounding is at most one ulp above Q
-// (Q = 7 or 127), so |q| <= Q and -Q-1 is never reached.
-__device__ __forceinline__ uint32_t dec_q4(float a, float b, float c, float d, float s) {
-  const uint32_t qa = __float_as_uint(__fadd_rn(__fmul_rn(a, s), 12582912.0f));
-  const uint32_t qb = __float_as_uint(__fadd_rn(__fmul_rn(b, s), 12582912.0f));
-  const uint32_t qc = __float_as_uint(__fadd_rn(__fmul_rn(c, s), 12582912.0f));
-  const uint32_t qd = __float_as_uint(__fadd_rn(__fmul_rn(d, s), 12582912.0f));
-  return __byte_perm(__byte_perm(qa, qb, 0x0040), __byte_perm(qc, qd, 0x0040), 0x5410);
-}
-
+// Eight codes without their sum (the register path forms it per lane).
 __device__ __forceinline__ uint2 dec_quant8(uint4 v, float s) {
-  return make_uint2(dec_q4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), s),
-                    dec_q4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w), s));
+  return make_uint2(codes4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), s),
+                    codes4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w), s));
 }
 
 __device__ __forceinline__ uint2 dec_quant8_f32(const float (&h)[8], float s) {
-  return make_uint2(dec_q4(h[0], h[1], h[2], h[3], s), dec_q4(h[4], h[5], h[6], h[7], s));
+  return make_uint2(codes4(h[0], h[1], h[2], h[3], s), codes4(h[4], h[5], h[6], h[7], s));
 }
 
 // minus the sum of the int8 codes in four words (four independent chains)
@@ -516,7 +496,7 @@ __global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
     } else {
       uint32_t a2 = 0u;   // chunks past the row end are zero
 #pragma unroll
-      for (int u = 0; u < U; ++u) a2 = __vmaxu2(a2, dec_absmax2(xv[u]));
+      for (int u = 0; u < U; ++u) a2 = __vmaxu2(a2, absmax2_bf16x8(xv[u]));
       am = max(a2 & 0xffffu, a2 >> 16) << 16;   // bf16 bits -> fp32 bits
     }
     const uint32_t wmax = __reduce_max_sync(0xffffffffu, am);

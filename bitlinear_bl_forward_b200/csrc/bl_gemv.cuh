@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
       block_reduce_max_f(amax, red_f);
       const float s = __fdiv_rn(static_cast<float>(Q), fmaxf(red_f[0], 1e-5f));
       for (int c = threadIdx.x; c < nch; c += kGemvThreads) {
-        const uint2 q = quant8_bf16(__ldg(xr + c), s, Q, rsum);
+        const uint2 q = quant8_bf16(__ldg(xr + c), s, rsum);
         const uint32_t off = m * KL + act_swz(static_cast<uint32_t>(c) << 3);
         *reinterpret_cast<uint2*>(smem + off) = q;
       }
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(THREADS, MINB)
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int c = threadIdx.x + THREADS * u;
-        if (c < nch) *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = quant8_bf16(xv[m][u], s[m], Q, rsum[m]);
+        if (c < nch) *reinterpret_cast<uint2*>(&s_act[m][act_swz(8u * c)]) = quant8_bf16(xv[m][u], s[m], rsum[m]);
       }
     }
   } else {

@@ -610,10 +610,10 @@ __global__ void __launch_bounds__(kActRowThreads, 4) bl_act_quant_norm_kernel(
 #pragma unroll
   for (int i = 0; i < kNormCache; ++i) {
     const int c = t + kActRowThreads * i;
-    if (c < nch) qr[c] = quant8_bf16(cache[i], s, Q, sum);
+    if (c < nch) qr[c] = quant8_bf16(cache[i], s, sum);
   }
   for (int c = t + kActRowThreads * kNormCache; c < nch; c += kActRowThreads)
-    qr[c] = quant8_bf16(apply(__ldg(xr + c), c), s, Q, sum);
+    qr[c] = quant8_bf16(apply(__ldg(xr + c), c), s, sum);
   const int wsum = __reduce_add_sync(0xffffffffu, sum);
   if (lane == 0) s_sum[warp] = wsum;
   __syncthreads();
