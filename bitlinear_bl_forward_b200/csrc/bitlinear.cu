@@ -178,13 +178,13 @@ bl_status launch_gemv1_t(const void* X, int x_is_i8, int K, int N, const uint8_t
 template <int A, int PRE, int FMT, int MODE>
 bl_status launch_dec_t(const bl::G2Table& tab, int grid, int in_mode, int Q, int out_mode, cudaStream_t stream) {
   auto kern = bl::bl_decode_kernel<A, PRE, FMT, MODE>;
-  constexpr int smem = MODE == bl::kModeBig ? bl::kDecBigSmemBytes : bl::kDecSmemBytes;
+  constexpr int smem = bl::dec_smem_bytes(MODE, FMT);
   static std::atomic<uint64_t> done{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
   if (!(done.load(std::memory_order_acquire) & (uint64_t(1) << dev))) {
-    // resident mode: two CTAs per SM (this launch's and the next one's) need
-    // the largest shared-memory carve-out; big mode: one CTA takes most of it
+    // two CTAs per SM (this launch's and the next one's) need the largest
+    // shared-memory carve-out; big mode with base-3 rows: one CTA takes most of it
     if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess ||
         cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -194,9 +194,9 @@ bl_status launch_dec_t(const bl::G2Table& tab, int grid, int in_mode, int Q, int
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(bl::kDecThreads);
-  // the same footprint for every launch: in resident mode a third CTA never
-  // fits on an SM, so two CTAs of one launch never share an SM
+  cfg.blockDim = dim3(bl::dec_threads(MODE, FMT));
+  // the same footprint for every launch: a third CTA never fits on an SM, so
+  // two CTAs of one launch never share an SM
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -365,8 +365,8 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
     c[best] += 1;
     sum += 1;
   }
-  const int ring = mode == bl::kModeBig ? bl::kDecBigRingBytes : bl::kDecRingBytes;
-  const int chunk_max = mode == bl::kModeBig ? bl::kDecBigChunkMax : bl::kDecChunkMax;
+  const int ring = bl::dec_ring_bytes(mode, fmt);
+  const int chunk_max = bl::dec_chunk_max(mode, fmt);
   int grid = 0;
   for (int i = 0; i < n; ++i) {
     const bl_linear& p = *probs[i];
@@ -378,7 +378,7 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
       cr = std::min(cr, bl::kDecSplitRows / rt * rt);   // split rows: the chunk's totals in shared memory
     if (mode == bl::kModeBig) {
       // one group per consumer warp per chunk
-      cr = std::min(cr, bl::kDecWarps * rt);
+      cr = std::min(cr, bl::dec_warps(mode, fmt) * rt);
       slots = std::min(bl::kDecMaxSlots, ring / (cr * rb));
     } else {
       const int cr_max = cr;

@@ -52,8 +52,7 @@
 
 namespace bl {
 
-constexpr int kDecWarps = 16;                        // consumer warps
-constexpr int kDecThreads = (kDecWarps + 1) * 32;    // + one producer warp
+constexpr int kDecWarps = 16;                        // consumer warps (+ one producer warp)
 constexpr int kDecMaxSlots = 16;
 constexpr int kDecMaxK = 8192;
 constexpr int kDecRegMaxWpl = 5;                     // resident register path: K <= 2560
@@ -62,12 +61,28 @@ constexpr int kDecActBytes = kDecMaxK + 128;
 // resident mode: two CTAs per SM
 constexpr int kDecRingBytes = 96 * 1024;
 constexpr int kDecChunkMax = 32 * 1024;
-constexpr int kDecSmemBytes = kDecRingBytes + kDecActBytes;
-// big mode: one CTA per SM
-constexpr int kDecBigRingBytes = 192 * 1024;
-constexpr int kDecBigChunkMax = 64 * 1024;
-constexpr int kDecBigSmemBytes = kDecBigRingBytes + kDecActBytes;
+// big mode, 2-bit rows: 8 consumer warps and a 96 KB ring, so that two CTAs
+// fit on an SM and the next launch's CTA fetches its first chunks while the
+// current one streams; base-3 rows (more instructions a byte) keep 16 warps
+// and a 192 KB ring, one CTA per SM
+constexpr int kDecBigWarps = 8;
+constexpr int kDecBigRingBytes = 96 * 1024;
+constexpr int kDecBigChunkMax = 32 * 1024;
+constexpr int kDecB3BigRingBytes = 192 * 1024;
+constexpr int kDecB3BigChunkMax = 64 * 1024;
 constexpr int kDecBigMaxCpl = kDecMaxK / 2048;       // 16-byte chunks a lane
+
+// Launch shape of a (mode, format) pair.
+__host__ __device__ constexpr bool dec_big2(int mode, int fmt) { return mode == 1 && fmt == 0; }
+__host__ __device__ constexpr int dec_warps(int mode, int fmt) { return dec_big2(mode, fmt) ? kDecBigWarps : kDecWarps; }
+__host__ __device__ constexpr int dec_threads(int mode, int fmt) { return (dec_warps(mode, fmt) + 1) * 32; }
+__host__ __device__ constexpr int dec_ring_bytes(int mode, int fmt) {
+  return mode == 0 ? kDecRingBytes : (fmt == 0 ? kDecBigRingBytes : kDecB3BigRingBytes);
+}
+__host__ __device__ constexpr int dec_chunk_max(int mode, int fmt) {
+  return mode == 0 ? kDecChunkMax : (fmt == 0 ? kDecBigChunkMax : kDecB3BigChunkMax);
+}
+__host__ __device__ constexpr int dec_smem_bytes(int mode, int fmt) { return dec_ring_bytes(mode, fmt) + kDecActBytes; }
 
 // What the token prologue forms before the quantisation: nothing (bf16
 // activations or int8 codes), the squared-ReLU input, or the RMS- or
@@ -281,17 +296,17 @@ __device__ __forceinline__ void dec3_dot(const uint8_t* rowp, int row_bytes, int
 // takes it when ceil(K / 512) == A); big mode with 2-bit rows, 16-byte chunks
 // per lane (ceil(K / 2048) of at most A for every problem of the launch).
 template <int A, int PRE, int FMT, int MODE>
-__global__ void __launch_bounds__(kDecThreads, MODE == kModeBig ? 1 : 2)
+__global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && FMT == kFmtBase3) ? 1 : 2)
     bl_decode_kernel(const __grid_constant__ G2Table tab, int in_mode, int Q, int out_mode,
                      unsigned long long limit_ns) {
-  constexpr int CW = kDecWarps;
+  constexpr int CW = dec_warps(MODE, FMT);
   constexpr bool RELU2 = PRE == kDecRelu2;
   constexpr bool RMS = PRE == kDecRms;
   constexpr bool LN = PRE == kDecLn;
   constexpr bool NORM = RMS || LN;
   constexpr bool B3 = FMT == kFmtBase3;
   constexpr bool BIG = MODE == kModeBig;
-  constexpr int RING = BIG ? kDecBigRingBytes : kDecRingBytes;
+  constexpr int RING = dec_ring_bytes(MODE, FMT);
   static_assert(!B3 || (A == 0 && PRE == kDecPlain), "base-3 rows take the shared-memory token path");
   static_assert(!BIG || B3 || (A >= 1 && A <= kDecBigMaxCpl), "big mode keeps 1..4 chunks a lane");
   static_assert(B3 || BIG || (A >= 1 && A <= kDecRegMaxWpl), "resident register path: 1..5 words a lane");
