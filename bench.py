@@ -292,6 +292,7 @@ class GpuWorkload:
             ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=device)
             self.layers.append(dict(L=L, copies=copies, X=X, Y=Y, ws=ws, xb=xb, own_x=own_x))
         self.rotations = rotations
+        self.prepared = {}
         # layers run together in one grouped call (e.g. up and gate of a feed-forward block)
         self.groups = [list(gr) for gr in self.w.groups] or [[i] for i in range(len(self.layers))]
         self.group_ws = []
@@ -324,9 +325,16 @@ class GpuWorkload:
             else:
                 bl.bl_forward(d["X"], Wp, gamma, d["L"].N, self.w.bits, out=d["Y"], workspace=d["ws"])
         else:
+            # the grouped call prepared once per rotation (argument packing
+            # outside the step); rebuilt when a layer's buffers are replaced
             ds = [self.layers[j] for j in gr]
-            bl.bl_forward_grouped([(d["X"], *d["copies"][r], d["L"].N) for d in ds], self.w.bits,
-                                  outs=[d["Y"] for d in ds], workspace=self.group_ws[gi])
+            key = (gi, r, tuple(d["X"].data_ptr() for d in ds), tuple(d["Y"].data_ptr() for d in ds))
+            call = self.prepared.get(key)
+            if call is None:
+                call = bl.PreparedGrouped([(d["X"], *d["copies"][r], d["L"].N) for d in ds], self.w.bits,
+                                          outs=[d["Y"] for d in ds], workspace=self.group_ws[gi])
+                self.prepared[key] = call
+            call()
 
     def step(self, i):
         r = i % self.rotations
@@ -486,11 +494,13 @@ def time_workload(wl, steps, warmup, dist_ctx, sample_clocks=True, chunk=None):
 
 
 def time_e2e(wl, steps, warmup, dist_ctx):
-    """Same metric through the public API with host buffers: each step copies
-    the step's inputs from pinned host memory in one transfer, runs the
-    library calls and reads all outputs back to pinned host memory in one
-    transfer (the layers' input and output tensors are views of one device
-    buffer each, 128-byte aligned)."""
+    """Same metric through the public API with host buffers.  A step that is
+    one grouped call goes through the library's host-buffer entry point
+    (bl_forward_grouped_host: a copy per distinct input from pinned host
+    memory, the grouped forward, a copy per output back, one C call a step).
+    Other steps copy the inputs from pinned host memory in one transfer, run
+    the library calls and read all outputs back in one transfer (the layers'
+    tensors are views of one device buffer each, 128-byte aligned)."""
     import torch
     own = [j for j, d in enumerate(wl.layers) if d["own_x"]]
 
@@ -523,12 +533,33 @@ def time_e2e(wl, steps, warmup, dist_ctx):
     h2d = sum(int(np.prod(tuple(wl.layers[j]["X"].shape))) * 2 for j in own)
     d2h = sum(d["Y"].numel() * 2 for d in wl.layers)
 
-    def one(i):
-        r = i % wl.rotations
-        dev_in.copy_(host_in, non_blocking=True)
-        for gi in range(len(wl.groups)):
-            wl.run_group(gi, r)
-        host_out.copy_(dev_out, non_blocking=True)
+    if len(wl.groups) == 1 and len(wl.groups[0]) > 1 and wl.fmt == "2bit":
+        # one grouped call a step: the library's host-buffer entry point
+        # copies the step's inputs in, runs the group and copies the outputs
+        # back, all on the stream (one C call a step)
+        from bitlinear_bl_forward_b200 import bl
+        gr = wl.groups[0]
+        hx, hy = {}, {}
+        for j, off in zip(own, in_offs):
+            shp = tuple(wl.layers[j]["X"].shape)
+            hx[j] = host_in[off:off + int(np.prod(shp))].view(shp)
+        for j, d in enumerate(wl.layers):
+            hx.setdefault(j, hx[d["L"].x_layer if d["L"].x_layer >= 0 else j])
+        for j, (d, off) in enumerate(zip(wl.layers, out_offs)):
+            shp = tuple(d["Y"].shape)
+            hy[j] = host_out[off:off + int(np.prod(shp))].view(shp)
+        calls = [bl.PreparedGroupedHost([(hx[j], *wl.layers[j]["copies"][r], wl.layers[j]["L"].N) for j in gr],
+                                        [hy[j] for j in gr], wl.w.bits) for r in range(wl.rotations)]
+
+        def one(i):
+            calls[i % wl.rotations]()
+    else:
+        def one(i):
+            r = i % wl.rotations
+            dev_in.copy_(host_in, non_blocking=True)
+            for gi in range(len(wl.groups)):
+                wl.run_group(gi, r)
+            host_out.copy_(dev_out, non_blocking=True)
 
     for i in range(warmup):
         one(i)

@@ -52,6 +52,8 @@ SIGNATURES = {
     "bl_forward_layernorm_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "bl_forward_layernorm": (_int, [_p, ctypes.c_float, _i64, _i64, _i64, _p, _p, _int, _p, _p, _sz, _p]),
     "bl_quant_act_layernorm": (_int, [_p, ctypes.c_float, _i64, _i64, _int, _p, _p, _p, _p, _p]),
+    "bl_forward_grouped_host_staging_bytes": (_sz, [_int, _p]),
+    "bl_forward_grouped_host": (_int, [_int, _p, _int, _p, _sz, _p, _sz, _p]),
     "bl_forward_norm_grouped_workspace_bytes": (_sz, [_int, _p, _int]),
     "bl_forward_norm_grouped": (_int, [_int, _p, _int, _p, ctypes.c_float, _int, _p, _sz, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
@@ -252,6 +254,97 @@ def bl_forward_grouped(problems, bits: int = 8, outs=None, workspace: torch.Tens
         ws = _workspace(need, problems[0][0].device if problems else "cuda")
     _check(lib().bl_forward_grouped(len(problems), arr, bits, ws.data_ptr() if ws is not None else None,
                                     ws.numel() if ws is not None else 0, _stream()), "bl_forward_grouped")
+    return outs
+
+
+class PreparedGrouped:
+    """A bl_forward_grouped call whose arguments are checked and packed once
+    (the bl_linear array, the workspace pointer): calling it issues the same
+    C call on the current stream with no per-call marshalling.  The tensors
+    must stay alive and in place; their contents may change between calls."""
+
+    def __init__(self, problems, bits: int = 8, outs=None, workspace: torch.Tensor | None = None):
+        if outs is None:
+            outs = [torch.empty((X.shape[0], N), dtype=torch.bfloat16, device=X.device) for (X, _, _, N) in problems]
+        self.outs = outs
+        self._keep = (list(problems), list(outs), workspace)
+        self._n = len(problems)
+        self._arr = _grouped_structs(problems, outs)
+        self._bits = bits
+        ws = workspace
+        if ws is None:
+            need = int(lib().bl_forward_grouped_workspace_bytes(self._n, self._arr, bits))
+            ws = _workspace(need, problems[0][0].device if problems else "cuda")
+            self._keep = self._keep + (ws,)
+        self._wsp = ws.data_ptr() if ws is not None else None
+        self._wsn = ws.numel() if ws is not None else 0
+        self._fn = lib().bl_forward_grouped
+
+    def __call__(self):
+        _check(self._fn(self._n, self._arr, self._bits, self._wsp, self._wsn, _stream()), "bl_forward_grouped")
+        return self.outs
+
+
+def _host(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def bl_forward_grouped_host_staging_bytes(problems, outs) -> int:
+    """problems: list of (X host bf16 [M, K], Wp, gamma, N); outs: host bf16 [M, N]."""
+    arr = _host_structs(problems, outs)
+    return int(lib().bl_forward_grouped_host_staging_bytes(len(problems), arr))
+
+
+def _host_structs(problems, outs):
+    arr = (BLLinear * max(1, len(problems)))()
+    for i, ((X, Wp, gamma, N), Y) in enumerate(zip(problems, outs)):
+        M, K = X.shape
+        if tuple(Y.shape) != (M, N):
+            raise ValueError("output must be [M, N]")
+        arr[i] = BLLinear(_host(X, torch.bfloat16, "X"), M, K, N, _dev(Wp, torch.uint8, "Wp"),
+                          _dev(gamma, torch.float32, "gamma"), _host(Y, torch.bfloat16, "out"))
+    return arr
+
+
+class PreparedGroupedHost:
+    """bl_forward_grouped_host prepared once: problems is a list of
+    (X host bf16 [M, K], Wp, gamma, N) and outs the host bf16 [M, N] outputs
+    (pinned memory keeps the copies asynchronous).  Each call enqueues on the
+    current stream the input copies, the grouped forward and the output
+    copies; synchronise the stream before reading the outputs."""
+
+    def __init__(self, problems, outs, bits: int = 8, device="cuda"):
+        self.outs = outs
+        self._n = len(problems)
+        self._arr = _host_structs(problems, outs)
+        self._bits = bits
+        nst = int(lib().bl_forward_grouped_host_staging_bytes(self._n, self._arr))
+        if nst == 0:
+            raise ValueError("bad problem shapes")
+        self._stg = torch.empty(nst, dtype=torch.uint8, device=device)
+        nws = int(lib().bl_forward_grouped_workspace_bytes(self._n, self._arr, bits))
+        self._ws = torch.empty(nws, dtype=torch.uint8, device=device) if nws else None
+        self._keep = (list(problems), list(outs))
+        self._args = (self._stg.data_ptr(), nst, self._ws.data_ptr() if self._ws is not None else None, nws)
+        self._fn = lib().bl_forward_grouped_host
+
+    def __call__(self):
+        _check(self._fn(self._n, self._arr, self._bits, *self._args, _stream()), "bl_forward_grouped_host")
+        return self.outs
+
+
+def bl_forward_grouped_host(problems, outs, bits: int = 8):
+    """One grouped forward on host-resident activations (see PreparedGroupedHost,
+    which keeps its staging and workspace across calls); synchronises the
+    stream before returning the host outputs."""
+    PreparedGroupedHost(problems, outs, bits)()
+    torch.cuda.current_stream().synchronize()
     return outs
 
 

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -310,9 +311,8 @@ double dec_cta_cost(int64_t N, int64_t K, int ctas, int a, int fmt, int mode) {
 // range per CTA is cut into whole-group chunks: in resident mode as few as
 // fit the ring without reuse when possible; in big mode one group per warp
 // per chunk.  Returns the grid size.
-int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, int mode, int a,
-                      const void* const* Us, const float* bias, float eps, int fmt = bl::kFmt2Bit) {
-  std::memset(tab, 0, sizeof(*tab));
+void plan_decode(const bl_linear* const* probs, int n, int sms, int mode, int a, int fmt, int* c, int* crs,
+                 int* sls) {
   int64_t rows_total = 0;
   for (int i = 0; i < n; ++i) rows_total += probs[i]->N;
   const int target = static_cast<int>(rows_total < sms ? rows_total : sms);
@@ -334,7 +334,6 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
   double lo_t = 0.0, hi_t = 0.0;
   for (int i = 0; i < n; ++i)
     hi_t = std::max(hi_t, dec_cta_cost(probs[i]->N, probs[i]->K, 1, a, fmt, mode));
-  int c[bl::kG2MaxProblems];
   for (int it = 0; it < 60; ++it) {
     const double mid = 0.5 * (lo_t + hi_t);
     int sum = 0;
@@ -367,7 +366,6 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
   }
   const int ring = bl::dec_ring_bytes(mode, fmt);
   const int chunk_max = bl::dec_chunk_max(mode, fmt);
-  int grid = 0;
   for (int i = 0; i < n; ++i) {
     const bl_linear& p = *probs[i];
     const int rb = dec_row_bytes(p.K, fmt);
@@ -391,6 +389,73 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
         slots = std::min(bl::kDecMaxSlots, ring / (cr * rb));
       }
     }
+    crs[i] = cr;
+    sls[i] = slots;
+  }
+}
+
+// The shape-only part of a launch table (CTAs per problem, chunk rows,
+// slots) depends on the problems' N and K, the mode, the register width and
+// the SM count alone; the search above costs more host time than the launch,
+// so recent plans are kept (a small round-robin table).
+struct DecPlan {
+  int n = 0, sms = 0, mode = 0, a = 0, fmt = 0;
+  int64_t N[bl::kG2MaxProblems] = {}, K[bl::kG2MaxProblems] = {};
+  int c[bl::kG2MaxProblems] = {}, cr[bl::kG2MaxProblems] = {}, slots[bl::kG2MaxProblems] = {};
+};
+constexpr int kDecPlanCache = 16;
+
+void plan_decode_cached(const bl_linear* const* probs, int n, int sms, int mode, int a, int fmt, int* c, int* crs,
+                        int* sls) {
+  static std::mutex mu;
+  static DecPlan plans[kDecPlanCache];
+  static int used = 0, next = 0;
+  auto same = [&](const DecPlan& q) {
+    if (q.n != n || q.sms != sms || q.mode != mode || q.a != a || q.fmt != fmt) return false;
+    for (int i = 0; i < n; ++i)
+      if (q.N[i] != probs[i]->N || q.K[i] != probs[i]->K) return false;
+    return true;
+  };
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int e = 0; e < used; ++e)
+      if (same(plans[e])) {
+        for (int i = 0; i < n; ++i) {
+          c[i] = plans[e].c[i];
+          crs[i] = plans[e].cr[i];
+          sls[i] = plans[e].slots[i];
+        }
+        return;
+      }
+  }
+  plan_decode(probs, n, sms, mode, a, fmt, c, crs, sls);
+  DecPlan q;
+  q.n = n;
+  q.sms = sms;
+  q.mode = mode;
+  q.a = a;
+  q.fmt = fmt;
+  for (int i = 0; i < n; ++i) {
+    q.N[i] = probs[i]->N;
+    q.K[i] = probs[i]->K;
+    q.c[i] = c[i];
+    q.cr[i] = crs[i];
+    q.slots[i] = sls[i];
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  plans[next] = q;
+  next = (next + 1) % kDecPlanCache;
+  if (used < kDecPlanCache) ++used;
+}
+
+int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, int sms, int mode, int a,
+                      const void* const* Us, const float* bias, float eps, int fmt = bl::kFmt2Bit) {
+  std::memset(tab, 0, sizeof(*tab));
+  int c[bl::kG2MaxProblems], crs[bl::kG2MaxProblems], sls[bl::kG2MaxProblems];
+  plan_decode_cached(probs, n, sms, mode, a, fmt, c, crs, sls);
+  int grid = 0;
+  for (int i = 0; i < n; ++i) {
+    const bl_linear& p = *probs[i];
     bl::G2Problem& q = tab->p[i];
     q.X = p.X;
     q.U = Us ? Us[i] : nullptr;
@@ -405,8 +470,8 @@ int fill_decode_table(bl::G2Table* tab, const bl_linear* const* probs, int n, in
     q.ctas = c[i];
     q.bias = bias;
     q.eps = eps;
-    q.chunk_rows = cr;
-    q.slots = slots;
+    q.chunk_rows = crs[i];
+    q.slots = sls[i];
     q.ksplit = (mode == bl::kModeResident && fmt == bl::kFmt2Bit) ? dec_split(p.K, a) : 1;
     grid += c[i];
   }
@@ -965,6 +1030,151 @@ bl_status bl_forward_grouped(int count, const bl_linear* problems, int bits, voi
     }
     if (st != BL_OK) return st;
   }
+  return BL_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Grouped forward on host-resident activations (end to end on one stream).
+// ---------------------------------------------------------------------------
+
+// Device staging of a host-buffer group.  Distinct inputs (the same host X
+// read by several problems is copied once) and the outputs are sorted by
+// host address; host regions that are exactly contiguous form one run,
+// staged contiguously (one copy a run), and every run starts 256-byte
+// aligned.  Inside a run a tensor keeps its host offset: for inputs a
+// multiple of 128 bytes (K % 64 == 0), so staged X stays 16-byte aligned;
+// outputs need no alignment.  Only the tensors' own bytes are ever copied.
+struct HostRun {
+  const uint8_t* host;   // first host byte of the run
+  size_t bytes;          // bytes of the run
+  size_t stage;          // offset of the run in the staging
+};
+struct HostStaging {
+  size_t x_off[bl::kG2MaxProblems], y_off[bl::kG2MaxProblems];
+  HostRun xr[bl::kG2MaxProblems], yr[bl::kG2MaxProblems];
+  int nxr = 0, nyr = 0;
+  size_t total = 0;
+};
+
+// Sort (host pointer, bytes, problem) triples by pointer, cut them into
+// exactly contiguous runs from `off` on; returns the offset after the runs.
+size_t host_runs(const uint8_t* const* ptr, const size_t* bytes, int m, HostRun* runs, int* nruns, size_t* stage_of,
+                 size_t off) {
+  int order[bl::kG2MaxProblems];
+  for (int i = 0; i < m; ++i) order[i] = i;
+  for (int i = 1; i < m; ++i)
+    for (int j = i; j > 0 && ptr[order[j]] < ptr[order[j - 1]]; --j) std::swap(order[j], order[j - 1]);
+  int r = -1;
+  for (int t = 0; t < m; ++t) {
+    const int i = order[t];
+    if (r < 0 || runs[r].host + runs[r].bytes != ptr[i]) {
+      if (r >= 0) off += align_up(runs[r].bytes, 256);
+      ++r;
+      runs[r] = HostRun{ptr[i], 0, off};
+    }
+    stage_of[i] = runs[r].stage + static_cast<size_t>(ptr[i] - runs[r].host);
+    runs[r].bytes += bytes[i];
+  }
+  if (r >= 0) off += align_up(runs[r].bytes, 256);
+  *nruns = r + 1;
+  return off;
+}
+
+// Returns false on a bad shape.
+bool host_staging_layout(int count, const bl_linear* problems, HostStaging* st) {
+  const uint8_t* xp[bl::kG2MaxProblems];
+  size_t xb[bl::kG2MaxProblems], xs[bl::kG2MaxProblems];
+  int xi[bl::kG2MaxProblems], first[bl::kG2MaxProblems];
+  int m = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    if (check_shape_nk(p.N, p.K) != BL_OK || check_m(p.M, p.K) != BL_OK) return false;
+    first[i] = -1;
+    for (int j = 0; j < i; ++j)
+      if (problems[j].X == p.X && problems[j].M == p.M && problems[j].K == p.K) {
+        first[i] = first[j] >= 0 ? first[j] : j;
+        break;
+      }
+    if (first[i] < 0) {
+      xp[m] = reinterpret_cast<const uint8_t*>(p.X);
+      xb[m] = static_cast<size_t>(p.M) * p.K * 2;
+      xi[i] = m++;
+    }
+  }
+  size_t off = host_runs(xp, xb, m, st->xr, &st->nxr, xs, 0);
+  for (int i = 0; i < count; ++i) st->x_off[i] = xs[xi[first[i] >= 0 ? first[i] : i]];
+  const uint8_t* yp[bl::kG2MaxProblems];
+  size_t yb[bl::kG2MaxProblems];
+  for (int i = 0; i < count; ++i) {
+    yp[i] = reinterpret_cast<const uint8_t*>(problems[i].Y);
+    yb[i] = static_cast<size_t>(problems[i].M) * problems[i].N * 2;
+  }
+  off = host_runs(yp, yb, count, st->yr, &st->nyr, st->y_off, off);
+  st->total = off;
+  return true;
+}
+
+size_t bl_forward_grouped_host_staging_bytes(int count, const bl_linear* problems) {
+  if (count <= 0 || count > bl::kG2MaxProblems || problems == nullptr) return 0;
+  HostStaging st;
+  return host_staging_layout(count, problems, &st) ? st.total : 0;
+}
+
+bl_status bl_forward_grouped_host(int count, const bl_linear* problems, int bits, void* staging, size_t staging_bytes,
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx_range("bl_forward_grouped_host");
+  if (problems == nullptr) return BL_ERR_INVALID_ARG;
+  if (count < 0 || count > bl::kG2MaxProblems) return BL_ERR_UNSUPPORTED;
+  if (count == 0) return BL_OK;
+  for (int i = 0; i < count; ++i)
+    if (problems[i].M == 0 || !problems[i].X || !problems[i].Y) return BL_ERR_INVALID_ARG;
+  HostStaging st;
+  if (!host_staging_layout(count, problems, &st)) return BL_ERR_SHAPE;
+  if (!staging || staging_bytes < st.total) return BL_ERR_WORKSPACE;
+  if (!aligned16(staging)) return BL_ERR_ALIGNMENT;
+  if (bits != 8 && bits != 4) return BL_ERR_UNSUPPORTED;
+  // outputs may not overlap each other or an input
+  for (int i = 0; i < count; ++i) {
+    const uint8_t* y0 = reinterpret_cast<const uint8_t*>(problems[i].Y);
+    const uint8_t* y1 = y0 + static_cast<size_t>(problems[i].M) * problems[i].N * 2;
+    for (int j = 0; j < count; ++j) {
+      const uint8_t* x0 = reinterpret_cast<const uint8_t*>(problems[j].X);
+      const uint8_t* x1 = x0 + static_cast<size_t>(problems[j].M) * problems[j].K * 2;
+      if (y0 < x1 && x0 < y1) return BL_ERR_INVALID_ARG;
+      if (j != i) {
+        const uint8_t* z0 = reinterpret_cast<const uint8_t*>(problems[j].Y);
+        const uint8_t* z1 = z0 + static_cast<size_t>(problems[j].M) * problems[j].N * 2;
+        if (y0 < z1 && z0 < y1) return BL_ERR_INVALID_ARG;
+      }
+    }
+  }
+  bl_linear dev[bl::kG2MaxProblems];
+  uint8_t* base = static_cast<uint8_t*>(staging);
+  for (int i = 0; i < count; ++i) {
+    const bl_linear& p = problems[i];
+    if (!p.Wp || !p.gamma) return BL_ERR_INVALID_ARG;
+    if (!aligned16(p.Wp)) return BL_ERR_ALIGNMENT;
+    const size_t w = fwd_ws_bytes(p.M, p.K);
+    if (w > 0 && (!workspace || workspace_bytes < w)) return BL_ERR_WORKSPACE;
+    if (w > 0 && !aligned16(workspace)) return BL_ERR_ALIGNMENT;
+    dev[i] = p;
+    dev[i].X = reinterpret_cast<const uint16_t*>(base + st.x_off[i]);
+    dev[i].Y = reinterpret_cast<uint16_t*>(base + st.y_off[i]);
+  }
+  for (int r = 0; r < st.nxr; ++r)
+    if (cudaMemcpyAsync(base + st.xr[r].stage, st.xr[r].host, st.xr[r].bytes, cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+  bl_status rc = bl_forward_grouped(count, dev, bits, workspace, workspace_bytes, stream);
+  if (rc != BL_OK) return rc;
+  for (int r = 0; r < st.nyr; ++r)
+    if (cudaMemcpyAsync(const_cast<uint8_t*>(st.yr[r].host), base + st.yr[r].stage, st.yr[r].bytes,
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
   return BL_OK;
 }
 

@@ -224,6 +224,31 @@ BL_API bl_status bl_forward_grouped(int count, const bl_linear* problems, int bi
 
 
 /*
+ * bl_forward_grouped end to end on host-resident activations: problems[i].X
+ * and problems[i].Y are HOST pointers (pinned memory keeps the copies
+ * asynchronous); Wp and gamma are device pointers as usual; every problem
+ * has at least one token, and no output may overlap an input or another
+ * output (BL_ERR_INVALID_ARG).  On `stream`, in order: the inputs copied to
+ * the device (problems with the same X, M and K share one copy; inputs whose
+ * host bytes are exactly contiguous travel in one copy), the grouped forward
+ * of bl_forward_grouped on the staged tensors, the outputs copied back
+ * (exactly contiguous outputs in one copy).  Only the tensors' own bytes are
+ * read or written.  The call
+ * returns once everything is enqueued; the host buffers must stay valid
+ * until the stream reaches that point.
+ * staging: device memory of at least
+ * bl_forward_grouped_host_staging_bytes(count, problems) bytes, 16-byte
+ * aligned, owned by the caller (the staged inputs and outputs, 256-byte
+ * aligned inside it).  workspace: as bl_forward_grouped (its size query
+ * takes the same structs).  Errors: as bl_forward_grouped, plus
+ * BL_ERR_WORKSPACE for missing or short staging; nothing is copied or
+ * launched unless the whole group is valid.
+ */
+BL_API size_t bl_forward_grouped_host_staging_bytes(int count, const bl_linear* problems);
+BL_API bl_status bl_forward_grouped_host(int count, const bl_linear* problems, int bits, void* staging,
+                                         size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                                         cudaStream_t stream);
+/*
  * Squared-ReLU feed-forward: the down projection's input is formed from the
  * gate projection's output ("BitNet 2B4T Guide: Scaling Native 1.58-Bit
  * LLMs", section "2. Squared ReLU Activation", ReLU^2(x) = max(0, x)^2, and

@@ -248,6 +248,45 @@ def test_norm_grouped_validation(L):
     assert L.bl_forward_norm_grouped(0, arr, 1, None, 1e-5, 8, None, 0, None) == OK
 
 
+def test_grouped_host_validation(L):
+    from bitlinear_bl_forward_b200.bl import BLLinear
+    arr = (BLLinear * 3)()
+    H = 0x7f0000001000          # host pointers are only copied from, never checked for alignment
+    arr[0] = BLLinear(H, 1, 2560, 6912, A, A, H + 0x100000)
+    arr[1] = BLLinear(H, 1, 2560, 6912, A, A, H + 0x200000)    # same X: staged once
+    arr[2] = BLLinear(H + 0x300000, 1, 6912, 2560, A, A, H + 0x400000)
+    need = L.bl_forward_grouped_host_staging_bytes(3, arr)
+    # two distinct inputs and three outputs, none adjacent: five runs, 256-byte aligned each
+    assert need == 2560 * 2 + 6912 * 2 + 6912 * 2 + 6912 * 2 + 2560 * 2
+    # adjacent host regions share a run: X_a | X_b contiguous, outputs contiguous
+    adj = (BLLinear * 3)()
+    adj[0] = BLLinear(H, 1, 2560, 6912, A, A, H + 0x100000)
+    adj[1] = BLLinear(H, 1, 2560, 6912, A, A, H + 0x100000 + 6912 * 2)
+    adj[2] = BLLinear(H + 2560 * 2, 1, 6912, 2560, A, A, H + 0x100000 + 2 * 6912 * 2)
+    in_run = 2560 * 2 + 6912 * 2                         # 18944 bytes -> 19200 with the run's alignment
+    out_run = 2 * 6912 * 2 + 2560 * 2                    # 32768 bytes
+    assert L.bl_forward_grouped_host_staging_bytes(3, adj) == (in_run + 255) // 256 * 256 + out_run
+    # an output overlapping an input is rejected before any copy
+    ov = (BLLinear * 1)()
+    ov[0] = BLLinear(H, 1, 2560, 6912, A, A, H + 2048)
+    assert L.bl_forward_grouped_host(1, ov, 8, A, 1 << 20, A, 1 << 20, None) == INVALID
+    assert L.bl_forward_grouped_host_staging_bytes(9, arr) == 0
+    assert L.bl_forward_grouped_host(3, arr, 8, None, 0, A, 1 << 20, None) == WS
+    assert L.bl_forward_grouped_host(3, arr, 8, A, need - 1, A, 1 << 20, None) == WS
+    assert L.bl_forward_grouped_host(3, arr, 8, U, need, A, 1 << 20, None) == ALIGN
+    assert L.bl_forward_grouped_host(3, arr, 5, A, need, A, 1 << 20, None) == UNSUP
+    assert L.bl_forward_grouped_host(9, arr, 8, A, need, A, 1 << 20, None) == UNSUP
+    assert L.bl_forward_grouped_host(3, None, 8, A, need, A, 1 << 20, None) == INVALID
+    arr[1] = BLLinear(H, 1, 2560, 6912, None, A, H + 0x200000)
+    assert L.bl_forward_grouped_host(3, arr, 8, A, need, A, 1 << 20, None) == INVALID
+    arr[1] = BLLinear(H, 1, 100, 6912, A, A, H + 0x200000)
+    assert L.bl_forward_grouped_host_staging_bytes(3, arr) == 0
+    assert L.bl_forward_grouped_host(3, arr, 8, A, need, A, 1 << 20, None) == SHAPE
+    assert L.bl_forward_grouped_host(0, arr, 8, None, 0, None, 0, None) == OK
+    arr[1] = BLLinear(H, 0, 2560, 6912, A, A, H + 0x200000)
+    assert L.bl_forward_grouped_host(3, arr, 8, A, need, A, 1 << 20, None) == INVALID   # no empty problems
+
+
 def test_base3_host_checks(L):
     # sizes: 4 * ceil(ceil(K / 20) / 4) bytes a row
     assert L.bl_packed_weight_bytes_b3(1, 64) == 16

@@ -322,6 +322,78 @@ def test_grouped_decode_mixed_k_one_launch():
             assert bf16_ulp_distance(bf16_dev_to_bits(a), oracle_bf16(X, c, g, bits)).max() <= BF16_ULP_TOL
 
 
+def test_prepared_grouped_call_matches_and_sees_new_inputs():
+    # the prepared form issues the same C call: equal outputs, and new input
+    # contents (same buffers) are picked up by the next call
+    cases = [(1, 2560, 700), (1, 2560, 33), (1, 6912, 130)]
+    probs, Xs = [], []
+    for j, (M, K, N) in enumerate(cases):
+        X, W = random_case(M, K, N, seed=1300 + j)
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        Xd = x_to_dev(X)
+        probs.append((Xd, Wp, gd, N))
+        Xs.append(Xd)
+    call = bl.PreparedGrouped(probs)
+    a = [y.clone() for y in call()]
+    b = bl.bl_forward_grouped(probs)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    for j, Xd in enumerate(Xs):
+        X2, _ = random_case(1, Xd.shape[1], 8, seed=1400 + j)
+        Xd.copy_(x_to_dev(X2))
+    c = [y.clone() for y in call()]
+    d = bl.bl_forward_grouped(probs)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(c, d))
+    assert not all(torch.equal(x, y) for x, y in zip(a, c))
+
+
+@pytest.mark.parametrize("M", [1, 3, 130])
+def test_grouped_host_buffers_match_device_path(M):
+    # host-resident X and Y through bl_forward_grouped_host: one staged copy
+    # for the shared input, the same kernels, outputs copied back
+    shapes = [(2560, 700), (2560, 264), (6912, 130)]
+    Xs, probs_d, probs_h, outs_h = {}, [], [], []
+    for j, (K, N) in enumerate(shapes):
+        X, W = random_case(M, K, N, seed=1500 + j)
+        key = K
+        if key not in Xs:
+            Xs[key] = X
+        Xh = torch.from_numpy(Xs[key].view(np.int16)).view(torch.bfloat16).pin_memory()
+        Wp, gd = bl.bl_quantize_weights(torch.from_numpy(W).cuda())
+        probs_d.append((x_to_dev(Xs[key]), Wp, gd, N))
+        probs_h.append((Xh, Wp, gd, N))
+        outs_h.append(torch.full((M, N), float("nan"), dtype=torch.bfloat16).pin_memory())
+    # the two K = 2560 problems read one host tensor
+    probs_h[1] = (probs_h[0][0],) + probs_h[1][1:]
+    ref = bl.bl_forward_grouped(probs_d)
+    call = bl.PreparedGroupedHost(probs_h, outs_h)
+    for _ in range(2):
+        call()
+        torch.cuda.synchronize()
+        for a, b in zip(outs_h, ref):
+            assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16))
+    outs2 = [torch.empty_like(o).pin_memory() for o in outs_h]
+    bl.bl_forward_grouped_host(probs_h, outs2)
+    assert all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(outs2, outs_h))
+    # inputs and outputs as adjacent views of one pinned buffer each: one
+    # copy in and one copy out (the staged tensors keep their offsets)
+    xin = torch.empty(M * (2560 + 6912), dtype=torch.bfloat16).pin_memory()
+    xa, xb = xin[:M * 2560].view(M, 2560), xin[M * 2560:].view(M, 6912)
+    xa.copy_(probs_h[0][0])
+    xb.copy_(probs_h[2][0])
+    yout = torch.full((M * (700 + 264 + 130),), float("nan"), dtype=torch.bfloat16).pin_memory()
+    ys = [yout[:M * 700].view(M, 700), yout[M * 700:M * 964].view(M, 264), yout[M * 964:].view(M, 130)]
+    adj = [(xa, probs_h[0][1], probs_h[0][2], 700), (xa, probs_h[1][1], probs_h[1][2], 264),
+           (xb, probs_h[2][1], probs_h[2][2], 130)]
+    a256 = lambda n: (n + 255) // 256 * 256   # noqa: E731 -- each run starts 256-byte aligned
+    assert bl.bl_forward_grouped_host_staging_bytes(adj, ys) == a256(M * 9472 * 2) + a256(M * 1094 * 2)
+    bl.PreparedGroupedHost(adj, ys)()
+    torch.cuda.synchronize()
+    for a, b in zip(ys, ref):
+        assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16))
+
+
 def test_grouped_mixed_shapes_fall_back_to_sequential():
     cases = [(1, 256, 300), (3, 512, 129), (1, 4096, 64), (2, 192, 100), (0, 64, 8)]
     probs, singles = [], []
