@@ -168,15 +168,6 @@ __device__ __forceinline__ int dec_warp_totals(const int (&part)[RT], int lane) 
   return t;
 }
 
-// Warp sum of each row's partial; lane r of the group rescales and stores
-// row r (one store instruction for the group).
-template <int RT, int OUT>
-__device__ __forceinline__ void dec_store(const int (&part)[RT], int n0, int nlive, int lane, float f,
-                                          void* __restrict__ Y, const float* __restrict__ bias, int out_mode) {
-  const int t = dec_warp_totals<RT>(part, lane);
-  if (lane < nlive) dec_put<OUT>(t, n0 + lane, f, Y, bias, out_mode);
-}
-
 __device__ __forceinline__ int dec_fold(const int (&a)[4]) { return a[0] + (a[1] >> 2) + (a[2] >> 4) + (a[3] >> 6); }
 
 // 2-bit rows, resident mode: lane l takes words word0 + l + 32 i (i < WPL)
