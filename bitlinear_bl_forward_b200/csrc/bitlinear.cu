@@ -284,10 +284,22 @@ inline int dec_rt(int mode, int fmt) {
 // reductions and stores; shared adds when rows are split), plus a penalty
 // for bytes that do not fit the ring (fetched after the dependency wait).
 // Big mode: the weight bytes a CTA streams.
+// Row-lane mode: issue slots of one SM sub-partition (items go round-robin
+// to 16 warps, four per sub-partition): per 16-byte column of a 32-row tile
+// about 37 instructions, per item (tile x 512-weight segment) about 25 more;
+// bytes beyond the ring as above; more than 512 rows a CTA is not allowed.
 double dec_cta_cost(int64_t N, int64_t K, int ctas, int a, int fmt, int mode) {
   const int64_t rows = (N + ctas - 1) / ctas;
   const double bytes = static_cast<double>(rows) * static_cast<double>(dec_row_bytes(K, fmt));
   if (mode == bl::kModeBig) return bytes;
+  if (mode == bl::kModeRowLane) {
+    if (rows > bl::kDecLaneMaxRows) return 1e12;
+    const int64_t tiles = (rows + bl::kDecLaneRows - 1) / bl::kDecLaneRows;
+    const int64_t upr = K / 64, segs = (upr + 7) / 8;
+    const double pb = static_cast<double>(rows) * bl::dec_lane_stride(static_cast<int>(K / 4));
+    const double over = pb > bl::kDecRingBytes ? (pb - bl::kDecRingBytes) / 8.0 : 0.0;
+    return (static_cast<double>(tiles * upr) * 37.0 + static_cast<double>(tiles * segs) * 25.0) / 4.0 + over;
+  }
   const int rt = dec_rt(mode, fmt);
   const int64_t groups = (rows + rt - 1) / rt;
   double group;
@@ -372,6 +384,16 @@ void plan_decode(const bl_linear* const* probs, int n, int sms, int mode, int a,
     const int rt = dec_rt(mode, fmt);
     const int maxrows = static_cast<int>((p.N + c[i] - 1) / c[i]);
     int cr = (chunk_max / rb) / rt * rt, slots = 0;
+    if (mode == bl::kModeRowLane) {
+      // one 32-row tile a chunk; every chunk resident when the padded rows fit
+      const int st = bl::dec_lane_stride(rb);
+      cr = bl::kDecLaneRows;
+      const int nch = (maxrows + cr - 1) / cr;
+      slots = (static_cast<int64_t>(maxrows) * st <= ring) ? nch : ring / (cr * st);
+      crs[i] = cr;
+      sls[i] = std::max(1, std::min(bl::kDecMaxSlots, slots));
+      continue;
+    }
     if (mode == bl::kModeResident && fmt == bl::kFmt2Bit && dec_split(p.K, a) > 1)
       cr = std::min(cr, bl::kDecSplitRows / rt * rt);   // split rows: the chunk's totals in shared memory
     if (mode == bl::kModeBig) {
@@ -497,11 +519,26 @@ bl_status launch_decode(const bl_linear* const* probs, int n, int in_mode, int Q
   }
   const bool norm = in_mode == bl::kInRmsNorm || in_mode == bl::kInLayerNorm;
   const bool big = !norm && wbytes > static_cast<double>(sms) * bl::kDecRingBytes;
+  const bool relu2 = in_mode == bl::kInRelu2 || in_mode == bl::kInRelu2Gated;
+  bl::G2Table tab;
+  if (!big) {
+    // row-lane mode when every CTA's rows fit its shared row totals
+    const int grid = fill_decode_table(&tab, probs, n, sms, bl::kModeRowLane, 0, Us, bias, eps);
+    bool fits = true;
+    for (int i = 0; i < n; ++i)
+      fits = fits && tab.p[i].rows_per_cta + (tab.p[i].rows_rem ? 1 : 0) <= bl::kDecLaneMaxRows;
+    if (fits) {
+      if (relu2) return launch_dec_t<0, bl::kDecRelu2, bl::kFmt2Bit, bl::kModeRowLane>(tab, grid, in_mode, Q, out_mode, stream);
+      if (in_mode == bl::kInRmsNorm)
+        return launch_dec_t<0, bl::kDecRms, bl::kFmt2Bit, bl::kModeRowLane>(tab, grid, in_mode, Q, out_mode, stream);
+      if (in_mode == bl::kInLayerNorm)
+        return launch_dec_t<0, bl::kDecLn, bl::kFmt2Bit, bl::kModeRowLane>(tab, grid, in_mode, Q, out_mode, stream);
+      return launch_dec_t<0, bl::kDecPlain, bl::kFmt2Bit, bl::kModeRowLane>(tab, grid, in_mode, Q, out_mode, stream);
+    }
+  }
   const int mode = big ? bl::kModeBig : bl::kModeResident;
   const int a = big ? dec_cpl(maxK) : dec_pick_wplr(probs, n);
-  bl::G2Table tab;
   const int grid = fill_decode_table(&tab, probs, n, sms, mode, a, Us, bias, eps);
-  const bool relu2 = in_mode == bl::kInRelu2 || in_mode == bl::kInRelu2Gated;
   if (big) {
     if (relu2) return launch_dec_big<bl::kDecRelu2>(a, tab, grid, in_mode, Q, out_mode, stream);
     return launch_dec_big<bl::kDecPlain>(a, tab, grid, in_mode, Q, out_mode, stream);

@@ -77,10 +77,10 @@ __host__ __device__ constexpr bool dec_big2(int mode, int fmt) { return mode == 
 __host__ __device__ constexpr int dec_warps(int mode, int fmt) { return dec_big2(mode, fmt) ? kDecBigWarps : kDecWarps; }
 __host__ __device__ constexpr int dec_threads(int mode, int fmt) { return (dec_warps(mode, fmt) + 1) * 32; }
 __host__ __device__ constexpr int dec_ring_bytes(int mode, int fmt) {
-  return mode == 0 ? kDecRingBytes : (fmt == 0 ? kDecBigRingBytes : kDecB3BigRingBytes);
+  return mode != 1 ? kDecRingBytes : (fmt == 0 ? kDecBigRingBytes : kDecB3BigRingBytes);
 }
 __host__ __device__ constexpr int dec_chunk_max(int mode, int fmt) {
-  return mode == 0 ? kDecChunkMax : (fmt == 0 ? kDecBigChunkMax : kDecB3BigChunkMax);
+  return mode != 1 ? kDecChunkMax : (fmt == 0 ? kDecBigChunkMax : kDecB3BigChunkMax);
 }
 __host__ __device__ constexpr int dec_smem_bytes(int mode, int fmt) { return dec_ring_bytes(mode, fmt) + kDecActBytes; }
 
@@ -92,7 +92,21 @@ enum DecPre : int { kDecPlain = 0, kDecRelu2 = 1, kDecRms = 2, kDecLn = 3 };
 // Weight storage: 2 bits a weight, or base 3 (five weights a byte, see
 // bl_weights.cuh).
 enum DecFmt : int { kFmt2Bit = 0, kFmtBase3 = 1 };
-enum DecMode : int { kModeResident = 0, kModeBig = 1 };
+// kModeRowLane: resident layers of 2-bit rows with each lane owning a whole
+// row (see the consumer loop); kModeResident keeps the column-split register
+// path for row ranges that this mode does not take.
+enum DecMode : int { kModeResident = 0, kModeBig = 1, kModeRowLane = 2 };
+
+// Row-lane mode: rows of a 32-row tile sit in shared memory at a stride of an
+// odd number of 16-byte units (the row's bytes plus 16 or 32), so the eight
+// lanes of a quarter-warp that read the same 16-byte column of eight rows hit
+// eight different bank groups; a tile is one ring chunk.
+constexpr int kDecLaneRows = 32;
+constexpr int kDecLaneMaxRows = 512;             // rows of one CTA (shared row totals)
+constexpr int kDecSegs = kDecMaxK / 512;          // 512-weight segments of the longest row
+__host__ __device__ constexpr int dec_lane_stride(int row_bytes) {
+  return row_bytes + (((row_bytes >> 4) & 1) ? 32 : 16);
+}
 
 // Rows a warp (or a team of warps) takes at once.
 constexpr int kDecRegRows = 2;     // 2-bit rows, token codes in registers
@@ -297,10 +311,12 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   constexpr bool NORM = RMS || LN;
   constexpr bool B3 = FMT == kFmtBase3;
   constexpr bool BIG = MODE == kModeBig;
+  constexpr bool LANES = MODE == kModeRowLane;
   constexpr int RING = dec_ring_bytes(MODE, FMT);
   static_assert(!B3 || (A == 0 && PRE == kDecPlain), "base-3 rows take the shared-memory token path");
+  static_assert(!LANES || (A == 0 && !B3), "row-lane mode: 2-bit rows, token codes read from shared memory");
   static_assert(!BIG || B3 || (A >= 1 && A <= kDecBigMaxCpl), "big mode keeps 1..4 chunks a lane");
-  static_assert(B3 || BIG || (A >= 1 && A <= kDecRegMaxWpl), "resident register path: 1..5 words a lane");
+  static_assert(B3 || BIG || LANES || (A >= 1 && A <= kDecRegMaxWpl), "resident register path: 1..5 words a lane");
   int pi = 0;
   while (pi + 1 < tab.count && static_cast<int>(blockIdx.x) >= tab.p[pi + 1].cta_begin) ++pi;
   const void* __restrict__ X = tab.p[pi].X;
@@ -329,12 +345,19 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   __shared__ unsigned long long s_s1[LN ? kS1Limbs : 1];
   __shared__ long long s_w1[LN ? CW : 1];
   __shared__ float s_rms, s_mu;
+  // row totals of split rows (resident register path: two chunks' worth;
+  // row-lane mode: one per row of the CTA), and minus the sum of the token's
+  // codes in each 512-weight segment (row-lane mode)
+  __shared__ int s_rowsum[kDecLaneMaxRows];
+  __shared__ int s_negseg[LANES ? kDecSegs : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = B3 ? base3_row_words(K) : (K >> 4);   // 32-bit words of a row
   const int row_bytes = 4 * words;
   const int nch = rows > 0 ? (rows + CR - 1) / CR : 0;
-  const int chunk_bytes = CR * row_bytes;
+  // row-lane mode: rows at a padded stride in the ring
+  const int rstride = LANES ? dec_lane_stride(row_bytes) : row_bytes;
+  const int chunk_bytes = CR * rstride;
   volatile int* abort_v = &abort_flag;
 
   if (threadIdx.x == 0) {
@@ -351,9 +374,60 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   if constexpr (LN) {
     if (threadIdx.x < kS1Limbs) s_s1[threadIdx.x] = 0ull;
   }
+  if constexpr (LANES) {
+    for (int t = threadIdx.x; t < kDecLaneMaxRows; t += blockDim.x) s_rowsum[t] = 0;
+    if (threadIdx.x < kDecSegs) s_negseg[threadIdx.x] = 0;
+  }
   __syncthreads();
   pdl_launch_dependents();
 
+  if (warp == CW && LANES) {
+    // ---------------- producer, row-lane mode: one copy per row, padded stride ----------------
+    const uint8_t* base = Wp + static_cast<size_t>(r0) * row_bytes;
+    const int pre = min(nch, slots);
+    if (lane == 0)
+      for (int c = 0; c < pre; ++c)
+        mbar_arrive_expect_tx(&full[c], static_cast<uint32_t>(min(CR, rows - c * CR) * row_bytes));
+    __syncwarp();
+    for (int c = 0; c < pre; ++c) {
+      const int cr = min(CR, rows - c * CR);
+      for (int r = lane; r < cr; r += 32)
+        bulk_load(dec_smem + c * chunk_bytes + r * rstride, base + static_cast<size_t>(c * CR + r) * row_bytes,
+                  static_cast<uint32_t>(row_bytes), &full[c]);
+    }
+    if (lane == 0 && nch > pre) {
+      const size_t off0 = static_cast<size_t>(pre) * CR * row_bytes;
+      const size_t bytes = static_cast<size_t>(rows) * row_bytes;
+      for (size_t off = off0; off < bytes; off += kPrefetchChunk)
+        bulk_prefetch_l2(base + off, static_cast<uint32_t>(min(static_cast<size_t>(kPrefetchChunk), bytes - off)));
+    }
+    int issued = pre;
+    int s = 0, ph = 1;   // slot and phase parity of chunk c
+    for (int c = pre; c < nch; ++c) {
+      const int cr = min(CR, rows - c * CR);
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(&empty[s], ph ^ 1u, abort_v, limit_ns, 21);
+        if (ok) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(cr * row_bytes));
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      for (int r = lane; r < cr; r += 32)
+        bulk_load(dec_smem + s * chunk_bytes + r * rstride, base + static_cast<size_t>(c * CR + r) * row_bytes,
+                  static_cast<uint32_t>(row_bytes), &full[s]);
+      issued = c + 1;
+      if (++s == slots) {
+        s = 0;
+        ph ^= 1;
+      }
+    }
+    // no copy may be in flight when the CTA exits
+    if (lane == 0)
+      for (int s = 0; s < slots && s < issued; ++s) {
+        const int last = s + slots * ((issued - 1 - s) / slots);
+        mbar_wait(&full[s], (last / slots) & 1, nullptr, limit_ns, 22);
+      }
+    return;
+  }
   if (warp == CW) {
     // ---------------- producer (never waits on the preceding kernel) ----------------
     if (lane == 0) {
@@ -518,21 +592,39 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = threadIdx.x + CT * u;
+      uint2 q = make_uint2(0u, 0u);
       if (c < nchx) {
         if constexpr (RELU2) {
           float h[8];
           relu2_8(xv[u], uv[u], gated, h);
-          *reinterpret_cast<uint2*>(&s_act[8 * c]) = dec_quant8_f32(h, sc);
+          q = dec_quant8_f32(h, sc);
         } else {
-          *reinterpret_cast<uint2*>(&s_act[8 * c]) = dec_quant8(xv[u], sc);
+          q = dec_quant8(xv[u], sc);
         }
+        *reinterpret_cast<uint2*>(&s_act[8 * c]) = q;
+      }
+      if constexpr (LANES) {
+        // the warp's 256 codes lie in one 512-code segment
+        const int ns = __reduce_add_sync(0xffffffffu, __dp4a(static_cast<int>(q.x), -1, __dp4a(static_cast<int>(q.y), -1, 0)));
+        if (lane == 0 && c - lane < nchx) atomicAdd(&s_negseg[(c - lane) >> 6], ns);
       }
     }
   } else {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = threadIdx.x + CT * u;
-      if (c < nchx) *reinterpret_cast<uint4*>(&s_act[16 * c]) = xv[u];
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (c < nchx) {
+        v = xv[u];
+        *reinterpret_cast<uint4*>(&s_act[16 * c]) = v;
+      }
+      if constexpr (LANES) {
+        // the warp's 512 codes are one segment
+        int r4[4] = {0, 0, 0, 0};
+        dec_negsum4(v, r4);
+        const int ns = __reduce_add_sync(0xffffffffu, (r4[0] + r4[1]) + (r4[2] + r4[3]));
+        if (lane == 0 && c - lane < nchx) atomicAdd(&s_negseg[(c - lane) >> 5], ns);
+      }
     }
   }
   if constexpr (B3) {
@@ -549,11 +641,11 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   // 32 A p + l + 32 i (i < A); big mode, lane l keeps the codes of the 16-byte
   // chunks l + 32 i (i < A), word g of chunk i at [4 i + g].  Base-3 rows read
   // the codes from shared memory.
-  constexpr bool REGP = !B3;
-  const int S = BIG ? 1 : tab.p[pi].ksplit;
+  constexpr bool REGP = !B3 && !LANES;
+  const int S = (BIG || LANES) ? 1 : tab.p[pi].ksplit;
   const int team = warp / S, part = warp - team * S, teams = CW / S;
   const int word0 = BIG ? 0 : 32 * A * part;
-  constexpr int AW = B3 ? 1 : (BIG ? 4 * A : A);
+  constexpr int AW = (B3 || LANES) ? 1 : (BIG ? 4 * A : A);
   uint32_t act[AW][4];
   int nr[4] = {0, 0, 0, 0};
   if constexpr (REGP) {
@@ -568,7 +660,7 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
       act[i][3] = v.w;
       dec_negsum4(v, nr);
     }
-  } else {
+  } else if constexpr (B3) {
     for (int wi = lane; wi < words; wi += 32) {
       const uint32_t* a = reinterpret_cast<const uint32_t*>(&s_act[20 * wi]);
       dec_negsum4(make_uint4(a[0], a[1], a[2], a[3]), nr);
@@ -586,12 +678,72 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   // kDecSplitRows rows; otherwise once per chunk (chunks of split rows hold
   // at most kDecSplitRows rows), with the chunk waits agreed CTA-wide so a
   // timeout unwinds every consumer together.
+  if constexpr (LANES) {
+    // ---------------- consumers, row-lane mode ----------------
+    // Lane l of a warp owns row l of a 32-row tile (one ring chunk) and takes
+    // one 512-weight segment of it per item: per 16-byte column of 64
+    // weights, its own row's 16 bytes (eight lanes of a quarter-warp hit eight
+    // bank groups thanks to the padded stride) and the matching 64 token codes
+    // (one address for the whole warp), four masked dp4a per 32-bit word.
+    // Items run chunk by chunk, segment-major inside a chunk: item i goes to
+    // warp i % 16.  Each item adds its rows' partial totals into shared row
+    // totals (integer adds, any order); one store pass ends the CTA.
+    const int upr = K >> 6;               // 16-byte columns of a row
+    const int segs = (upr + 7) >> 3;
+    const uint4* act4 = reinterpret_cast<const uint4*>(s_act);
+    int it = warp, ibase = 0;
+    int s = 0, ph = 0;
+    for (int c = 0; c < nch; ++c) {
+      bool ok = mbar_wait(&full[s], ph, abort_v, limit_ns, 23);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int c0 = c * CR;
+      const int crow = min(CR, rows - c0);
+      const uint8_t* sbase = dec_smem + s * chunk_bytes;
+      const uint4* wrow = reinterpret_cast<const uint4*>(sbase + (lane < crow ? lane : 0) * rstride);
+      for (; it < ibase + segs; it += CW) {
+        const int seg = it - ibase;
+        const uint4* wp = wrow + 8 * seg;
+        const uint4* ap = act4 + 32 * seg;
+        int acc[4] = {s_negseg[seg], 0, 0, 0};
+        const int nu = min(8, upr - 8 * seg);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (t < nu) {
+            const uint4 w = wp[t];
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint4 a = ap[4 * t + g];
+              acc[0] = dp4a_us(wv[g] & 0x03030303u, a.x, acc[0]);
+              acc[1] = dp4a_us(wv[g] & 0x0c0c0c0cu, a.y, acc[1]);
+              acc[2] = dp4a_us(wv[g] & 0x30303030u, a.z, acc[2]);
+              acc[3] = dp4a_us(wv[g] & 0xc0c0c0c0u, a.w, acc[3]);
+            }
+          }
+        }
+        if (lane < crow) atomicAdd(&s_rowsum[c0 + lane], dec_fold(acc));
+      }
+      ibase += segs;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == slots) {
+        s = 0;
+        ph ^= 1;
+      }
+    }
+    // every consumer leaves the loop (a bounded wait that gives up ends it
+    // too), so all of them reach this barrier; a stalled CTA stores nothing
+    const bool all_ok = named_bar_and(1, CT, !*abort_v);
+    if (all_ok)
+      for (int t = threadIdx.x; t < rows; t += CT) dec_put<kOutAny>(s_rowsum[t], r0 + t, f, Y, bias, out_mode);
+    return;
+  }
   constexpr int RT = dec_group_rows<FMT, MODE>();
-  __shared__ int s_rowsum[2][kDecSplitRows];
   const bool active = team < teams;
   const bool once = rows <= kDecSplitRows;   // split rows: one final store pass
   if (S > 1) {
-    for (int t = threadIdx.x; t < 2 * kDecSplitRows; t += CT) (&s_rowsum[0][0])[t] = 0;
+    for (int t = threadIdx.x; t < 2 * kDecSplitRows; t += CT) s_rowsum[t] = 0;
     named_bar_sync(1, CT);
   }
   auto walk = [&](auto out_tag) {
@@ -621,7 +773,7 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
       const int cend = min(c0 + CR, rows);
       const uint8_t* sbase = dec_smem + s * chunk_bytes;
       // split rows: row r of the CTA at rs[r - rbase]
-      int* rs = once ? &s_rowsum[0][0] : s_rowsum[c & 1];
+      int* rs = once ? s_rowsum : s_rowsum + (c & 1) * kDecSplitRows;
       const int rbase = once ? 0 : c0;
       if (active) {
         for (; g * RT < cend; g += teams) {
@@ -670,7 +822,7 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
       // nothing (its status word records the timeout)
       const bool all_ok = named_bar_and(1, CT, !*abort_v);
       if (all_ok)
-        for (int t = threadIdx.x; t < rows; t += CT) dec_put<OUT>(s_rowsum[0][t], r0 + t, f, Y, bias, out_mode);
+        for (int t = threadIdx.x; t < rows; t += CT) dec_put<OUT>(s_rowsum[t], r0 + t, f, Y, bias, out_mode);
     }
   };
   // one copy of the loop for every output type: a smaller kernel runs faster
