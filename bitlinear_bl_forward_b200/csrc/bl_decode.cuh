@@ -103,7 +103,8 @@ enum DecMode : int { kModeResident = 0, kModeBig = 1, kModeRowLane = 2 };
 // eight different bank groups; a tile is one ring chunk.
 constexpr int kDecLaneRows = 32;
 constexpr int kDecLaneMaxRows = 512;             // rows of one CTA (shared row totals)
-constexpr int kDecSegs = kDecMaxK / 512;          // 512-weight segments of the longest row
+constexpr int kDecLaneMaxRT = 2;                 // rows a lane takes at once (measured best of 1, 2, 4)
+constexpr int kDecHalfSegs = kDecMaxK / 256;     // 256-weight (four-column) items of the longest row
 __host__ __device__ constexpr int dec_lane_stride(int row_bytes) {
   return row_bytes + (((row_bytes >> 4) & 1) ? 32 : 16);
 }
@@ -293,6 +294,58 @@ __device__ __forceinline__ void dec3_dot(const uint8_t* rowp, int row_bytes, int
   for (int r = 0; r < RT; ++r) part[r] = acc[r];
 }
 
+// Row-lane mode, one item: lane l takes rows l + 32 j (j < RT) of the rows
+// at row0 (stride rstride; rows at or past `live` read row 0 again and are
+// discarded), nu <= 4 16-byte columns from row0 on, with the token codes of
+// those columns at ap (16 bytes per 32-bit weight word); each row starts at
+// neg (minus the codes' sum) and its folded total is added to rs[row].
+template <int RT>
+__device__ __forceinline__ void dec_lane_item(const uint8_t* row0, int rstride, int live, int lane, const uint4* ap,
+                                              int nu, int neg, int* rs) {
+  const uint4* wp[RT];
+#pragma unroll
+  for (int j = 0; j < RT; ++j) {
+    const int r = 32 * j + lane;
+    wp[j] = reinterpret_cast<const uint4*>(row0 + (r < live ? r : 0) * rstride);
+  }
+  int acc[RT][4];
+#pragma unroll
+  for (int j = 0; j < RT; ++j) {
+    acc[j][0] = neg;
+    acc[j][1] = acc[j][2] = acc[j][3] = 0;
+  }
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    if (t < nu) {
+      uint32_t w[RT][4];
+#pragma unroll
+      for (int j = 0; j < RT; ++j) {
+        const uint4 v = wp[j][t];
+        w[j][0] = v.x;
+        w[j][1] = v.y;
+        w[j][2] = v.z;
+        w[j][3] = v.w;
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const uint4 a = ap[4 * t + g];
+#pragma unroll
+        for (int j = 0; j < RT; ++j) {
+          acc[j][0] = dp4a_us(w[j][g] & 0x03030303u, a.x, acc[j][0]);
+          acc[j][1] = dp4a_us(w[j][g] & 0x0c0c0c0cu, a.y, acc[j][1]);
+          acc[j][2] = dp4a_us(w[j][g] & 0x30303030u, a.z, acc[j][2]);
+          acc[j][3] = dp4a_us(w[j][g] & 0xc0c0c0c0u, a.w, acc[j][3]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < RT; ++j) {
+    const int r = 32 * j + lane;
+    if (r < live) atomicAdd(rs + r, dec_fold(acc[j]));
+  }
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -349,7 +402,7 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   // row-lane mode: one per row of the CTA), and minus the sum of the token's
   // codes in each 512-weight segment (row-lane mode)
   __shared__ int s_rowsum[kDecLaneMaxRows];
-  __shared__ int s_negseg[LANES ? kDecSegs : 1];
+  __shared__ int s_negseg[LANES ? kDecHalfSegs : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = B3 ? base3_row_words(K) : (K >> 4);   // 32-bit words of a row
@@ -376,7 +429,7 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   }
   if constexpr (LANES) {
     for (int t = threadIdx.x; t < kDecLaneMaxRows; t += blockDim.x) s_rowsum[t] = 0;
-    if (threadIdx.x < kDecSegs) s_negseg[threadIdx.x] = 0;
+    if (threadIdx.x < kDecHalfSegs) s_negseg[threadIdx.x] = 0;
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -604,9 +657,9 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
         *reinterpret_cast<uint2*>(&s_act[8 * c]) = q;
       }
       if constexpr (LANES) {
-        // the warp's 256 codes lie in one 512-code segment
+        // the warp's 256 codes are one four-column item's
         const int ns = __reduce_add_sync(0xffffffffu, __dp4a(static_cast<int>(q.x), -1, __dp4a(static_cast<int>(q.y), -1, 0)));
-        if (lane == 0 && c - lane < nchx) atomicAdd(&s_negseg[(c - lane) >> 6], ns);
+        if (lane == 0 && c - lane < nchx) atomicAdd(&s_negseg[(c - lane) >> 5], ns);
       }
     }
   } else {
@@ -619,11 +672,14 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
         *reinterpret_cast<uint4*>(&s_act[16 * c]) = v;
       }
       if constexpr (LANES) {
-        // the warp's 512 codes are one segment
+        // each half-warp's 256 codes are one four-column item's
         int r4[4] = {0, 0, 0, 0};
         dec_negsum4(v, r4);
-        const int ns = __reduce_add_sync(0xffffffffu, (r4[0] + r4[1]) + (r4[2] + r4[3]));
-        if (lane == 0 && c - lane < nchx) atomicAdd(&s_negseg[(c - lane) >> 5], ns);
+        int ns = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) ns += __shfl_xor_sync(0xffffffffu, ns, o);
+        const int c0 = c - (lane & 15);
+        if ((lane & 15) == 0 && c0 < nchx) atomicAdd(&s_negseg[c0 >> 4], ns);
       }
     }
   }
@@ -680,56 +736,65 @@ __global__ void __launch_bounds__(dec_threads(MODE, FMT), (MODE == kModeBig && F
   // timeout unwinds every consumer together.
   if constexpr (LANES) {
     // ---------------- consumers, row-lane mode ----------------
-    // Lane l of a warp owns row l of a 32-row tile (one ring chunk) and takes
-    // one 512-weight segment of it per item: per 16-byte column of 64
-    // weights, its own row's 16 bytes (eight lanes of a quarter-warp hit eight
-    // bank groups thanks to the padded stride) and the matching 64 token codes
-    // (one address for the whole warp), four masked dp4a per 32-bit word.
-    // Items run chunk by chunk, segment-major inside a chunk: item i goes to
-    // warp i % 16.  Each item adds its rows' partial totals into shared row
-    // totals (integer adds, any order); one store pass ends the CTA.
+    // Lane l of a warp owns rows l, l + 32, ... of a group of up to 128 rows
+    // (one to four 32-row ring chunks) and takes four 16-byte columns (256
+    // weights) of them per item: per column, its rows' 16 bytes (the eight
+    // lanes of a quarter-warp hit eight bank groups thanks to the padded
+    // stride) and the matching 64 token codes (one address for the whole
+    // warp, shared by the lane's rows), four masked dp4a per 32-bit word.
+    // Item i goes to warp i % 16.  Each item adds its rows' partial totals
+    // into shared row totals (integer adds, any order); one store pass ends
+    // the CTA.  When the ring must be reused, chunks are taken one at a time
+    // (one row a lane) and released in order.
     const int upr = K >> 6;               // 16-byte columns of a row
-    const int segs = (upr + 7) >> 3;
+    const int nhs = (upr + 3) >> 2;       // four-column items of a row
     const uint4* act4 = reinterpret_cast<const uint4*>(s_act);
-    int it = warp, ibase = 0;
-    int s = 0, ph = 0;
-    for (int c = 0; c < nch; ++c) {
-      bool ok = mbar_wait(&full[s], ph, abort_v, limit_ns, 23);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const int c0 = c * CR;
-      const int crow = min(CR, rows - c0);
-      const uint8_t* sbase = dec_smem + s * chunk_bytes;
-      const uint4* wrow = reinterpret_cast<const uint4*>(sbase + (lane < crow ? lane : 0) * rstride);
-      for (; it < ibase + segs; it += CW) {
-        const int seg = it - ibase;
-        const uint4* wp = wrow + 8 * seg;
-        const uint4* ap = act4 + 32 * seg;
-        int acc[4] = {s_negseg[seg], 0, 0, 0};
-        const int nu = min(8, upr - 8 * seg);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (t < nu) {
-            const uint4 w = wp[t];
-            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint4 a = ap[4 * t + g];
-              acc[0] = dp4a_us(wv[g] & 0x03030303u, a.x, acc[0]);
-              acc[1] = dp4a_us(wv[g] & 0x0c0c0c0cu, a.y, acc[1]);
-              acc[2] = dp4a_us(wv[g] & 0x30303030u, a.z, acc[2]);
-              acc[3] = dp4a_us(wv[g] & 0xc0c0c0c0u, a.w, acc[3]);
-            }
-          }
-        }
-        if (lane < crow) atomicAdd(&s_rowsum[c0 + lane], dec_fold(acc));
+    if (nch <= slots) {
+      // every chunk resident: row r at r * rstride
+      constexpr int GR = kDecLaneRows * kDecLaneMaxRT;   // rows of a group
+      const int ngroups = (rows + GR - 1) / GR;
+      for (int it = warp; it < ngroups * nhs; it += CW) {
+        const int g = it / nhs, h = it - g * nhs;
+        const int live = rows - GR * g;
+        const int rt = min(kDecLaneMaxRT, (live + 31) >> 5);
+        bool ok = true;
+        for (int j = 0; j < rt; ++j) ok = ok && mbar_wait(&full[kDecLaneMaxRT * g + j], 0, abort_v, limit_ns, 23);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const uint8_t* row0 = dec_smem + static_cast<size_t>(GR * g) * rstride + 64 * h;
+        const uint4* ap = act4 + 16 * h;
+        const int nu = min(4, upr - 4 * h);
+        const int neg = s_negseg[h];
+        int* rs = s_rowsum + GR * g;
+        if (kDecLaneMaxRT >= 4 && rt == 4)
+          dec_lane_item<(kDecLaneMaxRT >= 4 ? 4 : 1)>(row0, rstride, live, lane, ap, nu, neg, rs);
+        else if (kDecLaneMaxRT >= 3 && rt == 3)
+          dec_lane_item<(kDecLaneMaxRT >= 3 ? 3 : 1)>(row0, rstride, live, lane, ap, nu, neg, rs);
+        else if (kDecLaneMaxRT >= 2 && rt == 2)
+          dec_lane_item<(kDecLaneMaxRT >= 2 ? 2 : 1)>(row0, rstride, live, lane, ap, nu, neg, rs);
+        else
+          dec_lane_item<1>(row0, rstride, live, lane, ap, nu, neg, rs);
       }
-      ibase += segs;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (++s == slots) {
-        s = 0;
-        ph ^= 1;
+    } else {
+      int it = warp, ibase = 0;
+      int s = 0, ph = 0;
+      for (int c = 0; c < nch; ++c) {
+        bool ok = mbar_wait(&full[s], ph, abort_v, limit_ns, 23);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const int c0 = c * CR;
+        const uint8_t* sbase = dec_smem + s * chunk_bytes;
+        for (; it < ibase + nhs; it += CW) {
+          const int h = it - ibase;
+          dec_lane_item<1>(sbase + 64 * h, rstride, min(CR, rows - c0), lane, act4 + 16 * h, min(4, upr - 4 * h),
+                           s_negseg[h], s_rowsum + c0);
+        }
+        ibase += nhs;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (++s == slots) {
+          s = 0;
+          ph ^= 1;
+        }
       }
     }
     // every consumer leaves the loop (a bounded wait that gives up ends it
