@@ -54,6 +54,9 @@ SIGNATURES = {
     "bl_quant_act_layernorm": (_int, [_p, ctypes.c_float, _i64, _i64, _int, _p, _p, _p, _p, _p]),
     "bl_forward_grouped_host_staging_bytes": (_sz, [_int, _p]),
     "bl_forward_grouped_host": (_int, [_int, _p, _int, _p, _sz, _p, _sz, _p]),
+    "bl_forward_grouped_host_graph": (_int, [_int, _p, _int, _p, _sz, _p, _sz, _p, ctypes.POINTER(_p)]),
+    "bl_graph_launch": (_int, [_p, _p]),
+    "bl_graph_destroy": (None, [_p]),
     "bl_forward_norm_grouped_workspace_bytes": (_sz, [_int, _p, _int]),
     "bl_forward_norm_grouped": (_int, [_int, _p, _int, _p, ctypes.c_float, _int, _p, _sz, _p]),
     "bl_matmul_i32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
@@ -317,9 +320,13 @@ class PreparedGroupedHost:
     (X host bf16 [M, K], Wp, gamma, N) and outs the host bf16 [M, N] outputs
     (pinned memory keeps the copies asynchronous).  Each call enqueues on the
     current stream the input copies, the grouped forward and the output
-    copies; synchronise the stream before reading the outputs."""
+    copies; synchronise the stream before reading the outputs.  graph=True
+    records the call once as a CUDA graph (bl_forward_grouped_host_graph:
+    this runs the step once on the current stream and waits for it) and each
+    call replays it (bl_graph_launch), reading the current contents of the
+    same host inputs."""
 
-    def __init__(self, problems, outs, bits: int = 8, device="cuda"):
+    def __init__(self, problems, outs, bits: int = 8, device="cuda", graph: bool = False):
         self.outs = outs
         self._n = len(problems)
         self._arr = _host_structs(problems, outs)
@@ -333,10 +340,39 @@ class PreparedGroupedHost:
         self._keep = (list(problems), list(outs))
         self._args = (self._stg.data_ptr(), nst, self._ws.data_ptr() if self._ws is not None else None, nws)
         self._fn = lib().bl_forward_grouped_host
+        self._graph = bl_forward_grouped_host_graph(self._n, self._arr, bits, *self._args) if graph else None
 
     def __call__(self):
-        _check(self._fn(self._n, self._arr, self._bits, *self._args, _stream()), "bl_forward_grouped_host")
+        if self._graph is not None:
+            bl_graph_launch(self._graph)
+        else:
+            _check(self._fn(self._n, self._arr, self._bits, *self._args, _stream()), "bl_forward_grouped_host")
         return self.outs
+
+    def __del__(self):
+        g = getattr(self, "_graph", None)
+        if g is not None and _lib is not None:
+            bl_graph_destroy(g)
+            self._graph = None
+
+
+def bl_forward_grouped_host_graph(count, structs, bits, staging, staging_bytes, workspace, workspace_bytes):
+    """Record a host-buffer grouped forward as a CUDA graph (returns the
+    handle; see PreparedGroupedHost, which owns one)."""
+    h = ctypes.c_void_p(None)
+    _check(lib().bl_forward_grouped_host_graph(count, structs, bits, staging, staging_bytes, workspace,
+                                               workspace_bytes, _stream(), ctypes.byref(h)),
+           "bl_forward_grouped_host_graph")
+    return h
+
+
+def bl_graph_launch(graph):
+    """One replay of a recorded graph on the current stream."""
+    _check(lib().bl_graph_launch(graph, _stream()), "bl_graph_launch")
+
+
+def bl_graph_destroy(graph):
+    lib().bl_graph_destroy(graph)
 
 
 def bl_forward_grouped_host(problems, outs, bits: int = 8):

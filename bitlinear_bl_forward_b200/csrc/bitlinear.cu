@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -1689,6 +1690,84 @@ bl_status bl_selftest_wait_timeout(unsigned long long limit_ns, int* waited_ok, 
   if (limit_ns > 10ull * kWaitLimitNs) return BL_ERR_INVALID_ARG;
   bl::bl_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, waited_ok);
   return last_cuda();
+}
+
+// ---------------------------------------------------------------------------
+// A host-buffer grouped forward recorded once as a CUDA graph and replayed.
+// ---------------------------------------------------------------------------
+
+struct bl_graph_s {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+
+bl_status bl_forward_grouped_host_graph(int count, const bl_linear* problems, int bits, void* staging,
+                                        size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                                        cudaStream_t stream, bl_graph* out) {
+  const NvtxRange nvtx_range("bl_forward_grouped_host_graph");
+  if (out == nullptr) return BL_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (problems == nullptr) return BL_ERR_INVALID_ARG;
+  if (count <= 0 || count > bl::kG2MaxProblems) return BL_ERR_UNSUPPORTED;
+  // one plain call first, on the caller's stream (after the caller's work
+  // there): it validates the arguments and does the kernels' one-time set-up
+  // on this device outside the capture
+  bl_status rc = bl_forward_grouped_host(count, problems, bits, staging, staging_bytes, workspace, workspace_bytes,
+                                         stream);
+  if (rc != BL_OK) return rc;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BL_ERR_CUDA;
+  }
+  cudaStream_t s = nullptr;   // the capture runs on a private stream
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BL_ERR_CUDA;
+  }
+  cudaGraph_t g = nullptr;
+  if (rc == BL_OK) {
+    if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+      rc = BL_ERR_CUDA;
+    } else {
+      rc = bl_forward_grouped_host(count, problems, bits, staging, staging_bytes, workspace, workspace_bytes, s);
+      if (cudaStreamEndCapture(s, &g) != cudaSuccess && rc == BL_OK) rc = BL_ERR_CUDA;
+    }
+  }
+  cudaGraphExec_t ex = nullptr;
+  if (rc == BL_OK && cudaGraphInstantiate(&ex, g, 0) != cudaSuccess) rc = BL_ERR_CUDA;
+  bl_graph h = nullptr;
+  if (rc == BL_OK) {
+    h = new (std::nothrow) bl_graph_s;
+    if (h == nullptr) rc = BL_ERR_CUDA;
+  }
+  if (rc != BL_OK) {
+    (void)cudaGetLastError();
+    if (ex) cudaGraphExecDestroy(ex);
+    if (g) cudaGraphDestroy(g);
+    cudaStreamDestroy(s);
+    return rc;
+  }
+  h->graph = g;
+  h->exec = ex;
+  cudaStreamDestroy(s);
+  *out = h;
+  return BL_OK;
+}
+
+bl_status bl_graph_launch(bl_graph graph, cudaStream_t stream) {
+  if (graph == nullptr) return BL_ERR_INVALID_ARG;
+  if (cudaGraphLaunch(graph->exec, stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BL_ERR_CUDA;
+  }
+  return BL_OK;
+}
+
+void bl_graph_destroy(bl_graph graph) {
+  if (graph == nullptr) return;
+  if (graph->exec) cudaGraphExecDestroy(graph->exec);
+  if (graph->graph) cudaGraphDestroy(graph->graph);
+  delete graph;
 }
 
 }  // extern "C"

@@ -249,6 +249,36 @@ BL_API bl_status bl_forward_grouped_host(int count, const bl_linear* problems, i
                                          size_t staging_bytes, void* workspace, size_t workspace_bytes,
                                          cudaStream_t stream);
 /*
+ * The host-buffer grouped forward above, recorded once as a CUDA graph and
+ * replayed.  No counterpart on the pages: it serves callers that run the
+ * same step over and over on fixed buffers (a serving loop that writes each
+ * new token into the same pinned host buffer), for whom the host work of a
+ * call -- argument checks, the launch table, one API call per copy and per
+ * kernel -- costs several times the GPU time of a one-token step; a replay
+ * is one graph launch.
+ * bl_forward_grouped_host_graph takes the arguments of
+ * bl_forward_grouped_host and keeps their pointers: every replay copies the
+ * CURRENT contents of the same host inputs in, runs the same forward and
+ * copies the outputs back to the same host outputs, using the same staging,
+ * workspace and weights, which must all stay valid (and keep their sizes)
+ * until bl_graph_destroy.  Creating it runs the step once on `stream`
+ * (the outputs are written) and waits for it, then records the step on a
+ * private stream; it must not be called while the calling thread captures
+ * a stream.  Errors: as
+ * bl_forward_grouped_host (count must be 1..8), plus BL_ERR_CUDA when the
+ * capture fails; on error *graph is NULL.
+ * bl_graph_launch enqueues one replay on `stream` (asynchronous; replays
+ * that overlap on the GPU share the staging and workspace and race).
+ * bl_graph_destroy frees the recorded graph (NULL is ignored); no replay may
+ * still be running.
+ */
+typedef struct bl_graph_s* bl_graph;
+BL_API bl_status bl_forward_grouped_host_graph(int count, const bl_linear* problems, int bits, void* staging,
+                                               size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                                               cudaStream_t stream, bl_graph* graph);
+BL_API bl_status bl_graph_launch(bl_graph graph, cudaStream_t stream);
+BL_API void bl_graph_destroy(bl_graph graph);
+/*
  * Squared-ReLU feed-forward: the down projection's input is formed from the
  * gate projection's output ("BitNet 2B4T Guide: Scaling Native 1.58-Bit
  * LLMs", section "2. Squared ReLU Activation", ReLU^2(x) = max(0, x)^2, and

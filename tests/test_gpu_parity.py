@@ -137,6 +137,24 @@ def test_few_tiles_long_k(M, K, N):
     check_forward(X, Wp, g, c, 8)
 
 
+# One-token shapes that reach each path of the row-lane decode kernel: rows
+# that overflow the shared ring (K = 8192, 47-48 rows a CTA: chunks taken one
+# at a time), more than 512 rows a CTA (the column-split fallback), rows of an
+# odd number of 16-byte columns (the wider padding) with a partial last item,
+# and fewer rows than CTAs.
+ROW_LANE = [(8192, 7000, 8), (64, 80000, 8), (192, 5000, 4), (320, 33, 8), (6912, 2561, 8)]
+
+
+@pytest.mark.parametrize("K,N,bits", ROW_LANE)
+def test_decode_row_lane_paths(K, N, bits):
+    X, W = random_case(1, K, N, seed=K + N)
+    g = o.absmean_scale(W)
+    c = o.ternary_codes(W, g)
+    Wp, gd = check_weights(W, g, c, o.pack_ternary(c))
+    check_act(X, bits)
+    check_forward(X, Wp, g, c, bits)
+
+
 def test_zero_inputs_and_degenerate_rows():
     M, K, N = 5, 128, 96
     X, W = random_case(M, K, N, seed=7)
@@ -392,6 +410,34 @@ def test_grouped_host_buffers_match_device_path(M):
     torch.cuda.synchronize()
     for a, b in zip(ys, ref):
         assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("M", [1, 130])
+def test_grouped_host_graph_replays_current_inputs(M):
+    # the step recorded as a CUDA graph: each replay copies the host inputs'
+    # current contents in and gives the outputs of a fresh device-path call
+    shapes = [(2560, 700), (2560, 264), (6912, 130)]
+    ws = []
+    for j, (K, N) in enumerate(shapes):
+        _, W = random_case(1, K, N, seed=1700 + j)
+        ws.append(bl.bl_quantize_weights(torch.from_numpy(W).cuda()))
+    xa = torch.empty((M, 2560), dtype=torch.bfloat16).pin_memory()
+    xb = torch.empty((M, 6912), dtype=torch.bfloat16).pin_memory()
+    xs = [xa, xa, xb]
+    outs = [torch.full((M, N), float("nan"), dtype=torch.bfloat16).pin_memory() for _, N in shapes]
+    probs_h = [(x, Wp, gd, N) for x, (Wp, gd), (_, N) in zip(xs, ws, shapes)]
+    for trial in range(3):
+        xa.copy_(torch.from_numpy(random_case(M, 2560, 1, seed=1800 + trial)[0].view(np.int16)).view(torch.bfloat16))
+        xb.copy_(torch.from_numpy(random_case(M, 6912, 1, seed=1900 + trial)[0].view(np.int16)).view(torch.bfloat16))
+        if trial == 0:
+            call = bl.PreparedGroupedHost(probs_h, outs, graph=True)   # records (and runs) the step
+        else:
+            call()
+        torch.cuda.synchronize()
+        ref = bl.bl_forward_grouped([(x.cuda(), Wp, gd, N) for x, (Wp, gd), (_, N) in zip(xs, ws, shapes)])
+        for a, b in zip(outs, ref):
+            assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16)), trial
+    del call
 
 
 def test_grouped_mixed_shapes_fall_back_to_sequential():
