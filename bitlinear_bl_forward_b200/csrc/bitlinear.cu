@@ -19,6 +19,7 @@
 #include "../../include/bitlinear.h"
 #include "bl_act.cuh"
 #include "bl_common.cuh"
+#include "bl_copy.cuh"
 #include "bl_tc_common.cuh"
 #include "bl_gemm_tc2.cuh"
 #include "bl_gemm_2sm.cuh"
@@ -1152,6 +1153,46 @@ bool host_staging_layout(int count, const bl_linear* problems, HostStaging* st) 
   return true;
 }
 
+// One host-buffer run: a copy kernel when the host side is pinned memory the
+// device can address (and both sides are 16-byte aligned), else a
+// copy-engine transfer.  h2d: host -> staging.
+// The device address of pinned host memory the device can address, else null.
+const uint8_t* host_dev_ptr(const void* host) {
+  cudaPointerAttributes a{};
+  const uint8_t* d = nullptr;
+  if (cudaPointerGetAttributes(&a, host) == cudaSuccess && a.type == cudaMemoryTypeHost && a.devicePointer)
+    d = static_cast<const uint8_t*>(a.devicePointer);
+  (void)cudaGetLastError();
+  return d;
+}
+
+bl_status copy_run(const uint8_t* host, uint8_t* stage, size_t bytes, bool h2d, cudaStream_t stream) {
+  const uint8_t* hdev = host_dev_ptr(host);
+  if (hdev == nullptr || !aligned16(hdev) || !aligned16(stage)) {
+    if (cudaMemcpyAsync(h2d ? static_cast<void*>(stage) : const_cast<uint8_t*>(host), h2d ? static_cast<const void*>(host) : stage,
+                        bytes, h2d ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    return BL_OK;
+  }
+  const size_t n16 = bytes >> 4;
+  const unsigned grid = static_cast<unsigned>(std::max<size_t>(1, std::min<size_t>((n16 + 255) / 256, 148)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint8_t* src = h2d ? hdev : stage;
+  uint8_t* dst = h2d ? stage : const_cast<uint8_t*>(hdev);
+  if (cudaLaunchKernelEx(&cfg, bl::bl_copy_run_kernel, src, dst, bytes) != cudaSuccess) return BL_ERR_CUDA;
+  return last_cuda();
+}
+
 size_t bl_forward_grouped_host_staging_bytes(int count, const bl_linear* problems) {
   if (count <= 0 || count > bl::kG2MaxProblems || problems == nullptr) return 0;
   HostStaging st;
@@ -1199,20 +1240,13 @@ bl_status bl_forward_grouped_host(int count, const bl_linear* problems, int bits
     dev[i].X = reinterpret_cast<const uint16_t*>(base + st.x_off[i]);
     dev[i].Y = reinterpret_cast<uint16_t*>(base + st.y_off[i]);
   }
+  bl_status rc;
   for (int r = 0; r < st.nxr; ++r)
-    if (cudaMemcpyAsync(base + st.xr[r].stage, st.xr[r].host, st.xr[r].bytes, cudaMemcpyHostToDevice, stream) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      return BL_ERR_CUDA;
-    }
-  bl_status rc = bl_forward_grouped(count, dev, bits, workspace, workspace_bytes, stream);
+    if ((rc = copy_run(st.xr[r].host, base + st.xr[r].stage, st.xr[r].bytes, true, stream)) != BL_OK) return rc;
+  rc = bl_forward_grouped(count, dev, bits, workspace, workspace_bytes, stream);
   if (rc != BL_OK) return rc;
   for (int r = 0; r < st.nyr; ++r)
-    if (cudaMemcpyAsync(const_cast<uint8_t*>(st.yr[r].host), base + st.yr[r].stage, st.yr[r].bytes,
-                        cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return BL_ERR_CUDA;
-    }
+    if ((rc = copy_run(st.yr[r].host, base + st.yr[r].stage, st.yr[r].bytes, false, stream)) != BL_OK) return rc;
   return BL_OK;
 }
 
