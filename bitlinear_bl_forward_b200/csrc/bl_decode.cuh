@@ -12,35 +12,41 @@
 // stream of weight rows through the SMs.  One launch serves a table of
 // independent one-token problems with any mix of K (e.g. the up, gate and
 // down projections of a feed-forward block); the host gives each problem
-// CTAs by a cost model, one CTA per SM.  Two ring modes:
+// CTAs by a cost model, one CTA per SM.  Ring modes:
 //
-//   * resident (layers of a few MB): a CTA takes a little under half an SM
-//     (a 96 KB ring plus the token codes, <= 56 registers a thread), so the
-//     CTAs of the next launch on the stream (programmatic dependent launch,
-//     triggered at the start) become resident beside this launch's CTAs and
-//     fetch their weights while this launch runs;
-//   * big (layers of tens of MB): one CTA per SM with a 192 KB ring (three
-//     64 KB chunks in flight per SM keep HBM busy) and the token codes of a
-//     lane's 16-byte chunks kept in registers.
+//   * row-lane (2-bit layers of a few MB, the usual case): a CTA takes a
+//     little under half an SM (a 96 KB ring plus the token codes, <= 56
+//     registers a thread), so the CTAs of the next launch on the stream
+//     (programmatic dependent launch, triggered at the start) become
+//     resident beside this launch's CTAs and fetch their weights while this
+//     launch runs.  Rows sit in the ring at a padded stride and each lane
+//     owns whole rows (see the row-lane consumer loop);
+//   * resident, column-split (the same footprint; rows of more than 512 a
+//     CTA, and base-3 rows): lane l takes 32-bit words l, l + 32, ... of
+//     every row, with its columns' token codes in registers (base-3 rows:
+//     read from shared memory);
+//   * big (layers of tens of MB): 2-bit rows with 8 consumer warps and a
+//     96 KB ring, two CTAs per SM (base-3 rows: 16 warps, a 192 KB ring, one
+//     CTA per SM), column-split with a lane's 16-byte chunks' token codes in
+//     registers.
 //
-// In both, a producer warp copies the CTA's row range into the ring
-// (cp.async.bulk, whole-row chunks, one mbarrier each) BEFORE the dependency
-// wait: the weights and gamma are parameters, not produced by the preceding
-// kernel.  Sixteen consumer warps wait for the token, quantise it once per
-// CTA into shared memory, then walk groups of rows (group g -> warp g % 16;
-// chunks hold whole groups):
+// In all of them a producer warp copies the CTA's row range into the ring
+// (cp.async.bulk, one mbarrier per chunk) BEFORE the dependency wait: the
+// weights and gamma are parameters, not produced by the preceding kernel.
+// The consumer warps wait for the token and quantise it once per CTA into
+// shared memory.  Then:
 //
-//   * 2-bit rows: lane l takes 32-bit words (resident) or 16-byte chunks
-//     (big) of each row; per word four masked unsigned-by-signed dp4a (slice
+//   * 2-bit rows: per 32-bit word four masked unsigned-by-signed dp4a (slice
 //     j of a word holds 4^j * (c+1) in each byte) into four accumulators,
 //     folded exactly as acc0 + acc1/4 + acc2/16 + acc3/64;
 //   * base-3 rows: five digits a byte, recovered by tripling (see dec3_dot);
-//   * the stored digits are c + 1, so sum_k c*q = sum_k (c+1)*q - sum_k q.  A
-//     lane visits the same columns of every row, so it starts each row at
-//     minus the sum of its own columns' codes: the warp sum is then the exact
-//     dot product, with no CTA-wide reduction of sum_k q;
-//   * one warp reduction per row, then lane r of the group rescales and
-//     stores row r (one store instruction per group).
+//   * the stored digits are c + 1, so sum_k c*q = sum_k (c+1)*q - sum_k q:
+//     each partial sum starts at minus the sum of the codes of the columns
+//     it covers (per lane in the column-split modes, per 256-column block in
+//     row-lane mode), so the totals are the exact dot products;
+//   * column-split: one warp reduction per row, then lane r of the group
+//     rescales and stores row r; row-lane: shared row totals and one store
+//     pass per CTA.
 #pragma once
 
 #include <type_traits>
