@@ -287,6 +287,31 @@ def test_grouped_host_validation(L):
     assert L.bl_forward_grouped_host(3, arr, 8, A, need, A, 1 << 20, None) == INVALID   # no empty problems
 
 
+def test_grouped_host_graph_validation(L):
+    # the recording entry validates like bl_forward_grouped_host before any
+    # CUDA call, and clears the handle on error
+    from bitlinear_bl_forward_b200.bl import BLLinear
+    H = 0x7f0000001000
+    ov = (BLLinear * 1)()
+    ov[0] = BLLinear(H, 1, 2560, 6912, A, A, H + 2048)          # output overlaps the input
+    h = ctypes.c_void_p(0x1234)
+    assert L.bl_forward_grouped_host_graph(1, ov, 8, A, 1 << 20, A, 1 << 20, None, ctypes.byref(h)) == INVALID
+    assert h.value is None
+    h = ctypes.c_void_p(0x1234)
+    assert L.bl_forward_grouped_host_graph(0, ov, 8, A, 1 << 20, A, 1 << 20, None, ctypes.byref(h)) == UNSUP
+    assert h.value is None
+    assert L.bl_forward_grouped_host_graph(9, ov, 8, A, 1 << 20, A, 1 << 20, None, ctypes.byref(h)) == UNSUP
+    assert L.bl_forward_grouped_host_graph(1, None, 8, A, 1 << 20, A, 1 << 20, None, ctypes.byref(h)) == INVALID
+    assert L.bl_forward_grouped_host_graph(1, ov, 8, A, 1 << 20, A, 1 << 20, None, None) == INVALID
+    ok = (BLLinear * 1)()
+    ok[0] = BLLinear(H, 1, 2560, 6912, A, A, H + 0x100000)
+    assert L.bl_forward_grouped_host_graph(1, ok, 8, None, 0, A, 1 << 20, None, ctypes.byref(h)) == WS
+    assert L.bl_forward_grouped_host_graph(1, ok, 5, A, 1 << 20, A, 1 << 20, None, ctypes.byref(h)) == UNSUP
+    assert h.value is None
+    assert L.bl_graph_launch(None, None) == INVALID
+    L.bl_graph_destroy(None)   # a no-op
+
+
 def test_base3_host_checks(L):
     # sizes: 4 * ceil(ceil(K / 20) / 4) bytes a row
     assert L.bl_packed_weight_bytes_b3(1, 64) == 16
