@@ -1153,9 +1153,6 @@ bool host_staging_layout(int count, const bl_linear* problems, HostStaging* st) 
   return true;
 }
 
-// One host-buffer run: a copy kernel when the host side is pinned memory the
-// device can address (and both sides are 16-byte aligned), else a
-// copy-engine transfer.  h2d: host -> staging.
 // The device address of pinned host memory the device can address, else null.
 const uint8_t* host_dev_ptr(const void* host) {
   cudaPointerAttributes a{};
@@ -1166,8 +1163,14 @@ const uint8_t* host_dev_ptr(const void* host) {
   return d;
 }
 
+// One host-buffer run: a copy kernel when the run is small (the copy
+// engine's fixed latency dominates), the host side is pinned memory the
+// device can address and both sides are 16-byte aligned; else a copy-engine
+// transfer (which also keeps large transfers off the SMs).  h2d: host ->
+// staging.
+constexpr size_t kCopyKernelMaxBytes = size_t(1) << 20;
 bl_status copy_run(const uint8_t* host, uint8_t* stage, size_t bytes, bool h2d, cudaStream_t stream) {
-  const uint8_t* hdev = host_dev_ptr(host);
+  const uint8_t* hdev = bytes <= kCopyKernelMaxBytes ? host_dev_ptr(host) : nullptr;
   if (hdev == nullptr || !aligned16(hdev) || !aligned16(stage)) {
     if (cudaMemcpyAsync(h2d ? static_cast<void*>(stage) : const_cast<uint8_t*>(host), h2d ? static_cast<const void*>(host) : stage,
                         bytes, h2d ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost, stream) != cudaSuccess) {

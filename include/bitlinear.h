@@ -232,9 +232,10 @@ BL_API bl_status bl_forward_grouped(int count, const bl_linear* problems, int bi
  * the device (problems with the same X, M and K share one copy; inputs whose
  * host bytes are exactly contiguous travel in one copy), the grouped forward
  * of bl_forward_grouped on the staged tensors, the outputs copied back
- * (exactly contiguous outputs in one copy).  A copy is a small kernel that
- * reads or writes the host bytes directly when they are pinned memory the
- * device can address (16-byte aligned), else a copy-engine transfer.  Only
+ * (exactly contiguous outputs in one copy).  A copy of at most 1 MiB is a
+ * small kernel that reads or writes the host bytes directly when they are
+ * pinned memory the device can address (16-byte aligned); other copies are
+ * copy-engine transfers.  Only
  * the tensors' own bytes are read or written.  The call
  * returns once everything is enqueued; the host buffers must stay valid
  * until the stream reaches that point.
