@@ -3,7 +3,7 @@
 This module only draws random numbers; it holds none of the BitLinear
 arithmetic.  Both the CUDA-path tests/benchmark and the CPU oracle consume the
 same arrays, generated on the host with torch's CPU generator so that every
-run (here or on a GPU machine) sees identical bits.
+run, on any machine with or without a GPU, sees identical bits.
 
 Recipe (per workload; ``seed`` defaults to 0):
   * weights:  W fp32 [N, K] = std * N(0, 1), generator seed = seed + 10*i for
