@@ -352,6 +352,10 @@ class PreparedGroupedHost:
     def __del__(self):
         g = getattr(self, "_graph", None)
         if g is not None and _lib is not None:
+            try:
+                torch.cuda.synchronize()   # no replay may still be running when the graph is freed
+            except Exception:
+                pass
             bl_graph_destroy(g)
             self._graph = None
 
